@@ -1,0 +1,179 @@
+"""fp64 CPU oracle for D = act(alpha * A.B + bias) and its ReLU sign mask.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py``'s CPU-baseline leg (``cpu_baseline`` / ``--impl reference``) may
+import this package.  The product path (the C-ABI library and its binding)
+never imports, links or runs anything here, and this package never imports the
+product: the two meet only at the seeded input generators, which hold no
+arithmetic of the method.
+
+The arithmetic lives in ``gemm_epi_oracle.c`` (plain C, IEEE double, OpenMP
+over output rows); this module compiles it with gcc on first use and marshals
+numpy arrays through ctypes.  Inputs are raw storage arrays (``uint16`` for
+fp16/bf16 bit patterns, ``uint8`` for e4m3 bytes); the C code decodes them
+itself.  Every function's docstring names the page passage it follows; the
+file header of ``gemm_epi_oracle.c`` lists them all.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gemm_epi_oracle.c")
+_LIB = os.path.join(_HERE, "libgemm_epi_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+DTYPES = ("f16", "bf16", "e4m3")
+EPILOGUES = ("none", "bias", "relu_bias", "relu_aux_bias", "gelu_bias")
+AXES = ("row", "col")
+LAYOUTS = ("kn", "nk")
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library with gcc (no fast-math: IEEE double)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared", "-Wall", "-Werror",
+             _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            # A test may point the loader at a deliberately mutated build of the
+            # same source (tests/test_oracle_mutants.py) to check that the pins
+            # catch the mutation.
+            path = os.environ.get("GEMM_EPI_ORACLE_LIB") or build()
+            lib = ctypes.CDLL(path)
+            i64, vp, dp, cp = ctypes.c_int64, ctypes.c_void_p, ctypes.c_double, ctypes.c_char_p
+            lib.oracle_decode_f16.argtypes = [ctypes.c_uint16]
+            lib.oracle_decode_f16.restype = dp
+            lib.oracle_decode_bf16.argtypes = [ctypes.c_uint16]
+            lib.oracle_decode_bf16.restype = dp
+            lib.oracle_decode_e4m3.argtypes = [ctypes.c_uint8]
+            lib.oracle_decode_e4m3.restype = dp
+            lib.oracle_gelu.argtypes = [dp]
+            lib.oracle_gelu.restype = dp
+            lib.oracle_gemm_epi.argtypes = [i64, i64, i64, cp, cp, cp, cp, vp, vp, vp, dp, dp,
+                                            vp, vp, vp]
+            lib.oracle_gemm_epi.restype = ctypes.c_int
+            lib.oracle_gemm_epi_sampled.argtypes = [i64, i64, i64, cp, cp, cp, cp, vp, vp, vp,
+                                                    dp, dp, i64, vp, vp, vp, vp, vp]
+            lib.oracle_gemm_epi_sampled.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _storage(a, dtype):
+    """Check a raw storage array against the input format and make it contiguous."""
+    want = np.uint8 if dtype == "e4m3" else np.uint16
+    a = np.ascontiguousarray(a)
+    if a.dtype != want:
+        raise TypeError(f"{dtype} storage must be {np.dtype(want).name}, got {a.dtype}")
+    return a
+
+
+def decode(bits, dtype: str) -> np.ndarray:
+    """Decode raw fp16 / bf16 / e4m3 bit patterns to float64 with the C decoders."""
+    lib = _load()
+    fn = {"f16": lib.oracle_decode_f16, "bf16": lib.oracle_decode_bf16,
+          "e4m3": lib.oracle_decode_e4m3}[dtype]
+    flat = np.asarray(bits).ravel()
+    return np.array([fn(int(v)) for v in flat], dtype=np.float64).reshape(np.shape(bits))
+
+
+def gelu(x: float) -> float:
+    """Exact GELU x*Phi(x) (erf form), as the oracle applies it."""
+    return _load().oracle_gelu(float(x))
+
+
+def _names(dtype, epilogue, bias_axis, b_layout):
+    if dtype not in DTYPES or epilogue not in EPILOGUES or bias_axis not in AXES \
+            or b_layout not in LAYOUTS:
+        raise ValueError(f"unknown oracle option {(dtype, epilogue, bias_axis, b_layout)}")
+    return tuple(s.encode() for s in (dtype, epilogue, bias_axis, b_layout))
+
+
+def gemm_epi(A, B, bias, *, dtype: str, epilogue: str, bias_axis: str = "row",
+             b_layout: str = "kn", scale_a: float = 1.0, scale_b: float = 1.0):
+    """Full fp64 result (D, pre-activation, mask) of act(alpha*A.B + bias).
+
+    A is (m, k) row-major storage; B is (k, n) for ``b_layout="kn"`` or (n, k)
+    for ``"nk"``; bias has length m (``"row"``: one value per output row,
+    added to every column -- the pages' default broadcast) or n (``"col"``).
+    Returns float64 D and pre (m, n) and a uint8 0/1 mask (m, n).
+    """
+    A = _storage(A, dtype)
+    B = _storage(B, dtype)
+    m, k = A.shape
+    n = B.shape[1] if b_layout == "kn" else B.shape[0]
+    if (B.shape[0] if b_layout == "kn" else B.shape[1]) != k:
+        raise ValueError("inner dimensions differ")
+    if bias is not None:
+        bias = _storage(bias, "bf16" if dtype == "e4m3" else dtype)
+        if bias.size != (m if bias_axis == "row" else n):
+            raise ValueError("bias length does not match its axis")
+    D = np.empty((m, n), np.float64)
+    pre = np.empty((m, n), np.float64)
+    mask = np.empty((m, n), np.uint8)
+    rc = _load().oracle_gemm_epi(m, n, k, *_names(dtype, epilogue, bias_axis, b_layout),
+                                 _ptr(A), _ptr(B), _ptr(bias), float(scale_a), float(scale_b),
+                                 _ptr(D), _ptr(pre), _ptr(mask))
+    if rc != 0:
+        raise RuntimeError(f"oracle_gemm_epi failed with status {rc}")
+    return D, pre, mask
+
+
+def gemm_epi_sampled(A, B, bias, rows, cols, *, dtype: str, epilogue: str,
+                     bias_axis: str = "row", b_layout: str = "kn", scale_a: float = 1.0,
+                     scale_b: float = 1.0, m: int | None = None, k: int | None = None):
+    """(D, pre, mask) at positions (rows[s], cols[s]); one fp64 dot product each.
+
+    ``A`` may be given as the full (m, k) storage array.  Same conventions as
+    :func:`gemm_epi`.
+    """
+    A = _storage(A, dtype)
+    B = _storage(B, dtype)
+    m_, k_ = A.shape
+    m = m_ if m is None else m
+    k = k_ if k is None else k
+    n = B.shape[1] if b_layout == "kn" else B.shape[0]
+    if bias is not None:
+        bias = _storage(bias, "bf16" if dtype == "e4m3" else dtype)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    cols = np.ascontiguousarray(cols, dtype=np.int64)
+    if rows.shape != cols.shape:
+        raise ValueError("rows and cols differ in length")
+    cnt = rows.size
+    D = np.empty(cnt, np.float64)
+    pre = np.empty(cnt, np.float64)
+    mask = np.empty(cnt, np.uint8)
+    rc = _load().oracle_gemm_epi_sampled(m, n, k, *_names(dtype, epilogue, bias_axis, b_layout),
+                                         _ptr(A), _ptr(B), _ptr(bias), float(scale_a),
+                                         float(scale_b), cnt, _ptr(rows), _ptr(cols), _ptr(D),
+                                         _ptr(pre), _ptr(mask))
+    if rc != 0:
+        raise RuntimeError(f"oracle_gemm_epi_sampled failed with status {rc}")
+    return D, pre, mask
+
+
+def threads() -> int:
+    """OpenMP threads the oracle will use (OMP_NUM_THREADS, else the CPU count)."""
+    env = os.environ.get("OMP_NUM_THREADS")
+    if env and env.isdigit():
+        return int(env)
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()

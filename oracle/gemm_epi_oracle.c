@@ -1,0 +1,260 @@
+/*
+ * gemm_epi_oracle.c -- plain, slow, obviously correct CPU reference for
+ *
+ *     D = act(alpha * (A . B) + bias)      and     mask = (alpha * (A . B) + bias) > 0
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may include, link,
+ * load or call this file; only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg do.  It shares no code, header, table or constant with the
+ * CUDA library: it decodes every input format itself from the format's
+ * definition and does all arithmetic in IEEE double.
+ *
+ * What is computed, and where the pages define it:
+ *   - the product A.B with a wide accumulator ("compute type 32F"): page
+ *     "PyTorch inference: cuBLASLt bias fusion optimization" (blog.hotdry.top),
+ *     paragraph 3.  The oracle accumulates in double, wider than the method.
+ *   - a bias vector added to the product: same page, paragraph 2 (EPILOGUE_BIAS);
+ *     its broadcast -- a length-m bias is added to every column of the (m,n)
+ *     result, a (1,n) bias to every row -- from "nvmath-python epilog bias
+ *     fusion parameters" (blog.hotdry.top), body paragraph 3, and
+ *     "nvmath-python cuBLASLt bias fusion for PyTorch inference"
+ *     (blog.hotdry.top), paragraph 5 (shape constraints).
+ *   - ReLU applied after the bias (RELU_BIAS): "nvmath-python epilog bias
+ *     fusion parameters", body paragraph 2.
+ *   - the auxiliary output of RELU_AUX_BIAS, the sign mask of the ReLU input
+ *     kept for the backward pass: same paragraph, and "nvmath-python cuBLASLt
+ *     bias fusion for PyTorch inference", paragraph 6.  Read as: bit set
+ *     exactly when the pre-activation is strictly greater than zero.
+ *   - GELU after the bias: "PyTorch inference: cuBLASLt bias fusion
+ *     optimization", paragraph 2; torch.nn.GELU() in "PyTorch 2.14 NVGEMM
+ *     epilogue fusion" (zdabc.icu), section "verifying torch.compile".  Read
+ *     as the exact erf form, 0.5 x (1 + erf(x / sqrt 2)).
+ *   - a scaling factor applied in the epilogue: "PyTorch 2.14 NVGEMM epilogue
+ *     fusion", section "why epilogue fusion matters".  Read as the FP8
+ *     per-tensor dequantisation alpha = s_A * s_B applied to the product,
+ *     before the bias; alpha = 1 for 16-bit inputs.
+ *
+ * Formats decoded here (from their definitions, not from any library):
+ *   fp16  IEEE binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits.
+ *   bf16  upper half of IEEE binary32: 1 sign, 8 exponent (bias 127), 7 fraction.
+ *   e4m3  OCP FP8 E4M3 ("fn" variant): 1 sign, 4 exponent (bias 7), 3 fraction,
+ *         no infinities, S.1111.111 is NaN, largest finite 448.
+ *
+ * Result of the full variant: D_ref (double, m x n, row-major) holds the
+ * activation output before any rounding to the output type; pre_ref (double,
+ * optional) holds the pre-activation p; mask_ref (uint8, optional) holds
+ * 1 where p > 0 else 0 for every epilogue.  The sampled variant computes the
+ * same three quantities at a list of (row, col) positions, one dot product
+ * each.
+ *
+ * Status codes: 0 ok, -1 bad argument (unknown name, non-positive size, NULL
+ * buffer where one is required), -2 out of memory.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---- the oracle's own vocabulary (independent of the CUDA library's enums) --- */
+enum { OR_F16 = 1, OR_BF16 = 2, OR_E4M3 = 3 };
+enum { OR_NONE = 10, OR_BIAS = 11, OR_RELU_BIAS = 12, OR_RELU_AUX_BIAS = 13, OR_GELU_BIAS = 14 };
+enum { OR_ROW = 20, OR_COL = 21 };
+enum { OR_KN = 30, OR_NK = 31 };
+
+static int dtype_code(const char *s) {
+    if (!s) return 0;
+    if (!strcmp(s, "f16")) return OR_F16;
+    if (!strcmp(s, "bf16")) return OR_BF16;
+    if (!strcmp(s, "e4m3")) return OR_E4M3;
+    return 0;
+}
+static int epi_code(const char *s) {
+    if (!s) return 0;
+    if (!strcmp(s, "none")) return OR_NONE;
+    if (!strcmp(s, "bias")) return OR_BIAS;
+    if (!strcmp(s, "relu_bias")) return OR_RELU_BIAS;
+    if (!strcmp(s, "relu_aux_bias")) return OR_RELU_AUX_BIAS;
+    if (!strcmp(s, "gelu_bias")) return OR_GELU_BIAS;
+    return 0;
+}
+static int axis_code(const char *s) {
+    if (!s) return 0;
+    if (!strcmp(s, "row")) return OR_ROW;
+    if (!strcmp(s, "col")) return OR_COL;
+    return 0;
+}
+static int layout_code(const char *s) {
+    if (!s) return 0;
+    if (!strcmp(s, "kn")) return OR_KN;
+    if (!strcmp(s, "nk")) return OR_NK;
+    return 0;
+}
+
+/* ---- format decoding, written from each format's bit-level definition ----- */
+
+double oracle_decode_f16(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    double v;
+    if (e == 0) {
+        v = ldexp((double)f, -24);                 /* subnormal: f * 2^(1-15-10) */
+    } else if (e == 31) {
+        v = f ? NAN : INFINITY;
+    } else {
+        v = ldexp(1.0 + (double)f / 1024.0, e - 15);
+    }
+    return sign ? -v : v;
+}
+
+double oracle_decode_bf16(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int e = (h >> 7) & 0xff;
+    int f = h & 0x7f;
+    double v;
+    if (e == 0) {
+        v = ldexp((double)f, -133);                /* subnormal: f * 2^(1-127-7) */
+    } else if (e == 255) {
+        v = f ? NAN : INFINITY;
+    } else {
+        v = ldexp(1.0 + (double)f / 128.0, e - 127);
+    }
+    return sign ? -v : v;
+}
+
+double oracle_decode_e4m3(uint8_t b) {
+    int sign = (b >> 7) & 1;
+    int e = (b >> 3) & 0xf;
+    int f = b & 0x7;
+    double v;
+    if (e == 15 && f == 7) {
+        v = NAN;                                   /* the only NaN pattern; no infinities */
+    } else if (e == 0) {
+        v = ldexp((double)f, -9);                  /* subnormal: f * 2^(1-7-3) */
+    } else {
+        v = ldexp(1.0 + (double)f / 8.0, e - 7);
+    }
+    return sign ? -v : v;
+}
+
+/* GELU, exact form: x * Phi(x) with Phi the standard normal CDF. */
+double oracle_gelu(double x) { return 0.5 * x * (1.0 + erf(x / sqrt(2.0))); }
+
+static double load(const void *base, int dt, int64_t idx) {
+    switch (dt) {
+    case OR_F16: return oracle_decode_f16(((const uint16_t *)base)[idx]);
+    case OR_BF16: return oracle_decode_bf16(((const uint16_t *)base)[idx]);
+    case OR_E4M3: return oracle_decode_e4m3(((const uint8_t *)base)[idx]);
+    }
+    return NAN;
+}
+
+/* The bias and the output share the input type for 16-bit inputs; for e4m3
+ * inputs they are bf16. */
+static int bias_dtype(int dt) { return dt == OR_E4M3 ? OR_BF16 : dt; }
+
+/* One output element after the product p = sum_t a(i,t) b(t,j) is known. */
+static void finish(double p, int epi, int axis, int bdt, const void *bias, int64_t i, int64_t j,
+                   double alpha, double *d, double *pre, uint8_t *mask) {
+    p = alpha * p;
+    if (epi != OR_NONE) p += load(bias, bdt, axis == OR_ROW ? i : j);
+    double y;
+    switch (epi) {
+    case OR_RELU_BIAS:
+    case OR_RELU_AUX_BIAS: y = p > 0.0 ? p : 0.0; break;
+    case OR_GELU_BIAS: y = oracle_gelu(p); break;
+    default: y = p; break;                         /* NONE and BIAS */
+    }
+    *d = y;
+    if (pre) *pre = p;
+    if (mask) *mask = (uint8_t)(p > 0.0);
+}
+
+static int check_args(int64_t m, int64_t n, int64_t k, int dt, int epi, int axis, int lay,
+                      const void *A, const void *B, const void *bias) {
+    if (m <= 0 || n <= 0 || k <= 0) return -1;
+    if (!dt || !epi || !axis || !lay) return -1;
+    if (!A || !B) return -1;
+    if (epi != OR_NONE && !bias) return -1;
+    return 0;
+}
+
+/*
+ * Full result.  Loop order i (rows, OpenMP) -> t (reduction) -> j (columns):
+ * each output row is accumulated in a double row buffer; B is decoded once
+ * into a (k, n) double array whatever its stored layout.
+ */
+int oracle_gemm_epi(int64_t m, int64_t n, int64_t k, const char *dtype, const char *epilogue,
+                    const char *bias_axis, const char *b_layout, const void *A, const void *B,
+                    const void *bias, double scale_a, double scale_b, double *D_ref,
+                    double *pre_ref, uint8_t *mask_ref) {
+    int dt = dtype_code(dtype), epi = epi_code(epilogue), axis = axis_code(bias_axis);
+    int lay = layout_code(b_layout);
+    if (check_args(m, n, k, dt, epi, axis, lay, A, B, bias) || !D_ref) return -1;
+    double alpha = dt == OR_E4M3 ? scale_a * scale_b : 1.0;
+    int bdt = bias_dtype(dt);
+
+    double *Bd = (double *)malloc((size_t)k * (size_t)n * sizeof(double));
+    if (!Bd) return -2;
+    for (int64_t t = 0; t < k; ++t)
+        for (int64_t j = 0; j < n; ++j)
+            Bd[t * n + j] = load(B, dt, lay == OR_KN ? t * n + j : j * k + t);
+
+    int err = 0;
+#pragma omp parallel
+    {
+        double *row = (double *)malloc((size_t)n * sizeof(double));
+        if (!row) {
+#pragma omp atomic write
+            err = -2;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < m; ++i) {
+            if (!row) continue;
+            for (int64_t j = 0; j < n; ++j) row[j] = 0.0;
+            for (int64_t t = 0; t < k; ++t) {
+                double a = load(A, dt, i * k + t);
+                const double *brow = Bd + t * n;
+                for (int64_t j = 0; j < n; ++j) row[j] += a * brow[j];
+            }
+            for (int64_t j = 0; j < n; ++j)
+                finish(row[j], epi, axis, bdt, bias, i, j, alpha, &D_ref[i * n + j],
+                       pre_ref ? &pre_ref[i * n + j] : NULL,
+                       mask_ref ? &mask_ref[i * n + j] : NULL);
+        }
+        free(row);
+    }
+    free(Bd);
+    return err;
+}
+
+/*
+ * The same quantities at `count` positions (rows[s], cols[s]): one plain dot
+ * product over t per position, read straight from the stored operands.
+ */
+int oracle_gemm_epi_sampled(int64_t m, int64_t n, int64_t k, const char *dtype,
+                            const char *epilogue, const char *bias_axis, const char *b_layout,
+                            const void *A, const void *B, const void *bias, double scale_a,
+                            double scale_b, int64_t count, const int64_t *rows,
+                            const int64_t *cols, double *D_ref, double *pre_ref,
+                            uint8_t *mask_ref) {
+    int dt = dtype_code(dtype), epi = epi_code(epilogue), axis = axis_code(bias_axis);
+    int lay = layout_code(b_layout);
+    if (check_args(m, n, k, dt, epi, axis, lay, A, B, bias) || !D_ref || !rows || !cols ||
+        count < 0)
+        return -1;
+    for (int64_t s = 0; s < count; ++s)
+        if (rows[s] < 0 || rows[s] >= m || cols[s] < 0 || cols[s] >= n) return -1;
+    double alpha = dt == OR_E4M3 ? scale_a * scale_b : 1.0;
+    int bdt = bias_dtype(dt);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t s = 0; s < count; ++s) {
+        int64_t i = rows[s], j = cols[s];
+        double p = 0.0;
+        for (int64_t t = 0; t < k; ++t)
+            p += load(A, dt, i * k + t) * load(B, dt, lay == OR_KN ? t * n + j : j * k + t);
+        finish(p, epi, axis, bdt, bias, i, j, alpha, &D_ref[s], pre_ref ? &pre_ref[s] : NULL,
+               mask_ref ? &mask_ref[s] : NULL);
+    }
+    return 0;
+}

@@ -1,0 +1,303 @@
+"""Pins for the fp64 CPU oracle against facts that do not come from the oracle.
+
+Each test checks the oracle against something fixed independently of it: a
+hand-computed case (tests/golden/tiny_cases.json), a textbook value, a
+library routine on a special case (numpy matmul, numpy/torch float
+conversions), or an invariant of the definition.  Together they are chosen so
+that a plausible slip anywhere in the oracle -- a dropped bias, a bias on the
+wrong axis, a transposed operand, a sign error in GELU, a ">=" for ">" in the
+mask, a wrong exponent bias in a decoder, a missing FP8 scale -- fails at least
+one of them (tests/test_oracle_mutants.py plants such slips and checks that).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import load_golden, to_storage_values
+
+from activation_epilogue_tcgen05_b200.workloads import Workload, make_problem, storage
+
+
+# ----------------------------------------------------------------------------- golden cases
+CASES = load_golden("tiny_cases.json")["cases"]
+
+
+def _case_inputs(c):
+    dt = c["dtype"]
+    if "e4m3_codes" in c:
+        a = np.array(c["e4m3_codes"]["a"], dtype=np.uint8)
+        b = np.array(c["e4m3_codes"]["b"], dtype=np.uint8)
+    else:
+        a = to_storage_values(c["a"], dt)
+        b = to_storage_values(c["b"], dt)
+    bias = to_storage_values(c["bias"], "bf16" if dt == "e4m3" else dt)
+    return a, b, bias
+
+
+@pytest.mark.parametrize("c", CASES, ids=[c["id"] for c in CASES])
+def test_golden_tiny_case(oracle_lib, c):
+    a, b, bias = _case_inputs(c)
+    D, pre, mask = oracle_lib.gemm_epi(
+        a, b, bias, dtype=c["dtype"], epilogue=c["epilogue"], bias_axis=c["bias_axis"],
+        b_layout=c["b_layout"], scale_a=c.get("scale_a", 1.0), scale_b=c.get("scale_b", 1.0))
+    want = np.array(c["d"], dtype=np.float64)
+    rtol = c.get("rtol", 0.0)
+    np.testing.assert_allclose(D, want, rtol=rtol, atol=0.0)
+    np.testing.assert_array_equal(mask, np.array(c["mask"], dtype=np.uint8))
+    # the sampled variant agrees at every position
+    rows, cols = np.meshgrid(np.arange(D.shape[0]), np.arange(D.shape[1]), indexing="ij")
+    Ds, pres, masks = oracle_lib.gemm_epi_sampled(
+        a, b, bias, rows.ravel(), cols.ravel(), dtype=c["dtype"], epilogue=c["epilogue"],
+        bias_axis=c["bias_axis"], b_layout=c["b_layout"], scale_a=c.get("scale_a", 1.0),
+        scale_b=c.get("scale_b", 1.0))
+    np.testing.assert_array_equal(Ds, D.ravel())
+    np.testing.assert_array_equal(masks, mask.ravel())
+
+
+# ----------------------------------------------------------------------------- decoders
+def test_decode_f16_every_code_matches_numpy(oracle_lib):
+    codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle_lib.decode(codes, "f16")
+    want = codes.view(np.float16).astype(np.float64)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    np.testing.assert_array_equal(got[ok], want[ok])
+
+
+def test_decode_bf16_every_code_matches_torch(oracle_lib):
+    codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle_lib.decode(codes, "bf16")
+    want = torch.from_numpy(codes.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    np.testing.assert_array_equal(got[ok], want[ok])
+
+
+def test_decode_e4m3_fixed_points(oracle_lib):
+    d = lambda code: float(oracle_lib.decode(np.array([code], np.uint8), "e4m3")[0])
+    assert d(0x38) == 1.0
+    assert d(0x7E) == 448.0
+    assert d(0x01) == 2.0 ** -9
+    assert d(0x08) == 2.0 ** -6           # smallest normal
+    assert d(0x07) == 7 * 2.0 ** -9       # largest subnormal
+    assert d(0x00) == 0.0 and math.copysign(1.0, d(0x80)) == -1.0
+    assert math.isnan(d(0x7F)) and math.isnan(d(0xFF))
+    for code in range(0x80):
+        if code != 0x7F:
+            assert d(code | 0x80) == -d(code)
+
+
+def test_decode_e4m3_every_code_matches_torch(oracle_lib):
+    codes = np.arange(256, dtype=np.uint16).astype(np.uint8)
+    got = oracle_lib.decode(codes, "e4m3")
+    want = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    assert ok.sum() == 254
+    np.testing.assert_array_equal(got[ok], want[ok])
+    # round trip of every finite code through the value
+    back = torch.from_numpy(got[ok]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(back[codes[ok] != 0x80], codes[ok][codes[ok] != 0x80])
+
+
+# ----------------------------------------------------------------------------- GELU
+def test_gelu_textbook_values(oracle_lib):
+    # Phi from a standard normal table: Phi(1), Phi(2), Phi(3)
+    assert oracle_lib.gelu(1.0) == pytest.approx(0.841344746068543, rel=1e-14)
+    assert oracle_lib.gelu(-1.0) == pytest.approx(-0.158655253931457, rel=1e-13)
+    assert oracle_lib.gelu(2.0) == pytest.approx(1.954499736103642, rel=1e-14)
+    assert oracle_lib.gelu(3.0) == pytest.approx(3 * 0.998650101968370, rel=1e-14)
+    assert oracle_lib.gelu(0.0) == 0.0
+
+
+@pytest.mark.parametrize("x", [0.25, 0.5, 1.0, 1.7, 3.0, 6.0])
+def test_gelu_odd_part_is_identity(oracle_lib, x):
+    # x*Phi(x) - (-x)*Phi(-x) = x*(Phi(x) + Phi(-x)) = x
+    assert oracle_lib.gelu(x) - oracle_lib.gelu(-x) == pytest.approx(x, rel=1e-15, abs=1e-15)
+
+
+def test_gelu_limits(oracle_lib):
+    assert oracle_lib.gelu(10.0) == pytest.approx(10.0, rel=1e-15)
+    assert abs(oracle_lib.gelu(-10.0)) < 1e-20
+
+
+# ----------------------------------------------------------------------------- vs numpy matmul
+def _decoded(arr, dtype):
+    if dtype == "f16":
+        return arr.view(np.float16).astype(np.float64)
+    t = torch.from_numpy(arr.view(np.int16 if dtype == "bf16" else np.uint8).copy())
+    t = t.view(torch.bfloat16 if dtype == "bf16" else torch.float8_e4m3fn)
+    return t.double().numpy()
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "e4m3"])
+@pytest.mark.parametrize("b_layout", ["kn", "nk"])
+@pytest.mark.parametrize("bias_axis", ["row", "col"])
+def test_pre_activation_equals_numpy_matmul_plus_bias(oracle_lib, dtype, b_layout, bias_axis):
+    wl = Workload("t", 37, 29, 53, dtype, "relu_aux_bias", bias_axis, b_layout, seed=3)
+    p = make_problem(wl)
+    A, B, bias = storage(p.A), storage(p.B), storage(p.bias)
+    D, pre, mask = oracle_lib.gemm_epi(A, B, bias, dtype=dtype, epilogue="relu_aux_bias",
+                                       bias_axis=bias_axis, b_layout=b_layout,
+                                       scale_a=p.scale_a, scale_b=p.scale_b)
+    a = _decoded(A, dtype)
+    b = _decoded(B, dtype)
+    if b_layout == "nk":
+        b = b.T
+    bias_v = _decoded(bias, "bf16" if dtype == "e4m3" else dtype)
+    want = (p.scale_a * p.scale_b) * (a @ b)
+    want = want + (bias_v[:, None] if bias_axis == "row" else bias_v[None, :])
+    np.testing.assert_allclose(pre, want, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(mask, (want > 0).astype(np.uint8))
+    np.testing.assert_array_equal(D, np.maximum(pre, 0.0))
+
+
+def test_none_is_bare_product(oracle_lib):
+    wl = Workload("t", 16, 24, 40, "f16", "none", "row", "kn", seed=4)
+    p = make_problem(wl)
+    A, B = storage(p.A), storage(p.B)
+    D, pre, _ = oracle_lib.gemm_epi(A, B, storage(p.bias), dtype="f16", epilogue="none")
+    np.testing.assert_allclose(D, _decoded(A, "f16") @ _decoded(B, "f16"), rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(D, pre)
+
+
+# ----------------------------------------------------------------------------- invariants
+@pytest.mark.parametrize("epilogue", ["bias", "relu_bias", "gelu_bias"])
+def test_identity_b(oracle_lib, epilogue):
+    """B = I (k = n): D = act(A + bias) elementwise."""
+    m, k = 9, 12
+    wl = Workload("t", m, k, k, "bf16", epilogue, "col", "kn", seed=5)
+    p = make_problem(wl)
+    A, bias = storage(p.A), storage(p.bias)
+    eye = to_storage_values(np.eye(k).tolist(), "bf16")
+    D, pre, _ = oracle_lib.gemm_epi(A, eye, bias, dtype="bf16", epilogue=epilogue,
+                                    bias_axis="col")
+    x = _decoded(A, "bf16") + _decoded(bias, "bf16")[None, :]
+    np.testing.assert_array_equal(pre, x)
+    if epilogue == "bias":
+        np.testing.assert_array_equal(D, x)
+    elif epilogue == "relu_bias":
+        np.testing.assert_array_equal(D, np.maximum(x, 0))
+    else:
+        for v, dv in zip(x.ravel(), D.ravel()):
+            assert dv == pytest.approx(0.5 * v * (1 + math.erf(v / math.sqrt(2))), rel=1e-15,
+                                       abs=1e-300)
+
+
+def test_zero_bias_equals_bias_free_product(oracle_lib):
+    wl = Workload("t", 11, 13, 17, "f16", "relu_bias", "row", "kn", seed=6,
+                  dist_bias=("zeros", 0))
+    p = make_problem(wl)
+    D, pre, _ = oracle_lib.gemm_epi(storage(p.A), storage(p.B), storage(p.bias), dtype="f16",
+                                    epilogue="relu_bias")
+    Dn, _, _ = oracle_lib.gemm_epi(storage(p.A), storage(p.B), None, dtype="f16",
+                                   epilogue="none")
+    np.testing.assert_array_equal(pre, Dn)
+    np.testing.assert_array_equal(D, np.maximum(Dn, 0))
+
+
+def test_relu_properties(oracle_lib):
+    wl = Workload("t", 33, 47, 64, "bf16", "relu_bias", "row", "kn", seed=7)
+    p = make_problem(wl)
+    D, pre, mask = oracle_lib.gemm_epi(storage(p.A), storage(p.B), storage(p.bias),
+                                       dtype="bf16", epilogue="relu_bias")
+    assert (D >= 0).all()
+    np.testing.assert_array_equal(D[pre > 0], pre[pre > 0])
+    assert (D[pre <= 0] == 0).all()
+    np.testing.assert_array_equal(mask, (pre > 0).astype(np.uint8))
+    frac = mask.mean()
+    assert 0.3 < frac < 0.7          # symmetric data: about half positive
+
+
+def test_bias_axis_swap_is_transpose(oracle_lib):
+    """ROW bias on (A, B) equals COL bias on (B^T, A^T), transposed."""
+    m, n, k = 10, 14, 20
+    wl = Workload("t", m, n, k, "f16", "gelu_bias", "row", "kn", seed=8)
+    p = make_problem(wl)
+    A, B, bias = storage(p.A), storage(p.B), storage(p.bias)
+    D1, _, _ = oracle_lib.gemm_epi(A, B, bias, dtype="f16", epilogue="gelu_bias",
+                                   bias_axis="row", b_layout="kn")
+    # (B^T)(n,k) as the A operand; A^T (k,m) as a kn B operand
+    D2, _, _ = oracle_lib.gemm_epi(np.ascontiguousarray(B.T), np.ascontiguousarray(A.T), bias,
+                                   dtype="f16", epilogue="gelu_bias", bias_axis="col",
+                                   b_layout="kn")
+    np.testing.assert_allclose(D2.T, D1, rtol=1e-13, atol=1e-13)
+
+
+def test_nk_layout_equals_kn(oracle_lib):
+    wl = Workload("t", 7, 19, 23, "bf16", "relu_aux_bias", "col", "kn", seed=9)
+    p = make_problem(wl)
+    A, B, bias = storage(p.A), storage(p.B), storage(p.bias)
+    D1, pre1, m1 = oracle_lib.gemm_epi(A, B, bias, dtype="bf16", epilogue="relu_aux_bias",
+                                       bias_axis="col", b_layout="kn")
+    D2, pre2, m2 = oracle_lib.gemm_epi(A, np.ascontiguousarray(B.T), bias, dtype="bf16",
+                                       epilogue="relu_aux_bias", bias_axis="col",
+                                       b_layout="nk")
+    np.testing.assert_array_equal(pre1, pre2)
+    np.testing.assert_array_equal(m1, m2)
+
+
+def test_fp8_unit_scales_equal_16bit_path(oracle_lib):
+    """e4m3 with s_A = s_B = 1 on integer values equals the fp16 path on the same values."""
+    wl = Workload("t", 12, 20, 32, "e4m3", "relu_aux_bias", "col", "kn", seed=10,
+                  dist_a=("int", 4), dist_b=("int", 4), dist_bias=("int", 8))
+    p = make_problem(wl, int_scales=True)
+    A8, B8, bias = storage(p.A), storage(p.B), storage(p.bias)
+    D8, pre8, m8 = oracle_lib.gemm_epi(A8, B8, bias, dtype="e4m3", epilogue="relu_aux_bias",
+                                       bias_axis="col", scale_a=1.0, scale_b=1.0)
+    A16 = to_storage_values(p.A.double().tolist(), "bf16")
+    B16 = to_storage_values(p.B.double().tolist(), "bf16")
+    D16, pre16, m16 = oracle_lib.gemm_epi(A16, B16, bias, dtype="bf16",
+                                          epilogue="relu_aux_bias", bias_axis="col")
+    np.testing.assert_array_equal(pre8, pre16)
+    np.testing.assert_array_equal(D8, D16)
+    np.testing.assert_array_equal(m8, m16)
+    # with scales s_A = 2, s_B = 0.5 (alpha = 1) nothing changes; with s_A = 2, s_B = 2
+    # the product (but not the bias) is multiplied by 4
+    D8b, pre8b, _ = oracle_lib.gemm_epi(A8, B8, bias, dtype="e4m3", epilogue="relu_aux_bias",
+                                        bias_axis="col", scale_a=2.0, scale_b=0.5)
+    np.testing.assert_array_equal(pre8b, pre8)
+    Dn, _, _ = oracle_lib.gemm_epi(A8, B8, None, dtype="e4m3", epilogue="none")
+    _, pre4, _ = oracle_lib.gemm_epi(A8, B8, bias, dtype="e4m3", epilogue="relu_aux_bias",
+                                     bias_axis="col", scale_a=2.0, scale_b=2.0)
+    np.testing.assert_array_equal(pre4 - 4 * Dn, pre8 - Dn)
+
+
+def test_integer_inputs_exact(oracle_lib):
+    """Integer operands in {-2..2}: every partial sum is an exact integer."""
+    wl = Workload("t", 24, 40, 64, "f16", "bias", "row", "kn", seed=11, dist_a=("int", 2),
+                  dist_b=("int", 2), dist_bias=("int", 2))
+    p = make_problem(wl)
+    D, _, _ = oracle_lib.gemm_epi(storage(p.A), storage(p.B), storage(p.bias), dtype="f16",
+                                  epilogue="bias")
+    want = (p.A.long() @ p.B.long() + p.bias.long()[:, None]).double().numpy()
+    np.testing.assert_array_equal(D, want)
+
+
+def test_sampled_matches_full(oracle_lib):
+    wl = Workload("t", 40, 36, 50, "e4m3", "gelu_bias", "col", "nk", seed=12)
+    p = make_problem(wl)
+    A, B, bias = storage(p.A), storage(p.B), storage(p.bias)
+    kw = dict(dtype="e4m3", epilogue="gelu_bias", bias_axis="col", b_layout="nk",
+              scale_a=p.scale_a, scale_b=p.scale_b)
+    D, pre, mask = oracle_lib.gemm_epi(A, B, bias, **kw)
+    rng = np.random.default_rng(0)
+    rows = rng.integers(0, 40, 200)
+    cols = rng.integers(0, 36, 200)
+    Ds, pres, masks = oracle_lib.gemm_epi_sampled(A, B, bias, rows, cols, **kw)
+    np.testing.assert_allclose(Ds, D[rows, cols], rtol=1e-13, atol=1e-15)
+    np.testing.assert_array_equal(masks, mask[rows, cols])
+
+
+def test_bad_arguments_rejected(oracle_lib):
+    a = to_storage_values([[1.0]], "f16")
+    with pytest.raises(ValueError):
+        oracle_lib.gemm_epi(a, a, a, dtype="f32", epilogue="bias")
+    with pytest.raises(ValueError):
+        oracle_lib.gemm_epi(a, a, a, dtype="f16", epilogue="tanh")
+    with pytest.raises(RuntimeError):
+        oracle_lib.gemm_epi(a, a, None, dtype="f16", epilogue="bias")
+    with pytest.raises(RuntimeError):
+        oracle_lib.gemm_epi_sampled(a, a, a, [1], [0], dtype="f16", epilogue="bias")
