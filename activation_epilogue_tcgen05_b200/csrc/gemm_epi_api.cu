@@ -1,0 +1,504 @@
+// gemm_epi_api.cu -- the C ABI declared in include/gemm_epi.h: plan creation
+// and kernel choice, argument and alignment checks, TMA tensor-map encoding
+// (cached per plan), launches, status-word handling.
+//
+// The plan / run / free life cycle mirrors the stateful interface of
+// "nvmath-python cuBLASLt bias fusion for PyTorch inference" (blog.hotdry.top),
+// paragraphs 3 and 5 (Matmul.plan(epilog=..., epilog_inputs=...), execute(),
+// free()); the epilogue set, the bias broadcast and the 16-byte alignment rule
+// follow "nvmath-python epilog bias fusion parameters" (blog.hotdry.top), body
+// paragraphs 2-3.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <unordered_set>
+
+#include "../../include/gemm_epi.h"
+#include "kernels.h"
+
+using namespace gemm_epi;
+
+namespace {
+
+constexpr uint64_t kPlanMagic = 0x67656d6d5f657069ull;   // "gemm_epi"
+
+struct Plan {
+    uint64_t magic;
+    int64_t m, n, k;
+    int dtype, epilogue, axis, b_layout;
+    gemm_epi_options opts;
+    int device, num_sms;
+    // kernel choice
+    int kernel;          // GEMM_EPI_KERNEL_TC1 / TC2 / SPLITK
+    int block_n;         // TC: tile width; SPLITK: 128
+    int nm;              // SPLITK: MMA N (batch rows rounded up)
+    int split;           // SPLITK: cluster size along k
+    int kb_per_cta;
+    int grid;
+    int group_m;
+    TcLauncher tc_launch = nullptr, tc_none_launch = nullptr;
+    SkLauncher sk_launch = nullptr, sk_none_launch = nullptr;
+    BiasActLauncher ba_launch = nullptr;
+    KernelInfo info{};
+    // FP8 scales (device pointers, borrowed)
+    const float *scale_a = nullptr, *scale_b = nullptr;
+    // device status word (owned)
+    unsigned int *status = nullptr;
+    // tensor-map cache, keyed on the operand pointers
+    bool maps_valid = false;
+    const void *cA = nullptr, *cB = nullptr;
+    void *cD = nullptr;
+    CUtensorMap tmA, tmB, tmD;
+};
+
+std::mutex g_mu;
+std::unordered_set<Plan *> g_plans;
+
+bool live(gemm_epi_plan_t h) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    Plan *p = reinterpret_cast<Plan *>(h);
+    return h && g_plans.count(p) && p->magic == kPlanMagic;
+}
+
+int esize(int dt) { return dt == GEMM_EPI_E4M3 ? 1 : 2; }
+
+// ----------------------------------------------------------------- tensor maps
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                              const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                              CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                              CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(ptr);
+    });
+    return fn;
+}
+
+CUtensorMapDataType tmap_type(int dt) {
+    switch (dt) {
+    case GEMM_EPI_F16: return CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    case GEMM_EPI_BF16: return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    default: return CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    }
+}
+
+// Row-major 2-D tensor: `inner` contiguous elements per row, `outer` rows.
+bool make_map(CUtensorMap *map, int dt, const void *ptr, int64_t inner, int64_t outer, uint32_t box_inner,
+              uint32_t box_outer) {
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+    cuuint64_t strides[1] = {(cuuint64_t)(inner * esize(dt))};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, tmap_type(dt), 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ----------------------------------------------------------------- kernel choice
+int num_sms_of(int dev) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    return v > 0 ? v : 148;
+}
+
+int round_nm(int64_t m) {
+    if (m <= 16) return 16;
+    if (m <= 32) return 32;
+    if (m <= 64) return 64;
+    return 128;
+}
+
+int choose(Plan *P) {
+    const int64_t m = P->m, n = P->n;
+    int kernel = P->opts.kernel;
+    if (kernel == GEMM_EPI_KERNEL_AUTO) kernel = m <= 64 ? GEMM_EPI_KERNEL_SPLITK : GEMM_EPI_KERNEL_TC1;
+    if (kernel == GEMM_EPI_KERNEL_SPLITK && m > 128) return GEMM_EPI_ERR_UNSUPPORTED;
+    P->kernel = kernel;
+    const bool b_mn = P->b_layout == GEMM_EPI_B_KN;
+    const int bk = 128 / esize(P->dtype);
+    const int64_t num_kb = (P->k + bk - 1) / bk;
+    const int sms = P->opts.max_ctas > 0 ? std::min(P->opts.max_ctas, P->num_sms) : P->num_sms;
+
+    if (kernel == GEMM_EPI_KERNEL_SPLITK) {
+        P->nm = round_nm(m);
+        P->block_n = 128;
+        const int64_t tiles_n = (n + 127) / 128;
+        const int max_split = sk_max_split(P->nm);
+        int split = P->opts.split_k;
+        if (split <= 0) {
+            split = (int)std::max<int64_t>(1, sms / std::max<int64_t>(1, tiles_n));
+            if (split > max_split) split = max_split;
+        }
+        if (split > max_split || split < 1) return GEMM_EPI_ERR_ARG;
+        if (split > num_kb) split = (int)num_kb;
+        P->kb_per_cta = (int)((num_kb + split - 1) / split);
+        split = (int)((num_kb + P->kb_per_cta - 1) / P->kb_per_cta);   // no CTA without work
+        P->split = split;
+        P->grid = (int)(tiles_n * split);
+        KernelInfo none_info;
+        if (!find_sk(P->dtype, GEMM_EPI_NONE, 0, b_mn, P->nm, &P->sk_none_launch, &none_info))
+            return GEMM_EPI_ERR_UNSUPPORTED;
+        if (!find_sk(P->dtype, P->epilogue, P->axis, b_mn, P->nm, &P->sk_launch, &P->info))
+            return GEMM_EPI_ERR_UNSUPPORTED;
+    } else {
+        const int cg = kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
+        const int bm = 128 * cg;
+        int bn = P->opts.block_n;
+        if (bn == 0) {
+            const int64_t tiles256 = ((m + bm - 1) / bm) * ((n + 255) / 256);
+            bn = tiles256 >= sms / cg ? 256 : 128;
+        }
+        if (bn != 128 && bn != 256) return GEMM_EPI_ERR_ARG;
+        P->block_n = bn;
+        const int64_t tiles = ((m + bm - 1) / bm) * ((n + bn - 1) / bn);
+        const int64_t units = std::min<int64_t>(tiles, cg == 2 ? sms / 2 : sms);
+        P->grid = (int)(units * cg);
+        P->group_m = 8;
+        KernelInfo none_info;
+        if (!find_tc(cg, P->dtype, GEMM_EPI_NONE, 0, b_mn, bn, &P->tc_none_launch, &none_info))
+            return GEMM_EPI_ERR_UNSUPPORTED;
+        if (!find_tc(cg, P->dtype, P->epilogue, P->axis, b_mn, bn, &P->tc_launch, &P->info))
+            return GEMM_EPI_ERR_UNSUPPORTED;
+        P->split = 1;
+    }
+    if (P->epilogue != GEMM_EPI_NONE && !find_bias_act(P->dtype, P->epilogue, P->axis, &P->ba_launch))
+        return GEMM_EPI_ERR_UNSUPPORTED;
+    return GEMM_EPI_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_run_args(Plan *P, const void *A, const void *B, const void *bias, void *D, uint32_t *aux) {
+    if (!A || !B || !D) return GEMM_EPI_ERR_NULL;
+    if (P->epilogue != GEMM_EPI_NONE && !bias) return GEMM_EPI_ERR_NULL;
+    if (P->epilogue == GEMM_EPI_RELU_AUX_BIAS && !aux) return GEMM_EPI_ERR_NULL;
+    if (P->dtype == GEMM_EPI_E4M3 && (!P->scale_a || !P->scale_b)) return GEMM_EPI_ERR_NULL;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return GEMM_EPI_ERR_ALIGN;
+    if (P->epilogue != GEMM_EPI_NONE && !aligned16(bias)) return GEMM_EPI_ERR_ALIGN;
+    if (P->epilogue == GEMM_EPI_RELU_AUX_BIAS && !aligned16(aux)) return GEMM_EPI_ERR_ALIGN;
+    return GEMM_EPI_OK;
+}
+
+int ensure_maps(Plan *P, const void *A, const void *B, void *D) {
+    if (P->maps_valid && P->cA == A && P->cB == B && P->cD == D) return GEMM_EPI_OK;
+    const int dt = P->dtype;
+    const int64_t m = P->m, n = P->n, k = P->k;
+    const int bk = 128 / esize(dt);
+    const bool b_kn = P->b_layout == GEMM_EPI_B_KN;
+    const int box_n = 128 / esize(dt);            // elements in one 128-byte row
+    bool ok = true;
+    if (P->kernel == GEMM_EPI_KERNEL_SPLITK) {
+        // operand "W" = B (128 output columns per tile), operand "X" = A (nm rows)
+        ok = ok && (b_kn ? make_map(&P->tmA, dt, B, n, k, box_n, bk) : make_map(&P->tmA, dt, B, k, n, bk, 128));
+        ok = ok && make_map(&P->tmB, dt, A, k, m, bk, P->nm);
+    } else {
+        const int cg = P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
+        const int bn_local = P->block_n / cg;
+        ok = ok && make_map(&P->tmA, dt, A, k, m, bk, 128);
+        ok = ok && (b_kn ? make_map(&P->tmB, dt, B, n, k, box_n, bk) : make_map(&P->tmB, dt, B, k, n, bk, bn_local));
+        const int out_dt = dt == GEMM_EPI_E4M3 ? GEMM_EPI_BF16 : dt;
+        ok = ok && make_map(&P->tmD, out_dt, D, n, m, 64, 32);
+    }
+    if (!ok) {
+        P->maps_valid = false;
+        return GEMM_EPI_ERR_CUDA;
+    }
+    P->cA = A;
+    P->cB = B;
+    P->cD = D;
+    P->maps_valid = true;
+    return GEMM_EPI_OK;
+}
+
+int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, cudaStream_t stream) {
+    const int bk = 128 / esize(P->dtype);
+    const int num_kb = (int)((P->k + bk - 1) / bk);
+    const int64_t pitch_words = ((P->n + 127) / 128) * 4;
+    cudaError_t e;
+    if (P->kernel == GEMM_EPI_KERNEL_SPLITK) {
+        SkLaunch L;
+        L.tmW = P->tmA;
+        L.tmX = P->tmB;
+        L.p.m = (int)P->m;
+        L.p.n = (int)P->n;
+        L.p.k = (int)P->k;
+        L.p.num_kb = num_kb;
+        L.p.kb_per_cta = P->kb_per_cta;
+        L.p.bias = bias;
+        L.p.D = D;
+        L.p.aux = aux;
+        L.p.aux_pitch_words = pitch_words;
+        L.p.scale_a = P->scale_a;
+        L.p.scale_b = P->scale_b;
+        L.p.status = P->status;
+        L.grid = P->grid;
+        L.cluster = P->split;
+        L.stream = stream;
+        e = (fused ? P->sk_launch : P->sk_none_launch)(L);
+    } else {
+        const int cg = P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
+        TcLaunch L;
+        L.tmA = P->tmA;
+        L.tmB = P->tmB;
+        L.tmD = P->tmD;
+        L.p.m = (int)P->m;
+        L.p.n = (int)P->n;
+        L.p.k = (int)P->k;
+        L.p.tiles_m = (int)((P->m + 128 * cg - 1) / (128 * cg));
+        L.p.tiles_n = (int)((P->n + P->block_n - 1) / P->block_n);
+        L.p.num_tiles = L.p.tiles_m * L.p.tiles_n;
+        L.p.num_kb = num_kb;
+        L.p.group_m = P->group_m;
+        L.p.bias = bias;
+        L.p.aux = aux;
+        L.p.aux_pitch_words = pitch_words;
+        L.p.scale_a = P->scale_a;
+        L.p.scale_b = P->scale_b;
+        L.p.status = P->status;
+        L.p.inject_stall = P->opts.inject_stall;
+        L.grid = P->grid;
+        L.stream = stream;
+        e = (fused ? P->tc_launch : P->tc_none_launch)(L);
+    }
+    return e == cudaSuccess ? GEMM_EPI_OK : GEMM_EPI_ERR_CUDA;
+}
+
+int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis, int b_layout,
+              const gemm_epi_options *opts, gemm_epi_plan_t *out) {
+    if (!out) return GEMM_EPI_ERR_ARG;
+    if (m <= 0 || n <= 0 || k <= 0) return GEMM_EPI_ERR_ARG;
+    if (m > 0x7fffffffll || n > 0x7fffffffll || k > 0x7fffffffll) return GEMM_EPI_ERR_ARG;
+    if (dtype < GEMM_EPI_F16 || dtype > GEMM_EPI_E4M3) return GEMM_EPI_ERR_ARG;
+    if (epilogue < GEMM_EPI_NONE || epilogue > GEMM_EPI_GELU_BIAS) return GEMM_EPI_ERR_ARG;
+    if (bias_axis != GEMM_EPI_BIAS_ROW && bias_axis != GEMM_EPI_BIAS_COL) return GEMM_EPI_ERR_ARG;
+    if (b_layout != GEMM_EPI_B_KN && b_layout != GEMM_EPI_B_NK) return GEMM_EPI_ERR_ARG;
+    gemm_epi_options o{};
+    if (opts) o = *opts;
+    if (o.kernel < GEMM_EPI_KERNEL_AUTO || o.kernel > GEMM_EPI_KERNEL_SPLITK) return GEMM_EPI_ERR_ARG;
+    if (o.block_n != 0 && o.block_n != 128 && o.block_n != 256) return GEMM_EPI_ERR_ARG;
+    if (o.split_k < 0 || o.split_k > 8 || o.max_ctas < 0) return GEMM_EPI_ERR_ARG;
+    if (o.inject_stall != 0 && o.inject_stall != 1) return GEMM_EPI_ERR_ARG;
+    if (o.inject_stall && o.kernel == GEMM_EPI_KERNEL_SPLITK) return GEMM_EPI_ERR_UNSUPPORTED;
+    // 16-byte row pitches (TMA strides; the pages' 16-byte alignment rule)
+    const int es = esize(dtype);
+    const int out_es = 2;
+    if ((k * es) % 16 != 0) return GEMM_EPI_ERR_ALIGN;
+    if ((n * es) % 16 != 0 || (n * out_es) % 16 != 0) return GEMM_EPI_ERR_ALIGN;
+
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return GEMM_EPI_ERR_NO_DEVICE;
+    }
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0) return GEMM_EPI_ERR_NO_DEVICE;
+
+    Plan *P = new (std::nothrow) Plan();
+    if (!P) return GEMM_EPI_ERR_CUDA;
+    P->magic = kPlanMagic;
+    P->m = m;
+    P->n = n;
+    P->k = k;
+    P->dtype = dtype;
+    P->epilogue = epilogue;
+    P->axis = epilogue == GEMM_EPI_NONE ? GEMM_EPI_BIAS_ROW : bias_axis;
+    P->b_layout = b_layout;
+    P->opts = o;
+    P->device = dev;
+    P->num_sms = num_sms_of(dev);
+    int rc = choose(P);
+    if (rc != GEMM_EPI_OK) {
+        delete P;
+        return rc;
+    }
+    if (cudaMalloc(&P->status, 256) != cudaSuccess || cudaMemset(P->status, 0, 256) != cudaSuccess) {
+        cudaGetLastError();
+        if (P->status) cudaFree(P->status);
+        delete P;
+        return GEMM_EPI_ERR_CUDA;
+    }
+    if (getenv("GEMM_EPI_LOG")) {
+        fprintf(stderr,
+                "gemm_epi plan m=%lld n=%lld k=%lld dtype=%d epi=%d axis=%d b=%d -> kernel=%d bn=%d nm=%d "
+                "split=%d grid=%d stages=%d smem=%d\n",
+                (long long)m, (long long)n, (long long)k, dtype, epilogue, bias_axis, b_layout, P->kernel,
+                P->block_n, P->nm, P->split, P->grid, P->info.stages, P->info.smem_bytes);
+    }
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        g_plans.insert(P);
+    }
+    *out = reinterpret_cast<gemm_epi_plan_t>(P);
+    return GEMM_EPI_OK;
+}
+
+}  // namespace
+
+// ----------------------------------------------------------------- lookups
+namespace gemm_epi {
+bool find_tc(int cg, int dt, int epi, int axis, bool b_mn, int bn, TcLauncher *l, KernelInfo *i) {
+    KernelInfo tmp;
+    if (!i) i = &tmp;
+    switch (dt) {
+    case DT_F16: return find_tc_f16(cg, epi, axis, b_mn, bn, l, i);
+    case DT_BF16: return find_tc_bf16(cg, epi, axis, b_mn, bn, l, i);
+    case DT_E4M3: return find_tc_e4m3(cg, epi, axis, b_mn, bn, l, i);
+    }
+    return false;
+}
+bool find_sk(int dt, int epi, int axis, bool w_mn, int nm, SkLauncher *l, KernelInfo *i) {
+    KernelInfo tmp;
+    if (!i) i = &tmp;
+    switch (dt) {
+    case DT_F16: return find_sk_f16(epi, axis, w_mn, nm, l, i);
+    case DT_BF16: return find_sk_bf16(epi, axis, w_mn, nm, l, i);
+    case DT_E4M3: return find_sk_e4m3(epi, axis, w_mn, nm, l, i);
+    }
+    return false;
+}
+}  // namespace gemm_epi
+
+// ----------------------------------------------------------------- C ABI
+extern "C" {
+
+int gemm_epi_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis,
+                  gemm_epi_plan_t *out) {
+    return make_plan(m, n, k, dtype, epilogue, bias_axis, GEMM_EPI_B_KN, nullptr, out);
+}
+
+int gemm_epi_plan_ex(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis, int b_layout,
+                     gemm_epi_plan_t *out) {
+    return make_plan(m, n, k, dtype, epilogue, bias_axis, b_layout, nullptr, out);
+}
+
+int gemm_epi_plan_opts(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis, int b_layout,
+                       const gemm_epi_options *opts, gemm_epi_plan_t *out) {
+    return make_plan(m, n, k, dtype, epilogue, bias_axis, b_layout, opts, out);
+}
+
+int gemm_epi_set_scales(gemm_epi_plan_t plan, const float *d_scale_a, const float *d_scale_b) {
+    if (!live(plan)) return GEMM_EPI_ERR_ARG;
+    Plan *P = reinterpret_cast<Plan *>(plan);
+    if (P->dtype != GEMM_EPI_E4M3) return GEMM_EPI_ERR_ARG;
+    if (!d_scale_a || !d_scale_b) return GEMM_EPI_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(d_scale_a) & 3u) || (reinterpret_cast<uintptr_t>(d_scale_b) & 3u))
+        return GEMM_EPI_ERR_ALIGN;
+    P->scale_a = d_scale_a;
+    P->scale_b = d_scale_b;
+    return GEMM_EPI_OK;
+}
+
+int gemm_epi_run(gemm_epi_plan_t plan, const void *A, const void *B, const void *bias, void *D, uint32_t *aux,
+                 void *stream) {
+    if (!live(plan)) return GEMM_EPI_ERR_ARG;
+    Plan *P = reinterpret_cast<Plan *>(plan);
+    int rc = check_run_args(P, A, B, bias, D, aux);
+    if (rc != GEMM_EPI_OK) return rc;
+    rc = ensure_maps(P, A, B, D);
+    if (rc != GEMM_EPI_OK) return rc;
+    return launch_main(P, true, bias, D, aux, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gemm_epi_unfused_run(gemm_epi_plan_t plan, const void *A, const void *B, const void *bias, void *D,
+                         uint32_t *aux, void *stream) {
+    if (!live(plan)) return GEMM_EPI_ERR_ARG;
+    Plan *P = reinterpret_cast<Plan *>(plan);
+    int rc = check_run_args(P, A, B, bias, D, aux);
+    if (rc != GEMM_EPI_OK) return rc;
+    rc = ensure_maps(P, A, B, D);
+    if (rc != GEMM_EPI_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    rc = launch_main(P, false, bias, D, aux, s);
+    if (rc != GEMM_EPI_OK || P->epilogue == GEMM_EPI_NONE) return rc;
+    const int64_t pitch_words = ((P->n + 127) / 128) * 4;
+    const int64_t total = P->m * pitch_words;
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, (int64_t)P->num_sms * 16);
+    cudaError_t e = P->ba_launch(D, bias, aux, (int)P->m, (int)P->n, pitch_words, (int)blocks, s);
+    return e == cudaSuccess ? GEMM_EPI_OK : GEMM_EPI_ERR_CUDA;
+}
+
+int gemm_epi_check(gemm_epi_plan_t plan, void *stream) {
+    if (!live(plan)) return GEMM_EPI_ERR_ARG;
+    Plan *P = reinterpret_cast<Plan *>(plan);
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GEMM_EPI_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpy(&word, P->status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GEMM_EPI_ERR_CUDA;
+    if (word != 0) {
+        cudaMemset(P->status, 0, sizeof(word));
+        return GEMM_EPI_ERR_TIMEOUT;
+    }
+    return GEMM_EPI_OK;
+}
+
+int gemm_epi_plan_query(gemm_epi_plan_t plan, gemm_epi_plan_info *info) {
+    if (!live(plan) || !info) return GEMM_EPI_ERR_ARG;
+    Plan *P = reinterpret_cast<Plan *>(plan);
+    info->kernel = P->kernel;
+    info->block_m = P->kernel == GEMM_EPI_KERNEL_SPLITK ? P->nm : P->info.block_m;
+    info->block_n = P->block_n;
+    info->block_k = P->info.block_k;
+    info->stages = P->info.stages;
+    info->split_k = P->split;
+    info->grid = P->grid;
+    info->cluster = P->kernel == GEMM_EPI_KERNEL_SPLITK ? P->split : (P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1);
+    info->threads = P->info.threads;
+    info->smem_bytes = P->info.smem_bytes;
+    if (P->kernel == GEMM_EPI_KERNEL_SPLITK) {
+        info->tiles = (int)((P->n + 127) / 128);
+    } else {
+        const int bm = P->kernel == GEMM_EPI_KERNEL_TC2 ? 256 : 128;
+        info->tiles = (int)(((P->m + bm - 1) / bm) * ((P->n + P->block_n - 1) / P->block_n));
+    }
+    return GEMM_EPI_OK;
+}
+
+int gemm_epi_free(gemm_epi_plan_t plan) {
+    Plan *P = reinterpret_cast<Plan *>(plan);
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!plan || !g_plans.count(P)) return GEMM_EPI_ERR_ARG;
+        g_plans.erase(P);
+    }
+    if (P->status) cudaFree(P->status);
+    P->magic = 0;
+    delete P;
+    return GEMM_EPI_OK;
+}
+
+const char *gemm_epi_status_string(int status) {
+    switch (status) {
+    case GEMM_EPI_OK: return "ok";
+    case GEMM_EPI_ERR_ARG: return "invalid argument (size, enum, option or plan handle)";
+    case GEMM_EPI_ERR_ALIGN: return "pointer not 16-byte aligned or row pitch not a multiple of 16 bytes";
+    case GEMM_EPI_ERR_NULL: return "required pointer is NULL (operand, bias, aux or FP8 scales)";
+    case GEMM_EPI_ERR_UNSUPPORTED: return "combination not supported by this build";
+    case GEMM_EPI_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case GEMM_EPI_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case GEMM_EPI_ERR_NO_DEVICE: return "no current sm_100 (B200-class) CUDA device";
+    }
+    return "unknown status";
+}
+
+int64_t gemm_epi_aux_pitch_bytes(int64_t n) { return n <= 0 ? 0 : ((n + 127) / 128) * 16; }
+
+int gemm_epi_version(void) { return 100; }
+
+}  // extern "C"

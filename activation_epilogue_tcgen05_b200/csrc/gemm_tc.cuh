@@ -1,0 +1,502 @@
+// gemm_tc.cuh -- persistent, warp-specialised tcgen05 GEMM with the bias /
+// ReLU / GELU / sign-mask / FP8-scale epilogue fused in.
+//
+//   D = act(alpha * A.B + bias),   aux bit = (alpha * A.B + bias) > 0
+//
+// The fused epilogue follows "PyTorch inference: cuBLASLt bias fusion
+// optimization" (blog.hotdry.top), paragraph 2 (bias -- and GELU -- applied in
+// the GEMM kernel itself, no separate add kernel, no write-back of the
+// intermediate) and "nvmath-python epilog bias fusion parameters"
+// (blog.hotdry.top), body paragraphs 2-3 (BIAS / RELU_BIAS / RELU_AUX_BIAS,
+// the ReLU input's sign mask, length-m bias added to every column).  The FP8
+// scale is the epilogue "scaling factor" of "PyTorch 2.14 NVGEMM epilogue
+// fusion" (zdabc.icu), section "why epilogue fusion matters".  The kernel
+// design is this library's own, for sm_100a.
+//
+// Roles (one CTA per SM, or one CTA pair per two SMs when CG == 2):
+//   warp 0      TMA producer: streams A and B k-blocks into a STAGES-deep
+//               ring of 128-byte-swizzled shared-memory stages.
+//   warp 1      TMEM allocator and MMA issuer: one thread issues
+//               tcgen05.mma (M = 128*CG, N = BN, K = 32 bytes per step) into
+//               one of two fp32 accumulators in tensor memory; tcgen05.commit
+//               frees ring stages and publishes finished accumulators.
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time, then
+//               scale, bias, activation, sign-mask bits, RNE cast, 128-byte
+//               swizzled staging in shared memory and TMA stores of D; the
+//               mask goes out as 16-byte vector stores.  With two
+//               accumulators the epilogue of tile t overlaps the mainloop of
+//               tile t+1.
+//
+// Every wait is bounded: after TIMEOUT_NS without progress the waiting thread
+// records a code in the caller's status word, raises a CTA-wide abort flag and
+// every role winds down (waiting, again bounded, for its own copies and MMAs
+// in flight) so that tensor memory is always released and the kernel returns.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace gemm_epi {
+
+enum : int { DT_F16 = 0, DT_BF16 = 1, DT_E4M3 = 2 };
+enum : int { EPI_NONE = 0, EPI_BIAS = 1, EPI_RELU = 2, EPI_RELU_AUX = 3, EPI_GELU = 4 };
+enum : int { AXIS_ROW = 0, AXIS_COL = 1 };
+
+// Status-word bits written by kernels that gave up waiting.
+enum : unsigned int {
+    ST_TIMEOUT_PRODUCER = 1u << 0,
+    ST_TIMEOUT_MMA = 1u << 1,
+    ST_TIMEOUT_EPILOGUE = 1u << 2,
+    ST_TIMEOUT_DRAIN = 1u << 3,
+    ST_TIMEOUT_SPLITK = 1u << 4,
+};
+
+constexpr uint64_t TIMEOUT_NS = 1000000000ull;    // 1 s without progress on one wait
+constexpr uint64_t DRAIN_TIMEOUT_NS = 100000000ull;  // 100 ms for the wind-down waits
+
+struct TcParams {
+    int m, n, k;
+    int tiles_m, tiles_n, num_tiles, num_kb;
+    int group_m;                 // tile-raster group height (in tiles along m)
+    const void *bias;            // length m (ROW) or n (COL), output type
+    uint32_t *aux;               // RELU_AUX only
+    int64_t aux_pitch_words;     // ceil(n/128)*4
+    const float *scale_a;        // E4M3 only (device scalars)
+    const float *scale_b;
+    unsigned int *status;        // device status word
+    int inject_stall;            // testing only: 1 = the MMA issuer publishes no accumulator
+};
+
+// Bounded mbarrier wait.  Returns false when this CTA is aborting (this wait
+// timed out, or another role already raised the abort flag).
+template <bool CLUSTER_SCOPE>
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                             unsigned int *status, unsigned int code,
+                                             uint64_t limit_ns = TIMEOUT_NS) {
+    auto poll = [&]() {
+        return CLUSTER_SCOPE ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity);
+    };
+    if (poll()) return true;
+    const uint64_t t0 = ptx::globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (poll()) return true;
+        if ((i & 15u) == 0u) {
+            if (*abort_flag) return false;
+            if (ptx::globaltimer() - t0 > limit_ns) {
+                *abort_flag = 1;
+                atomicOr(status, code);
+                return false;
+            }
+        }
+    }
+}
+
+// Wind-down wait used after an abort: waits for this CTA's own copies or MMAs
+// still in flight, ignoring the abort flag, for at most DRAIN_TIMEOUT_NS.
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, unsigned int *status) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((i & 15u) == 0u && ptx::globaltimer() - t0 > DRAIN_TIMEOUT_NS) {
+            atomicOr(status, ST_TIMEOUT_DRAIN);
+            return false;
+        }
+    }
+}
+
+template <int DT>
+struct OutT;
+template <>
+struct OutT<DT_F16> {
+    using type = __half;
+    static __device__ __forceinline__ uint32_t pack(float a, float b) {
+        __half2 h = __floats2half2_rn(a, b);
+        return *reinterpret_cast<uint32_t *>(&h);
+    }
+    static __device__ __forceinline__ float load(const void *p, int64_t i) {
+        return __half2float(reinterpret_cast<const __half *>(p)[i]);
+    }
+};
+template <>
+struct OutT<DT_BF16> {
+    using type = __nv_bfloat16;
+    static __device__ __forceinline__ uint32_t pack(float a, float b) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<uint32_t *>(&h);
+    }
+    static __device__ __forceinline__ float load(const void *p, int64_t i) {
+        return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+    }
+};
+template <>
+struct OutT<DT_E4M3> : OutT<DT_BF16> {};   // e4m3 operands -> bf16 bias and output
+
+// 16-bit bias values -> fp32 (8 packed values from one 16-byte load).
+template <int DT>
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if constexpr (DT == DT_F16) {
+            __half2 h = *reinterpret_cast<const __half2 *>(&w[i]);
+            float2 t = __half22float2(h);
+            f[2 * i] = t.x;
+            f[2 * i + 1] = t.y;
+        } else {
+            __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&w[i]);
+            float2 t = __bfloat1622float2(h);
+            f[2 * i] = t.x;
+            f[2 * i + 1] = t.y;
+        }
+    }
+}
+
+template <int EPI>
+__device__ __forceinline__ float activate(float x) {
+    if constexpr (EPI == EPI_RELU || EPI == EPI_RELU_AUX) {
+        return x > 0.0f ? x : 0.0f;
+    } else if constexpr (EPI == EPI_GELU) {
+        return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+    } else {
+        return x;
+    }
+}
+
+template <int DT_, int EPI_, int AXIS_, bool B_MN_, int BN_, int CG_, int STAGES_>
+struct TcCfg {
+    static constexpr int DT = DT_, EPI = EPI_, AXIS = AXIS_, BN = BN_, CG = CG_, STAGES = STAGES_;
+    static constexpr bool B_MN = B_MN_;             // B stored (k, n): N contiguous
+    static constexpr int ESIZE = DT == DT_E4M3 ? 1 : 2;
+    static constexpr int KIND = DT == DT_E4M3 ? 1 : 0;
+    static constexpr uint32_t FMT = DT == DT_BF16 ? 1u : 0u;
+    static constexpr int BM = 128;                  // output rows per CTA
+    static constexpr int BK = 128 / ESIZE;          // k per stage: one 128-byte swizzle row
+    static constexpr int UMMA_K = 32 / ESIZE;       // k per tcgen05.mma
+    static constexpr int KSTEPS = BK / UMMA_K;      // 4
+    static constexpr int BN_LOCAL = BN / CG;        // B rows (n) this CTA loads
+    static constexpr int A_BYTES = BM * 128;
+    static constexpr int B_BYTES = BN_LOCAL * 128;
+    static constexpr int B_BOX_N = 128 / ESIZE;     // n per 128-byte MN-major box
+    static constexpr int B_BOXES = B_MN ? BN_LOCAL / B_BOX_N : 1;
+    static constexpr int B_BOX_BYTES = B_MN ? BK * 128 : B_BYTES;
+    static constexpr int EPI_WARPS = 4;
+    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+    static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                   : (2 * BN <= 256) ? 256 : 512;
+    static constexpr int STG_BYTES = 32 * 128;      // per epilogue warp: 32 rows x 64 outputs
+    // shared-memory layout (offsets from a 1024-byte aligned base)
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_BIAS = OFF_STG + EPI_WARPS * STG_BYTES;
+    static constexpr int BIAS_FLOATS = (EPI != EPI_NONE && AXIS == AXIS_COL) ? BN : 0;
+    static constexpr int OFF_BAR = OFF_BIAS + EPI_WARPS * BIAS_FLOATS * 4;
+    static constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
+    static_assert(BN % 128 == 0 && BN <= 256, "BN must be 128 or 256");
+    static_assert(2 * BN <= 512, "two accumulators must fit in tensor memory");
+    static_assert(B_MN == false || BN_LOCAL % B_BOX_N == 0, "MN-major B tile must be whole boxes");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "stage alignment");
+};
+
+// Tile index -> (tile_m, tile_n) with a grouped raster: GROUP_M tile-rows are
+// walked column by column so that concurrently resident CTAs share A and B
+// panels in L2.
+__device__ __forceinline__ void tile_coords(const TcParams &p, int t, int &tm, int &tn) {
+    const int per_group = p.group_m * p.tiles_n;
+    const int g = t / per_group;
+    const int first = g * p.group_m;
+    const int rows = min(p.group_m, p.tiles_m - first);
+    const int r = t - g * per_group;
+    tm = first + r % rows;
+    tn = r / rows;
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmD, const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sb = ptx::smem_addr(smem);
+    const uint32_t sA = sb + C::OFF_A, sB = sb + C::OFF_B, sStg = sb + C::OFF_STG;
+    float *bias_smem = reinterpret_cast<float *>(smem + C::OFF_BIAS);
+    const uint32_t bar0 = sb + C::OFF_BAR;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+    auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
+    auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
+    const uint32_t done_bar = bar0 + 8u * (2 * C::STAGES + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+
+    const int warp = ptx::warp_id();
+    const int lane = ptx::lane_id();
+    const uint32_t rank = C::CG == 2 ? ptx::cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int unit = C::CG == 2 ? (blockIdx.x >> 1) : blockIdx.x;        // tile-processing unit
+    const int units = C::CG == 2 ? (gridDim.x >> 1) : gridDim.x;
+
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&tmA);
+        ptx::prefetch_tmap(&tmB);
+        ptx::prefetch_tmap(&tmD);
+        for (int s = 0; s < C::STAGES; ++s) {
+            ptx::mbar_init(full_bar(s), 1);
+            ptx::mbar_init(empty_bar(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            ptx::mbar_init(tfull_bar(a), 1);
+            ptx::mbar_init(tempty_bar(a), C::EPI_WARPS * C::CG);
+        }
+        ptx::mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        ptx::fence_mbarrier_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc<C::CG>(ptx::smem_addr(tmem_slot), C::TMEM_COLS);
+        ptx::tmem_relinquish<C::CG>();
+    }
+    ptx::tc_fence_before();
+    if constexpr (C::CG == 2) ptx::cluster_sync(); else __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            uint32_t issued = 0;
+            bool ok = true;
+            for (int t = unit; ok && t < p.num_tiles; t += units) {
+                int tm, tn;
+                tile_coords(p, t, tm, tn);
+                const int m0 = tm * (C::BM * C::CG) + (int)rank * C::BM;
+                const int nb = tn * C::BN + (int)rank * C::BN_LOCAL;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!wait_bounded<false>(empty_bar(stage), phase ^ 1u, abort_flag, p.status,
+                                             ST_TIMEOUT_PRODUCER)) {
+                        ok = false;
+                        break;
+                    }
+                    uint32_t fb = full_bar(stage);
+                    if constexpr (C::CG == 2) {
+                        fb = ptx::mapa(fb, 0);      // the pair's leader counts both CTAs' bytes
+                        if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * (C::A_BYTES + C::B_BYTES));
+                    } else {
+                        ptx::mbar_arrive_expect_tx(fb, C::A_BYTES + C::B_BYTES);
+                    }
+                    const int k0 = kb * C::BK;
+                    const uint32_t a_dst = sA + stage * C::A_BYTES;
+                    const uint32_t b_dst = sB + stage * C::B_BYTES;
+                    auto load = [&](uint32_t dst, const CUtensorMap *map, int c0, int c1) {
+                        if constexpr (C::CG == 2)
+                            ptx::tma_load_2d_pair(dst, map, fb, c0, c1, 0x1000000000000000ull);
+                        else
+                            ptx::tma_load_2d(dst, map, fb, c0, c1, 0x1000000000000000ull);
+                    };
+                    load(a_dst, &tmA, k0, m0);
+                    if constexpr (C::B_MN) {
+#pragma unroll
+                        for (int b = 0; b < C::B_BOXES; ++b)
+                            load(b_dst + b * C::B_BOX_BYTES, &tmB, nb + b * C::B_BOX_N, k0);
+                    } else {
+                        load(b_dst, &tmB, k0, nb);
+                    }
+                    ++issued;
+                    if (++stage == (uint32_t)C::STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok && (C::CG == 1 || leader)) {
+                // wind down: wait (bounded) until the loads still in flight have landed
+                const uint32_t back = issued < (uint32_t)C::STAGES ? issued : (uint32_t)C::STAGES;
+                for (uint32_t j = issued - back; j < issued; ++j)
+                    wait_drain(full_bar(j % C::STAGES), (j / C::STAGES) & 1u, p.status);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && leader) {
+            constexpr uint32_t idesc = make_idesc(C::FMT, false, C::B_MN, 128 * C::CG, C::BN);
+            uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+            bool ok = true;
+            // with inject_stall nothing is issued or committed: the epilogue's
+            // bounded wait for the first accumulator runs out (failure-path test)
+            for (int t = unit; ok && !p.inject_stall && t < p.num_tiles; t += units) {
+                if (!wait_bounded<C::CG == 2>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status,
+                                              ST_TIMEOUT_MMA)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * C::BN;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!wait_bounded<false>(full_bar(stage), phase, abort_flag, p.status, ST_TIMEOUT_MMA)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t a_base = sA + stage * C::A_BYTES;
+                    const uint32_t b_base = sB + stage * C::B_BYTES;
+#pragma unroll
+                    for (int ks = 0; ks < C::KSTEPS; ++ks) {
+                        const uint64_t ad = make_sdesc(a_base + ks * 32, 16, 1024);
+                        const uint64_t bd = C::B_MN ? make_sdesc(b_base + ks * C::UMMA_K * 128, C::B_BOX_BYTES, 1024)
+                                                    : make_sdesc(b_base + ks * 32, 16, 1024);
+                        ptx::mma<C::CG, C::KIND>(d_tmem, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+                    }
+                    if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(empty_bar(stage), 0x3);
+                    else ptx::mma_commit(empty_bar(stage));
+                    if (++stage == (uint32_t)C::STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(tfull_bar(acc), 0x3);
+                else ptx::mma_commit(tfull_bar(acc));
+                if (++acc == 2u) { acc = 0; acc_phase ^= 1u; }
+            }
+            // every MMA issued by this thread has completed once done_bar flips
+            if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(done_bar, 0x1);
+            else ptx::mma_commit(done_bar);
+            wait_drain(done_bar, 0, p.status);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        using O = OutT<C::DT>;
+        const int ew = warp - 2;                 // epilogue warp 0..3
+        const int q = warp & 3;                  // TMEM lane quadrant this warp may access
+        const uint32_t stg = sStg + ew * C::STG_BYTES;
+        float *bsm = bias_smem + ew * C::BIAS_FLOATS;
+        float alpha = 1.0f;
+        if constexpr (C::DT == DT_E4M3) alpha = __ldg(p.scale_a) * __ldg(p.scale_b);
+        uint32_t acc = 0, acc_phase = 0;
+        bool ok = true;
+        for (int t = unit; ok && t < p.num_tiles; t += units) {
+            int tm, tn;
+            tile_coords(p, t, tm, tn);
+            const int m0 = tm * (C::BM * C::CG) + (int)rank * C::BM;
+            const int n0 = tn * C::BN;
+            const int row = m0 + 32 * q + lane;
+            const bool row_ok = row < p.m;
+            float rbias = 0.0f;
+            if constexpr (C::EPI != EPI_NONE && C::AXIS == AXIS_ROW) {
+                if (row_ok) rbias = O::load(p.bias, row);
+            }
+            if constexpr (C::BIAS_FLOATS > 0) {
+                // this warp's copy of bias[n0 .. n0+BN) as fp32 (read once per tile)
+                __syncwarp();
+                if (n0 + C::BN <= p.n) {
+#pragma unroll
+                    for (int j = lane * 8; j < C::BN; j += 256) {
+                        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
+                            reinterpret_cast<const typename O::type *>(p.bias) + n0 + j));
+                        float f[8];
+                        unpack8<C::DT == DT_F16 ? DT_F16 : DT_BF16>(u, f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) bsm[j + e] = f[e];
+                    }
+                } else {
+                    for (int j = lane; j < C::BN; j += 32) bsm[j] = n0 + j < p.n ? O::load(p.bias, n0 + j) : 0.0f;
+                }
+                __syncwarp();
+            }
+            if (!wait_bounded<false>(tfull_bar(acc), acc_phase, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + acc * C::BN;
+#pragma unroll 1
+            for (int g = 0; g < C::BN / 128; ++g) {       // 128 output columns per group
+                uint32_t words[4];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {          // 32 columns per chunk
+                    const int c = 4 * g + cc;
+                    uint32_t v[32];
+                    ptx::tmem_ld_32x32b_x32(tbase + c * 32, v);
+                    ptx::tmem_wait_ld(v);
+                    if (cc == 3 && g == C::BN / 128 - 1) {
+                        // accumulator fully read: hand it back to the MMA issuer
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if constexpr (C::CG == 2) ptx::mbar_arrive_cluster(ptx::mapa(tempty_bar(acc), 0));
+                            else ptx::mbar_arrive(tempty_bar(acc));
+                        }
+                    }
+                    const int col0 = n0 + 32 * c;
+                    uint32_t packed[16];
+                    uint32_t bits = 0;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        float x0 = __uint_as_float(v[j]), x1 = __uint_as_float(v[j + 1]);
+                        if constexpr (C::DT == DT_E4M3) { x0 *= alpha; x1 *= alpha; }
+                        if constexpr (C::EPI != EPI_NONE) {
+                            if constexpr (C::AXIS == AXIS_ROW) { x0 += rbias; x1 += rbias; }
+                            else { x0 += bsm[32 * c + j]; x1 += bsm[32 * c + j + 1]; }
+                        }
+                        if constexpr (C::EPI == EPI_RELU_AUX) {
+                            bits |= (x0 > 0.0f ? 1u : 0u) << j;
+                            bits |= (x1 > 0.0f ? 1u : 0u) << (j + 1);
+                        }
+                        packed[j / 2] = O::pack(activate<C::EPI>(x0), activate<C::EPI>(x1));
+                    }
+                    if constexpr (C::EPI == EPI_RELU_AUX) {
+                        const int valid = p.n - col0;
+                        const uint32_t keep = valid >= 32 ? 0xFFFFFFFFu : (valid <= 0 ? 0u : ((1u << valid) - 1u));
+                        words[cc] = bits & keep;
+                    }
+                    // stage 32 rows x 64 outputs (two chunks) in the 128-byte swizzled layout
+                    if ((cc & 1) == 0) {
+                        if (lane == 0) ptx::bulk_wait_read<0>();     // previous store has read the buffer
+                        __syncwarp();
+                    }
+                    uint8_t *stg_row = smem + C::OFF_STG + ew * C::STG_BYTES + lane * 128;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int chunk = ((cc & 1) * 4 + i) ^ (lane & 7);
+                        *reinterpret_cast<uint4 *>(stg_row + chunk * 16) =
+                            make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                    }
+                    if ((cc & 1) == 1) {
+                        ptx::fence_proxy_async_smem();
+                        __syncwarp();
+                        // boxes starting past the last row or column hold nothing to store
+                        if (lane == 0 && m0 + 32 * q < p.m && n0 + 32 * (c - 1) < p.n) {
+                            ptx::tma_store_2d(&tmD, stg, n0 + 32 * (c - 1), m0 + 32 * q);
+                            ptx::bulk_commit();
+                        }
+                    }
+                }
+                if constexpr (C::EPI == EPI_RELU_AUX) {
+                    const int wcol = n0 + 128 * g;
+                    if (row_ok && wcol < p.n) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.aux + (int64_t)row * p.aux_pitch_words + wcol / 32);
+                        *dst = make_uint4(words[0], words[1], words[2], words[3]);
+                    }
+                }
+            }
+            if (++acc == 2u) { acc = 0; acc_phase ^= 1u; }
+        }
+        if (lane == 0) ptx::bulk_wait<0>();
+        __syncwarp();
+    }
+
+    // ---------------------------------------------------------------- teardown
+    __syncwarp();
+    ptx::tc_fence_before();
+    if constexpr (C::CG == 2) ptx::cluster_sync(); else __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc<C::CG>(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace gemm_epi

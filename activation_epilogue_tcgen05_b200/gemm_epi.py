@@ -1,0 +1,240 @@
+"""ctypes binding of the C ABI in ``include/gemm_epi.h`` (argument marshalling only).
+
+The functions keep the C names and signatures; every step of the computation
+runs in the CUDA library.  ``Plan`` is a small convenience wrapper that takes
+torch tensors (device memory, the current stream) and passes their raw
+pointers through the same entry points.
+
+If ``libgemm_epi.so`` has not been built, loading raises ``RuntimeError``:
+there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libgemm_epi.so")
+
+# enums (include/gemm_epi.h)
+F16, BF16, E4M3 = 0, 1, 2
+NONE, BIAS, RELU_BIAS, RELU_AUX_BIAS, GELU_BIAS = 0, 1, 2, 3, 4
+BIAS_ROW, BIAS_COL = 0, 1
+B_KN, B_NK = 0, 1
+KERNEL_AUTO, KERNEL_TC1, KERNEL_TC2, KERNEL_SPLITK = 0, 1, 2, 3
+OK, ERR_ARG, ERR_ALIGN, ERR_NULL, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NO_DEVICE = \
+    0, -1, -2, -3, -4, -5, -6, -7
+
+DTYPE = {"f16": F16, "bf16": BF16, "e4m3": E4M3}
+EPILOGUE = {"none": NONE, "bias": BIAS, "relu_bias": RELU_BIAS, "relu_aux_bias": RELU_AUX_BIAS,
+            "gelu_bias": GELU_BIAS}
+AXIS = {"row": BIAS_ROW, "col": BIAS_COL}
+LAYOUT = {"kn": B_KN, "nk": B_NK}
+KERNEL = {"auto": KERNEL_AUTO, "tc1": KERNEL_TC1, "tc2": KERNEL_TC2, "splitk": KERNEL_SPLITK}
+
+# every symbol include/gemm_epi.h declares
+EXPORTS = ("gemm_epi_plan", "gemm_epi_plan_ex", "gemm_epi_plan_opts", "gemm_epi_set_scales",
+           "gemm_epi_run", "gemm_epi_unfused_run", "gemm_epi_check", "gemm_epi_plan_query",
+           "gemm_epi_free", "gemm_epi_status_string", "gemm_epi_aux_pitch_bytes",
+           "gemm_epi_version")
+
+
+class Options(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int32), ("block_n", ctypes.c_int32),
+                ("split_k", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
+                ("inject_stall", ctypes.c_int32)]
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_int32) for f in
+                ("kernel", "block_m", "block_n", "block_k", "stages", "split_k", "grid", "cluster",
+                 "threads", "smem_bytes", "tiles")]
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+class GemmEpiError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib():
+    """Load libgemm_epi.so (raises RuntimeError when it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m activation_epilogue_tcgen05_b200.build` (no fallback exists)")
+            L = ctypes.CDLL(LIB_PATH)
+            i64, i32, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+            pp = ctypes.POINTER(vp)
+            L.gemm_epi_plan.argtypes = [i64, i64, i64, i32, i32, i32, pp]
+            L.gemm_epi_plan_ex.argtypes = [i64, i64, i64, i32, i32, i32, i32, pp]
+            L.gemm_epi_plan_opts.argtypes = [i64, i64, i64, i32, i32, i32, i32,
+                                             ctypes.POINTER(Options), pp]
+            L.gemm_epi_set_scales.argtypes = [vp, vp, vp]
+            L.gemm_epi_run.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+            L.gemm_epi_unfused_run.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+            L.gemm_epi_check.argtypes = [vp, vp]
+            L.gemm_epi_plan_query.argtypes = [vp, ctypes.POINTER(PlanInfo)]
+            L.gemm_epi_free.argtypes = [vp]
+            L.gemm_epi_status_string.argtypes = [i32]
+            L.gemm_epi_status_string.restype = ctypes.c_char_p
+            L.gemm_epi_aux_pitch_bytes.argtypes = [i64]
+            L.gemm_epi_aux_pitch_bytes.restype = i64
+            L.gemm_epi_version.argtypes = []
+            for name in ("gemm_epi_plan", "gemm_epi_plan_ex", "gemm_epi_plan_opts",
+                         "gemm_epi_set_scales", "gemm_epi_run", "gemm_epi_unfused_run",
+                         "gemm_epi_check", "gemm_epi_plan_query", "gemm_epi_free",
+                         "gemm_epi_version"):
+                getattr(L, name).restype = i32
+            _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------- C-named wrappers
+def gemm_epi_plan(m, n, k, dtype, epilogue, bias_axis) -> int:
+    h = ctypes.c_void_p()
+    _check(lib().gemm_epi_plan(m, n, k, dtype, epilogue, bias_axis, ctypes.byref(h)), "gemm_epi_plan")
+    return h.value
+
+
+def gemm_epi_plan_ex(m, n, k, dtype, epilogue, bias_axis, b_layout) -> int:
+    h = ctypes.c_void_p()
+    _check(lib().gemm_epi_plan_ex(m, n, k, dtype, epilogue, bias_axis, b_layout, ctypes.byref(h)),
+           "gemm_epi_plan_ex")
+    return h.value
+
+
+def gemm_epi_plan_opts(m, n, k, dtype, epilogue, bias_axis, b_layout, opts: Options | None) -> int:
+    h = ctypes.c_void_p()
+    _check(lib().gemm_epi_plan_opts(m, n, k, dtype, epilogue, bias_axis, b_layout,
+                                    ctypes.byref(opts) if opts is not None else None,
+                                    ctypes.byref(h)), "gemm_epi_plan_opts")
+    return h.value
+
+
+def gemm_epi_set_scales(plan, d_scale_a, d_scale_b) -> None:
+    _check(lib().gemm_epi_set_scales(plan, d_scale_a, d_scale_b), "gemm_epi_set_scales")
+
+
+def gemm_epi_run(plan, A, B, bias, D, aux, stream) -> None:
+    _check(lib().gemm_epi_run(plan, A, B, bias, D, aux, stream), "gemm_epi_run")
+
+
+def gemm_epi_unfused_run(plan, A, B, bias, D, aux, stream) -> None:
+    _check(lib().gemm_epi_unfused_run(plan, A, B, bias, D, aux, stream), "gemm_epi_unfused_run")
+
+
+def gemm_epi_check(plan, stream) -> None:
+    _check(lib().gemm_epi_check(plan, stream), "gemm_epi_check")
+
+
+def gemm_epi_plan_query(plan) -> dict:
+    info = PlanInfo()
+    _check(lib().gemm_epi_plan_query(plan, ctypes.byref(info)), "gemm_epi_plan_query")
+    return info.as_dict()
+
+
+def gemm_epi_free(plan) -> None:
+    _check(lib().gemm_epi_free(plan), "gemm_epi_free")
+
+
+def gemm_epi_status_string(status: int) -> str:
+    return lib().gemm_epi_status_string(status).decode()
+
+
+def gemm_epi_aux_pitch_bytes(n: int) -> int:
+    return lib().gemm_epi_aux_pitch_bytes(n)
+
+
+def gemm_epi_version() -> int:
+    return lib().gemm_epi_version()
+
+
+def status_string(status: int) -> str:
+    try:
+        return gemm_epi_status_string(status)
+    except Exception:  # library not loadable: still report the number
+        return "status"
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != OK:
+        raise GemmEpiError(rc, what)
+
+
+# ---------------------------------------------------------------- torch convenience
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+class Plan:
+    """Owns one gemm_epi plan; ``run`` passes torch tensors' device pointers.
+
+    ``dtype``/``epilogue``/``bias_axis``/``b_layout``/``kernel`` take the
+    names used across the package ("bf16", "relu_aux_bias", "row", "kn", ...).
+    """
+
+    def __init__(self, m, n, k, dtype="bf16", epilogue="bias", bias_axis="row", b_layout="kn",
+                 kernel="auto", block_n=0, split_k=0, max_ctas=0, inject_stall=0):
+        self.m, self.n, self.k = int(m), int(n), int(k)
+        self.dtype, self.epilogue, self.bias_axis, self.b_layout = dtype, epilogue, bias_axis, b_layout
+        opts = Options(KERNEL[kernel], int(block_n), int(split_k), int(max_ctas), int(inject_stall))
+        self.handle = gemm_epi_plan_opts(self.m, self.n, self.k, DTYPE[dtype], EPILOGUE[epilogue],
+                                         AXIS[bias_axis], LAYOUT[b_layout], opts)
+        self._scales = None
+
+    @property
+    def info(self) -> dict:
+        return gemm_epi_plan_query(self.handle)
+
+    def set_scales(self, scale_a, scale_b):
+        """fp32 device scalars (torch tensors); kept alive by the plan object."""
+        self._scales = (scale_a, scale_b)
+        gemm_epi_set_scales(self.handle, _ptr(scale_a), _ptr(scale_b))
+
+    def run(self, A, B, bias, D, aux=None, stream=None, fused=True):
+        s = _stream_ptr(stream)
+        f = gemm_epi_run if fused else gemm_epi_unfused_run
+        f(self.handle, _ptr(A), _ptr(B), _ptr(bias), _ptr(D), _ptr(aux), s)
+
+    def check(self, stream=None):
+        gemm_epi_check(self.handle, _stream_ptr(stream))
+
+    def close(self):
+        if getattr(self, "handle", None):
+            gemm_epi_free(self.handle)
+            self.handle = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream) if hasattr(stream, "cuda_stream") else stream
+
+
+def aux_pitch_words(n: int) -> int:
+    return gemm_epi_aux_pitch_bytes(n) // 4

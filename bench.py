@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark: fused GEMM + bias (+ ReLU / GELU, + sign mask) TFLOP/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one call of gemm_epi_run over one batch of seeded synthetic inputs
+already resident in HBM: a single launch of the fused persistent kernel that
+loads A and B tiles with TMA, multiplies on the tcgen05 tensor cores into
+tensor memory, and finishes each tile (bias, activation, sign mask, rounding)
+before its one store.  Throughput counts 2*m*n*k flops per step (epilogue
+work is not counted).  Between timed steps the inputs rotate over enough
+distinct buffer sets to exceed the 126 MB L2, so every step reads its
+operands from HBM.
+
+N > 1 (torchrun, one process per GPU): every rank runs its own independent
+replica of the problem (weak scaling, no data-path collective); the timed
+region is bracketed by a barrier and the slowest rank's time is used.
+
+Printed on rank 0: one JSON line with the contract's keys plus ``roofline``
+(dominant kernel vs. the measured tensor / HBM peak), ``cpu_baseline`` (the
+fp64 oracle on the host cores, a bounded sample), ``e2e`` (host buffers,
+copies inside the timed region), ``unfused`` (the library's own GEMM-then-
+elementwise path), ``clocks`` and ``gpu_launches``.
+
+``--impl reference`` times the CPU oracle itself, as it stands, on the same
+workload and metric (bounded samples per step); under torchrun only rank 0
+runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused GEMM+bias(+act) TFLOP/s on 1 B200 and % of dense tensor peak"
+DEFAULT_WORKLOAD = "relu_aux_bias_bf16_4096x4096x4096"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0        # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--kernel", default="auto", choices=["auto", "tc1", "tc2", "splitk"])
+    ap.add_argument("--block-n", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-unfused", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured (MEASURED_PEAKS.json)"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback (profiling recipe)"
+
+
+def kernel_source_hash():
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "activation_epilogue_tcgen05_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(workload: str, kernel_hash: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on this kernel source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and not line.startswith("#") and parts[0] == workload \
+                    and parts[1] == kernel_hash:
+                return int(parts[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples (SM clock, throttle reasons) over a window."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, period_ms: int = 50):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 f"-lms={period_ms}"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 10:
+                self.samples.append((time.time(), parts))
+
+    def wait_first(self, timeout=10.0):
+        t0 = time.time()
+        while self.proc and not self.samples and time.time() - t0 < timeout:
+            time.sleep(0.05)
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        win = [p for (t, p) in self.samples if t0 - 0.1 <= t <= t1 + 0.1]
+        if len(win) < 3:                      # short region: nearest samples around it
+            near = sorted(self.samples, key=lambda s: abs(s[0] - (t0 + t1) / 2))[:5]
+            win = [p for (_, p) in near]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(p[2]) for p in win if num(p[2]) is not None]
+        mx = [num(p[3]) for p in win if num(p[3]) is not None]
+        power = [num(p[4]) for p in win if num(p[4]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in win for i in range(4) if p[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "power_w_max": max(power) if power else None, "samples": len(win)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle legs
+def oracle_rows_rate(wl, prob, target_s: float, max_rows=None):
+    """Time the oracle (as it stands) on the first R rows of the workload; R sized to ~target_s.
+
+    Returns (TFLOP/s, rows, seconds, threads)."""
+    import numpy as np
+    import oracle
+    from activation_epilogue_tcgen05_b200.workloads import storage
+
+    Bs = storage(prob.B)
+    bias_full = storage(prob.bias)
+
+    def run(rows):
+        As = storage(prob.A[:rows])
+        bias = bias_full[:rows] if wl.bias_axis == "row" else bias_full
+        t0 = time.perf_counter()
+        oracle.gemm_epi(As, Bs, bias, dtype=wl.dtype, epilogue=wl.epilogue, bias_axis=wl.bias_axis,
+                        b_layout=wl.b_layout, scale_a=prob.scale_a, scale_b=prob.scale_b)
+        return time.perf_counter() - t0
+
+    threads = oracle.threads()
+    rows = min(wl.m, max(1, threads))
+    dt = run(rows)
+    if dt < target_s:
+        rows = int(min(wl.m if max_rows is None else max_rows,
+                       max(rows, rows * target_s / max(dt, 1e-6))))
+        dt = run(rows)
+    flops = 2.0 * rows * wl.n * wl.k
+    return flops / dt / 1e12, rows, dt, threads
+
+
+def reference_arm(args):
+    """--impl reference: the fp64 CPU oracle as it stands, on this workload."""
+    from activation_epilogue_tcgen05_b200 import replicas
+    rank, world, _ = replicas.env_rank()
+    if rank != 0:
+        return 0
+    import numpy as np
+    import oracle
+    from activation_epilogue_tcgen05_b200.workloads import WORKLOADS, make_problem, storage
+    wl = WORKLOADS[args.workload]
+    gen_dev = "cpu"
+    if wl.m * wl.k > (1 << 28):              # very large operands: draw only what the samples need
+        wl_small = wl.with_(m=min(wl.m, 4096))
+        prob = make_problem(wl_small, device=gen_dev)
+    else:
+        prob = make_problem(wl, device=gen_dev)
+    As, Bs, bias = storage(prob.A), storage(prob.B), storage(prob.bias)
+    m_avail = As.shape[0]
+    rng = np.random.default_rng(0)
+
+    def step(count):
+        rows = rng.integers(0, m_avail, count)
+        cols = rng.integers(0, wl.n, count)
+        t0 = time.perf_counter()
+        oracle.gemm_epi_sampled(As, Bs, bias if wl.bias_axis == "col" else bias[:m_avail], rows, cols,
+                                dtype=wl.dtype, epilogue=wl.epilogue, bias_axis=wl.bias_axis,
+                                b_layout=wl.b_layout, scale_a=prob.scale_a, scale_b=prob.scale_b)
+        return time.perf_counter() - t0
+
+    threads = oracle.threads()
+    # size one step so that warmup + steps take about a minute in total
+    probe = max(threads * 4, 64)
+    t_probe = step(probe)
+    per_pos = t_probe / probe
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    count = int(max(threads, min(1 << 20, budget / max(per_pos, 1e-9))))
+    for _ in range(args.warmup):
+        step(count)
+    total = 0.0
+    for _ in range(args.steps):
+        total += step(count)
+    flops = 2.0 * wl.k * count * args.steps
+    value = flops / total / 1e12
+    sample = f"{count} seeded output positions per step (one fp64 dot product of length k each)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "m": wl.m, "n": wl.n, "k": wl.k, "dtype": wl.dtype,
+                   "epilogue": wl.epilogue, "bias_axis": wl.bias_axis, "b_layout": wl.b_layout},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def main(argv=None):
+    args = parse(argv)
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    from activation_epilogue_tcgen05_b200 import gemm_epi as g
+    from activation_epilogue_tcgen05_b200 import replicas
+    from activation_epilogue_tcgen05_b200.workloads import TORCH_DTYPE, WORKLOADS, make_problem
+
+    rank, world, local_rank = replicas.env_rank()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback exists)")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    have_pg = replicas.init("nccl", timeout_s=120, device_id=dev)
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+
+    wl = WORKLOADS[args.workload]
+    out_t = TORCH_DTYPE[wl.out_dtype]
+    big = wl.m * wl.k > (1 << 28)
+    prob = make_problem(wl, device="cuda" if big else "cpu")
+    A0, B0, bias0 = prob.A.to(dev), prob.B.to(dev), prob.bias.to(dev)
+    aux_words = wl.m * g.aux_pitch_words(wl.n) if wl.epilogue == "relu_aux_bias" else 0
+    esz = 1 if wl.dtype == "e4m3" else 2
+    in_bytes = (wl.m * wl.k + wl.k * wl.n) * esz + bias0.numel() * 2
+    out_bytes = wl.m * wl.n * 2 + aux_words * 4
+    set_bytes = in_bytes + out_bytes
+    n_sets = 1 if set_bytes > 2 * L2_BYTES else max(2, math.ceil(3 * L2_BYTES / set_bytes))
+
+    sets = []
+    for i in range(n_sets):
+        A = A0 if i == 0 else A0.clone()
+        B = B0 if i == 0 else B0.clone()
+        bias = bias0 if i == 0 else bias0.clone()
+        D = torch.empty((wl.m, wl.n), dtype=out_t, device=dev)
+        aux = torch.empty((aux_words,), dtype=torch.int32, device=dev) if aux_words else None
+        sets.append((A, B, bias, D, aux))
+    plan = g.Plan(wl.m, wl.n, wl.k, wl.dtype, wl.epilogue, wl.bias_axis, wl.b_layout,
+                  kernel=args.kernel, block_n=args.block_n)
+    if wl.dtype == "e4m3":
+        plan.set_scales(torch.tensor([prob.scale_a], dtype=torch.float32, device=dev),
+                        torch.tensor([prob.scale_b], dtype=torch.float32, device=dev))
+    info = plan.info
+    stream = torch.cuda.current_stream(dev)
+    flops = 2.0 * wl.m * wl.n * wl.k
+
+    # first call (tensor-map encode) timed apart from the steady state
+    t0 = time.perf_counter()
+    plan.run(*sets[0], stream=stream)
+    torch.cuda.synchronize(dev)
+    first_call_ms = 1000 * (time.perf_counter() - t0)
+    plan.check(stream)
+
+    for i in range(args.warmup):
+        plan.run(*sets[i % n_sets], stream=stream)
+    torch.cuda.synchronize(dev)
+    plan.check(stream)
+    if sampler:
+        sampler.wait_first()
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    replicas.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.time()
+    start.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        plan.run(*sets[i % n_sets], stream=stream)
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    wall1 = time.time()
+    replicas.barrier()
+    plan.check(stream)
+    elapsed_ms = start.elapsed_time(end)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    elapsed_ms_max = replicas.max_over_ranks(elapsed_ms, device=dev)
+    avg_launch_s = statistics.fmean(launch_ms) / 1000.0
+    clocks = sampler.summary(wall0, wall1) if sampler else None
+
+    value = flops * world * K / (elapsed_ms_max / 1000.0) / 1e12
+    ms_per_step = elapsed_ms_max / K
+
+    # ---- roofline of the dominant (only) kernel: one launch per step
+    peaks, peak_src = load_peaks()
+    khash = kernel_source_hash()
+    traffic = recorded_traffic(wl.name, khash)
+    if info["kernel"] == g.KERNEL_SPLITK:
+        alg_bytes = in_bytes + out_bytes
+        achieved = alg_bytes / avg_launch_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "algorithmic_bytes": alg_bytes, "peak_source": peak_src + ", hbm copy"}
+    else:
+        peak = peaks["bf16_tflops"] * (FP8_OVER_BF16 if wl.dtype == "e4m3" else 1.0)
+        achieved = flops / avg_launch_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": in_bytes + out_bytes,
+                "peak_source": peak_src + (", bf16 burst x nominal fp8/bf16 ratio 2"
+                                           if wl.dtype == "e4m3" else ", bf16 burst")}
+    roof["kernel_source"] = khash
+
+    # ---- the library's own unfused path (bare GEMM, then the elementwise kernel)
+    unfused = None
+    if not args.no_unfused and wl.epilogue != "none":
+        Ku = min(K, 200)
+        for i in range(3):
+            plan.run(*sets[i % n_sets], stream=stream, fused=False)
+        torch.cuda.synchronize(dev)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for i in range(Ku):
+            plan.run(*sets[i % n_sets], stream=stream, fused=False)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        plan.check(stream)
+        ums = replicas.max_over_ranks(s0.elapsed_time(s1), device=dev) / Ku
+        unfused = {"ms_per_step": ums, "value": flops * world / (ums / 1000) / 1e12, "unit": "TFLOP/s",
+                   "steps": Ku, "launches_per_step": 2, "fused_speedup": ums / ms_per_step}
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Ke = min(K, 50)
+        hA = torch.empty(A0.shape, dtype=A0.dtype, pin_memory=True)
+        hB = torch.empty(B0.shape, dtype=B0.dtype, pin_memory=True)
+        hbias = torch.empty(bias0.shape, dtype=bias0.dtype, pin_memory=True)
+        hA.copy_(A0)
+        hB.copy_(B0)
+        hbias.copy_(bias0)
+        hD = torch.empty((wl.m, wl.n), dtype=out_t, pin_memory=True)
+        haux = torch.empty((aux_words,), dtype=torch.int32, pin_memory=True) if aux_words else None
+        A, B, bias, D, aux = sets[0]
+
+        def e2e_step():
+            A.copy_(hA, non_blocking=True)
+            B.copy_(hB, non_blocking=True)
+            bias.copy_(hbias, non_blocking=True)
+            plan.run(A, B, bias, D, aux, stream=stream)
+            hD.copy_(D, non_blocking=True)
+            if aux is not None:
+                haux.copy_(aux, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        replicas.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        plan.check(stream)
+        ems = replicas.max_over_ranks(s0.elapsed_time(s1), device=dev) / Ke
+        e2e = {"value": flops * world / (ems / 1000) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(out_bytes),
+               "ms_per_step": ems, "steps": Ke, "api": "gemm_epi_run (C ABI) + pinned host copies"}
+
+    if sampler:
+        sampler.stop()
+
+    # ---- CPU oracle baseline: rank 0, N = 1 only
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if big:
+            prob_cpu = make_problem(wl.with_(m=min(wl.m, 2048)), device="cpu")
+        else:
+            prob_cpu = make_problem(wl, device="cpu")
+        tf, rows, secs, threads = oracle_rows_rate(wl, prob_cpu, args.cpu_seconds,
+                                                   max_rows=prob_cpu.A.shape[0])
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"first {rows} of {wl.m} output rows, all {wl.n} columns ({secs:.1f} s; "
+                         f"fp64, OpenMP over rows)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "m": wl.m, "n": wl.n, "k": wl.k, "dtype": wl.dtype,
+                       "out_dtype": wl.out_dtype, "epilogue": wl.epilogue, "bias_axis": wl.bias_axis,
+                       "b_layout": wl.b_layout, "parallelism": f"replicas x{world}",
+                       "l2": (f"inputs rotate over {n_sets} buffer sets ({n_sets * set_bytes / 2**20:.0f} MiB"
+                              f" > 126 MB L2)" if n_sets > 1 else
+                              f"one set of {set_bytes / 2**20:.0f} MiB > 126 MB L2"),
+                       "plan": info, "first_call_ms": first_call_ms},
+            "pct_of_peak": 100.0 * roof["frac"],
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "unfused": unfused,
+            "gpu_launches": K, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    plan.close()
+    if have_pg:
+        replicas.barrier()
+        replicas.finalize()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,200 @@
+/*
+ * gemm_epi.h -- fused GEMM + bias + activation for NVIDIA B200 (sm_100a).
+ *
+ *     D = act(alpha * (A . B) + bias)          aux = packed bits of (alpha*(A.B) + bias) > 0
+ *
+ * One persistent kernel computes the product on the tcgen05 tensor cores with
+ * the fp32 accumulator in tensor memory, finishes every accumulator tile in
+ * registers (scale, bias, activation, sign mask, rounding to the output type)
+ * and writes it to HBM once.
+ *
+ * Where the pages define the operation
+ *   [bias-fusion]   "PyTorch inference: cuBLASLt bias fusion optimization"
+ *                   (blog.hotdry.top/posts/2025/09/22/pytorch-inference-cublaslt-bias-fusion-optimization)
+ *   [nvmath-fusion] "nvmath-python cuBLASLt bias fusion for PyTorch inference"
+ *                   (blog.hotdry.top/posts/2025/09/22/nvmath-python-cublaslt-bias-fusion-for-pytorch-inference)
+ *   [epilog-params] "nvmath-python epilog bias fusion parameters"
+ *                   (blog.hotdry.top/agent/posts/2025/09/22/nvmath-python-epilog-bias-fusion-parameters)
+ *   [nvgemm]        "PyTorch 2.14 NVGEMM epilogue fusion" (zdabc.icu/article/2026/9/3/3582.html)
+ *
+ * Conventions for every entry point
+ *   - A is row-major (m, k).  B is row-major (k, n) (GEMM_EPI_B_KN, default)
+ *     or row-major (n, k) (GEMM_EPI_B_NK: an nn.Linear weight, D = A . B^T).
+ *   - D is row-major (m, n), densely packed (row pitch n elements).
+ *   - Accumulation and all epilogue arithmetic are fp32; D is rounded to
+ *     nearest even.  fp16 inputs give fp16 bias and D; bf16 gives bf16; e4m3
+ *     inputs give bf16 bias and D ([nvmath-fusion] paragraph 5: input, weight
+ *     and bias types agree; FP8 keeps a 16-bit output).
+ *   - Every pointer passed to run() is a DEVICE pointer into memory of the
+ *     current CUDA device, owned by the caller, 16-byte aligned ([epilog-params]
+ *     body paragraph 3).  Row pitches k*esize and n*esize must be multiples of
+ *     16 bytes: k and n multiples of 8 for 16-bit types, of 16 for e4m3.
+ *   - Calls are asynchronous on the given stream (a cudaStream_t passed as
+ *     void*, NULL = legacy default stream) and never synchronise.
+ *   - On any error nothing is launched and a negative status is returned.
+ */
+#ifndef GEMM_EPI_H
+#define GEMM_EPI_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- enumerations -------------------------------------------------------- */
+
+/* Operand types ([nvmath-fusion] paragraph 5: FP16, BF16, FP8). */
+enum gemm_epi_dtype { GEMM_EPI_F16 = 0, GEMM_EPI_BF16 = 1, GEMM_EPI_E4M3 = 2 };
+
+/* Epilogues ([epilog-params] body paragraph 2; [bias-fusion] paragraph 2 for GELU).
+ *   NONE           D = alpha*A.B                   (the bare GEMM; bias ignored)
+ *   BIAS           D = alpha*A.B + bias
+ *   RELU_BIAS      D = max(alpha*A.B + bias, 0)
+ *   RELU_AUX_BIAS  as RELU_BIAS, plus aux = sign mask of the ReLU input
+ *   GELU_BIAS      D = GELU(x) = 0.5 x (1 + erf(x / sqrt 2)), x = alpha*A.B + bias */
+enum gemm_epi_epilogue {
+    GEMM_EPI_NONE = 0,
+    GEMM_EPI_BIAS = 1,
+    GEMM_EPI_RELU_BIAS = 2,
+    GEMM_EPI_RELU_AUX_BIAS = 3,
+    GEMM_EPI_GELU_BIAS = 4
+};
+
+/* Bias broadcast ([epilog-params] body paragraph 3; [nvmath-fusion] paragraph 5):
+ *   ROW  bias has length m; bias[i] is added to every column of output row i
+ *        (a (m,1) bias -- the pages' default).
+ *   COL  bias has length n; bias[j] is added to every row of output column j
+ *        (a (1,n) bias). */
+enum gemm_epi_bias_axis { GEMM_EPI_BIAS_ROW = 0, GEMM_EPI_BIAS_COL = 1 };
+
+/* Storage of B. */
+enum gemm_epi_b_layout { GEMM_EPI_B_KN = 0, GEMM_EPI_B_NK = 1 };
+
+/* Kernel families a plan can use (GEMM_EPI_KERNEL_AUTO lets the plan choose). */
+enum gemm_epi_kernel {
+    GEMM_EPI_KERNEL_AUTO = 0,
+    GEMM_EPI_KERNEL_TC1 = 1,    /* persistent, one CTA per 128 x block_n tile           */
+    GEMM_EPI_KERNEL_TC2 = 2,    /* persistent, CTA pair (cta_group::2) per 256 x block_n */
+    GEMM_EPI_KERNEL_SPLITK = 3  /* small m: operand roles swapped, K split over a cluster */
+};
+
+/* Status codes. */
+enum gemm_epi_status {
+    GEMM_EPI_OK = 0,
+    GEMM_EPI_ERR_ARG = -1,          /* size <= 0, unknown enum, bad option, bad plan handle */
+    GEMM_EPI_ERR_ALIGN = -2,        /* pointer not 16-byte aligned, or row pitch not a multiple of 16 B */
+    GEMM_EPI_ERR_NULL = -3,         /* required pointer NULL (A, B, D; bias for a bias epilogue;
+                                       aux for RELU_AUX_BIAS; scales unset for E4M3) */
+    GEMM_EPI_ERR_UNSUPPORTED = -4,  /* valid request this build cannot serve (option combination) */
+    GEMM_EPI_ERR_CUDA = -5,         /* a CUDA runtime/driver call failed (launch, tensor map) */
+    GEMM_EPI_ERR_TIMEOUT = -6,      /* a kernel gave up on a bounded wait (reported by check()) */
+    GEMM_EPI_ERR_NO_DEVICE = -7     /* current device is not sm_100 (B200 class) */
+};
+
+/* Opaque plan.  Created by gemm_epi_plan*, owned by the caller until
+ * gemm_epi_free; holds host metadata, a tensor-map cache and one 256-byte
+ * device status word.  A plan may be run any number of times, on any stream,
+ * from one host thread at a time. */
+typedef struct gemm_epi_plan_s *gemm_epi_plan_t;
+
+/* Optional tuning knobs; zero-initialise for automatic choices. */
+typedef struct gemm_epi_options {
+    int32_t kernel;    /* enum gemm_epi_kernel                                        */
+    int32_t block_n;   /* output tile width (128 or 256; 0 = auto)                    */
+    int32_t split_k;   /* SPLITK only: CTAs per cluster along k (1..8; 0 = auto)       */
+    int32_t max_ctas;  /* persistent kernels: cap on resident CTAs (0 = one per SM)    */
+    int32_t inject_stall; /* testing only (TC1/TC2): 1 = the MMA issuer never publishes an
+                             accumulator, so the epilogue's bounded wait runs out after about
+                             one second and gemm_epi_check() reports GEMM_EPI_ERR_TIMEOUT;
+                             D is left unwritten.  0 for real work.                        */
+} gemm_epi_options;
+
+/* What a plan decided (for logging and tests). */
+typedef struct gemm_epi_plan_info {
+    int32_t kernel, block_m, block_n, block_k, stages, split_k;
+    int32_t grid, cluster, threads, smem_bytes, tiles;
+} gemm_epi_plan_info;
+
+/* ---- entry points -------------------------------------------------------- */
+
+/* Create a plan for D = act(alpha*A.B + bias) with B stored (k, n).
+ * The stateful plan / execute / free life cycle follows [nvmath-fusion]
+ * paragraphs 3 and 5 (Matmul.plan(epilog=..., epilog_inputs={"bias": ...}),
+ * execute(), free()).
+ * m, n, k >= 1; dtype/epilogue/bias_axis from the enums above.
+ * Returns GEMM_EPI_OK and *out, or ERR_ARG / ERR_ALIGN (pitch rule) /
+ * ERR_NO_DEVICE / ERR_CUDA; *out is untouched on error.  Needs a current CUDA
+ * device of compute capability 10.0 (allocates the status word there). */
+int gemm_epi_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis,
+                  gemm_epi_plan_t *out);
+
+/* As gemm_epi_plan, with the storage of B given explicitly. */
+int gemm_epi_plan_ex(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis,
+                     int b_layout, gemm_epi_plan_t *out);
+
+/* As gemm_epi_plan_ex, with tuning options (opts may be NULL). */
+int gemm_epi_plan_opts(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis,
+                       int b_layout, const gemm_epi_options *opts, gemm_epi_plan_t *out);
+
+/* E4M3 plans only: per-tensor fp32 scales s_A, s_B as DEVICE pointers to one
+ * float each, read by every run; alpha = s_A * s_B multiplies the product
+ * before the bias (the epilogue scaling factor of [nvgemm], section "why
+ * epilogue fusion matters").  16-bit plans have alpha = 1 and reject this
+ * call with ERR_ARG.  The pointers are borrowed, not owned. */
+int gemm_epi_set_scales(gemm_epi_plan_t plan, const float *d_scale_a, const float *d_scale_b);
+
+/* Enqueue the fused kernel: one launch, D (and aux) written once.
+ *   A     (m, k) operand, B (k, n) or (n, k) operand, device pointers.
+ *   bias  length m (ROW) or n (COL), output type; ignored (may be NULL) for NONE.
+ *   D     (m, n) output.
+ *   aux   RELU_AUX_BIAS only (else ignored, may be NULL): packed sign mask,
+ *         row-major uint32 words, row pitch gemm_epi_aux_pitch_bytes(n);
+ *         bit b of word w in row i is 1 iff the fp32 pre-activation of
+ *         element (i, 32w + b) is > 0 (taken before rounding to the output
+ *         type); bits past column n-1 are 0.  ([epilog-params] body
+ *         paragraph 2: the ReLU input's sign mask kept for the backward pass.)
+ *   stream  cudaStream_t as void*.
+ * Returns OK, ERR_ARG (bad plan), ERR_NULL, ERR_ALIGN or ERR_CUDA.  A kernel
+ * that gives up on a bounded internal wait records it in the plan's status
+ * word; gemm_epi_check() reports it. */
+int gemm_epi_run(gemm_epi_plan_t plan, const void *A, const void *B, const void *bias, void *D,
+                 uint32_t *aux, void *stream);
+
+/* The library's own UNFUSED baseline on the same plan and arguments: the bare
+ * GEMM (epilogue NONE) writes alpha*A.B to D in the output type, then a
+ * separate elementwise kernel reads D back, adds the bias, applies the
+ * activation, writes D (in place) and aux.  Two launches and one extra round
+ * trip of D through HBM: the sequence the pages' fusion removes ([epilog-params]
+ * body paragraphs 1 and 5: validate the stepwise result first).  Its result
+ * rounds the pre-activation to the output type before the bias, so it may
+ * differ from gemm_epi_run within the tolerance. */
+int gemm_epi_unfused_run(gemm_epi_plan_t plan, const void *A, const void *B, const void *bias,
+                         void *D, uint32_t *aux, void *stream);
+
+/* Synchronise `stream`, read and clear the plan's device status word.
+ * Returns OK, ERR_TIMEOUT (some kernel of this plan gave up waiting since the
+ * last check), ERR_CUDA (a sticky CUDA error) or ERR_ARG. */
+int gemm_epi_check(gemm_epi_plan_t plan, void *stream);
+
+/* Fill *info with the plan's kernel choice.  ERR_ARG on a bad handle. */
+int gemm_epi_plan_query(gemm_epi_plan_t plan, gemm_epi_plan_info *info);
+
+/* Release the plan (host metadata, tensor maps, status word).  Must not
+ * overlap a run still executing on the GPU that uses this plan's status word:
+ * synchronise first.  ERR_ARG for an unknown or already freed handle. */
+int gemm_epi_free(gemm_epi_plan_t plan);
+
+/* Static description of a status code (never NULL). */
+const char *gemm_epi_status_string(int status);
+
+/* Row pitch of the aux mask in bytes: ceil(n / 128) * 16 (0 for n <= 0). */
+int64_t gemm_epi_aux_pitch_bytes(int64_t n);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int gemm_epi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GEMM_EPI_H */

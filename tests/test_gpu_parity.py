@@ -1,0 +1,322 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small shapes that span several tiles plus ragged edges in m, n and k are
+compared element by element for every dtype x epilogue x bias axis x B layout
+and every kernel family; the five named workloads are checked at full size
+(element by element where the oracle is fast enough, on seeded sampled
+positions otherwise, plus invariants that hold at any size).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import TOL, aux_padding_bits, unpack_aux, band, tolerance
+from parity import (alloc_outputs, check_against_oracle, compare, device_inputs, gpu_run,
+                    make_plan, oracle_full, sampled_oracle, sigmas)
+
+from activation_epilogue_tcgen05_b200 import gemm_epi as g
+from activation_epilogue_tcgen05_b200.workloads import (TORCH_DTYPE, WORKLOADS, Workload,
+                                                        make_problem, sample_positions, storage)
+
+pytestmark = pytest.mark.gpu
+
+DTYPES = ["f16", "bf16", "e4m3"]
+EPILOGUES = ["none", "bias", "relu_bias", "relu_aux_bias", "gelu_bias"]
+
+
+def small(dtype, epilogue, axis, layout, m=200, n=272, seed=1):
+    k = 336 if dtype == "e4m3" else 328          # ragged last k-block
+    return Workload(f"small_{dtype}_{epilogue}", m, n, k, dtype, epilogue, axis, layout, seed=seed)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    major, minor = torch.cuda.get_device_capability()
+    if (major, minor) != (10, 0):
+        pytest.skip("needs sm_100")
+    from activation_epilogue_tcgen05_b200 import build
+    build.build()
+    oracle.build()
+
+
+# ------------------------------------------------------------------ persistent TC kernels
+@pytest.mark.parametrize("layout", ["kn", "nk"])
+@pytest.mark.parametrize("axis", ["row", "col"])
+@pytest.mark.parametrize("epilogue", EPILOGUES)
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("kernel,block_n", [("tc1", 128), ("tc1", 256), ("tc2", 256), ("tc2", 128)])
+def test_small_all_variants(kernel, block_n, dtype, epilogue, axis, layout):
+    if kernel == "tc2" and block_n == 128 and dtype == "e4m3" and layout == "kn":
+        pytest.skip("not instantiated: a 64-column e4m3 half-tile is narrower than one 128-byte box")
+    wl = small(dtype, epilogue, axis, layout)
+    prob = make_problem(wl)
+    worst, info = check_against_oracle(wl, prob, kernel=kernel, block_n=block_n)
+    assert info["kernel"] == g.KERNEL[kernel] and info["block_n"] == block_n
+    assert worst <= 1.0
+
+
+@pytest.mark.parametrize("kernel", ["tc1", "tc2"])
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_persistent_many_tiles_per_cta(kernel, dtype):
+    """Few CTAs, many tiles each: accumulator double-buffer and ring phases wrap many times."""
+    k = 1024 if dtype == "e4m3" else 1000
+    wl = Workload("persist", 600, 528, k, dtype, "relu_aux_bias", "col", "kn", seed=2)
+    prob = make_problem(wl)
+    worst, info = check_against_oracle(wl, prob, kernel=kernel, block_n=128, max_ctas=4)
+    assert info["grid"] <= 4 and info["tiles"] >= 10
+    assert worst <= 1.0
+
+
+@pytest.mark.parametrize("kernel", ["tc1", "tc2"])
+@pytest.mark.parametrize("m,n,k", [(1, 16, 16), (7, 24, 40), (129, 136, 72), (257, 264, 64)])
+def test_tiny_and_edge_shapes(kernel, m, n, k):
+    wl = Workload("edge", m, n, k, "bf16", "relu_aux_bias", "row", "kn", seed=3)
+    prob = make_problem(wl)
+    worst, _ = check_against_oracle(wl, prob, kernel=kernel)
+    assert worst <= 1.0
+
+
+@pytest.mark.parametrize("kernel", ["tc1", "tc2", "splitk"])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("epilogue", ["bias", "relu_aux_bias", "none"])
+def test_integer_inputs_bit_exact(kernel, dtype, epilogue):
+    """Integer operands in {-2..2}: fp32 sums are exact, so D must equal RNE(oracle) bit for bit."""
+    m = 48 if kernel == "splitk" else 300
+    wl = Workload("int", m, 264, 200, dtype, epilogue, "row", "kn", seed=4, dist_a=("int", 2),
+                  dist_b=("int", 2), dist_bias=("int", 2))
+    prob = make_problem(wl)
+    D, words, _ = gpu_run(wl, prob, kernel=kernel)
+    ref, pre, mask = oracle_full(wl, prob)
+    want = torch.from_numpy(ref).to(TORCH_DTYPE[dtype])
+    assert torch.equal(D.view(torch.int16), want.view(torch.int16))
+    if epilogue == "relu_aux_bias":
+        np.testing.assert_array_equal(unpack_aux(words, wl.m, wl.n), mask)
+
+
+# ------------------------------------------------------------------ small-m split-K kernel
+@pytest.mark.parametrize("layout", ["nk", "kn"])
+@pytest.mark.parametrize("axis", ["col", "row"])
+@pytest.mark.parametrize("epilogue", EPILOGUES)
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("m", [16, 40, 100])
+def test_splitk_variants(m, dtype, epilogue, axis, layout):
+    k = 1024 if dtype == "e4m3" else 1000
+    wl = Workload("sk", m, 400, k, dtype, epilogue, axis, layout, seed=5)
+    prob = make_problem(wl)
+    worst, info = check_against_oracle(wl, prob, kernel="splitk")
+    assert info["kernel"] == g.KERNEL_SPLITK
+    assert worst <= 1.0
+
+
+@pytest.mark.parametrize("split", [1, 2, 3, 8])
+def test_splitk_cluster_sizes(split):
+    wl = Workload("sk_split", 16, 512, 2048, "f16", "gelu_bias", "col", "nk", seed=6,
+                  dist_b=("uniform", 1 / 64), dist_bias=("uniform", 1 / 64))
+    prob = make_problem(wl)
+    worst, info = check_against_oracle(wl, prob, kernel="splitk", split_k=split)
+    assert info["split_k"] == split
+    assert worst <= 1.0
+
+
+# ------------------------------------------------------------------ fused vs unfused, determinism
+@pytest.mark.parametrize("kernel", ["tc1", "tc2", "splitk"])
+@pytest.mark.parametrize("epilogue", ["bias", "relu_bias", "relu_aux_bias", "gelu_bias"])
+def test_unfused_path_matches_oracle_and_fused(kernel, epilogue):
+    m = 64 if kernel == "splitk" else 384
+    wl = Workload("unf", m, 384, 512, "bf16", epilogue, "row", "kn", seed=7)
+    prob = make_problem(wl)
+    inputs = device_inputs(prob)
+    Df, wf, _ = gpu_run(wl, prob, fused=True, inputs=inputs, kernel=kernel)
+    Du, wu, _ = gpu_run(wl, prob, fused=False, inputs=inputs, kernel=kernel)
+    ref, pre, mask = oracle_full(wl, prob)
+    sa, sb = sigmas(prob)
+    compare(wl, Df, wf, ref, pre, mask, sa, sb)
+    compare(wl, Du, wu, ref, pre, mask, sa, sb)
+
+
+@pytest.mark.parametrize("kernel", ["tc1", "tc2", "splitk"])
+def test_run_to_run_bit_identical(kernel):
+    m = 32 if kernel == "splitk" else 512
+    wl = Workload("det", m, 512, 768, "bf16", "relu_aux_bias", "col", "kn", seed=8)
+    prob = make_problem(wl)
+    inputs = device_inputs(prob)
+    D1, w1, _ = gpu_run(wl, prob, inputs=inputs, kernel=kernel)
+    D2, w2, _ = gpu_run(wl, prob, inputs=inputs, kernel=kernel)
+    assert torch.equal(D1.view(torch.int16), D2.view(torch.int16))
+    np.testing.assert_array_equal(w1, w2)
+
+
+@pytest.mark.parametrize("kernel", ["tc1", "tc2", "splitk"])
+def test_guard_regions_untouched(kernel):
+    """D and aux live inside larger buffers; the bytes around them must not change."""
+    m = 24 if kernel == "splitk" else 136
+    wl = Workload("guard", m, 200, 136, "f16", "relu_aux_bias", "row", "kn", seed=9)
+    prob = make_problem(wl)
+    A, B, bias = device_inputs(prob)
+    G = 4096                                              # guard elements (16-byte multiple)
+    pattern = -12345
+    Dbuf = torch.full((G + wl.m * wl.n + G,), pattern, dtype=torch.int16, device="cuda")
+    D = Dbuf[G:G + wl.m * wl.n].view(torch.float16).view(wl.m, wl.n)
+    words = wl.m * g.aux_pitch_words(wl.n)
+    Abuf = torch.full((G + words + G,), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    aux = Abuf[G:G + words]
+    plan = make_plan(wl, prob, kernel=kernel)
+    plan.run(A, B, bias, D, aux)
+    plan.check()
+    plan.close()
+    torch.cuda.synchronize()
+    assert (Dbuf[:G] == pattern).all() and (Dbuf[G + wl.m * wl.n:] == pattern).all()
+    assert (Abuf[:G] == 0x5A5A5A5A).all() and (Abuf[G + words:] == 0x5A5A5A5A).all()
+    ref, pre, mask = oracle_full(wl, prob)
+    sa, sb = sigmas(prob)
+    compare(wl, D.cpu(), aux.cpu().numpy().view(np.uint32), ref, pre, mask, sa, sb)
+
+
+def test_non_default_stream():
+    wl = Workload("stream", 256, 256, 256, "bf16", "gelu_bias", "col", "nk", seed=10)
+    prob = make_problem(wl)
+    A, B, bias = device_inputs(prob)
+    D, _ = alloc_outputs(wl)
+    s = torch.cuda.Stream()
+    plan = make_plan(wl, prob)
+    with torch.cuda.stream(s):
+        plan.run(A, B, bias, D, None, stream=s)
+    plan.check(stream=s)
+    plan.close()
+    ref, pre, mask = oracle_full(wl, prob)
+    compare(wl, D.cpu(), None, ref, pre, mask, *sigmas(prob))
+
+
+# ------------------------------------------------------------------ errors and failure paths
+def test_run_argument_errors():
+    wl = Workload("err", 128, 128, 128, "bf16", "relu_aux_bias", "row", "kn")
+    prob = make_problem(wl)
+    A, B, bias = device_inputs(prob)
+    D, aux = alloc_outputs(wl)
+    plan = make_plan(wl, prob)
+    L, h = g.lib(), plan.handle
+    s = None
+    p = lambda t: None if t is None else t.data_ptr()
+    assert L.gemm_epi_run(h, None, p(B), p(bias), p(D), p(aux), s) == g.ERR_NULL
+    assert L.gemm_epi_run(h, p(A), p(B), None, p(D), p(aux), s) == g.ERR_NULL
+    assert L.gemm_epi_run(h, p(A), p(B), p(bias), p(D), None, s) == g.ERR_NULL
+    assert L.gemm_epi_run(h, p(A) + 2, p(B), p(bias), p(D), p(aux), s) == g.ERR_ALIGN
+    assert L.gemm_epi_run(h, p(A), p(B), p(bias) + 2, p(D), p(aux), s) == g.ERR_ALIGN
+    assert L.gemm_epi_run(h, p(A), p(B), p(bias), p(D), p(aux) + 4, s) == g.ERR_ALIGN
+    assert L.gemm_epi_set_scales(h, p(A), p(A)) == g.ERR_ARG           # not an e4m3 plan
+    plan.close()
+    assert L.gemm_epi_run(h, p(A), p(B), p(bias), p(D), p(aux), s) == g.ERR_ARG  # freed
+    # e4m3 without scales
+    wl8 = Workload("err8", 128, 128, 128, "e4m3", "bias", "row", "kn")
+    plan8 = g.Plan(128, 128, 128, "e4m3", "bias", "row", "kn")
+    p8 = make_problem(wl8)
+    A8, B8, b8 = device_inputs(p8)
+    D8, _ = alloc_outputs(wl8)
+    assert L.gemm_epi_run(plan8.handle, p(A8), p(B8), p(b8), p(D8), None, s) == g.ERR_NULL
+    plan8.close()
+
+
+@pytest.mark.parametrize("kernel", ["tc1", "tc2"])
+def test_bounded_wait_reports_timeout_and_context_survives(kernel):
+    """A wait that can never complete (nothing publishes the accumulator) must end in about a
+    second with GEMM_EPI_ERR_TIMEOUT, and the next normal run must work."""
+    wl = Workload("stall", 256, 256, 256, "bf16", "bias", "row", "kn", seed=11)
+    prob = make_problem(wl)
+    A, B, bias = device_inputs(prob)
+    D, _ = alloc_outputs(wl)
+    plan = make_plan(wl, prob, kernel=kernel, inject_stall=1)
+    plan.run(A, B, bias, D, None)
+    with pytest.raises(g.GemmEpiError) as e:
+        plan.check()
+    assert e.value.status == g.ERR_TIMEOUT
+    plan.check()                               # the status word was cleared
+    plan.close()
+    worst, _ = check_against_oracle(wl, prob, kernel=kernel)
+    assert worst <= 1.0
+
+
+# ------------------------------------------------------------------ the five named workloads
+def _named(name):
+    return WORKLOADS[name]
+
+
+def test_workload_gemm_bias_f16_full():
+    wl = _named("gemm_bias_f16_1024x512x2048")
+    prob = make_problem(wl)
+    worst, info = check_against_oracle(wl, prob)
+    assert worst <= 1.0
+
+
+def test_workload_linear_gelu_f16_full_splitk():
+    wl = _named("linear_gelu_f16_16x4096x4096")
+    prob = make_problem(wl)
+    worst, info = check_against_oracle(wl, prob)
+    assert info["kernel"] == g.KERNEL_SPLITK
+    assert worst <= 1.0
+
+
+def _properties_relu(D, words, wl):
+    """Invariants at any size: D >= 0; mask bit => D >= 0; D > 0 => mask bit; zero padding."""
+    d = D.float()
+    assert (d >= 0).all()
+    if words is not None:
+        bits = torch.from_numpy(unpack_aux(words, wl.m, wl.n).astype(np.bool_))
+        assert not (bits & (d < 0)).any()
+        assert not ((d > 0) & ~bits).any()
+        assert aux_padding_bits(words, wl.m, wl.n) == 0
+
+
+def _sampled_check(wl, prob, D, words):
+    rows, cols = sample_positions(wl.m, wl.n, 64, 64, seed=0)
+    ref, pre, mask = sampled_oracle(wl, prob, rows, cols)
+    sa, sb = sigmas(prob)
+    d = D[torch.as_tensor(rows), torch.as_tensor(cols)].double().numpy()
+    tol = tolerance(ref, wl.dtype, wl.k, sa, sb)
+    bad = ~(np.abs(d - ref) <= tol)
+    assert not bad.any(), f"{int(bad.sum())} sampled outputs outside tolerance"
+    if words is not None:
+        bits = unpack_aux(words, wl.m, wl.n)[rows, cols]
+        exact = band(pre, wl.dtype, wl.k, sa, sb)
+        assert not (exact & (bits != mask)).any()
+
+
+def test_workload_relu_aux_bias_bf16_4096():
+    wl = _named("relu_aux_bias_bf16_4096x4096x4096")
+    prob = make_problem(wl)
+    inputs = device_inputs(prob)
+    D, words, info = gpu_run(wl, prob, inputs=inputs)
+    _properties_relu(D, words, wl)
+    _sampled_check(wl, prob, D, words)
+    # the unfused baseline agrees with the fused result within the tolerance
+    Du, wu, _ = gpu_run(wl, prob, inputs=inputs, fused=False)
+    sa, sb = sigmas(prob)
+    tol = TOL["bf16"][0] * D.double().abs() + TOL["bf16"][1] * np.sqrt(wl.k) * sa * sb
+    assert ((Du.double() - D.double()).abs() <= 2 * tol).all()
+
+
+@pytest.mark.slow
+def test_workload_relu_aux_bias_bf16_4096_full_oracle():
+    wl = _named("relu_aux_bias_bf16_4096x4096x4096")
+    prob = make_problem(wl)
+    worst, _ = check_against_oracle(wl, prob)
+    assert worst <= 1.0
+
+
+def test_workload_fp8_gelu_bias():
+    wl = _named("fp8_gelu_bias_8192x14336x4096")
+    prob = make_problem(wl)
+    D, words, _ = gpu_run(wl, prob)
+    _sampled_check(wl, prob, D, words)
+
+
+def test_workload_large_relu_bias_sampled():
+    wl = _named("relu_bias_bf16_65536x8192x16384")
+    prob = make_problem(wl, device="cuda")
+    D, words, _ = gpu_run(wl, prob, inputs=(prob.A, prob.B, prob.bias))
+    _properties_relu(D, words, wl)
+    _sampled_check(wl, prob, D, words)
+    del prob
+    torch.cuda.empty_cache()
