@@ -166,9 +166,10 @@ int gemm_epi_run(gemm_epi_plan_t plan, const void *A, const void *B, const void 
  * separate elementwise kernel reads D back, adds the bias, applies the
  * activation, writes D (in place) and aux.  Two launches and one extra round
  * trip of D through HBM: the sequence the pages' fusion removes ([epilog-params]
- * body paragraphs 1 and 5: validate the stepwise result first).  Its result
- * rounds the pre-activation to the output type before the bias, so it may
- * differ from gemm_epi_run within the tolerance. */
+ * body paragraphs 1 and 5: validate the stepwise result first).  It rounds
+ * alpha*A.B to the output type before adding the bias, so where the bias
+ * cancels a large product its error can exceed the fused path's by up to one
+ * unit in the last place of alpha*A.B in the output type. */
 int gemm_epi_unfused_run(gemm_epi_plan_t plan, const void *A, const void *B, const void *bias,
                          void *D, uint32_t *aux, void *stream);
 

@@ -77,12 +77,17 @@ def oracle_full(wl: Workload, prob: Problem):
                            scale_a=prob.scale_a, scale_b=prob.scale_b)
 
 
-def compare(wl, D_gpu, words, ref, pre, mask, sa, sb, rows=None, cols=None):
-    """Assert elementwise tolerance on D and exactness of the mask outside the band."""
+def compare(wl, D_gpu, words, ref, pre, mask, sa, sb, rows=None, cols=None, extra=None):
+    """Assert elementwise tolerance on D and exactness of the mask outside the band.
+
+    ``extra`` (same shape as ref) widens both bounds, for paths with an
+    additional rounding step (the unfused baseline)."""
     d = D_gpu.double().numpy()
     if rows is not None:
         d = d[rows, cols]
     tol = tolerance(ref, wl.dtype, wl.k, sa, sb)
+    if extra is not None:
+        tol = tol + extra
     err = np.abs(d - ref)
     ok = err <= tol                       # NaN (unwritten) compares False
     if not ok.all():
@@ -96,6 +101,8 @@ def compare(wl, D_gpu, words, ref, pre, mask, sa, sb, rows=None, cols=None):
         if rows is not None:
             bits = bits[rows, cols]
         exact = band(pre, wl.dtype, wl.k, sa, sb)
+        if extra is not None:
+            exact &= np.abs(pre) > tolerance(pre, wl.dtype, wl.k, sa, sb) + extra
         wrong = exact & (bits != mask)
         assert not wrong.any(), f"{int(wrong.sum())} mask bits differ outside the tolerance band"
         assert aux_padding_bits(words, wl.m, wl.n) == 0, "mask padding bits are not zero"
@@ -121,3 +128,16 @@ def sampled_oracle(wl: Workload, prob: Problem, rows, cols):
     return oracle.gemm_epi_sampled(A_rows, Bs, bias, inv.astype(np.int64), np.asarray(cols, np.int64),
                                    dtype=wl.dtype, epilogue=wl.epilogue, bias_axis=wl.bias_axis,
                                    b_layout=wl.b_layout, scale_a=prob.scale_a, scale_b=prob.scale_b)
+
+
+# One unit in the last place, relative, of the output type: the unfused path
+# rounds alpha*A.B to the output type before the bias is added.
+OUT_ULP = {"f16": 2.0 ** -10, "bf16": 2.0 ** -7, "e4m3": 2.0 ** -7}
+
+
+def unfused_extra(wl: Workload, prob: Problem, pre):
+    """|alpha*A.B| * ulp(out): the unfused path's additional rounding of the product."""
+    from oracle import decode
+    b = decode(storage(prob.bias), wl.out_dtype)
+    b = b[:, None] if wl.bias_axis == "row" else b[None, :]
+    return OUT_ULP[wl.out_dtype] * np.abs(pre - b)
