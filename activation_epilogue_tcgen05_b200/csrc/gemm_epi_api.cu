@@ -502,3 +502,106 @@ int64_t gemm_epi_aux_pitch_bytes(int64_t n) { return n <= 0 ? 0 : ((n + 127) / 1
 int gemm_epi_version(void) { return 100; }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------- allocation-free entry point
+//
+// gemm_epi_run_noalloc serves callers that may not allocate device memory
+// themselves or through this library.  Its kernels still need scratch beyond
+// the caller's inputs and outputs -- the 4-byte status word that a bounded
+// wait writes when it gives up -- so that word lives in the file-scope array
+// below instead of in a plan's cudaMalloc'd block.
+namespace {
+
+constexpr size_t kNoallocScratchBytes = 256;                  // reserved on every device
+constexpr size_t kNoallocNeededBytes = sizeof(unsigned int);  // used by one call: the status word
+static_assert(kNoallocNeededBytes <= kNoallocScratchBytes, "no-alloc scratch array too small");
+
+static __device__ __align__(256) unsigned int g_noalloc_scratch[kNoallocScratchBytes / sizeof(unsigned int)];
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+unsigned int *g_noalloc_addr[kNoallocMaxDevices] = {};        // device address of the array, per device
+
+// Device address of g_noalloc_scratch on `dev` (the current device).  In host
+// code the array's name is only a host-side stand-in, so the address is taken
+// once per device with cudaGetSymbolAddress and cached.
+int noalloc_scratch(int dev, unsigned int **out) {
+    if (dev < 0 || dev >= kNoallocMaxDevices) return GEMM_EPI_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return GEMM_EPI_ERR_CUDA;
+        }
+        g_noalloc_addr[dev] = static_cast<unsigned int *>(p);
+    }
+    *out = g_noalloc_addr[dev];
+    return GEMM_EPI_OK;
+}
+
+}  // namespace
+
+extern "C" int gemm_epi_run_noalloc(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis,
+                                    int b_layout, const void *A, const void *B, const void *bias,
+                                    const float *d_scale_a, const float *d_scale_b, void *D, uint32_t *aux,
+                                    int wait, void *stream) {
+    // the same argument rules as a plan (sizes are limited to 2^31 - 1)
+    if (m <= 0 || n <= 0 || k <= 0) return GEMM_EPI_ERR_ARG;
+    if (m > 0x7fffffffll || n > 0x7fffffffll || k > 0x7fffffffll) return GEMM_EPI_ERR_ARG;
+    if (dtype < GEMM_EPI_F16 || dtype > GEMM_EPI_E4M3) return GEMM_EPI_ERR_ARG;
+    if (epilogue < GEMM_EPI_NONE || epilogue > GEMM_EPI_GELU_BIAS) return GEMM_EPI_ERR_ARG;
+    if (bias_axis != GEMM_EPI_BIAS_ROW && bias_axis != GEMM_EPI_BIAS_COL) return GEMM_EPI_ERR_ARG;
+    if (b_layout != GEMM_EPI_B_KN && b_layout != GEMM_EPI_B_NK) return GEMM_EPI_ERR_ARG;
+    if (wait != 0 && wait != 1) return GEMM_EPI_ERR_ARG;
+    const int es = esize(dtype);
+    if ((k * es) % 16 != 0 || (n * es) % 16 != 0 || (n * 2) % 16 != 0) return GEMM_EPI_ERR_ALIGN;
+    // the call needs kNoallocNeededBytes of scratch; anything larger than the array is refused
+    if (kNoallocNeededBytes > kNoallocScratchBytes) return GEMM_EPI_ERR_UNSUPPORTED;
+
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return GEMM_EPI_ERR_NO_DEVICE;
+    }
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0) return GEMM_EPI_ERR_NO_DEVICE;
+
+    Plan P{};                                   // on the stack: nothing is allocated
+    P.magic = kPlanMagic;
+    P.m = m;
+    P.n = n;
+    P.k = k;
+    P.dtype = dtype;
+    P.epilogue = epilogue;
+    P.axis = epilogue == GEMM_EPI_NONE ? GEMM_EPI_BIAS_ROW : bias_axis;
+    P.b_layout = b_layout;
+    P.device = dev;
+    P.num_sms = num_sms_of(dev);
+    int rc = choose(&P);
+    if (rc != GEMM_EPI_OK) return rc;
+    if (dtype == GEMM_EPI_E4M3) {
+        P.scale_a = d_scale_a;
+        P.scale_b = d_scale_b;
+    }
+    rc = check_run_args(&P, A, B, bias, D, aux);
+    if (rc != GEMM_EPI_OK) return rc;
+    unsigned int *scratch = nullptr;
+    rc = noalloc_scratch(dev, &scratch);
+    if (rc != GEMM_EPI_OK) return rc;
+    P.status = scratch;
+    rc = ensure_maps(&P, A, B, D);
+    if (rc != GEMM_EPI_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // the array keeps the previous call's contents: the status word must start at zero
+    if (cudaMemsetAsync(scratch, 0, kNoallocNeededBytes, s) != cudaSuccess) return GEMM_EPI_ERR_CUDA;
+    rc = launch_main(&P, true, bias, D, aux, s);
+    if (rc != GEMM_EPI_OK || !wait) return rc;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GEMM_EPI_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpy(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return GEMM_EPI_ERR_CUDA;
+    return word != 0 ? GEMM_EPI_ERR_TIMEOUT : GEMM_EPI_OK;
+}

@@ -37,7 +37,7 @@ KERNEL = {"auto": KERNEL_AUTO, "tc1": KERNEL_TC1, "tc2": KERNEL_TC2, "splitk": K
 EXPORTS = ("gemm_epi_plan", "gemm_epi_plan_ex", "gemm_epi_plan_opts", "gemm_epi_set_scales",
            "gemm_epi_run", "gemm_epi_unfused_run", "gemm_epi_check", "gemm_epi_plan_query",
            "gemm_epi_free", "gemm_epi_status_string", "gemm_epi_aux_pitch_bytes",
-           "gemm_epi_version")
+           "gemm_epi_version", "gemm_epi_run_noalloc")
 
 
 class Options(ctypes.Structure):
@@ -92,10 +92,12 @@ def lib():
             L.gemm_epi_aux_pitch_bytes.argtypes = [i64]
             L.gemm_epi_aux_pitch_bytes.restype = i64
             L.gemm_epi_version.argtypes = []
+            L.gemm_epi_run_noalloc.argtypes = [i64, i64, i64, i32, i32, i32, i32, vp, vp, vp, vp,
+                                               vp, vp, vp, i32, vp]
             for name in ("gemm_epi_plan", "gemm_epi_plan_ex", "gemm_epi_plan_opts",
                          "gemm_epi_set_scales", "gemm_epi_run", "gemm_epi_unfused_run",
                          "gemm_epi_check", "gemm_epi_plan_query", "gemm_epi_free",
-                         "gemm_epi_version"):
+                         "gemm_epi_version", "gemm_epi_run_noalloc"):
                 getattr(L, name).restype = i32
             _lib = L
     return _lib
@@ -159,6 +161,14 @@ def gemm_epi_aux_pitch_bytes(n: int) -> int:
 
 def gemm_epi_version() -> int:
     return lib().gemm_epi_version()
+
+
+def gemm_epi_run_noalloc(m, n, k, dtype, epilogue, bias_axis, b_layout, A, B, bias, d_scale_a,
+                         d_scale_b, D, aux, wait, stream) -> None:
+    """Allocation-free fused run (see include/gemm_epi.h); raises on a non-zero status."""
+    _check(lib().gemm_epi_run_noalloc(m, n, k, dtype, epilogue, bias_axis, b_layout, A, B, bias,
+                                      d_scale_a, d_scale_b, D, aux, wait, stream),
+           "gemm_epi_run_noalloc")
 
 
 def status_string(status: int) -> str:

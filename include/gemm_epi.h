@@ -181,6 +181,37 @@ int gemm_epi_check(gemm_epi_plan_t plan, void *stream);
 /* Fill *info with the plan's kernel choice.  ERR_ARG on a bad handle. */
 int gemm_epi_plan_query(gemm_epi_plan_t plan, gemm_epi_plan_info *info);
 
+/* Fused run that allocates nothing (the pages have no counterpart; this is a
+ * service of this library).  For callers that must not allocate device memory:
+ * code inside a host framework that hands out all device memory from its own
+ * pool and forbids side allocations, or code on a latency-critical path that
+ * cannot afford cudaMalloc/cudaFree and their implicit synchronisation.  Such
+ * callers cannot create a plan (a plan allocates its status word), so this
+ * call takes the problem description and the buffers directly and computes
+ * exactly what gemm_epi_plan_ex + gemm_epi_run would (same kernels, same
+ * automatic kernel choice, same argument rules and errors).
+ *
+ * Arguments: as gemm_epi_plan_ex and gemm_epi_run; d_scale_a/d_scale_b as in
+ * gemm_epi_set_scales (E4M3 only, else ignored).  wait = 0: enqueue and
+ * return; a kernel that gives up on a bounded wait goes unreported.  wait = 1:
+ * also synchronise `stream` and return GEMM_EPI_ERR_TIMEOUT if it did.
+ *
+ * Scratch and its limits: the kernels' only scratch is a 4-byte status word,
+ * kept in a 256-byte static device array that every GPU which loads this
+ * library holds until the process exits.  A call that needed more than 256
+ * bytes would be refused with GEMM_EPI_ERR_UNSUPPORTED; m, n and k are limited
+ * to 2^31 - 1 (GEMM_EPI_ERR_ARG beyond).  Every call on a device shares the
+ * array and clears the status word on `stream` before its launch, so calls
+ * that overlap on the GPU (other streams, other host threads) race on it: one
+ * call's timeout may be reported by another, or lost.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  No
+ * cudaMalloc, cudaFree or allocating library routine is called. */
+int gemm_epi_run_noalloc(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis,
+                         int b_layout, const void *A, const void *B, const void *bias,
+                         const float *d_scale_a, const float *d_scale_b, void *D, uint32_t *aux,
+                         int wait, void *stream);
+
 /* Release the plan (host metadata, tensor maps, status word).  Must not
  * overlap a run still executing on the GPU that uses this plan's status word:
  * synchronise first.  ERR_ARG for an unknown or already freed handle. */
