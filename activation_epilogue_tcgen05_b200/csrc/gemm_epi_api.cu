@@ -41,6 +41,11 @@ struct Plan {
     int kb_per_cta;
     int grid;
     int group_m;
+    // stream-K tail (TC kernels): tiles [0, sk_tiles) split by k-blocks, sk_q per unit
+    int sk_tiles = 0, sk_q = 0;
+    float *workspace = nullptr;          // owned: units x CG x 128 x block_n fp32
+    unsigned int *flags = nullptr;       // owned: units x CG x 4 words, zero between launches
+    size_t flags_bytes = 0;
     TcLauncher tc_launch = nullptr, tc_none_launch = nullptr;
     SkLauncher sk_launch = nullptr, sk_none_launch = nullptr;
     BiasActLauncher ba_launch = nullptr;
@@ -126,7 +131,15 @@ int round_nm(int64_t m) {
 int choose(Plan *P) {
     const int64_t m = P->m, n = P->n;
     int kernel = P->opts.kernel;
-    if (kernel == GEMM_EPI_KERNEL_AUTO) kernel = m <= 64 ? GEMM_EPI_KERNEL_SPLITK : GEMM_EPI_KERNEL_TC1;
+    if (kernel == GEMM_EPI_KERNEL_AUTO) {
+        // small m: swapped split-K; enough 256 x 256 tiles for every SM pair: CTA pairs
+        // (half the operand traffic per SM); otherwise single CTAs
+        const int64_t pair_tiles = ((m + 255) / 256) * ((n + 255) / 256);
+        const int sms_auto = P->opts.max_ctas > 0 ? std::min(P->opts.max_ctas, P->num_sms) : P->num_sms;
+        if (m <= 64) kernel = GEMM_EPI_KERNEL_SPLITK;
+        else if (pair_tiles >= sms_auto / 2) kernel = GEMM_EPI_KERNEL_TC2;
+        else kernel = GEMM_EPI_KERNEL_TC1;
+    }
     if (kernel == GEMM_EPI_KERNEL_SPLITK && m > 128) return GEMM_EPI_ERR_UNSUPPORTED;
     P->kernel = kernel;
     const bool b_mn = P->b_layout == GEMM_EPI_B_KN;
@@ -166,8 +179,27 @@ int choose(Plan *P) {
         if (bn != 128 && bn != 256) return GEMM_EPI_ERR_ARG;
         P->block_n = bn;
         const int64_t tiles = ((m + bm - 1) / bm) * ((n + bn - 1) / bn);
-        const int64_t units = std::min<int64_t>(tiles, cg == 2 ? sms / 2 : sms);
-        P->grid = (int)(units * cg);
+        const int64_t units_max = cg == 2 ? sms / 2 : sms;
+        // stream-K: split the tiles of an incomplete last wave (or all tiles, when there are
+        // fewer tiles than units) by k-blocks over every unit
+        int64_t sk_tiles = 0;
+        const int sk_mode = P->opts.stream_k;          // 0 auto, 1 off, 2 on
+        if (sk_mode != 1 && tiles % units_max != 0) {
+            const int64_t waves = (tiles + units_max - 1) / units_max;
+            const double loss = 1.0 - (double)tiles / (double)(waves * units_max);
+            const bool worth = tiles < units_max ? num_kb >= 8 : loss > 0.02;
+            if (sk_mode == 2 || worth) sk_tiles = tiles < units_max ? tiles : tiles % units_max;
+        }
+        if (sk_tiles > 0) {
+            int64_t q = (sk_tiles * num_kb + units_max - 1) / units_max;
+            q = std::max<int64_t>(q, std::min<int64_t>(num_kb, 4));   // at least 4 k-blocks a run
+            P->sk_tiles = (int)sk_tiles;
+            P->sk_q = (int)q;
+            P->grid = (int)(units_max * cg);
+        } else {
+            const int64_t units = std::min<int64_t>(tiles, units_max);
+            P->grid = (int)(units * cg);
+        }
         P->group_m = 8;
         KernelInfo none_info;
         if (!find_tc(cg, P->dtype, GEMM_EPI_NONE, 0, b_mn, bn, &P->tc_none_launch, &none_info))
@@ -271,6 +303,10 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.scale_b = P->scale_b;
         L.p.status = P->status;
         L.p.inject_stall = P->opts.inject_stall;
+        L.p.sk_tiles = P->sk_tiles;
+        L.p.sk_q = P->sk_q;
+        L.p.workspace = P->workspace;
+        L.p.flags = P->flags;
         L.grid = P->grid;
         L.stream = stream;
         e = (fused ? P->tc_launch : P->tc_none_launch)(L);
@@ -293,6 +329,7 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     if (o.block_n != 0 && o.block_n != 128 && o.block_n != 256) return GEMM_EPI_ERR_ARG;
     if (o.split_k < 0 || o.split_k > 8 || o.max_ctas < 0) return GEMM_EPI_ERR_ARG;
     if (o.inject_stall != 0 && o.inject_stall != 1) return GEMM_EPI_ERR_ARG;
+    if (o.stream_k < 0 || o.stream_k > 2) return GEMM_EPI_ERR_ARG;
     if (o.inject_stall && o.kernel == GEMM_EPI_KERNEL_SPLITK) return GEMM_EPI_ERR_UNSUPPORTED;
     // 16-byte row pitches (TMA strides; the pages' 16-byte alignment rule)
     const int es = esize(dtype);
@@ -334,12 +371,28 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
         delete P;
         return GEMM_EPI_ERR_CUDA;
     }
+    if (P->sk_tiles > 0) {
+        const int cg = P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
+        const size_t units = (size_t)P->grid / cg;
+        const size_t ws_bytes = units * cg * 128 * (size_t)P->block_n * sizeof(float);
+        const size_t fl_bytes = units * cg * 4 * sizeof(unsigned int);
+        P->flags_bytes = fl_bytes;
+        if (cudaMalloc(&P->workspace, ws_bytes) != cudaSuccess || cudaMalloc(&P->flags, fl_bytes) != cudaSuccess ||
+            cudaMemset(P->flags, 0, fl_bytes) != cudaSuccess) {
+            cudaGetLastError();
+            if (P->workspace) cudaFree(P->workspace);
+            if (P->flags) cudaFree(P->flags);
+            cudaFree(P->status);
+            delete P;
+            return GEMM_EPI_ERR_CUDA;
+        }
+    }
     if (getenv("GEMM_EPI_LOG")) {
         fprintf(stderr,
                 "gemm_epi plan m=%lld n=%lld k=%lld dtype=%d epi=%d axis=%d b=%d -> kernel=%d bn=%d nm=%d "
-                "split=%d grid=%d stages=%d smem=%d\n",
+                "split=%d grid=%d stages=%d smem=%d sk_tiles=%d sk_q=%d\n",
                 (long long)m, (long long)n, (long long)k, dtype, epilogue, bias_axis, b_layout, P->kernel,
-                P->block_n, P->nm, P->split, P->grid, P->info.stages, P->info.smem_bytes);
+                P->block_n, P->nm, P->split, P->grid, P->info.stages, P->info.smem_bytes, P->sk_tiles, P->sk_q);
     }
     {
         std::lock_guard<std::mutex> lk(g_mu);
@@ -443,6 +496,8 @@ int gemm_epi_check(gemm_epi_plan_t plan, void *stream) {
         return GEMM_EPI_ERR_CUDA;
     if (word != 0) {
         cudaMemset(P->status, 0, sizeof(word));
+        // an aborted launch may have left stream-K flags raised: start the next one clean
+        if (P->flags) cudaMemset(P->flags, 0, P->flags_bytes);
         return GEMM_EPI_ERR_TIMEOUT;
     }
     return GEMM_EPI_OK;
@@ -461,6 +516,8 @@ int gemm_epi_plan_query(gemm_epi_plan_t plan, gemm_epi_plan_info *info) {
     info->cluster = P->kernel == GEMM_EPI_KERNEL_SPLITK ? P->split : (P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1);
     info->threads = P->info.threads;
     info->smem_bytes = P->info.smem_bytes;
+    info->sk_tiles = P->sk_tiles;
+    info->sk_q = P->sk_q;
     if (P->kernel == GEMM_EPI_KERNEL_SPLITK) {
         info->tiles = (int)((P->n + 127) / 128);
     } else {
@@ -478,6 +535,8 @@ int gemm_epi_free(gemm_epi_plan_t plan) {
         g_plans.erase(P);
     }
     if (P->status) cudaFree(P->status);
+    if (P->workspace) cudaFree(P->workspace);
+    if (P->flags) cudaFree(P->flags);
     P->magic = 0;
     delete P;
     return GEMM_EPI_OK;
@@ -581,6 +640,7 @@ extern "C" int gemm_epi_run_noalloc(int64_t m, int64_t n, int64_t k, int dtype, 
     P.b_layout = b_layout;
     P.device = dev;
     P.num_sms = num_sms_of(dev);
+    P.opts.stream_k = 1;                        // stream-K would need a workspace: off
     int rc = choose(&P);
     if (rc != GEMM_EPI_OK) return rc;
     if (dtype == GEMM_EPI_E4M3) {

@@ -27,6 +27,18 @@
 //               accumulators the epilogue of tile t overlaps the mainloop of
 //               tile t+1.
 //
+// Stream-K tail: when the tiles do not divide evenly over the units (CTAs, or
+// CTA pairs), the first sk_tiles tiles are not given out whole.  Their
+// k-blocks are laid end to end and cut into equal runs of sk_q k-blocks, one run
+// per unit.  A unit whose run ends inside a tile writes that fp32 partial tile
+// to its workspace slot and raises one flag per epilogue warp; the unit
+// whose run holds a tile's last k-block waits (bounded) for the flags of the
+// units before it, adds their partials in unit order, clears those flags and
+// runs the epilogue.  Each unit handles its unfinished (partial) run first, so
+// a partial never waits on anything, and waiters only wait on lower-indexed
+// units.  Because every flag is cleared by its one reader, a launch leaves the
+// flags as it found them (all zero), so launches can be replayed (CUDA graphs).
+//
 // Every wait is bounded: after TIMEOUT_NS without progress the waiting thread
 // records a code in the caller's status word, raises a CTA-wide abort flag and
 // every role winds down (waiting, again bounded, for its own copies and MMAs
@@ -69,6 +81,10 @@ struct TcParams {
     const float *scale_b;
     unsigned int *status;        // device status word
     int inject_stall;            // testing only: 1 = the MMA issuer publishes no accumulator
+    int sk_tiles;                // tiles [0, sk_tiles) are split over the units by k-blocks
+    int sk_q;                    // k-blocks per unit in that stream-K phase
+    float *workspace;            // partial tiles: [unit][cta rank][128 rows][BN] fp32
+    unsigned int *flags;         // [unit][cta rank][4 epilogue warps]: 1 while a partial is unread
 };
 
 // Bounded mbarrier wait.  Returns false when this CTA is aborting (this wait
@@ -108,6 +124,68 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, unsign
         }
     }
 }
+
+// Bounded wait until *flag is set (a partial tile published by another unit).
+__device__ __forceinline__ bool wait_flag(const unsigned int *flag, volatile int *abort_flag, unsigned int *status) {
+    if (ptx::ld_acquire_gpu(flag) != 0u) return true;
+    const uint64_t t0 = ptx::globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (ptx::ld_acquire_gpu(flag) != 0u) return true;
+        if ((i & 15u) == 0u) {
+            if (*abort_flag) return false;
+            if (ptx::globaltimer() - t0 > TIMEOUT_NS) {
+                *abort_flag = 1;
+                atomicOr(status, ST_TIMEOUT_EPILOGUE);
+                return false;
+            }
+        }
+    }
+}
+
+// One unit of work: k-blocks [kb0, kb1) of one output tile.
+struct WorkItem {
+    int tile, kb0, kb1;
+};
+
+// The work of one unit, in processing order: its stream-K run (the segment
+// that ends inside a tile first, then the one that finishes a tile), then its
+// data-parallel tiles sk_tiles + unit, + units, ...  A run never spans more
+// than two tiles (sk_q <= num_kb).
+struct WorkIter {
+    WorkItem s0, s1;        // stream-K segments in processing order (kept out of an indexed array)
+    int nseg, i, dp_t;
+    __device__ WorkIter(const TcParams &p, int unit, int units) : nseg(0), i(0), dp_t(p.sk_tiles + unit) {
+        const int total = p.sk_tiles * p.num_kb;
+        const int beg = min(unit * p.sk_q, total);
+        const int end = min(beg + p.sk_q, total);
+        if (beg < end) {
+            const int t1 = beg / p.num_kb;
+            const int k1 = beg - t1 * p.num_kb;
+            if (end <= (t1 + 1) * p.num_kb) {
+                s0 = WorkItem{t1, k1, end - t1 * p.num_kb};
+                nseg = 1;
+            } else {
+                s0 = WorkItem{t1 + 1, 0, end - (t1 + 1) * p.num_kb};   // unfinished tile first
+                s1 = WorkItem{t1, k1, p.num_kb};
+                nseg = 2;
+            }
+        }
+        (void)units;
+    }
+    __device__ bool next(const TcParams &p, int units, WorkItem &w) {
+        if (i < nseg) {
+            w = i == 0 ? s0 : s1;
+            ++i;
+            return true;
+        }
+        if (dp_t < p.num_tiles) {
+            w = WorkItem{dp_t, 0, p.num_kb};
+            dp_t += units;
+            return true;
+        }
+        return false;
+    }
+};
 
 template <int DT>
 struct OutT;
@@ -276,12 +354,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             uint32_t stage = 0, phase = 0;
             uint32_t issued = 0;
             bool ok = true;
-            for (int t = unit; ok && t < p.num_tiles; t += units) {
+            WorkIter it(p, unit, units);
+            WorkItem w;
+            while (ok && it.next(p, units, w)) {
                 int tm, tn;
-                tile_coords(p, t, tm, tn);
+                tile_coords(p, w.tile, tm, tn);
                 const int m0 = tm * (C::BM * C::CG) + (int)rank * C::BM;
                 const int nb = tn * C::BN + (int)rank * C::BN_LOCAL;
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!wait_bounded<false>(empty_bar(stage), phase ^ 1u, abort_flag, p.status,
                                              ST_TIMEOUT_PRODUCER)) {
                         ok = false;
@@ -330,7 +410,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             bool ok = true;
             // with inject_stall nothing is issued or committed: the epilogue's
             // bounded wait for the first accumulator runs out (failure-path test)
-            for (int t = unit; ok && !p.inject_stall && t < p.num_tiles; t += units) {
+            WorkIter it(p, unit, units);
+            WorkItem w;
+            while (ok && !p.inject_stall && it.next(p, units, w)) {
                 if (!wait_bounded<C::CG == 2>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status,
                                               ST_TIMEOUT_MMA)) {
                     ok = false;
@@ -338,7 +420,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * C::BN;
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!wait_bounded<false>(full_bar(stage), phase, abort_flag, p.status, ST_TIMEOUT_MMA)) {
                         ok = false;
                         break;
@@ -351,7 +433,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         const uint64_t ad = make_sdesc(a_base + ks * 32, 16, 1024);
                         const uint64_t bd = C::B_MN ? make_sdesc(b_base + ks * C::UMMA_K * 128, C::B_BOX_BYTES, 1024)
                                                     : make_sdesc(b_base + ks * 32, 16, 1024);
-                        ptx::mma<C::CG, C::KIND>(d_tmem, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+                        ptx::mma<C::CG, C::KIND>(d_tmem, ad, bd, idesc, (kb > w.kb0 || ks > 0) ? 1u : 0u);
                     }
                     if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(empty_bar(stage), 0x3);
                     else ptx::mma_commit(empty_bar(stage));
@@ -378,9 +460,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if constexpr (C::DT == DT_E4M3) alpha = __ldg(p.scale_a) * __ldg(p.scale_b);
         uint32_t acc = 0, acc_phase = 0;
         bool ok = true;
-        for (int t = unit; ok && t < p.num_tiles; t += units) {
+        WorkIter it(p, unit, units);
+        WorkItem w;
+        while (ok && it.next(p, units, w)) {
+            // partial_out: this unit holds a non-final slice of the tile -> publish a partial.
+            // Otherwise units [c_first, unit) published the slices before ours.
+            const bool partial_out = w.kb1 < p.num_kb;
+            const int c_first = w.kb0 > 0 ? (w.tile * p.num_kb) / p.sk_q : unit;
             int tm, tn;
-            tile_coords(p, t, tm, tn);
+            tile_coords(p, w.tile, tm, tn);
             const int m0 = tm * (C::BM * C::CG) + (int)rank * C::BM;
             const int n0 = tn * C::BN;
             const int row = m0 + 32 * q + lane;
@@ -389,7 +477,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if constexpr (C::EPI != EPI_NONE && C::AXIS == AXIS_ROW) {
                 if (row_ok) rbias = O::load(p.bias, row);
             }
-            if constexpr (C::BIAS_FLOATS > 0) {
+            if constexpr (C::BIAS_FLOATS > 0) if (!partial_out) {
                 // this warp's copy of bias[n0 .. n0+BN) as fp32 (read once per tile)
                 __syncwarp();
                 if (n0 + C::BN <= p.n) {
@@ -412,7 +500,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 break;
             }
             ptx::tc_fence_after();
+            // this warp's rows of each earlier slice are published by the same warp quadrant
+            for (int v = c_first; ok && v < unit && !partial_out; ++v)
+                ok = wait_flag(p.flags + ((size_t)v * C::CG + rank) * 4 + q, abort_flag, p.status);
+            if (!ok) break;
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + acc * C::BN;
+            float *ws_own = p.workspace + (((size_t)unit * C::CG + rank) * 128 + 32 * q + lane) * C::BN;
 #pragma unroll 1
             for (int g = 0; g < C::BN / 128; ++g) {       // 128 output columns per group
                 uint32_t words[4];
@@ -429,6 +522,27 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         if (lane == 0) {
                             if constexpr (C::CG == 2) ptx::mbar_arrive_cluster(ptx::mapa(tempty_bar(acc), 0));
                             else ptx::mbar_arrive(tempty_bar(acc));
+                        }
+                    }
+                    if (partial_out) {
+                        // non-final slice: hand the fp32 partial to the tile's finishing unit
+                        float4 *dst = reinterpret_cast<float4 *>(ws_own + 32 * c);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                        continue;
+                    }
+                    for (int u = c_first; u < unit; ++u) {       // earlier slices, in unit order
+                        const float4 *src = reinterpret_cast<const float4 *>(
+                            p.workspace + (((size_t)u * C::CG + rank) * 128 + 32 * q + lane) * C::BN + 32 * c);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float4 f = __ldcg(src + j);
+                            v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + f.x);
+                            v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + f.y);
+                            v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + f.z);
+                            v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + f.w);
                         }
                     }
                     const int col0 = n0 + 32 * c;
@@ -475,6 +589,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         }
                     }
                 }
+                if (partial_out) continue;
                 if constexpr (C::EPI == EPI_RELU_AUX) {
                     const int wcol = n0 + 128 * g;
                     if (row_ok && wcol < p.n) {
@@ -482,6 +597,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         *dst = make_uint4(words[0], words[1], words[2], words[3]);
                     }
                 }
+            }
+            if (partial_out) {
+                // publish: every lane's stores are ordered before the warp's flag
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) ptx::st_release_gpu(p.flags + ((size_t)unit * C::CG + rank) * 4 + q, 1u);
+            } else if (lane == 0) {
+                // the earlier slices have been read: clear their flags for the next launch
+                for (int v = c_first; v < unit; ++v) p.flags[((size_t)v * C::CG + rank) * 4 + q] = 0u;
             }
             if (++acc == 2u) { acc = 0; acc_phase ^= 1u; }
         }

@@ -32,6 +32,7 @@ EPILOGUE = {"none": NONE, "bias": BIAS, "relu_bias": RELU_BIAS, "relu_aux_bias":
 AXIS = {"row": BIAS_ROW, "col": BIAS_COL}
 LAYOUT = {"kn": B_KN, "nk": B_NK}
 KERNEL = {"auto": KERNEL_AUTO, "tc1": KERNEL_TC1, "tc2": KERNEL_TC2, "splitk": KERNEL_SPLITK}
+STREAM_K = {"auto": 0, "off": 1, "on": 2}
 
 # every symbol include/gemm_epi.h declares
 EXPORTS = ("gemm_epi_plan", "gemm_epi_plan_ex", "gemm_epi_plan_opts", "gemm_epi_set_scales",
@@ -43,13 +44,13 @@ EXPORTS = ("gemm_epi_plan", "gemm_epi_plan_ex", "gemm_epi_plan_opts", "gemm_epi_
 class Options(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("block_n", ctypes.c_int32),
                 ("split_k", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
-                ("inject_stall", ctypes.c_int32)]
+                ("inject_stall", ctypes.c_int32), ("stream_k", ctypes.c_int32)]
 
 
 class PlanInfo(ctypes.Structure):
     _fields_ = [(f, ctypes.c_int32) for f in
                 ("kernel", "block_m", "block_n", "block_k", "stages", "split_k", "grid", "cluster",
-                 "threads", "smem_bytes", "tiles")]
+                 "threads", "smem_bytes", "tiles", "sk_tiles", "sk_q")]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -196,10 +197,11 @@ class Plan:
     """
 
     def __init__(self, m, n, k, dtype="bf16", epilogue="bias", bias_axis="row", b_layout="kn",
-                 kernel="auto", block_n=0, split_k=0, max_ctas=0, inject_stall=0):
+                 kernel="auto", block_n=0, split_k=0, max_ctas=0, inject_stall=0, stream_k="auto"):
         self.m, self.n, self.k = int(m), int(n), int(k)
         self.dtype, self.epilogue, self.bias_axis, self.b_layout = dtype, epilogue, bias_axis, b_layout
-        opts = Options(KERNEL[kernel], int(block_n), int(split_k), int(max_ctas), int(inject_stall))
+        opts = Options(KERNEL[kernel], int(block_n), int(split_k), int(max_ctas), int(inject_stall),
+                       STREAM_K[stream_k])
         self.handle = gemm_epi_plan_opts(self.m, self.n, self.k, DTYPE[dtype], EPILOGUE[epilogue],
                                          AXIS[bias_axis], LAYOUT[b_layout], opts)
         self._scales = None

@@ -58,11 +58,14 @@ def parse(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--kernel", default="auto", choices=["auto", "tc1", "tc2", "splitk"])
     ap.add_argument("--block-n", type=int, default=0)
+    ap.add_argument("--stream-k", default="auto", choices=["auto", "off", "on"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-unfused", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the timed steps directly instead of replaying them from a CUDA graph")
     return ap.parse_args(argv)
 
 
@@ -293,7 +296,7 @@ def main(argv=None):
         aux = torch.empty((aux_words,), dtype=torch.int32, device=dev) if aux_words else None
         sets.append((A, B, bias, D, aux))
     plan = g.Plan(wl.m, wl.n, wl.k, wl.dtype, wl.epilogue, wl.bias_axis, wl.b_layout,
-                  kernel=args.kernel, block_n=args.block_n)
+                  kernel=args.kernel, block_n=args.block_n, stream_k=args.stream_k)
     if wl.dtype == "e4m3":
         plan.set_scales(torch.tensor([prob.scale_a], dtype=torch.float32, device=dev),
                         torch.tensor([prob.scale_b], dtype=torch.float32, device=dev))
@@ -316,25 +319,55 @@ def main(argv=None):
         sampler.wait_first()
 
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    use_graph = not args.no_graph
+
+    def capture(fused: bool, count: int):
+        """The count steps (one launch each) captured into a CUDA graph."""
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cs = torch.cuda.current_stream(dev)
+            for i in range(count):
+                plan.run(*sets[i % n_sets], stream=cs, fused=fused)
+        return graph
+
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    replicas.barrier()
-    torch.cuda.synchronize(dev)
-    wall0 = time.time()
-    start.record(stream)
-    for i in range(K):
-        ev[i][0].record(stream)
-        plan.run(*sets[i % n_sets], stream=stream)
-        ev[i][1].record(stream)
-    end.record(stream)
-    torch.cuda.synchronize(dev)
-    wall1 = time.time()
-    replicas.barrier()
-    plan.check(stream)
-    elapsed_ms = start.elapsed_time(end)
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    if use_graph:
+        graph = capture(True, K)
+        graph.replay()                          # upload / first replay, untimed
+        torch.cuda.synchronize(dev)
+        plan.check(stream)
+        replicas.barrier()
+        torch.cuda.synchronize(dev)
+        wall0 = time.time()
+        start.record(stream)
+        graph.replay()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        wall1 = time.time()
+        replicas.barrier()
+        plan.check(stream)
+        elapsed_ms = start.elapsed_time(end)
+        # launches replay back to back: the average launch lasts the region over K
+        avg_launch_s = elapsed_ms / K / 1000.0
+        del graph
+    else:
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        replicas.barrier()
+        torch.cuda.synchronize(dev)
+        wall0 = time.time()
+        start.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            plan.run(*sets[i % n_sets], stream=stream)
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        wall1 = time.time()
+        replicas.barrier()
+        plan.check(stream)
+        elapsed_ms = start.elapsed_time(end)
+        avg_launch_s = statistics.fmean(a.elapsed_time(b) for a, b in ev) / 1000.0
     elapsed_ms_max = replicas.max_over_ranks(elapsed_ms, device=dev)
-    avg_launch_s = statistics.fmean(launch_ms) / 1000.0
     clocks = sampler.summary(wall0, wall1) if sampler else None
 
     value = flops * world * K / (elapsed_ms_max / 1000.0) / 1e12
@@ -367,17 +400,27 @@ def main(argv=None):
             plan.run(*sets[i % n_sets], stream=stream, fused=False)
         torch.cuda.synchronize(dev)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        for i in range(Ku):
-            plan.run(*sets[i % n_sets], stream=stream, fused=False)
-        s1.record(stream)
+        if use_graph:
+            ugraph = capture(False, Ku)
+            ugraph.replay()
+            torch.cuda.synchronize(dev)
+            s0.record(stream)
+            ugraph.replay()
+            s1.record(stream)
+        else:
+            s0.record(stream)
+            for i in range(Ku):
+                plan.run(*sets[i % n_sets], stream=stream, fused=False)
+            s1.record(stream)
         torch.cuda.synchronize(dev)
         plan.check(stream)
         ums = replicas.max_over_ranks(s0.elapsed_time(s1), device=dev) / Ku
         unfused = {"ms_per_step": ums, "value": flops * world / (ums / 1000) / 1e12, "unit": "TFLOP/s",
                    "steps": Ku, "launches_per_step": 2, "fused_speedup": ums / ms_per_step}
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers: every step copies its inputs
+    # from pinned host memory and reads its result back; copies of neighbouring steps overlap
+    # the compute (H2D, compute and D2H on three streams, two device buffer sets)
     e2e = None
     if not args.no_e2e:
         Ke = min(K, 50)
@@ -387,34 +430,60 @@ def main(argv=None):
         hA.copy_(A0)
         hB.copy_(B0)
         hbias.copy_(bias0)
-        hD = torch.empty((wl.m, wl.n), dtype=out_t, pin_memory=True)
-        haux = torch.empty((aux_words,), dtype=torch.int32, pin_memory=True) if aux_words else None
-        A, B, bias, D, aux = sets[0]
+        e_sets = [sets[0], sets[1] if n_sets > 1 else (
+            torch.empty_like(A0), torch.empty_like(B0), torch.empty_like(bias0),
+            torch.empty((wl.m, wl.n), dtype=out_t, device=dev),
+            torch.empty((aux_words,), dtype=torch.int32, device=dev) if aux_words else None)]
+        hD = [torch.empty((wl.m, wl.n), dtype=out_t, pin_memory=True) for _ in range(2)]
+        haux = [torch.empty((aux_words,), dtype=torch.int32, pin_memory=True) if aux_words else None
+                for _ in range(2)]
+        h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            A.copy_(hA, non_blocking=True)
-            B.copy_(hB, non_blocking=True)
-            bias.copy_(hbias, non_blocking=True)
-            plan.run(A, B, bias, D, aux, stream=stream)
-            hD.copy_(D, non_blocking=True)
-            if aux is not None:
-                haux.copy_(aux, non_blocking=True)
+        def e2e_steps(count, t_start=None, t_end=None):
+            used = [False, False]
+            for i in range(count):
+                j = i % 2
+                A, B, bias, D, aux = e_sets[j]
+                with torch.cuda.stream(h2d_s):
+                    if i == 0 and t_start is not None:
+                        t_start.record(h2d_s)
+                    if used[j]:
+                        h2d_s.wait_event(ev_comp[j])      # step i-2 has finished reading set j
+                    A.copy_(hA, non_blocking=True)
+                    B.copy_(hB, non_blocking=True)
+                    bias.copy_(hbias, non_blocking=True)
+                    ev_in[j].record(h2d_s)
+                stream.wait_event(ev_in[j])
+                if used[j]:
+                    stream.wait_event(ev_out[j])          # step i-2's result has been read back
+                plan.run(A, B, bias, D, aux, stream=stream)
+                ev_comp[j].record(stream)
+                with torch.cuda.stream(d2h_s):
+                    d2h_s.wait_event(ev_comp[j])
+                    hD[j].copy_(D, non_blocking=True)
+                    if aux is not None:
+                        haux[j].copy_(aux, non_blocking=True)
+                    ev_out[j].record(d2h_s)
+                used[j] = True
+            if t_end is not None:
+                t_end.record(d2h_s)
 
-        for _ in range(2):
-            e2e_step()
+        e2e_steps(2)
         torch.cuda.synchronize(dev)
         replicas.barrier()
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        for _ in range(Ke):
-            e2e_step()
-        s1.record(stream)
+        e2e_steps(Ke, s0, s1)
         torch.cuda.synchronize(dev)
         plan.check(stream)
         ems = replicas.max_over_ranks(s0.elapsed_time(s1), device=dev) / Ke
         e2e = {"value": flops * world / (ems / 1000) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(out_bytes),
-               "ms_per_step": ems, "steps": Ke, "api": "gemm_epi_run (C ABI) + pinned host copies"}
+               "ms_per_step": ems, "steps": Ke,
+               "api": "gemm_epi_run (C ABI) with pinned host buffers; H2D, compute and D2H of "
+                      "neighbouring steps overlap on three streams"}
 
     if sampler:
         sampler.stop()
@@ -444,7 +513,9 @@ def main(argv=None):
                        "l2": (f"inputs rotate over {n_sets} buffer sets ({n_sets * set_bytes / 2**20:.0f} MiB"
                               f" > 126 MB L2)" if n_sets > 1 else
                               f"one set of {set_bytes / 2**20:.0f} MiB > 126 MB L2"),
-                       "plan": info, "first_call_ms": first_call_ms},
+                       "plan": info, "first_call_ms": first_call_ms,
+                       "launch": "CUDA graph of the K steps (one kernel launch each)" if use_graph
+                       else "direct launches"},
             "pct_of_peak": 100.0 * roof["frac"],
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "unfused": unfused,
             "gpu_launches": K, "clocks": clocks,

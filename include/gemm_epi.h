@@ -93,8 +93,9 @@ enum gemm_epi_status {
 };
 
 /* Opaque plan.  Created by gemm_epi_plan*, owned by the caller until
- * gemm_epi_free; holds host metadata, a tensor-map cache and one 256-byte
- * device status word.  A plan may be run any number of times, on any stream,
+ * gemm_epi_free; holds host metadata, a tensor-map cache, one 256-byte
+ * device status word and, when the plan uses stream-K, a workspace for
+ * partial tiles plus their flags.  A plan may be run any number of times, on any stream,
  * from one host thread at a time. */
 typedef struct gemm_epi_plan_s *gemm_epi_plan_t;
 
@@ -108,12 +109,17 @@ typedef struct gemm_epi_options {
                              accumulator, so the epilogue's bounded wait runs out after about
                              one second and gemm_epi_check() reports GEMM_EPI_ERR_TIMEOUT;
                              D is left unwritten.  0 for real work.                        */
+    int32_t stream_k;  /* TC1/TC2: 0 = auto, 1 = off, 2 = on.  Stream-K splits the tiles of an
+                          incomplete last wave (or all tiles, when there are fewer tiles than
+                          SMs) by k-blocks over every SM; partial tiles pass through a
+                          workspace the plan allocates (SMs x 128 x block_n fp32).            */
 } gemm_epi_options;
 
 /* What a plan decided (for logging and tests). */
 typedef struct gemm_epi_plan_info {
     int32_t kernel, block_m, block_n, block_k, stages, split_k;
     int32_t grid, cluster, threads, smem_bytes, tiles;
+    int32_t sk_tiles, sk_q;   /* stream-K: tiles split by k-blocks, k-blocks per SM (unit) */
 } gemm_epi_plan_info;
 
 /* ---- entry points -------------------------------------------------------- */

@@ -83,10 +83,11 @@ def test_plan_rejects_bad_enums(g, kw):
 
 @pytest.mark.parametrize("opts", [
     dict(kernel=4), dict(kernel=-1), dict(block_n=64), dict(block_n=192), dict(split_k=9),
-    dict(split_k=-1), dict(max_ctas=-1), dict(inject_stall=2),
+    dict(split_k=-1), dict(max_ctas=-1), dict(inject_stall=2), dict(stream_k=3), dict(stream_k=-1),
 ])
 def test_plan_rejects_bad_options(g, opts):
-    o = g.Options(**{**dict(kernel=0, block_n=0, split_k=0, max_ctas=0, inject_stall=0), **opts})
+    o = g.Options(**{**dict(kernel=0, block_n=0, split_k=0, max_ctas=0, inject_stall=0,
+                            stream_k=0), **opts})
     assert _plan_rc(g, 64, 64, 64, opts=o) == g.ERR_ARG
 
 

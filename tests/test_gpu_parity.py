@@ -99,6 +99,63 @@ def test_integer_inputs_bit_exact(kernel, dtype, epilogue):
         np.testing.assert_array_equal(unpack_aux(words, wl.m, wl.n), mask)
 
 
+# ------------------------------------------------------------------ stream-K tail
+@pytest.mark.parametrize("kernel,max_ctas,m,n", [
+    ("tc1", 4, 600, 528),     # 25 tiles on 4 CTAs: one tile split four ways
+    ("tc1", 7, 600, 528),     # 25 tiles on 7 CTAs: runs span two tiles
+    ("tc1", 16, 256, 256),    # fewer tiles than CTAs: every tile split
+    ("tc2", 8, 600, 528),     # pairs: 3 x 5 tiles on 4 pairs
+    ("tc2", 8, 256, 256),     # pairs, fewer tiles than pairs (2 tiles on 4 pairs)
+])
+@pytest.mark.parametrize("dtype,epilogue,axis,layout", [
+    ("bf16", "relu_aux_bias", "row", "kn"), ("f16", "gelu_bias", "col", "nk"),
+    ("e4m3", "bias", "col", "kn"), ("bf16", "none", "row", "nk"),
+])
+def test_stream_k(kernel, max_ctas, m, n, dtype, epilogue, axis, layout):
+    k = 1024 if dtype == "e4m3" else 1000
+    wl = Workload("sk_tail", m, n, k, dtype, epilogue, axis, layout, seed=12)
+    prob = make_problem(wl)
+    bn = 256 if (kernel == "tc2" and dtype == "e4m3") else 128
+    worst, info = check_against_oracle(wl, prob, kernel=kernel, block_n=bn, max_ctas=max_ctas,
+                                       stream_k="on")
+    assert info["sk_tiles"] > 0
+    assert worst <= 1.0
+
+
+@pytest.mark.parametrize("kernel", ["tc1", "tc2"])
+def test_stream_k_deterministic_and_unfused(kernel):
+    wl = Workload("sk_det", 600, 528, 1000, "bf16", "relu_aux_bias", "row", "kn", seed=13)
+    prob = make_problem(wl)
+    inputs = device_inputs(prob)
+    opts = dict(kernel=kernel, block_n=128, max_ctas=6 if kernel == "tc1" else 8, stream_k="on")
+    D1, w1, info = gpu_run(wl, prob, inputs=inputs, **opts)
+    D2, w2, _ = gpu_run(wl, prob, inputs=inputs, **opts)
+    assert info["sk_tiles"] > 0
+    assert torch.equal(D1.view(torch.int16), D2.view(torch.int16))
+    np.testing.assert_array_equal(w1, w2)
+    Du, wu, _ = gpu_run(wl, prob, inputs=inputs, fused=False, **opts)
+    ref, pre, mask = oracle_full(wl, prob)
+    compare(wl, Du, wu, ref, pre, mask, *sigmas(prob), extra=unfused_extra(wl, prob, pre))
+
+
+def test_stream_k_repeated_runs_on_one_plan():
+    """Many runs of one plan: each launch must leave the partial-tile flags cleared."""
+    wl = Workload("sk_rep", 384, 400, 512, "f16", "relu_bias", "col", "kn", seed=14)
+    prob = make_problem(wl)
+    A, B, bias = device_inputs(prob)
+    D, _ = alloc_outputs(wl)
+    plan = make_plan(wl, prob, kernel="tc1", block_n=128, max_ctas=5, stream_k="on")
+    assert plan.info["sk_tiles"] > 0
+    ref, pre, mask = oracle_full(wl, prob)
+    sa, sb = sigmas(prob)
+    for _ in range(20):
+        D.fill_(float("nan"))
+        plan.run(A, B, bias, D, None)
+    plan.check()
+    plan.close()
+    compare(wl, D.cpu(), None, ref, pre, mask, sa, sb)
+
+
 # ------------------------------------------------------------------ small-m split-K kernel
 @pytest.mark.parametrize("layout", ["nk", "kn"])
 @pytest.mark.parametrize("axis", ["col", "row"])
