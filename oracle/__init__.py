@@ -30,7 +30,8 @@ _lock = threading.Lock()
 _lib = None
 
 DTYPES = ("f16", "bf16", "e4m3")
-EPILOGUES = ("none", "bias", "relu_bias", "relu_aux_bias", "gelu_bias")
+EPILOGUES = ("none", "bias", "relu_bias", "relu_aux_bias", "gelu_bias", "tanh_bias", "relu",
+             "relu_aux", "gelu", "tanh")
 AXES = ("row", "col")
 LAYOUTS = ("kn", "nk")
 

@@ -29,10 +29,15 @@
  *     optimization", paragraph 2; torch.nn.GELU() in "PyTorch 2.14 NVGEMM
  *     epilogue fusion" (zdabc.icu), section "verifying torch.compile".  Read
  *     as the exact erf form, 0.5 x (1 + erf(x / sqrt 2)).
+ *   - tanh after the bias (TANH_BIAS), and the same activations without a bias
+ *     (RELU, RELU_AUX, GELU, TANH): the predefined epilogue list of
+ *     "nvmath-python cuBLASLt bias fusion for PyTorch inference", paragraph 6
+ *     (Bias, ReLU, Tanh and so on).
  *   - a scaling factor applied in the epilogue: "PyTorch 2.14 NVGEMM epilogue
- *     fusion", section "why epilogue fusion matters".  Read as the FP8
- *     per-tensor dequantisation alpha = s_A * s_B applied to the product,
- *     before the bias; alpha = 1 for 16-bit inputs.
+ *     fusion", section "why epilogue fusion matters".  Read as alpha = s_A * s_B
+ *     multiplying the product before the bias, for every input type (the FP8
+ *     per-tensor dequantisation scales, or a plain scale for 16-bit inputs;
+ *     callers pass 1 and 1 for no scaling).
  *
  * Formats decoded here (from their definitions, not from any library):
  *   fp16  IEEE binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits.
@@ -57,7 +62,8 @@
 
 /* ---- the oracle's own vocabulary (independent of the CUDA library's enums) --- */
 enum { OR_F16 = 1, OR_BF16 = 2, OR_E4M3 = 3 };
-enum { OR_NONE = 10, OR_BIAS = 11, OR_RELU_BIAS = 12, OR_RELU_AUX_BIAS = 13, OR_GELU_BIAS = 14 };
+enum { OR_NONE = 10, OR_BIAS = 11, OR_RELU_BIAS = 12, OR_RELU_AUX_BIAS = 13, OR_GELU_BIAS = 14,
+       OR_TANH_BIAS = 15, OR_RELU = 16, OR_RELU_AUX = 17, OR_GELU = 18, OR_TANH = 19 };
 enum { OR_ROW = 20, OR_COL = 21 };
 enum { OR_KN = 30, OR_NK = 31 };
 
@@ -75,6 +81,11 @@ static int epi_code(const char *s) {
     if (!strcmp(s, "relu_bias")) return OR_RELU_BIAS;
     if (!strcmp(s, "relu_aux_bias")) return OR_RELU_AUX_BIAS;
     if (!strcmp(s, "gelu_bias")) return OR_GELU_BIAS;
+    if (!strcmp(s, "tanh_bias")) return OR_TANH_BIAS;
+    if (!strcmp(s, "relu")) return OR_RELU;
+    if (!strcmp(s, "relu_aux")) return OR_RELU_AUX;
+    if (!strcmp(s, "gelu")) return OR_GELU;
+    if (!strcmp(s, "tanh")) return OR_TANH;
     return 0;
 }
 static int axis_code(const char *s) {
@@ -153,16 +164,27 @@ static double load(const void *base, int dt, int64_t idx) {
  * inputs they are bf16. */
 static int bias_dtype(int dt) { return dt == OR_E4M3 ? OR_BF16 : dt; }
 
+/* Epilogues that add a bias vector. */
+static int has_bias(int epi) {
+    return epi == OR_BIAS || epi == OR_RELU_BIAS || epi == OR_RELU_AUX_BIAS || epi == OR_GELU_BIAS ||
+           epi == OR_TANH_BIAS;
+}
+
 /* One output element after the product p = sum_t a(i,t) b(t,j) is known. */
 static void finish(double p, int epi, int axis, int bdt, const void *bias, int64_t i, int64_t j,
                    double alpha, double *d, double *pre, uint8_t *mask) {
     p = alpha * p;
-    if (epi != OR_NONE) p += load(bias, bdt, axis == OR_ROW ? i : j);
+    if (has_bias(epi)) p += load(bias, bdt, axis == OR_ROW ? i : j);
     double y;
     switch (epi) {
     case OR_RELU_BIAS:
-    case OR_RELU_AUX_BIAS: y = p > 0.0 ? p : 0.0; break;
-    case OR_GELU_BIAS: y = oracle_gelu(p); break;
+    case OR_RELU_AUX_BIAS:
+    case OR_RELU:
+    case OR_RELU_AUX: y = p > 0.0 ? p : 0.0; break;
+    case OR_GELU_BIAS:
+    case OR_GELU: y = oracle_gelu(p); break;
+    case OR_TANH_BIAS:
+    case OR_TANH: y = tanh(p); break;
     default: y = p; break;                         /* NONE and BIAS */
     }
     *d = y;
@@ -175,7 +197,7 @@ static int check_args(int64_t m, int64_t n, int64_t k, int dt, int epi, int axis
     if (m <= 0 || n <= 0 || k <= 0) return -1;
     if (!dt || !epi || !axis || !lay) return -1;
     if (!A || !B) return -1;
-    if (epi != OR_NONE && !bias) return -1;
+    if (has_bias(epi) && !bias) return -1;
     return 0;
 }
 
@@ -191,7 +213,7 @@ int oracle_gemm_epi(int64_t m, int64_t n, int64_t k, const char *dtype, const ch
     int dt = dtype_code(dtype), epi = epi_code(epilogue), axis = axis_code(bias_axis);
     int lay = layout_code(b_layout);
     if (check_args(m, n, k, dt, epi, axis, lay, A, B, bias) || !D_ref) return -1;
-    double alpha = dt == OR_E4M3 ? scale_a * scale_b : 1.0;
+    double alpha = scale_a * scale_b;
     int bdt = bias_dtype(dt);
 
     double *Bd = (double *)malloc((size_t)k * (size_t)n * sizeof(double));
@@ -245,7 +267,7 @@ int oracle_gemm_epi_sampled(int64_t m, int64_t n, int64_t k, const char *dtype,
         return -1;
     for (int64_t s = 0; s < count; ++s)
         if (rows[s] < 0 || rows[s] >= m || cols[s] < 0 || cols[s] >= n) return -1;
-    double alpha = dt == OR_E4M3 ? scale_a * scale_b : 1.0;
+    double alpha = scale_a * scale_b;
     int bdt = bias_dtype(dt);
 #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t s = 0; s < count; ++s) {

@@ -18,8 +18,8 @@ SRC = os.path.join(ROOT, "oracle", "gemm_epi_oracle.c")
 # (id, text to replace, replacement, which occurrence (0-based) or None for all)
 MUTANTS = [
     ("bias_axis_swapped", "axis == OR_ROW ? i : j", "axis == OR_ROW ? j : i", None),
-    ("bias_dropped", "if (epi != OR_NONE) p += load", "if (0) p += load", None),
-    ("bias_on_none_too", "if (epi != OR_NONE) p += load", "if (1) p += load", None),
+    ("bias_dropped", "if (has_bias(epi)) p += load", "if (0) p += load", None),
+    ("bias_on_none_too", "if (has_bias(epi)) p += load", "if (epi == OR_NONE || has_bias(epi)) p += load", None),
     ("b_transposed_full", "lay == OR_KN ? t * n + j : j * k + t",
      "lay == OR_KN ? j * k + t : t * n + j", 0),
     ("b_transposed_sampled", "lay == OR_KN ? t * n + j : j * k + t",
@@ -31,14 +31,18 @@ MUTANTS = [
     ("mask_ge", "(uint8_t)(p > 0.0)", "(uint8_t)(p >= 0.0)", None),
     ("relu_dropped", "y = p > 0.0 ? p : 0.0", "y = p", None),
     ("alpha_dropped", "p = alpha * p;", "p = p;", None),
-    ("alpha_after_bias", "p = alpha * p;\n    if (epi != OR_NONE) p += load(bias, bdt, axis == OR_ROW ? i : j);",
-     "if (epi != OR_NONE) p += load(bias, bdt, axis == OR_ROW ? i : j);\n    p = alpha * p;", None),
+    ("alpha_after_bias", "p = alpha * p;\n    if (has_bias(epi)) p += load(bias, bdt, axis == OR_ROW ? i : j);",
+     "if (has_bias(epi)) p += load(bias, bdt, axis == OR_ROW ? i : j);\n    p = alpha * p;", None),
     ("e4m3_exponent_bias", "ldexp(1.0 + (double)f / 8.0, e - 7)", "ldexp(1.0 + (double)f / 8.0, e - 8)", None),
     ("e4m3_subnormal", "ldexp((double)f, -9)", "ldexp((double)f, -10)", None),
     ("f16_subnormal", "ldexp((double)f, -24)", "ldexp((double)f, -25)", None),
     ("bf16_exponent_bias", "e - 127)", "e - 126)", None),
     ("bias_dtype_for_fp8", "return dt == OR_E4M3 ? OR_BF16 : dt;", "return dt;", None),
     ("accumulate_dropped_term", "for (int64_t t = 0; t < k; ++t) {", "for (int64_t t = 1; t < k; ++t) {", None),
+    ("tanh_sign", "y = tanh(p);", "y = -tanh(p);", None),
+    ("tanh_as_relu", "case OR_TANH: y = tanh(p); break;", "case OR_TANH: y = p > 0.0 ? p : 0.0; break;", None),
+    ("bias_free_adds_bias", "return epi == OR_BIAS ||", "return epi == OR_RELU || epi == OR_BIAS ||", None),
+    ("alpha_fp8_only", "double alpha = scale_a * scale_b;", "double alpha = dt == OR_E4M3 ? scale_a * scale_b : 1.0;", None),
 ]
 
 

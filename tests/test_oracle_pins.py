@@ -296,8 +296,48 @@ def test_bad_arguments_rejected(oracle_lib):
     with pytest.raises(ValueError):
         oracle_lib.gemm_epi(a, a, a, dtype="f32", epilogue="bias")
     with pytest.raises(ValueError):
-        oracle_lib.gemm_epi(a, a, a, dtype="f16", epilogue="tanh")
+        oracle_lib.gemm_epi(a, a, a, dtype="f16", epilogue="swish")
     with pytest.raises(RuntimeError):
         oracle_lib.gemm_epi(a, a, None, dtype="f16", epilogue="bias")
     with pytest.raises(RuntimeError):
         oracle_lib.gemm_epi_sampled(a, a, a, [1], [0], dtype="f16", epilogue="bias")
+
+
+# ----------------------------------------------------------------------------- more epilogues
+@pytest.mark.parametrize("x", [0.125, 0.5, 1.0, 2.0, 4.0])
+def test_tanh_is_odd_and_bounded(oracle_lib, x):
+    a = to_storage_values([[x], [-x]], "f16")
+    one = to_storage_values([[1.0]], "f16")
+    D, pre, mask = oracle_lib.gemm_epi(a, one, None, dtype="f16", epilogue="tanh")
+    assert D[0, 0] == -D[1, 0]
+    assert 0 < D[0, 0] < 1 and D[0, 0] < x
+    assert D[0, 0] == pytest.approx((math.exp(2 * x) - 1) / (math.exp(2 * x) + 1), rel=1e-14)
+
+
+@pytest.mark.parametrize("pair", [("relu", "relu_bias"), ("relu_aux", "relu_aux_bias"),
+                                  ("gelu", "gelu_bias"), ("tanh", "tanh_bias")])
+def test_bias_free_epilogue_equals_zero_bias(oracle_lib, pair):
+    nobias, withbias = pair
+    wl = Workload("t", 13, 21, 34, "bf16", withbias, "col", "kn", seed=15, dist_bias=("zeros", 0))
+    p = make_problem(wl)
+    A, B, zero = storage(p.A), storage(p.B), storage(p.bias)
+    D0, pre0, m0 = oracle_lib.gemm_epi(A, B, zero, dtype="bf16", epilogue=withbias, bias_axis="col")
+    # a non-zero bias must be ignored by the bias-free epilogue
+    junk = to_storage_values(np.arange(21, dtype=np.float64).tolist(), "bf16")
+    D1, pre1, m1 = oracle_lib.gemm_epi(A, B, junk, dtype="bf16", epilogue=nobias, bias_axis="col")
+    np.testing.assert_array_equal(D0, D1)
+    np.testing.assert_array_equal(pre0, pre1)
+    np.testing.assert_array_equal(m0, m1)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_scaling_factor_applies_to_16bit_inputs(oracle_lib, dtype):
+    """alpha = s_A*s_B multiplies the product (not the bias) for 16-bit inputs too."""
+    wl = Workload("t", 9, 17, 24, dtype, "bias", "row", "kn", seed=16)
+    p = make_problem(wl)
+    A, B, bias = storage(p.A), storage(p.B), storage(p.bias)
+    _, pre1, _ = oracle_lib.gemm_epi(A, B, bias, dtype=dtype, epilogue="bias")
+    _, pre3, _ = oracle_lib.gemm_epi(A, B, bias, dtype=dtype, epilogue="bias", scale_a=1.5,
+                                     scale_b=2.0)
+    Dn, _, _ = oracle_lib.gemm_epi(A, B, None, dtype=dtype, epilogue="none")
+    np.testing.assert_allclose(pre3 - pre1, 2.0 * Dn, rtol=1e-12, atol=1e-12)
