@@ -33,7 +33,9 @@ __global__ void __launch_bounds__(256) bias_act_kernel(void *D, const void *bias
         }
         T *row = d + i * (int64_t)n;
         float rb = 0.0f;
-        if constexpr (AXIS == AXIS_ROW) rb = O::load(bias, i);
+        if constexpr (AXIS == AXIS_ROW) {
+            if (bias != nullptr) rb = O::load(bias, i);
+        }
         uint32_t bits = 0;
         if (j0 + 32 <= n) {
             uint4 *src = reinterpret_cast<uint4 *>(row + j0);
@@ -41,7 +43,10 @@ __global__ void __launch_bounds__(256) bias_act_kernel(void *D, const void *bias
 #pragma unroll
             for (int s = 0; s < 4; ++s) u[s] = src[s];
             float bcol[32];
-            if constexpr (AXIS == AXIS_COL) {
+            if constexpr (AXIS == AXIS_COL) if (bias == nullptr) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) bcol[e] = 0.0f;
+            } else {
                 const uint4 *bsrc = reinterpret_cast<const uint4 *>(reinterpret_cast<const T *>(bias) + j0);
 #pragma unroll
                 for (int s = 0; s < 4; ++s) {
@@ -70,7 +75,7 @@ __global__ void __launch_bounds__(256) bias_act_kernel(void *D, const void *bias
             }
         } else {
             for (int j = j0; j < n; ++j) {
-                float x = O::load(row, j) + (AXIS == AXIS_ROW ? rb : O::load(bias, j));
+                float x = O::load(row, j) + (AXIS == AXIS_ROW ? rb : (bias != nullptr ? O::load(bias, j) : 0.0f));
                 if constexpr (EPI == EPI_RELU_AUX) bits |= (x > 0.0f ? 1u : 0u) << (j - j0);
                 const float y = activate<EPI>(x);
                 if constexpr (DT == DT_F16) row[j] = __float2half_rn(y);

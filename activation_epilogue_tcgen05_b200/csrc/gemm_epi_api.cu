@@ -31,6 +31,8 @@ struct Plan {
     uint64_t magic;
     int64_t m, n, k;
     int dtype, epilogue, axis, b_layout;
+    int kepi;            // kernel epilogue (EPI_*): the activation
+    bool has_bias;       // the public epilogue adds a bias
     gemm_epi_options opts;
     int device, num_sms;
     // kernel choice
@@ -41,8 +43,8 @@ struct Plan {
     int kb_per_cta;
     int grid;
     int group_m;
-    // stream-K tail (TC kernels): tiles [0, sk_tiles) split by k-blocks, sk_q per unit
-    int sk_tiles = 0, sk_q = 0;
+    // split tail (TC kernels): tiles [0, sk_tiles) cut along k into sk_split parts
+    int sk_tiles = 0, sk_split = 0;
     float *workspace = nullptr;          // owned: units x CG x 128 x block_n fp32
     unsigned int *flags = nullptr;       // owned: units x CG x 4 words, zero between launches
     size_t flags_bytes = 0;
@@ -71,6 +73,23 @@ bool live(gemm_epi_plan_t h) {
 }
 
 int esize(int dt) { return dt == GEMM_EPI_E4M3 ? 1 : 2; }
+
+// Public epilogue -> kernel activation, and whether it adds a bias.  The
+// bias-free epilogues run the bias kernels with a NULL bias pointer.
+int kernel_epi(int e) {
+    switch (e) {
+    case GEMM_EPI_BIAS: return EPI_BIAS;
+    case GEMM_EPI_RELU_BIAS: case GEMM_EPI_RELU: return EPI_RELU;
+    case GEMM_EPI_RELU_AUX_BIAS: case GEMM_EPI_RELU_AUX: return EPI_RELU_AUX;
+    case GEMM_EPI_GELU_BIAS: case GEMM_EPI_GELU: return EPI_GELU;
+    case GEMM_EPI_TANH_BIAS: case GEMM_EPI_TANH: return EPI_TANH;
+    default: return EPI_NONE;
+    }
+}
+bool epi_has_bias(int e) {
+    return e == GEMM_EPI_BIAS || e == GEMM_EPI_RELU_BIAS || e == GEMM_EPI_RELU_AUX_BIAS || e == GEMM_EPI_GELU_BIAS ||
+           e == GEMM_EPI_TANH_BIAS;
+}
 
 // ----------------------------------------------------------------- tensor maps
 using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -166,7 +185,7 @@ int choose(Plan *P) {
         KernelInfo none_info;
         if (!find_sk(P->dtype, GEMM_EPI_NONE, 0, b_mn, P->nm, &P->sk_none_launch, &none_info))
             return GEMM_EPI_ERR_UNSUPPORTED;
-        if (!find_sk(P->dtype, P->epilogue, P->axis, b_mn, P->nm, &P->sk_launch, &P->info))
+        if (!find_sk(P->dtype, P->kepi, P->axis, b_mn, P->nm, &P->sk_launch, &P->info))
             return GEMM_EPI_ERR_UNSUPPORTED;
     } else {
         const int cg = kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
@@ -180,49 +199,71 @@ int choose(Plan *P) {
         P->block_n = bn;
         const int64_t tiles = ((m + bm - 1) / bm) * ((n + bn - 1) / bn);
         const int64_t units_max = cg == 2 ? sms / 2 : sms;
-        // stream-K: split the tiles of an incomplete last wave (or all tiles, when there are
-        // fewer tiles than units) by k-blocks over every unit
-        int64_t sk_tiles = 0;
+        // split tail: the tiles of an incomplete last wave (or all tiles, when there are fewer
+        // tiles than units) are cut along k into `split` parts on separate units, so the last
+        // wave costs 1/split of a tile.  Two parts by default: the finishing unit then adds a
+        // single partial, which overlaps its next tile's mainloop.
+        int64_t sk_tiles = 0, split = 0;
         const int sk_mode = P->opts.stream_k;          // 0 auto, 1 off, 2 on
         if (sk_mode != 1 && tiles % units_max != 0) {
+            const int64_t rem = tiles < units_max ? tiles : tiles % units_max;
             const int64_t waves = (tiles + units_max - 1) / units_max;
             const double loss = 1.0 - (double)tiles / (double)(waves * units_max);
+            split = std::min<int64_t>({units_max / rem, P->opts.split_k > 0 ? P->opts.split_k : 2, num_kb});
             const bool worth = tiles < units_max ? num_kb >= 8 : loss > 0.02;
-            if (sk_mode == 2 || worth) sk_tiles = tiles < units_max ? tiles : tiles % units_max;
+            if (split >= 2 && (sk_mode == 2 || worth)) sk_tiles = rem;
         }
         if (sk_tiles > 0) {
-            int64_t q = (sk_tiles * num_kb + units_max - 1) / units_max;
-            q = std::max<int64_t>(q, std::min<int64_t>(num_kb, 4));   // at least 4 k-blocks a run
             P->sk_tiles = (int)sk_tiles;
-            P->sk_q = (int)q;
-            P->grid = (int)(units_max * cg);
+            P->sk_split = (int)split;
+            // whole waves of tiles remain for every unit, or only the split parts need units
+            const int64_t units = tiles > sk_tiles ? units_max : sk_tiles * split;
+            P->grid = (int)(units * cg);
         } else {
             const int64_t units = std::min<int64_t>(tiles, units_max);
             P->grid = (int)(units * cg);
         }
         P->group_m = 8;
+        if (const char *g = getenv("GEMM_EPI_GROUP_M")) {   // tuning knob: tile-raster group height
+            const int v = atoi(g);
+            if (v >= 1 && v <= 64) P->group_m = v;
+        }
         KernelInfo none_info;
         if (!find_tc(cg, P->dtype, GEMM_EPI_NONE, 0, b_mn, bn, &P->tc_none_launch, &none_info))
             return GEMM_EPI_ERR_UNSUPPORTED;
-        if (!find_tc(cg, P->dtype, P->epilogue, P->axis, b_mn, bn, &P->tc_launch, &P->info))
+        if (!find_tc(cg, P->dtype, P->kepi, P->axis, b_mn, bn, &P->tc_launch, &P->info))
             return GEMM_EPI_ERR_UNSUPPORTED;
         P->split = 1;
     }
-    if (P->epilogue != GEMM_EPI_NONE && !find_bias_act(P->dtype, P->epilogue, P->axis, &P->ba_launch))
+    if (P->kepi != EPI_NONE && !find_bias_act(P->dtype, P->kepi, P->axis, &P->ba_launch))
         return GEMM_EPI_ERR_UNSUPPORTED;
     return GEMM_EPI_OK;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Timeline buffer of a tracing build (GEMM_EPI_TRACE=1); NULL in a normal build.
+unsigned long long *trace_buffer() {
+#if GEMM_EPI_TRACE
+    static unsigned long long *buf = nullptr;
+    if (!buf) {
+        const size_t bytes = (2 + 2 * (size_t)TRACE_CAP) * sizeof(unsigned long long);
+        if (cudaMalloc(&buf, bytes) != cudaSuccess || cudaMemset(buf, 0, bytes) != cudaSuccess) buf = nullptr;
+    }
+    return buf;
+#else
+    return nullptr;
+#endif
+}
+
 int check_run_args(Plan *P, const void *A, const void *B, const void *bias, void *D, uint32_t *aux) {
     if (!A || !B || !D) return GEMM_EPI_ERR_NULL;
-    if (P->epilogue != GEMM_EPI_NONE && !bias) return GEMM_EPI_ERR_NULL;
-    if (P->epilogue == GEMM_EPI_RELU_AUX_BIAS && !aux) return GEMM_EPI_ERR_NULL;
+    if (P->has_bias && !bias) return GEMM_EPI_ERR_NULL;
+    if (P->kepi == EPI_RELU_AUX && !aux) return GEMM_EPI_ERR_NULL;
     if (P->dtype == GEMM_EPI_E4M3 && (!P->scale_a || !P->scale_b)) return GEMM_EPI_ERR_NULL;
     if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return GEMM_EPI_ERR_ALIGN;
-    if (P->epilogue != GEMM_EPI_NONE && !aligned16(bias)) return GEMM_EPI_ERR_ALIGN;
-    if (P->epilogue == GEMM_EPI_RELU_AUX_BIAS && !aligned16(aux)) return GEMM_EPI_ERR_ALIGN;
+    if (P->has_bias && !aligned16(bias)) return GEMM_EPI_ERR_ALIGN;
+    if (P->kepi == EPI_RELU_AUX && !aligned16(aux)) return GEMM_EPI_ERR_ALIGN;
     return GEMM_EPI_OK;
 }
 
@@ -258,6 +299,7 @@ int ensure_maps(Plan *P, const void *A, const void *B, void *D) {
 }
 
 int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, cudaStream_t stream) {
+    if (!P->has_bias) bias = nullptr;
     const int bk = 128 / esize(P->dtype);
     const int num_kb = (int)((P->k + bk - 1) / bk);
     const int64_t pitch_words = ((P->n + 127) / 128) * 4;
@@ -304,9 +346,10 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.status = P->status;
         L.p.inject_stall = P->opts.inject_stall;
         L.p.sk_tiles = P->sk_tiles;
-        L.p.sk_q = P->sk_q;
+        L.p.sk_split = P->sk_split;
         L.p.workspace = P->workspace;
         L.p.flags = P->flags;
+        L.p.trace = trace_buffer();
         L.grid = P->grid;
         L.stream = stream;
         e = (fused ? P->tc_launch : P->tc_none_launch)(L);
@@ -320,7 +363,7 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     if (m <= 0 || n <= 0 || k <= 0) return GEMM_EPI_ERR_ARG;
     if (m > 0x7fffffffll || n > 0x7fffffffll || k > 0x7fffffffll) return GEMM_EPI_ERR_ARG;
     if (dtype < GEMM_EPI_F16 || dtype > GEMM_EPI_E4M3) return GEMM_EPI_ERR_ARG;
-    if (epilogue < GEMM_EPI_NONE || epilogue > GEMM_EPI_GELU_BIAS) return GEMM_EPI_ERR_ARG;
+    if (epilogue < GEMM_EPI_NONE || epilogue > GEMM_EPI_TANH) return GEMM_EPI_ERR_ARG;
     if (bias_axis != GEMM_EPI_BIAS_ROW && bias_axis != GEMM_EPI_BIAS_COL) return GEMM_EPI_ERR_ARG;
     if (b_layout != GEMM_EPI_B_KN && b_layout != GEMM_EPI_B_NK) return GEMM_EPI_ERR_ARG;
     gemm_epi_options o{};
@@ -355,7 +398,9 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     P->k = k;
     P->dtype = dtype;
     P->epilogue = epilogue;
-    P->axis = epilogue == GEMM_EPI_NONE ? GEMM_EPI_BIAS_ROW : bias_axis;
+    P->kepi = kernel_epi(epilogue);
+    P->has_bias = epi_has_bias(epilogue);
+    P->axis = P->has_bias ? bias_axis : GEMM_EPI_BIAS_ROW;
     P->b_layout = b_layout;
     P->opts = o;
     P->device = dev;
@@ -390,9 +435,9 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     if (getenv("GEMM_EPI_LOG")) {
         fprintf(stderr,
                 "gemm_epi plan m=%lld n=%lld k=%lld dtype=%d epi=%d axis=%d b=%d -> kernel=%d bn=%d nm=%d "
-                "split=%d grid=%d stages=%d smem=%d sk_tiles=%d sk_q=%d\n",
+                "split=%d grid=%d stages=%d smem=%d sk_tiles=%d sk_split=%d\n",
                 (long long)m, (long long)n, (long long)k, dtype, epilogue, bias_axis, b_layout, P->kernel,
-                P->block_n, P->nm, P->split, P->grid, P->info.stages, P->info.smem_bytes, P->sk_tiles, P->sk_q);
+                P->block_n, P->nm, P->split, P->grid, P->info.stages, P->info.smem_bytes, P->sk_tiles, P->sk_split);
     }
     {
         std::lock_guard<std::mutex> lk(g_mu);
@@ -449,7 +494,10 @@ int gemm_epi_plan_opts(int64_t m, int64_t n, int64_t k, int dtype, int epilogue,
 int gemm_epi_set_scales(gemm_epi_plan_t plan, const float *d_scale_a, const float *d_scale_b) {
     if (!live(plan)) return GEMM_EPI_ERR_ARG;
     Plan *P = reinterpret_cast<Plan *>(plan);
-    if (P->dtype != GEMM_EPI_E4M3) return GEMM_EPI_ERR_ARG;
+    if (!d_scale_a && !d_scale_b && P->dtype != GEMM_EPI_E4M3) {   // 16-bit: back to alpha = 1
+        P->scale_a = P->scale_b = nullptr;
+        return GEMM_EPI_OK;
+    }
     if (!d_scale_a || !d_scale_b) return GEMM_EPI_ERR_NULL;
     if ((reinterpret_cast<uintptr_t>(d_scale_a) & 3u) || (reinterpret_cast<uintptr_t>(d_scale_b) & 3u))
         return GEMM_EPI_ERR_ALIGN;
@@ -479,7 +527,8 @@ int gemm_epi_unfused_run(gemm_epi_plan_t plan, const void *A, const void *B, con
     if (rc != GEMM_EPI_OK) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     rc = launch_main(P, false, bias, D, aux, s);
-    if (rc != GEMM_EPI_OK || P->epilogue == GEMM_EPI_NONE) return rc;
+    if (rc != GEMM_EPI_OK || P->kepi == EPI_NONE) return rc;
+    if (!P->has_bias) bias = nullptr;
     const int64_t pitch_words = ((P->n + 127) / 128) * 4;
     const int64_t total = P->m * pitch_words;
     const int64_t blocks = std::min<int64_t>((total + 255) / 256, (int64_t)P->num_sms * 16);
@@ -517,7 +566,7 @@ int gemm_epi_plan_query(gemm_epi_plan_t plan, gemm_epi_plan_info *info) {
     info->threads = P->info.threads;
     info->smem_bytes = P->info.smem_bytes;
     info->sk_tiles = P->sk_tiles;
-    info->sk_q = P->sk_q;
+    info->sk_split = P->sk_split;
     if (P->kernel == GEMM_EPI_KERNEL_SPLITK) {
         info->tiles = (int)((P->n + 127) / 128);
     } else {
@@ -610,7 +659,7 @@ extern "C" int gemm_epi_run_noalloc(int64_t m, int64_t n, int64_t k, int dtype, 
     if (m <= 0 || n <= 0 || k <= 0) return GEMM_EPI_ERR_ARG;
     if (m > 0x7fffffffll || n > 0x7fffffffll || k > 0x7fffffffll) return GEMM_EPI_ERR_ARG;
     if (dtype < GEMM_EPI_F16 || dtype > GEMM_EPI_E4M3) return GEMM_EPI_ERR_ARG;
-    if (epilogue < GEMM_EPI_NONE || epilogue > GEMM_EPI_GELU_BIAS) return GEMM_EPI_ERR_ARG;
+    if (epilogue < GEMM_EPI_NONE || epilogue > GEMM_EPI_TANH) return GEMM_EPI_ERR_ARG;
     if (bias_axis != GEMM_EPI_BIAS_ROW && bias_axis != GEMM_EPI_BIAS_COL) return GEMM_EPI_ERR_ARG;
     if (b_layout != GEMM_EPI_B_KN && b_layout != GEMM_EPI_B_NK) return GEMM_EPI_ERR_ARG;
     if (wait != 0 && wait != 1) return GEMM_EPI_ERR_ARG;
@@ -636,14 +685,17 @@ extern "C" int gemm_epi_run_noalloc(int64_t m, int64_t n, int64_t k, int dtype, 
     P.k = k;
     P.dtype = dtype;
     P.epilogue = epilogue;
-    P.axis = epilogue == GEMM_EPI_NONE ? GEMM_EPI_BIAS_ROW : bias_axis;
+    P.kepi = kernel_epi(epilogue);
+    P.has_bias = epi_has_bias(epilogue);
+    P.axis = P.has_bias ? bias_axis : GEMM_EPI_BIAS_ROW;
     P.b_layout = b_layout;
     P.device = dev;
     P.num_sms = num_sms_of(dev);
     P.opts.stream_k = 1;                        // stream-K would need a workspace: off
     int rc = choose(&P);
     if (rc != GEMM_EPI_OK) return rc;
-    if (dtype == GEMM_EPI_E4M3) {
+    if (dtype == GEMM_EPI_E4M3 || d_scale_a || d_scale_b) {      // 16-bit: optional alpha
+        if (!d_scale_a || !d_scale_b) return GEMM_EPI_ERR_NULL;
         P.scale_a = d_scale_a;
         P.scale_b = d_scale_b;
     }
@@ -665,3 +717,15 @@ extern "C" int gemm_epi_run_noalloc(int64_t m, int64_t n, int64_t k, int dtype, 
     if (cudaMemcpy(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return GEMM_EPI_ERR_CUDA;
     return word != 0 ? GEMM_EPI_ERR_TIMEOUT : GEMM_EPI_OK;
 }
+
+#if GEMM_EPI_TRACE
+// Tracing builds only: copy the timeline (counter word + records) to host memory and reset it.
+extern "C" int gemm_epi_trace_read(void *host, size_t bytes) {
+    unsigned long long *buf = trace_buffer();
+    if (!buf) return GEMM_EPI_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return GEMM_EPI_ERR_CUDA;
+    const size_t cap = (2 + 2 * (size_t)TRACE_CAP) * sizeof(unsigned long long);
+    if (cudaMemcpy(host, buf, bytes < cap ? bytes : cap, cudaMemcpyDeviceToHost) != cudaSuccess) return GEMM_EPI_ERR_CUDA;
+    return cudaMemset(buf, 0, sizeof(unsigned long long)) == cudaSuccess ? GEMM_EPI_OK : GEMM_EPI_ERR_CUDA;
+}
+#endif

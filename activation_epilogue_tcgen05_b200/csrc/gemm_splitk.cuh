@@ -242,10 +242,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const int col = n0 + row_in_tile;
         const bool col_ok = col < p.n;
         float alpha = 1.0f;
-        if constexpr (C::DT == DT_E4M3) alpha = __ldg(p.scale_a) * __ldg(p.scale_b);
+        if (p.scale_a != nullptr) alpha = __ldg(p.scale_a) * __ldg(p.scale_b);
+        const bool has_bias = p.bias != nullptr;
         float cbias = 0.0f;
         if constexpr (C::EPI != EPI_NONE && C::AXIS == AXIS_COL) {
-            if (col_ok) cbias = O::load(p.bias, col);
+            if (col_ok && has_bias) cbias = O::load(p.bias, col);
         }
         T *D = reinterpret_cast<T *>(p.D);
         // every word of the mask pitch belongs to exactly one warp of one tile;
@@ -255,10 +256,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int i = 0; i < C::NM; ++i) {
             if (i < p.m) {
                 float x = acc[i];
-                if constexpr (C::DT == DT_E4M3) x *= alpha;
+                x *= alpha;
                 if constexpr (C::EPI != EPI_NONE) {
                     if constexpr (C::AXIS == AXIS_COL) x += cbias;
-                    else x += O::load(p.bias, i);
+                    else if (has_bias) x += O::load(p.bias, i);
                 }
                 if constexpr (C::EPI == EPI_RELU_AUX) {
                     const uint32_t bits = __ballot_sync(0xFFFFFFFFu, col_ok && x > 0.0f);

@@ -27,17 +27,16 @@
 //               accumulators the epilogue of tile t overlaps the mainloop of
 //               tile t+1.
 //
-// Stream-K tail: when the tiles do not divide evenly over the units (CTAs, or
-// CTA pairs), the first sk_tiles tiles are not given out whole.  Their
-// k-blocks are laid end to end and cut into equal runs of sk_q k-blocks, one run
-// per unit.  A unit whose run ends inside a tile writes that fp32 partial tile
-// to its workspace slot and raises one flag per epilogue warp; the unit
-// whose run holds a tile's last k-block waits (bounded) for the flags of the
-// units before it, adds their partials in unit order, clears those flags and
-// runs the epilogue.  Each unit handles its unfinished (partial) run first, so
-// a partial never waits on anything, and waiters only wait on lower-indexed
-// units.  Because every flag is cleared by its one reader, a launch leaves the
-// flags as it found them (all zero), so launches can be replayed (CUDA graphs).
+// Split tail (stream-K style): when the tiles do not divide evenly over the
+// units (CTAs, or CTA pairs), the first sk_tiles tiles are not given out
+// whole.  Tile i is cut along k into sk_split equal parts handled by units
+// i*sk_split + j as their first piece of work.  Parts j < sk_split-1 write their
+// fp32 partial tile to the unit's workspace slot and raise one flag per
+// epilogue warp; the last part's unit waits (bounded) for those flags, adds the
+// partials in part order, clears the flags and runs the epilogue.  All parts
+// start together and waiters only wait on lower-indexed units.  Because every
+// flag is cleared by its one reader, a launch leaves the flags as it found
+// them (all zero), so launches can be replayed (CUDA graphs).
 //
 // Every wait is bounded: after TIMEOUT_NS without progress the waiting thread
 // records a code in the caller's status word, raises a CTA-wide abort flag and
@@ -55,7 +54,9 @@
 namespace gemm_epi {
 
 enum : int { DT_F16 = 0, DT_BF16 = 1, DT_E4M3 = 2 };
-enum : int { EPI_NONE = 0, EPI_BIAS = 1, EPI_RELU = 2, EPI_RELU_AUX = 3, EPI_GELU = 4 };
+// Kernel epilogues (activation after alpha*A.B + bias).  A bias pointer of
+// NULL means no bias: the bias-free public epilogues run these same kernels.
+enum : int { EPI_NONE = 0, EPI_BIAS = 1, EPI_RELU = 2, EPI_RELU_AUX = 3, EPI_GELU = 4, EPI_TANH = 5 };
 enum : int { AXIS_ROW = 0, AXIS_COL = 1 };
 
 // Status-word bits written by kernels that gave up waiting.
@@ -77,15 +78,40 @@ struct TcParams {
     const void *bias;            // length m (ROW) or n (COL), output type
     uint32_t *aux;               // RELU_AUX only
     int64_t aux_pitch_words;     // ceil(n/128)*4
-    const float *scale_a;        // E4M3 only (device scalars)
+    const float *scale_a;        // alpha = *scale_a * *scale_b when set (always for E4M3)
     const float *scale_b;
     unsigned int *status;        // device status word
     int inject_stall;            // testing only: 1 = the MMA issuer publishes no accumulator
-    int sk_tiles;                // tiles [0, sk_tiles) are split over the units by k-blocks
-    int sk_q;                    // k-blocks per unit in that stream-K phase
-    float *workspace;            // partial tiles: [unit][cta rank][128 rows][BN] fp32
+    int sk_tiles;                // tiles [0, sk_tiles) are split along k over units
+    int sk_split;                // parts per split tile (units per split tile)
+    float *workspace;            // partial tiles, 128 x BN fp32 per (unit, cta rank); see ws_slot()
     unsigned int *flags;         // [unit][cta rank][4 epilogue warps]: 1 while a partial is unread
+    unsigned long long *trace;   // timeline records; used only by builds with GEMM_EPI_TRACE=1
 };
+
+// Timeline tracing (off unless the library is compiled with -DGEMM_EPI_TRACE=1):
+// each record is two 64-bit words, %globaltimer and (cta << 40 | warp << 32 |
+// event << 24 | tile << 8 | k-block), appended at trace[2 + 2*i] with i from an
+// atomic counter in trace[0].
+#ifndef GEMM_EPI_TRACE
+#define GEMM_EPI_TRACE 0
+#endif
+constexpr unsigned int TRACE_CAP = 1u << 21;
+__device__ __forceinline__ void trace_event(unsigned long long *trace, int warp, unsigned int ev, int tile,
+                                            int kb) {
+    if constexpr (GEMM_EPI_TRACE != 0) {
+        if (trace == nullptr) return;
+        const unsigned long long i = atomicAdd(trace, 1ull);
+        if (i < TRACE_CAP) {
+            trace[2 + 2 * i] = ptx::globaltimer();
+            trace[3 + 2 * i] = ((unsigned long long)blockIdx.x << 40) | ((unsigned long long)warp << 32) |
+                               ((unsigned long long)ev << 24) | ((unsigned long long)(tile & 0xFFFF) << 8) |
+                               (unsigned long long)(kb & 0xFF);
+        }
+    } else {
+        (void)trace; (void)warp; (void)ev; (void)tile; (void)kb;
+    }
+}
 
 // Bounded mbarrier wait.  Returns false when this CTA is aborting (this wait
 // timed out, or another role already raised the abort flag).
@@ -142,40 +168,40 @@ __device__ __forceinline__ bool wait_flag(const unsigned int *flag, volatile int
     }
 }
 
+// Where a thread's 32 partial sums of chunk c live in a workspace slot (128 x BN
+// fp32 per unit and CTA rank).  The slot is laid out [warp q][chunk c][group
+// g < 8][lane][4 floats], so the eight float4 accesses of a chunk are each one
+// 512-byte contiguous run per warp (fully coalesced writes and reads).
+template <int BN>
+__device__ __forceinline__ float4 *ws_chunk(float *workspace, int unit, int cg, int rank, int q, int c, int lane) {
+    float *slot = workspace + ((size_t)unit * cg + rank) * 128 * BN;
+    return reinterpret_cast<float4 *>(slot) + ((size_t)(q * (BN / 32) + c) * 8) * 32 + lane;
+}
+
 // One unit of work: k-blocks [kb0, kb1) of one output tile.
 struct WorkItem {
     int tile, kb0, kb1;
 };
 
-// The work of one unit, in processing order: its stream-K run (the segment
-// that ends inside a tile first, then the one that finishes a tile), then its
-// data-parallel tiles sk_tiles + unit, + units, ...  A run never spans more
-// than two tiles (sk_q <= num_kb).
+// The work of one unit, in processing order: its part of a split tile (if
+// unit < sk_tiles * sk_split), then its data-parallel tiles sk_tiles + unit,
+// + units, ...
 struct WorkIter {
-    WorkItem s0, s1;        // stream-K segments in processing order (kept out of an indexed array)
-    int nseg, i, dp_t;
-    __device__ WorkIter(const TcParams &p, int unit, int units) : nseg(0), i(0), dp_t(p.sk_tiles + unit) {
-        const int total = p.sk_tiles * p.num_kb;
-        const int beg = min(unit * p.sk_q, total);
-        const int end = min(beg + p.sk_q, total);
-        if (beg < end) {
-            const int t1 = beg / p.num_kb;
-            const int k1 = beg - t1 * p.num_kb;
-            if (end <= (t1 + 1) * p.num_kb) {
-                s0 = WorkItem{t1, k1, end - t1 * p.num_kb};
-                nseg = 1;
-            } else {
-                s0 = WorkItem{t1 + 1, 0, end - (t1 + 1) * p.num_kb};   // unfinished tile first
-                s1 = WorkItem{t1, k1, p.num_kb};
-                nseg = 2;
-            }
+    WorkItem s0;
+    bool has_part;
+    int dp_t;
+    __device__ WorkIter(const TcParams &p, int unit, int units) : has_part(false), dp_t(p.sk_tiles + unit) {
+        if (unit < p.sk_tiles * p.sk_split) {
+            const int tile = unit / p.sk_split, part = unit - tile * p.sk_split;
+            s0 = WorkItem{tile, part * p.num_kb / p.sk_split, (part + 1) * p.num_kb / p.sk_split};
+            has_part = true;
         }
         (void)units;
     }
     __device__ bool next(const TcParams &p, int units, WorkItem &w) {
-        if (i < nseg) {
-            w = i == 0 ? s0 : s1;
-            ++i;
+        if (has_part) {
+            w = s0;
+            has_part = false;
             return true;
         }
         if (dp_t < p.num_tiles) {
@@ -240,6 +266,8 @@ __device__ __forceinline__ float activate(float x) {
         return x > 0.0f ? x : 0.0f;
     } else if constexpr (EPI == EPI_GELU) {
         return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+    } else if constexpr (EPI == EPI_TANH) {
+        return tanhf(x);
     } else {
         return x;
     }
@@ -357,6 +385,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             WorkIter it(p, unit, units);
             WorkItem w;
             while (ok && it.next(p, units, w)) {
+                trace_event(p.trace, warp, 1, w.tile, w.kb0);
                 int tm, tn;
                 tile_coords(p, w.tile, tm, tn);
                 const int m0 = tm * (C::BM * C::CG) + (int)rank * C::BM;
@@ -419,6 +448,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     break;
                 }
                 ptx::tc_fence_after();
+                trace_event(p.trace, warp, 3, w.tile, w.kb0);
                 const uint32_t d_tmem = tmem_base + acc * C::BN;
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!wait_bounded<false>(full_bar(stage), phase, abort_flag, p.status, ST_TIMEOUT_MMA)) {
@@ -442,6 +472,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 if (!ok) break;
                 if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(tfull_bar(acc), 0x3);
                 else ptx::mma_commit(tfull_bar(acc));
+                trace_event(p.trace, warp, 4, w.tile, w.kb1);
                 if (++acc == 2u) { acc = 0; acc_phase ^= 1u; }
             }
             // every MMA issued by this thread has completed once done_bar flips
@@ -457,7 +488,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const uint32_t stg = sStg + ew * C::STG_BYTES;
         float *bsm = bias_smem + ew * C::BIAS_FLOATS;
         float alpha = 1.0f;
-        if constexpr (C::DT == DT_E4M3) alpha = __ldg(p.scale_a) * __ldg(p.scale_b);
+        if (p.scale_a != nullptr) alpha = __ldg(p.scale_a) * __ldg(p.scale_b);
+        const bool has_bias = p.bias != nullptr;
         uint32_t acc = 0, acc_phase = 0;
         bool ok = true;
         WorkIter it(p, unit, units);
@@ -466,7 +498,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             // partial_out: this unit holds a non-final slice of the tile -> publish a partial.
             // Otherwise units [c_first, unit) published the slices before ours.
             const bool partial_out = w.kb1 < p.num_kb;
-            const int c_first = w.kb0 > 0 ? (w.tile * p.num_kb) / p.sk_q : unit;
+            const int c_first = w.kb0 > 0 ? w.tile * p.sk_split : unit;
             int tm, tn;
             tile_coords(p, w.tile, tm, tn);
             const int m0 = tm * (C::BM * C::CG) + (int)rank * C::BM;
@@ -475,12 +507,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const bool row_ok = row < p.m;
             float rbias = 0.0f;
             if constexpr (C::EPI != EPI_NONE && C::AXIS == AXIS_ROW) {
-                if (row_ok) rbias = O::load(p.bias, row);
+                if (row_ok && has_bias) rbias = O::load(p.bias, row);
             }
             if constexpr (C::BIAS_FLOATS > 0) if (!partial_out) {
                 // this warp's copy of bias[n0 .. n0+BN) as fp32 (read once per tile)
                 __syncwarp();
-                if (n0 + C::BN <= p.n) {
+                if (!has_bias) {
+                    for (int j = lane; j < C::BN; j += 32) bsm[j] = 0.0f;
+                } else if (n0 + C::BN <= p.n) {
 #pragma unroll
                     for (int j = lane * 8; j < C::BN; j += 256) {
                         const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
@@ -495,17 +529,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
                 __syncwarp();
             }
+            if (lane == 0) trace_event(p.trace, warp, 5, w.tile, w.kb0);
             if (!wait_bounded<false>(tfull_bar(acc), acc_phase, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
+            if (lane == 0) trace_event(p.trace, warp, 6, w.tile, w.kb0);
             // this warp's rows of each earlier slice are published by the same warp quadrant
             for (int v = c_first; ok && v < unit && !partial_out; ++v)
                 ok = wait_flag(p.flags + ((size_t)v * C::CG + rank) * 4 + q, abort_flag, p.status);
             if (!ok) break;
+            if (lane == 0) trace_event(p.trace, warp, 7, w.tile, c_first);
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + acc * C::BN;
-            float *ws_own = p.workspace + (((size_t)unit * C::CG + rank) * 128 + 32 * q + lane) * C::BN;
 #pragma unroll 1
             for (int g = 0; g < C::BN / 128; ++g) {       // 128 output columns per group
                 uint32_t words[4];
@@ -526,19 +562,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                     if (partial_out) {
                         // non-final slice: hand the fp32 partial to the tile's finishing unit
-                        float4 *dst = reinterpret_cast<float4 *>(ws_own + 32 * c);
+                        float4 *dst = ws_chunk<C::BN>(p.workspace, unit, C::CG, rank, q, c, lane);
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
-                            dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                            dst[32 * j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                      __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
                         continue;
                     }
                     for (int u = c_first; u < unit; ++u) {       // earlier slices, in unit order
-                        const float4 *src = reinterpret_cast<const float4 *>(
-                            p.workspace + (((size_t)u * C::CG + rank) * 128 + 32 * q + lane) * C::BN + 32 * c);
+                        const float4 *src = ws_chunk<C::BN>(p.workspace, u, C::CG, rank, q, c, lane);
+                        float4 f8[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) f8[j] = __ldcg(src + 32 * j);
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
-                            const float4 f = __ldcg(src + j);
+                            const float4 f = f8[j];
                             v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + f.x);
                             v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + f.y);
                             v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + f.z);
@@ -551,7 +589,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
                         float x0 = __uint_as_float(v[j]), x1 = __uint_as_float(v[j + 1]);
-                        if constexpr (C::DT == DT_E4M3) { x0 *= alpha; x1 *= alpha; }
+                        x0 *= alpha;
+                        x1 *= alpha;
                         if constexpr (C::EPI != EPI_NONE) {
                             if constexpr (C::AXIS == AXIS_ROW) { x0 += rbias; x1 += rbias; }
                             else { x0 += bsm[32 * c + j]; x1 += bsm[32 * c + j + 1]; }
@@ -598,6 +637,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                 }
             }
+            if (lane == 0) trace_event(p.trace, warp, 8, w.tile, partial_out ? 1 : 0);
             if (partial_out) {
                 // publish: every lane's stores are ordered before the warp's flag
                 __threadfence();
@@ -607,6 +647,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 // the earlier slices have been read: clear their flags for the next launch
                 for (int v = c_first; v < unit; ++v) p.flags[((size_t)v * C::CG + rank) * 4 + q] = 0u;
             }
+            if (lane == 0) trace_event(p.trace, warp, 9, w.tile, 0);
             if (++acc == 2u) { acc = 0; acc_phase ^= 1u; }
         }
         if (lane == 0) ptx::bulk_wait<0>();

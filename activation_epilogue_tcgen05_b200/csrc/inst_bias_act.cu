@@ -25,6 +25,7 @@ static BiasActLauncher pick_epi(int epi, int axis) {
     case EPI_RELU: return pick_axis<DT, EPI_RELU>(axis);
     case EPI_RELU_AUX: return pick_axis<DT, EPI_RELU_AUX>(axis);
     case EPI_GELU: return pick_axis<DT, EPI_GELU>(axis);
+    case EPI_TANH: return pick_axis<DT, EPI_TANH>(axis);
     }
     return nullptr;
 }

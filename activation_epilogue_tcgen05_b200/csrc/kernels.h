@@ -175,6 +175,8 @@ KernelInfo sk_info() {
                                        : NAME##_mn<CG, EPI_RELU_AUX, AXIS_ROW>(bmn, bn, l, i);          \
         case EPI_GELU: return axis ? NAME##_mn<CG, EPI_GELU, AXIS_COL>(bmn, bn, l, i)                   \
                                    : NAME##_mn<CG, EPI_GELU, AXIS_ROW>(bmn, bn, l, i);                  \
+        case EPI_TANH: return axis ? NAME##_mn<CG, EPI_TANH, AXIS_COL>(bmn, bn, l, i)                   \
+                                   : NAME##_mn<CG, EPI_TANH, AXIS_ROW>(bmn, bn, l, i);                  \
         }                                                                                               \
         return false;                                                                                   \
     }                                                                                                   \
@@ -217,6 +219,8 @@ KernelInfo sk_info() {
                                        : NAME##_mn<EPI_RELU_AUX, AXIS_ROW>(wmn, nm, l, i);              \
         case EPI_GELU: return axis ? NAME##_mn<EPI_GELU, AXIS_COL>(wmn, nm, l, i)                       \
                                    : NAME##_mn<EPI_GELU, AXIS_ROW>(wmn, nm, l, i);                      \
+        case EPI_TANH: return axis ? NAME##_mn<EPI_TANH, AXIS_COL>(wmn, nm, l, i)                       \
+                                   : NAME##_mn<EPI_TANH, AXIS_ROW>(wmn, nm, l, i);                      \
         }                                                                                               \
         return false;                                                                                   \
     }

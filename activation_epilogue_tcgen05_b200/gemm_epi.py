@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(PKG, "libgemm_epi.so")
 # enums (include/gemm_epi.h)
 F16, BF16, E4M3 = 0, 1, 2
 NONE, BIAS, RELU_BIAS, RELU_AUX_BIAS, GELU_BIAS = 0, 1, 2, 3, 4
+TANH_BIAS, RELU, RELU_AUX, GELU, TANH = 5, 6, 7, 8, 9
 BIAS_ROW, BIAS_COL = 0, 1
 B_KN, B_NK = 0, 1
 KERNEL_AUTO, KERNEL_TC1, KERNEL_TC2, KERNEL_SPLITK = 0, 1, 2, 3
@@ -28,7 +29,10 @@ OK, ERR_ARG, ERR_ALIGN, ERR_NULL, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NO
 
 DTYPE = {"f16": F16, "bf16": BF16, "e4m3": E4M3}
 EPILOGUE = {"none": NONE, "bias": BIAS, "relu_bias": RELU_BIAS, "relu_aux_bias": RELU_AUX_BIAS,
-            "gelu_bias": GELU_BIAS}
+            "gelu_bias": GELU_BIAS, "tanh_bias": TANH_BIAS, "relu": RELU, "relu_aux": RELU_AUX,
+            "gelu": GELU, "tanh": TANH}
+HAS_BIAS = {"bias", "relu_bias", "relu_aux_bias", "gelu_bias", "tanh_bias"}
+HAS_AUX = {"relu_aux_bias", "relu_aux"}
 AXIS = {"row": BIAS_ROW, "col": BIAS_COL}
 LAYOUT = {"kn": B_KN, "nk": B_NK}
 KERNEL = {"auto": KERNEL_AUTO, "tc1": KERNEL_TC1, "tc2": KERNEL_TC2, "splitk": KERNEL_SPLITK}
@@ -50,7 +54,7 @@ class Options(ctypes.Structure):
 class PlanInfo(ctypes.Structure):
     _fields_ = [(f, ctypes.c_int32) for f in
                 ("kernel", "block_m", "block_n", "block_k", "stages", "split_k", "grid", "cluster",
-                 "threads", "smem_bytes", "tiles", "sk_tiles", "sk_q")]
+                 "threads", "smem_bytes", "tiles", "sk_tiles", "sk_split")]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

@@ -56,6 +56,9 @@ def parse(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--shape", default=None,
+                    help="custom problem m,n,k,dtype,epilogue,bias_axis,b_layout (overrides --workload; "
+                         "operands N(0,1)/64, bias N(0,1), seed 0)")
     ap.add_argument("--kernel", default="auto", choices=["auto", "tc1", "tc2", "splitk"])
     ap.add_argument("--block-n", type=int, default=0)
     ap.add_argument("--stream-k", default="auto", choices=["auto", "off", "on"])
@@ -66,6 +69,9 @@ def parse(argv=None):
     ap.add_argument("--no-unfused", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps directly instead of replaying them from a CUDA graph")
+    ap.add_argument("--cublas", action="store_true",
+                    help="also time cuBLAS's bare GEMM (torch.matmul, no epilogue) at this shape, "
+                         "as context only (16-bit workloads)")
     return ap.parse_args(argv)
 
 
@@ -166,6 +172,16 @@ class ClockSampler:
                 "reasons": reasons, "power_w_max": max(power) if power else None, "samples": len(win)}
 
 
+def workload_from_args(args):
+    from activation_epilogue_tcgen05_b200.workloads import WORKLOADS, Workload
+    if not args.shape:
+        return WORKLOADS[args.workload]
+    m, n, k, dt, epi, axis, lay = args.shape.split(",")
+    std = 1.0 if dt == "e4m3" else 1.0 / 64
+    return Workload(f"custom_{dt}_{epi}_{m}x{n}x{k}_{lay}", int(m), int(n), int(k), dt, epi, axis, lay,
+                    ("normal", std), ("normal", std), ("normal", 1.0))
+
+
 # ----------------------------------------------------------------------------- CPU oracle legs
 def oracle_rows_rate(wl, prob, target_s: float, max_rows=None):
     """Time the oracle (as it stands) on the first R rows of the workload; R sized to ~target_s.
@@ -205,8 +221,8 @@ def reference_arm(args):
         return 0
     import numpy as np
     import oracle
-    from activation_epilogue_tcgen05_b200.workloads import WORKLOADS, make_problem, storage
-    wl = WORKLOADS[args.workload]
+    from activation_epilogue_tcgen05_b200.workloads import make_problem, storage
+    wl = workload_from_args(args)
     gen_dev = "cpu"
     if wl.m * wl.k > (1 << 28):              # very large operands: draw only what the samples need
         wl_small = wl.with_(m=min(wl.m, 4096))
@@ -275,12 +291,12 @@ def main(argv=None):
     have_pg = replicas.init("nccl", timeout_s=120, device_id=dev)
     sampler = ClockSampler(local_rank) if rank == 0 else None
 
-    wl = WORKLOADS[args.workload]
+    wl = workload_from_args(args)
     out_t = TORCH_DTYPE[wl.out_dtype]
     big = wl.m * wl.k > (1 << 28)
     prob = make_problem(wl, device="cuda" if big else "cpu")
     A0, B0, bias0 = prob.A.to(dev), prob.B.to(dev), prob.bias.to(dev)
-    aux_words = wl.m * g.aux_pitch_words(wl.n) if wl.epilogue == "relu_aux_bias" else 0
+    aux_words = wl.m * g.aux_pitch_words(wl.n) if wl.epilogue in g.HAS_AUX else 0
     esz = 1 if wl.dtype == "e4m3" else 2
     in_bytes = (wl.m * wl.k + wl.k * wl.n) * esz + bias0.numel() * 2
     out_bytes = wl.m * wl.n * 2 + aux_words * 4
@@ -485,6 +501,25 @@ def main(argv=None):
                "api": "gemm_epi_run (C ABI) with pinned host buffers; H2D, compute and D2H of "
                       "neighbouring steps overlap on three streams"}
 
+    # ---- context only: the vendor library's bare GEMM (no bias, no activation) at this shape
+    cublas = None
+    if args.cublas and wl.dtype in ("f16", "bf16"):
+        Bt = B0 if wl.b_layout == "kn" else B0.t()
+        outc = torch.empty((wl.m, wl.n), dtype=out_t, device=dev)
+        for _ in range(5):
+            torch.matmul(A0, Bt, out=outc)
+        Kc = min(K, 500)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        c0.record(stream)
+        for _ in range(Kc):
+            torch.matmul(A0, Bt, out=outc)
+        c1.record(stream)
+        torch.cuda.synchronize(dev)
+        cms = c0.elapsed_time(c1) / Kc
+        cublas = {"value": flops / (cms / 1000) / 1e12, "unit": "TFLOP/s", "ms_per_step": cms,
+                  "steps": Kc, "what": "torch.matmul (cuBLAS) bare GEMM, same operands, L2-warm"}
+
     if sampler:
         sampler.stop()
 
@@ -520,6 +555,8 @@ def main(argv=None):
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "unfused": unfused,
             "gpu_launches": K, "clocks": clocks,
         }
+        if cublas is not None:
+            line["cublas_bare_gemm"] = cublas
         print(json.dumps(line), flush=True)
     plan.close()
     if have_pg:

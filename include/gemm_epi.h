@@ -47,18 +47,28 @@ extern "C" {
 /* Operand types ([nvmath-fusion] paragraph 5: FP16, BF16, FP8). */
 enum gemm_epi_dtype { GEMM_EPI_F16 = 0, GEMM_EPI_BF16 = 1, GEMM_EPI_E4M3 = 2 };
 
-/* Epilogues ([epilog-params] body paragraph 2; [bias-fusion] paragraph 2 for GELU).
- *   NONE           D = alpha*A.B                   (the bare GEMM; bias ignored)
- *   BIAS           D = alpha*A.B + bias
- *   RELU_BIAS      D = max(alpha*A.B + bias, 0)
- *   RELU_AUX_BIAS  as RELU_BIAS, plus aux = sign mask of the ReLU input
- *   GELU_BIAS      D = GELU(x) = 0.5 x (1 + erf(x / sqrt 2)), x = alpha*A.B + bias */
+/* Epilogues ([epilog-params] body paragraph 2; [bias-fusion] paragraph 2 for GELU;
+ * [nvmath-fusion] paragraph 6 lists Tanh among the predefined ones).  x = alpha*A.B + bias
+ * for the *_BIAS epilogues and x = alpha*A.B for the others, which ignore the bias
+ * argument (it may be NULL).
+ *   NONE           D = alpha*A.B                   (the bare GEMM)
+ *   BIAS           D = x
+ *   RELU_BIAS      D = max(x, 0)
+ *   RELU_AUX_BIAS  as RELU_BIAS, plus aux = sign mask of the ReLU input x
+ *   GELU_BIAS      D = GELU(x) = 0.5 x (1 + erf(x / sqrt 2))
+ *   TANH_BIAS      D = tanh(x)
+ *   RELU, RELU_AUX, GELU, TANH: the same without a bias */
 enum gemm_epi_epilogue {
     GEMM_EPI_NONE = 0,
     GEMM_EPI_BIAS = 1,
     GEMM_EPI_RELU_BIAS = 2,
     GEMM_EPI_RELU_AUX_BIAS = 3,
-    GEMM_EPI_GELU_BIAS = 4
+    GEMM_EPI_GELU_BIAS = 4,
+    GEMM_EPI_TANH_BIAS = 5,
+    GEMM_EPI_RELU = 6,
+    GEMM_EPI_RELU_AUX = 7,
+    GEMM_EPI_GELU = 8,
+    GEMM_EPI_TANH = 9
 };
 
 /* Bias broadcast ([epilog-params] body paragraph 3; [nvmath-fusion] paragraph 5):
@@ -103,23 +113,24 @@ typedef struct gemm_epi_plan_s *gemm_epi_plan_t;
 typedef struct gemm_epi_options {
     int32_t kernel;    /* enum gemm_epi_kernel                                        */
     int32_t block_n;   /* output tile width (128 or 256; 0 = auto)                    */
-    int32_t split_k;   /* SPLITK only: CTAs per cluster along k (1..8; 0 = auto)       */
+    int32_t split_k;   /* SPLITK: CTAs per cluster along k (1..8; 0 = auto).  TC1/TC2:
+                          cap on the parts a tail tile is split into (0 = 2)          */
     int32_t max_ctas;  /* persistent kernels: cap on resident CTAs (0 = one per SM)    */
     int32_t inject_stall; /* testing only (TC1/TC2): 1 = the MMA issuer never publishes an
                              accumulator, so the epilogue's bounded wait runs out after about
                              one second and gemm_epi_check() reports GEMM_EPI_ERR_TIMEOUT;
                              D is left unwritten.  0 for real work.                        */
-    int32_t stream_k;  /* TC1/TC2: 0 = auto, 1 = off, 2 = on.  Stream-K splits the tiles of an
+    int32_t stream_k;  /* TC1/TC2: 0 = auto, 1 = off, 2 = on.  Splits the tiles of an
                           incomplete last wave (or all tiles, when there are fewer tiles than
-                          SMs) by k-blocks over every SM; partial tiles pass through a
-                          workspace the plan allocates (SMs x 128 x block_n fp32).            */
+                          SMs) along k over several SMs (stream-K style); partial tiles pass
+                          through a workspace the plan allocates (SMs x 128 x block_n fp32). */
 } gemm_epi_options;
 
 /* What a plan decided (for logging and tests). */
 typedef struct gemm_epi_plan_info {
     int32_t kernel, block_m, block_n, block_k, stages, split_k;
     int32_t grid, cluster, threads, smem_bytes, tiles;
-    int32_t sk_tiles, sk_q;   /* stream-K: tiles split by k-blocks, k-blocks per SM (unit) */
+    int32_t sk_tiles, sk_split;   /* split tail: tiles split along k, parts per split tile */
 } gemm_epi_plan_info;
 
 /* ---- entry points -------------------------------------------------------- */
@@ -143,18 +154,20 @@ int gemm_epi_plan_ex(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, i
 int gemm_epi_plan_opts(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis,
                        int b_layout, const gemm_epi_options *opts, gemm_epi_plan_t *out);
 
-/* E4M3 plans only: per-tensor fp32 scales s_A, s_B as DEVICE pointers to one
- * float each, read by every run; alpha = s_A * s_B multiplies the product
- * before the bias (the epilogue scaling factor of [nvgemm], section "why
- * epilogue fusion matters").  16-bit plans have alpha = 1 and reject this
- * call with ERR_ARG.  The pointers are borrowed, not owned. */
+/* Per-tensor fp32 scales s_A, s_B as DEVICE pointers to one float each, read
+ * by every run; alpha = s_A * s_B multiplies the product before the bias (the
+ * epilogue scaling factor of [nvgemm], section "why epilogue fusion matters").
+ * Required for E4M3 plans (the dequantisation scales); optional for 16-bit
+ * plans, whose alpha is 1 until set (both NULL resets it).  The pointers are
+ * borrowed, not owned.  ERR_NULL if only one is given. */
 int gemm_epi_set_scales(gemm_epi_plan_t plan, const float *d_scale_a, const float *d_scale_b);
 
 /* Enqueue the fused kernel: one launch, D (and aux) written once.
  *   A     (m, k) operand, B (k, n) or (n, k) operand, device pointers.
- *   bias  length m (ROW) or n (COL), output type; ignored (may be NULL) for NONE.
+ *   bias  length m (ROW) or n (COL), output type; ignored (may be NULL) for the
+ *         epilogues without a bias.
  *   D     (m, n) output.
- *   aux   RELU_AUX_BIAS only (else ignored, may be NULL): packed sign mask,
+ *   aux   RELU_AUX_BIAS and RELU_AUX only (else ignored, may be NULL): packed sign mask,
  *         row-major uint32 words, row pitch gemm_epi_aux_pitch_bytes(n);
  *         bit b of word w in row i is 1 iff the fp32 pre-activation of
  *         element (i, 32w + b) is > 0 (taken before rounding to the output

@@ -26,7 +26,7 @@ def device_inputs(prob: Problem, device="cuda"):
 def alloc_outputs(wl: Workload, device="cuda"):
     D = torch.full((wl.m, wl.n), float("nan"), dtype=TORCH_DTYPE[wl.out_dtype], device=device)
     aux = None
-    if wl.epilogue == "relu_aux_bias":
+    if wl.epilogue in g.HAS_AUX:
         words = wl.m * g.aux_pitch_words(wl.n)
         aux = torch.full((words,), int(SENTINEL_WORD), dtype=torch.int32, device=device)
     return D, aux
@@ -34,7 +34,7 @@ def alloc_outputs(wl: Workload, device="cuda"):
 
 def make_plan(wl: Workload, prob: Problem, device="cuda", **opts):
     plan = g.Plan(wl.m, wl.n, wl.k, wl.dtype, wl.epilogue, wl.bias_axis, wl.b_layout, **opts)
-    if wl.dtype == "e4m3":
+    if wl.dtype == "e4m3" or prob.scale_a != 1.0 or prob.scale_b != 1.0:
         sa = torch.tensor([prob.scale_a], dtype=torch.float32, device=device)
         sb = torch.tensor([prob.scale_b], dtype=torch.float32, device=device)
         plan.set_scales(sa, sb)
@@ -44,6 +44,8 @@ def make_plan(wl: Workload, prob: Problem, device="cuda", **opts):
 def gpu_run(wl: Workload, prob: Problem, fused=True, inputs=None, **opts):
     """One run through gemm_epi_run (or the unfused path); returns host D, aux words, plan info."""
     A, B, bias = inputs if inputs is not None else device_inputs(prob)
+    if wl.epilogue not in g.HAS_BIAS:
+        bias = None                      # bias-free epilogues take a NULL bias
     D, aux = alloc_outputs(wl)
     plan = make_plan(wl, prob, **opts)
     try:
@@ -68,7 +70,7 @@ def _pop_std(t: torch.Tensor, limit: int = 1 << 24) -> float:
 
 def sigmas(prob: Problem):
     """Population std (fp64) of the operand values the product uses (dequantised)."""
-    return _pop_std(prob.A) * prob.scale_a, _pop_std(prob.B) * prob.scale_b
+    return _pop_std(prob.A) * abs(prob.scale_a), _pop_std(prob.B) * abs(prob.scale_b)
 
 
 def oracle_full(wl: Workload, prob: Problem):
@@ -96,7 +98,7 @@ def compare(wl, D_gpu, words, ref, pre, mask, sa, sb, rows=None, cols=None, extr
                    float(tol[tuple(i)])) for i in idx]
         raise AssertionError(f"{int((~ok).sum())} of {ok.size} outputs outside tolerance; first "
                              f"(index, gpu, ref, tol): {detail}")
-    if wl.epilogue == "relu_aux_bias":
+    if wl.epilogue in g.HAS_AUX:
         bits = unpack_aux(words, wl.m, wl.n)
         if rows is not None:
             bits = bits[rows, cols]
@@ -138,6 +140,8 @@ OUT_ULP = {"f16": 2.0 ** -10, "bf16": 2.0 ** -7, "e4m3": 2.0 ** -7}
 def unfused_extra(wl: Workload, prob: Problem, pre):
     """|alpha*A.B| * ulp(out): the unfused path's additional rounding of the product."""
     from oracle import decode
+    if wl.epilogue not in g.HAS_BIAS:
+        return OUT_ULP[wl.out_dtype] * np.abs(pre)
     b = decode(storage(prob.bias), wl.out_dtype)
     b = b[:, None] if wl.bias_axis == "row" else b[None, :]
     return OUT_ULP[wl.out_dtype] * np.abs(pre - b)

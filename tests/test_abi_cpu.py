@@ -75,7 +75,7 @@ def test_plan_rejects_bad_sizes(g, args):
     assert _plan_rc(g, *args) == g.ERR_ARG
 
 
-@pytest.mark.parametrize("kw", [dict(dt=3), dict(dt=-1), dict(epi=5), dict(epi=-1), dict(axis=2),
+@pytest.mark.parametrize("kw", [dict(dt=3), dict(dt=-1), dict(epi=10), dict(epi=-1), dict(axis=2),
                                 dict(layout=2)])
 def test_plan_rejects_bad_enums(g, kw):
     assert _plan_rc(g, 64, 64, 64, **kw) == g.ERR_ARG

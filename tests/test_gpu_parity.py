@@ -22,7 +22,8 @@ from activation_epilogue_tcgen05_b200.workloads import (TORCH_DTYPE, WORKLOADS, 
 pytestmark = pytest.mark.gpu
 
 DTYPES = ["f16", "bf16", "e4m3"]
-EPILOGUES = ["none", "bias", "relu_bias", "relu_aux_bias", "gelu_bias"]
+EPILOGUES = ["none", "bias", "relu_bias", "relu_aux_bias", "gelu_bias", "tanh_bias", "relu",
+             "relu_aux", "gelu", "tanh"]
 
 
 def small(dtype, epilogue, axis, layout, m=200, n=272, seed=1):
@@ -99,26 +100,49 @@ def test_integer_inputs_bit_exact(kernel, dtype, epilogue):
         np.testing.assert_array_equal(unpack_aux(words, wl.m, wl.n), mask)
 
 
+# ------------------------------------------------------------------ epilogue scaling factor
+@pytest.mark.parametrize("kernel", ["tc1", "tc2", "splitk"])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_alpha_scaling_16bit(kernel, dtype):
+    """alpha = s_A*s_B multiplies the product of 16-bit operands when scales are set."""
+    from dataclasses import replace as dc_replace
+    m = 32 if kernel == "splitk" else 264
+    wl = Workload("alpha", m, 272, 328, dtype, "gelu_bias", "col", "kn", seed=17)
+    prob = dc_replace(make_problem(wl), scale_a=0.75, scale_b=-2.5)
+    worst, _ = check_against_oracle(wl, prob, kernel=kernel)
+    assert worst <= 1.0
+    # both scale pointers NULL again: alpha back to 1
+    A, B, bias = device_inputs(prob)
+    D, _ = alloc_outputs(wl)
+    plan = make_plan(wl, prob, kernel=kernel)
+    g.gemm_epi_set_scales(plan.handle, None, None)
+    plan.run(A, B, bias, D, None)
+    plan.check()
+    plan.close()
+    ref, pre, mask = oracle_full(wl, dc_replace(prob, scale_a=1.0, scale_b=1.0))
+    compare(wl, D.cpu(), None, ref, pre, mask, *sigmas(dc_replace(prob, scale_a=1.0, scale_b=1.0)))
+
+
 # ------------------------------------------------------------------ stream-K tail
-@pytest.mark.parametrize("kernel,max_ctas,m,n", [
-    ("tc1", 4, 600, 528),     # 25 tiles on 4 CTAs: one tile split four ways
-    ("tc1", 7, 600, 528),     # 25 tiles on 7 CTAs: runs span two tiles
-    ("tc1", 16, 256, 256),    # fewer tiles than CTAs: every tile split
-    ("tc2", 8, 600, 528),     # pairs: 3 x 5 tiles on 4 pairs
-    ("tc2", 8, 256, 256),     # pairs, fewer tiles than pairs (2 tiles on 4 pairs)
+@pytest.mark.parametrize("kernel,max_ctas,m,n,parts", [
+    ("tc1", 4, 600, 528, 2),    # 25 tiles on 4 CTAs: the last tile in two parts
+    ("tc1", 8, 600, 528, 3),    # 25 tiles on 8 CTAs: the last tile in three parts
+    ("tc1", 16, 256, 256, 4),   # fewer tiles than CTAs: every tile in four parts
+    ("tc2", 12, 600, 528, 2),   # pairs: 3 x 5 tiles on 6 pairs
+    ("tc2", 8, 256, 256, 2),    # pairs, fewer tiles than pairs (2 tiles on 4 pairs)
 ])
 @pytest.mark.parametrize("dtype,epilogue,axis,layout", [
     ("bf16", "relu_aux_bias", "row", "kn"), ("f16", "gelu_bias", "col", "nk"),
     ("e4m3", "bias", "col", "kn"), ("bf16", "none", "row", "nk"),
 ])
-def test_stream_k(kernel, max_ctas, m, n, dtype, epilogue, axis, layout):
+def test_stream_k(kernel, max_ctas, m, n, parts, dtype, epilogue, axis, layout):
     k = 1024 if dtype == "e4m3" else 1000
     wl = Workload("sk_tail", m, n, k, dtype, epilogue, axis, layout, seed=12)
     prob = make_problem(wl)
     bn = 256 if (kernel == "tc2" and dtype == "e4m3") else 128
     worst, info = check_against_oracle(wl, prob, kernel=kernel, block_n=bn, max_ctas=max_ctas,
-                                       stream_k="on")
-    assert info["sk_tiles"] > 0
+                                       stream_k="on", split_k=parts)
+    assert info["sk_tiles"] > 0 and info["sk_split"] == parts
     assert worst <= 1.0
 
 
@@ -127,7 +151,7 @@ def test_stream_k_deterministic_and_unfused(kernel):
     wl = Workload("sk_det", 600, 528, 1000, "bf16", "relu_aux_bias", "row", "kn", seed=13)
     prob = make_problem(wl)
     inputs = device_inputs(prob)
-    opts = dict(kernel=kernel, block_n=128, max_ctas=6 if kernel == "tc1" else 8, stream_k="on")
+    opts = dict(kernel=kernel, block_n=128, max_ctas=6 if kernel == "tc1" else 12, stream_k="on")
     D1, w1, info = gpu_run(wl, prob, inputs=inputs, **opts)
     D2, w2, _ = gpu_run(wl, prob, inputs=inputs, **opts)
     assert info["sk_tiles"] > 0
@@ -183,7 +207,8 @@ def test_splitk_cluster_sizes(split):
 
 # ------------------------------------------------------------------ fused vs unfused, determinism
 @pytest.mark.parametrize("kernel", ["tc1", "tc2", "splitk"])
-@pytest.mark.parametrize("epilogue", ["bias", "relu_bias", "relu_aux_bias", "gelu_bias"])
+@pytest.mark.parametrize("epilogue", ["bias", "relu_bias", "relu_aux_bias", "gelu_bias", "tanh_bias",
+                                      "relu", "relu_aux", "gelu", "tanh"])
 def test_unfused_path_matches_oracle_and_fused(kernel, epilogue):
     m = 64 if kernel == "splitk" else 384
     wl = Workload("unf", m, 384, 512, "bf16", epilogue, "row", "kn", seed=7)
@@ -267,7 +292,7 @@ def test_run_argument_errors():
     assert L.gemm_epi_run(h, p(A) + 2, p(B), p(bias), p(D), p(aux), s) == g.ERR_ALIGN
     assert L.gemm_epi_run(h, p(A), p(B), p(bias) + 2, p(D), p(aux), s) == g.ERR_ALIGN
     assert L.gemm_epi_run(h, p(A), p(B), p(bias), p(D), p(aux) + 4, s) == g.ERR_ALIGN
-    assert L.gemm_epi_set_scales(h, p(A), p(A)) == g.ERR_ARG           # not an e4m3 plan
+    assert L.gemm_epi_set_scales(h, p(A), None) == g.ERR_NULL          # one scale only
     plan.close()
     assert L.gemm_epi_run(h, p(A), p(B), p(bias), p(D), p(aux), s) == g.ERR_ARG  # freed
     # e4m3 without scales
