@@ -71,6 +71,9 @@ def _load():
             lib.oracle_gemm_epi_sampled.argtypes = [i64, i64, i64, cp, cp, cp, cp, vp, vp, vp,
                                                     dp, dp, i64, vp, vp, vp, vp, vp]
             lib.oracle_gemm_epi_sampled.restype = ctypes.c_int
+            lib.oracle_gemm_epi_bwd.argtypes = [i64, i64, i64, cp, cp, cp, cp, vp, vp, vp, dp, dp,
+                                                vp, vp]
+            lib.oracle_gemm_epi_bwd.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -170,6 +173,33 @@ def gemm_epi_sampled(A, B, bias, rows, cols, *, dtype: str, epilogue: str,
     if rc != 0:
         raise RuntimeError(f"oracle_gemm_epi_sampled failed with status {rc}")
     return D, pre, mask
+
+
+def gemm_epi_bwd(A, B, mask, *, dtype: str, epilogue: str, bias_axis: str = "row",
+                 b_layout: str = "kn", scale_a: float = 1.0, scale_b: float = 1.0):
+    """ReLU backward epilogues: D = mask * (alpha*A.B) and, for "drelu_bgrad", the bias
+    gradient (sums of D along the bias axis).  mask is an (m, n) 0/1 array.
+
+    Returns float64 D (m, n) and dbias (length m for "row", n for "col"; None for "drelu").
+    """
+    if epilogue not in ("drelu", "drelu_bgrad") or dtype not in DTYPES or bias_axis not in AXES \
+            or b_layout not in LAYOUTS:
+        raise ValueError(f"unknown oracle option {(dtype, epilogue, bias_axis, b_layout)}")
+    A = _storage(A, dtype)
+    B = _storage(B, dtype)
+    m, k = A.shape
+    n = B.shape[1] if b_layout == "kn" else B.shape[0]
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    if mask.shape != (m, n):
+        raise ValueError("mask must be (m, n)")
+    D = np.empty((m, n), np.float64)
+    dbias = np.empty(m if bias_axis == "row" else n, np.float64) if epilogue == "drelu_bgrad" else None
+    rc = _load().oracle_gemm_epi_bwd(m, n, k, dtype.encode(), epilogue.encode(), bias_axis.encode(),
+                                     b_layout.encode(), _ptr(A), _ptr(B), _ptr(mask),
+                                     float(scale_a), float(scale_b), _ptr(D), _ptr(dbias))
+    if rc != 0:
+        raise RuntimeError(f"oracle_gemm_epi_bwd failed with status {rc}")
+    return D, dbias
 
 
 def threads() -> int:

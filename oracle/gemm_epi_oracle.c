@@ -280,3 +280,78 @@ int oracle_gemm_epi_sampled(int64_t m, int64_t n, int64_t k, const char *dtype,
     }
     return 0;
 }
+
+/*
+ * Backward epilogues (the mask of a forward RELU_AUX(_BIAS) fed back in).
+ * "nvmath-python cuBLASLt bias fusion for PyTorch inference" (blog.hotdry.top),
+ * paragraph 6: the auxiliary output of RELU_AUX_BIAS is the mask the backward
+ * pass needs; paragraph 7: fusing dBias is the next step.  Read as the usual
+ * ReLU backward of a layer z = alpha*A.B + bias, y = relu(z):
+ *
+ *   "drelu":        D(i,j) = mask(i,j) ? alpha * sum_t a(i,t) b(t,j) : 0
+ *   "drelu_bgrad":  the same D, plus the bias gradient, the sum of D over the
+ *                   axis the bias was broadcast along:
+ *                     ROW bias (length m): dbias(i) = sum_j D(i,j)
+ *                     COL bias (length n): dbias(j) = sum_i D(i,j)
+ *
+ * mask is m x n bytes (0/1, row-major); dbias may be NULL for "drelu".
+ * Everything is accumulated in double; D_ref is not rounded.
+ */
+int oracle_gemm_epi_bwd(int64_t m, int64_t n, int64_t k, const char *dtype, const char *epilogue,
+                        const char *bias_axis, const char *b_layout, const void *A, const void *B,
+                        const uint8_t *mask, double scale_a, double scale_b, double *D_ref,
+                        double *dbias_ref) {
+    int dt = dtype_code(dtype), axis = axis_code(bias_axis), lay = layout_code(b_layout);
+    int bgrad;
+    if (!epilogue) return -1;
+    if (!strcmp(epilogue, "drelu")) bgrad = 0;
+    else if (!strcmp(epilogue, "drelu_bgrad")) bgrad = 1;
+    else return -1;
+    if (m <= 0 || n <= 0 || k <= 0 || !dt || !axis || !lay || !A || !B || !mask || !D_ref) return -1;
+    if (bgrad && !dbias_ref) return -1;
+    const double alpha = scale_a * scale_b;
+
+    double *Bd = (double *)malloc((size_t)k * (size_t)n * sizeof(double));
+    if (!Bd) return -2;
+    for (int64_t t = 0; t < k; ++t)
+        for (int64_t j = 0; j < n; ++j)
+            Bd[t * n + j] = load(B, dt, lay == OR_KN ? t * n + j : j * k + t);
+    int err = 0;
+#pragma omp parallel
+    {
+        double *row = (double *)malloc((size_t)n * sizeof(double));
+        if (!row) {
+#pragma omp atomic write
+            err = -2;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < m; ++i) {
+            if (!row) continue;
+            for (int64_t j = 0; j < n; ++j) row[j] = 0.0;
+            for (int64_t t = 0; t < k; ++t) {
+                double a = load(A, dt, i * k + t);
+                const double *brow = Bd + t * n;
+                for (int64_t j = 0; j < n; ++j) row[j] += a * brow[j];
+            }
+            for (int64_t j = 0; j < n; ++j)
+                D_ref[i * n + j] = mask[i * n + j] ? alpha * row[j] : 0.0;
+        }
+        free(row);
+    }
+    free(Bd);
+    if (err) return err;
+    if (bgrad) {
+        if (axis == OR_ROW) {
+            for (int64_t i = 0; i < m; ++i) {
+                double s = 0.0;
+                for (int64_t j = 0; j < n; ++j) s += D_ref[i * n + j];
+                dbias_ref[i] = s;
+            }
+        } else {
+            for (int64_t j = 0; j < n; ++j) dbias_ref[j] = 0.0;
+            for (int64_t i = 0; i < m; ++i)
+                for (int64_t j = 0; j < n; ++j) dbias_ref[j] += D_ref[i * n + j];
+        }
+    }
+    return 0;
+}

@@ -43,6 +43,12 @@ MUTANTS = [
     ("tanh_as_relu", "case OR_TANH: y = tanh(p); break;", "case OR_TANH: y = p > 0.0 ? p : 0.0; break;", None),
     ("bias_free_adds_bias", "return epi == OR_BIAS ||", "return epi == OR_RELU || epi == OR_BIAS ||", None),
     ("alpha_fp8_only", "double alpha = scale_a * scale_b;", "double alpha = dt == OR_E4M3 ? scale_a * scale_b : 1.0;", None),
+    ("bwd_mask_inverted", "D_ref[i * n + j] = mask[i * n + j] ? alpha * row[j] : 0.0;",
+     "D_ref[i * n + j] = mask[i * n + j] ? 0.0 : alpha * row[j];", None),
+    ("bwd_alpha_dropped", "D_ref[i * n + j] = mask[i * n + j] ? alpha * row[j] : 0.0;",
+     "D_ref[i * n + j] = mask[i * n + j] ? row[j] : 0.0;", None),
+    ("bwd_bgrad_wrong_axis", "if (axis == OR_ROW) {\n            for (int64_t i = 0; i < m; ++i) {\n                double s",
+     "if (axis != OR_ROW) {\n            for (int64_t i = 0; i < m; ++i) {\n                double s", None),
 ]
 
 

@@ -341,3 +341,50 @@ def test_scaling_factor_applies_to_16bit_inputs(oracle_lib, dtype):
                                      scale_b=2.0)
     Dn, _, _ = oracle_lib.gemm_epi(A, B, None, dtype=dtype, epilogue="none")
     np.testing.assert_allclose(pre3 - pre1, 2.0 * Dn, rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- backward epilogues
+BWD = load_golden("tiny_cases.json")["cases_bwd"]
+
+
+@pytest.mark.parametrize("c", BWD, ids=[c["id"] for c in BWD])
+def test_golden_backward_case(oracle_lib, c):
+    a = to_storage_values(c["a"], c["dtype"])
+    b = to_storage_values(c["b"], c["dtype"])
+    D, dbias = oracle_lib.gemm_epi_bwd(a, b, np.array(c["mask_in"], np.uint8), dtype=c["dtype"],
+                                       epilogue=c["epilogue"], bias_axis=c["bias_axis"],
+                                       b_layout=c["b_layout"], scale_a=c.get("scale_a", 1.0),
+                                       scale_b=c.get("scale_b", 1.0))
+    np.testing.assert_array_equal(D, np.array(c["d"], dtype=np.float64))
+    if "dbias" in c:
+        np.testing.assert_array_equal(dbias, np.array(c["dbias"], dtype=np.float64))
+
+
+@pytest.mark.parametrize("axis", ["row", "col"])
+@pytest.mark.parametrize("layout", ["kn", "nk"])
+def test_backward_equals_masked_numpy_product(oracle_lib, axis, layout):
+    wl = Workload("t", 23, 31, 40, "bf16", "relu_aux_bias", axis, layout, seed=18)
+    p = make_problem(wl)
+    A, B = storage(p.A), storage(p.B)
+    # the forward pass's own mask
+    _, _, mask = oracle_lib.gemm_epi(A, B, storage(p.bias), dtype="bf16", epilogue="relu_aux_bias",
+                                     bias_axis=axis, b_layout=layout)
+    D, dbias = oracle_lib.gemm_epi_bwd(A, B, mask, dtype="bf16", epilogue="drelu_bgrad",
+                                       bias_axis=axis, b_layout=layout, scale_a=2.0, scale_b=0.75)
+    a, b = _decoded(A, "bf16"), _decoded(B, "bf16")
+    prod = 1.5 * (a @ (b if layout == "kn" else b.T))
+    np.testing.assert_allclose(D, np.where(mask == 1, prod, 0.0), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dbias, D.sum(axis=1 if axis == "row" else 0), rtol=1e-12, atol=1e-12)
+
+
+def test_backward_mask_extremes(oracle_lib):
+    wl = Workload("t", 8, 16, 24, "f16", "none", "row", "kn", seed=19)
+    p = make_problem(wl)
+    A, B = storage(p.A), storage(p.B)
+    Dn, _, _ = oracle_lib.gemm_epi(A, B, None, dtype="f16", epilogue="none")
+    ones = np.ones((8, 16), np.uint8)
+    D1, db1 = oracle_lib.gemm_epi_bwd(A, B, ones, dtype="f16", epilogue="drelu_bgrad")
+    np.testing.assert_array_equal(D1, Dn)
+    D0, db0 = oracle_lib.gemm_epi_bwd(A, B, 0 * ones, dtype="f16", epilogue="drelu_bgrad",
+                                      bias_axis="col")
+    assert (D0 == 0).all() and (db0 == 0).all()
