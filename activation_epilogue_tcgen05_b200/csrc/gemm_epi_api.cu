@@ -120,7 +120,7 @@ CUtensorMapDataType tmap_type(int dt) {
 
 // Row-major 2-D tensor: `inner` contiguous elements per row, `outer` rows.
 bool make_map(CUtensorMap *map, int dt, const void *ptr, int64_t inner, int64_t outer, uint32_t box_inner,
-              uint32_t box_outer) {
+              uint32_t box_outer, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
@@ -128,7 +128,7 @@ bool make_map(CUtensorMap *map, int dt, const void *ptr, int64_t inner, int64_t 
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, tmap_type(dt), 2, const_cast<void *>(ptr), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -285,7 +285,8 @@ int ensure_maps(Plan *P, const void *A, const void *B, void *D) {
         ok = ok && make_map(&P->tmA, dt, A, k, m, bk, 128);
         ok = ok && (b_kn ? make_map(&P->tmB, dt, B, n, k, box_n, bk) : make_map(&P->tmB, dt, B, k, n, bk, bn_local));
         const int out_dt = dt == GEMM_EPI_E4M3 ? GEMM_EPI_BF16 : dt;
-        ok = ok && make_map(&P->tmD, out_dt, D, n, m, 64, 32);
+        // the epilogue stages 32 rows x 32 outputs (64 bytes a row, 64-byte swizzle) per store
+        ok = ok && make_map(&P->tmD, out_dt, D, n, m, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
     }
     if (!ok) {
         P->maps_valid = false;

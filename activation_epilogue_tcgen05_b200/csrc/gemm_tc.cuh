@@ -260,12 +260,30 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
     }
 }
 
+// GELU(x) = x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)), exact (erf) form.
+// erfc(z) for z = |x|/sqrt(2) >= 0 follows Abramowitz & Stegun, Handbook of
+// Mathematical Functions, formula 7.1.26:
+//     erfc(z) ~= t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2),  t = 1 / (1 + p z),
+// with p = 0.3275911, a1..a5 = 0.254829592, -0.284496736, 1.421413741,
+// -1.453152027, 1.061405429 and |error| <= 1.5e-7.  1 + erf(x/sqrt 2) is erfc(z)
+// for x < 0 (no cancellation on the negative tail) and 2 - erfc(z) for x >= 0.
+// Branch-free: one reciprocal, one exponential, five FMAs.
+__device__ __forceinline__ float gelu_erf(float x) {
+    const float z = fabsf(x) * 0.70710678118654752f;
+    const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
+    const float poly =
+        t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f), -0.284496736f),
+                 0.254829592f);
+    const float ec = poly * __expf(-z * z);
+    return 0.5f * x * (x >= 0.0f ? 2.0f - ec : ec);
+}
+
 template <int EPI>
 __device__ __forceinline__ float activate(float x) {
     if constexpr (EPI == EPI_RELU || EPI == EPI_RELU_AUX) {
         return x > 0.0f ? x : 0.0f;
     } else if constexpr (EPI == EPI_GELU) {
-        return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+        return gelu_erf(x);
     } else if constexpr (EPI == EPI_TANH) {
         return tanhf(x);
     } else {
@@ -290,17 +308,25 @@ struct TcCfg {
     static constexpr int B_BOX_N = 128 / ESIZE;     // n per 128-byte MN-major box
     static constexpr int B_BOXES = B_MN ? BN_LOCAL / B_BOX_N : 1;
     static constexpr int B_BOX_BYTES = B_MN ? BK * 128 : B_BYTES;
-    static constexpr int EPI_WARPS = 4;
+    // GELU / tanh cost ~20 instructions an element: two epilogue warps per TMEM lane
+    // quadrant (each taking half the columns) so that the epilogue keeps up with the
+    // next tile's mainloop; the cheap epilogues use one warp per quadrant.
+    static constexpr bool HEAVY_EPI = EPI == EPI_GELU || EPI == EPI_TANH;
+    static constexpr int EPI_WARPS = HEAVY_EPI ? 8 : 4;
     static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+    static constexpr int COLS_W = BN * 4 / EPI_WARPS;       // columns of a tile one epilogue warp handles
+    static constexpr int NCH_W = COLS_W / 32;                // its 32-column chunks
+    static constexpr int CPG = NCH_W < 4 ? NCH_W : 4;        // chunks per mask-word group
+    static_assert(NCH_W % CPG == 0 && (CPG == 2 || CPG == 4), "chunk grouping");
     static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                    : (2 * BN <= 256) ? 256 : 512;
-    static constexpr int STG_BYTES = 32 * 128;      // per epilogue warp: 32 rows x 64 outputs
+    static constexpr int STG_BYTES = 32 * 64;       // per epilogue warp: 32 rows x 32 16-bit outputs
     // shared-memory layout (offsets from a 1024-byte aligned base)
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_BIAS = OFF_STG + EPI_WARPS * STG_BYTES;
-    static constexpr int BIAS_FLOATS = (EPI != EPI_NONE && AXIS == AXIS_COL) ? BN : 0;
+    static constexpr int BIAS_FLOATS = (EPI != EPI_NONE && AXIS == AXIS_COL) ? COLS_W : 0;
     static constexpr int OFF_BAR = OFF_BIAS + EPI_WARPS * BIAS_FLOATS * 4;
     static constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -483,8 +509,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         using O = OutT<C::DT>;
-        const int ew = warp - 2;                 // epilogue warp 0..3
+        const int ew = warp - 2;                 // epilogue warp 0..EPI_WARPS-1
         const int q = warp & 3;                  // TMEM lane quadrant this warp may access
+        const int cbase = (ew >> 2) * C::NCH_W;  // its first 32-column chunk of the tile
         const uint32_t stg = sStg + ew * C::STG_BYTES;
         float *bsm = bias_smem + ew * C::BIAS_FLOATS;
         float alpha = 1.0f;
@@ -503,6 +530,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             tile_coords(p, w.tile, tm, tn);
             const int m0 = tm * (C::BM * C::CG) + (int)rank * C::BM;
             const int n0 = tn * C::BN;
+            const int nw = n0 + 32 * cbase;      // this warp's first output column
             const int row = m0 + 32 * q + lane;
             const bool row_ok = row < p.m;
             float rbias = 0.0f;
@@ -510,22 +538,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 if (row_ok && has_bias) rbias = O::load(p.bias, row);
             }
             if constexpr (C::BIAS_FLOATS > 0) if (!partial_out) {
-                // this warp's copy of bias[n0 .. n0+BN) as fp32 (read once per tile)
+                // this warp's copy of bias[nw .. nw+COLS_W) as fp32 (read once per tile)
                 __syncwarp();
                 if (!has_bias) {
-                    for (int j = lane; j < C::BN; j += 32) bsm[j] = 0.0f;
-                } else if (n0 + C::BN <= p.n) {
+                    for (int j = lane; j < C::COLS_W; j += 32) bsm[j] = 0.0f;
+                } else if (nw + C::COLS_W <= p.n) {
 #pragma unroll
-                    for (int j = lane * 8; j < C::BN; j += 256) {
+                    for (int j = lane * 8; j < C::COLS_W; j += 256) {
                         const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
-                            reinterpret_cast<const typename O::type *>(p.bias) + n0 + j));
+                            reinterpret_cast<const typename O::type *>(p.bias) + nw + j));
                         float f[8];
                         unpack8<C::DT == DT_F16 ? DT_F16 : DT_BF16>(u, f);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) bsm[j + e] = f[e];
                     }
                 } else {
-                    for (int j = lane; j < C::BN; j += 32) bsm[j] = n0 + j < p.n ? O::load(p.bias, n0 + j) : 0.0f;
+                    for (int j = lane; j < C::COLS_W; j += 32) bsm[j] = nw + j < p.n ? O::load(p.bias, nw + j) : 0.0f;
                 }
                 __syncwarp();
             }
@@ -543,16 +571,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if (lane == 0) trace_event(p.trace, warp, 7, w.tile, c_first);
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + acc * C::BN;
 #pragma unroll 1
-            for (int g = 0; g < C::BN / 128; ++g) {       // 128 output columns per group
-                uint32_t words[4];
+            for (int g = 0; g < C::NCH_W / C::CPG; ++g) {    // CPG chunks share a mask store
+                uint32_t words[C::CPG];
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {          // 32 columns per chunk
-                    const int c = 4 * g + cc;
+                for (int cc = 0; cc < C::CPG; ++cc) {          // 32 columns per chunk
+                    const int c = cbase + C::CPG * g + cc;     // chunk index within the tile
+                    const int cl = c - cbase;                  // chunk index within this warp
                     uint32_t v[32];
                     ptx::tmem_ld_32x32b_x32(tbase + c * 32, v);
                     ptx::tmem_wait_ld(v);
-                    if (cc == 3 && g == C::BN / 128 - 1) {
-                        // accumulator fully read: hand it back to the MMA issuer
+                    if (cc == C::CPG - 1 && g == C::NCH_W / C::CPG - 1) {
+                        // accumulator fully read by this warp: hand it back to the MMA issuer
                         ptx::tc_fence_before();
                         __syncwarp();
                         if (lane == 0) {
@@ -571,12 +600,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                     for (int u = c_first; u < unit; ++u) {       // earlier slices, in unit order
                         const float4 *src = ws_chunk<C::BN>(p.workspace, u, C::CG, rank, q, c, lane);
-                        float4 f8[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) f8[j] = __ldcg(src + 32 * j);
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
-                            const float4 f = f8[j];
+                            const float4 f = __ldcg(src + 32 * j);
                             v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + f.x);
                             v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + f.y);
                             v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + f.z);
@@ -593,7 +619,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         x1 *= alpha;
                         if constexpr (C::EPI != EPI_NONE) {
                             if constexpr (C::AXIS == AXIS_ROW) { x0 += rbias; x1 += rbias; }
-                            else { x0 += bsm[32 * c + j]; x1 += bsm[32 * c + j + 1]; }
+                            else { x0 += bsm[32 * cl + j]; x1 += bsm[32 * cl + j + 1]; }
                         }
                         if constexpr (C::EPI == EPI_RELU_AUX) {
                             bits |= (x0 > 0.0f ? 1u : 0u) << j;
@@ -606,34 +632,34 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         const uint32_t keep = valid >= 32 ? 0xFFFFFFFFu : (valid <= 0 ? 0u : ((1u << valid) - 1u));
                         words[cc] = bits & keep;
                     }
-                    // stage 32 rows x 64 outputs (two chunks) in the 128-byte swizzled layout
-                    if ((cc & 1) == 0) {
-                        if (lane == 0) ptx::bulk_wait_read<0>();     // previous store has read the buffer
-                        __syncwarp();
-                    }
-                    uint8_t *stg_row = smem + C::OFF_STG + ew * C::STG_BYTES + lane * 128;
+                    // stage 32 rows x 32 outputs in the 64-byte swizzled layout the TMA store reads:
+                    // 16-byte piece j of row r sits at r*64 + ((j ^ ((r >> 1) & 3)) * 16)
+                    if (lane == 0) ptx::bulk_wait_read<0>();     // previous store has read the buffer
+                    __syncwarp();
+                    uint8_t *stg_row = smem + C::OFF_STG + ew * C::STG_BYTES + lane * 64;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const int chunk = ((cc & 1) * 4 + i) ^ (lane & 7);
-                        *reinterpret_cast<uint4 *>(stg_row + chunk * 16) =
+                        const int piece = i ^ ((lane >> 1) & 3);
+                        *reinterpret_cast<uint4 *>(stg_row + piece * 16) =
                             make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
                     }
-                    if ((cc & 1) == 1) {
-                        ptx::fence_proxy_async_smem();
-                        __syncwarp();
-                        // boxes starting past the last row or column hold nothing to store
-                        if (lane == 0 && m0 + 32 * q < p.m && n0 + 32 * (c - 1) < p.n) {
-                            ptx::tma_store_2d(&tmD, stg, n0 + 32 * (c - 1), m0 + 32 * q);
-                            ptx::bulk_commit();
-                        }
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    // boxes starting past the last row or column hold nothing to store
+                    if (lane == 0 && m0 + 32 * q < p.m && col0 < p.n) {
+                        ptx::tma_store_2d(&tmD, stg, col0, m0 + 32 * q);
+                        ptx::bulk_commit();
                     }
                 }
                 if (partial_out) continue;
                 if constexpr (C::EPI == EPI_RELU_AUX) {
-                    const int wcol = n0 + 128 * g;
-                    if (row_ok && wcol < p.n) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(p.aux + (int64_t)row * p.aux_pitch_words + wcol / 32);
-                        *dst = make_uint4(words[0], words[1], words[2], words[3]);
+                    const int wcol = nw + 32 * C::CPG * g;
+                    if (row_ok && wcol < p.aux_pitch_words * 32) {      // padding words too (zero bits)
+                        uint32_t *dst = p.aux + (int64_t)row * p.aux_pitch_words + wcol / 32;
+                        if constexpr (C::CPG == 4)
+                            *reinterpret_cast<uint4 *>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
+                        else
+                            *reinterpret_cast<uint2 *>(dst) = make_uint2(words[0], words[1]);
                     }
                 }
             }

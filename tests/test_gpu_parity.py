@@ -100,6 +100,34 @@ def test_integer_inputs_bit_exact(kernel, dtype, epilogue):
         np.testing.assert_array_equal(unpack_aux(words, wl.m, wl.n), mask)
 
 
+# ------------------------------------------------------------------ activation accuracy
+@pytest.mark.parametrize("epilogue", ["gelu", "tanh"])
+@pytest.mark.parametrize("kernel", ["tc1", "splitk"])
+def test_activation_dense_grid(epilogue, kernel):
+    """act(A . I): every bf16 value in [-10, 10] through the kernel's activation.
+
+    The product with an identity B is exact, so the only errors are the
+    activation's and the final bf16 rounding: |gpu - ref| <= 2^-8 |ref| + 1e-6."""
+    vals = torch.arange(-10.0, 10.0, 2.0 ** -7, dtype=torch.float64).to(torch.bfloat16).unique()
+    n = 128
+    m = (vals.numel() + n - 1) // n
+    if kernel == "splitk":
+        m = 64
+        vals = vals[: m * n]
+    grid = torch.zeros(m * n, dtype=torch.bfloat16)
+    grid[: vals.numel()] = vals
+    A = grid.view(m, n)
+    eye = torch.eye(n, dtype=torch.bfloat16)
+    D = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    with g.Plan(m, n, n, "bf16", epilogue, "row", "kn", kernel=kernel) as plan:
+        plan.run(A.cuda(), eye.cuda(), None, D)
+        plan.check()
+    ref, _, _ = oracle.gemm_epi(storage(A), storage(eye), None, dtype="bf16", epilogue=epilogue)
+    err = np.abs(D.double().cpu().numpy() - ref)
+    bound = 2.0 ** -8 * np.abs(ref) + 1e-6
+    assert (err <= bound).all(), f"max excess {float((err - bound).max())}"
+
+
 # ------------------------------------------------------------------ epilogue scaling factor
 @pytest.mark.parametrize("kernel", ["tc1", "tc2", "splitk"])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
