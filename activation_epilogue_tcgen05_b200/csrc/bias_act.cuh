@@ -5,6 +5,9 @@
 // paragraph 1: matmul, write back, separate element-wise kernel), kept as the
 // library's own baseline for time and DRAM-traffic comparisons.
 //
+// EPI_DRELU is the backward step of the same baseline: it reads the packed mask
+// from aux and zeroes D where the mask bit is 0 (no bias).
+//
 // One thread owns 32 consecutive columns of one row -- exactly one 32-bit
 // mask word -- and moves them with four 16-byte loads and stores; consecutive
 // threads take consecutive words of a row, so a warp streams 2 KB contiguous.
@@ -37,6 +40,8 @@ __global__ void __launch_bounds__(256) bias_act_kernel(void *D, const void *bias
             if (bias != nullptr) rb = O::load(bias, i);
         }
         uint32_t bits = 0;
+        uint32_t mbits = 0;
+        if constexpr (EPI == EPI_DRELU) mbits = aux[idx];
         if (j0 + 32 <= n) {
             uint4 *src = reinterpret_cast<uint4 *>(row + j0);
             uint4 u[4];
@@ -65,6 +70,10 @@ __global__ void __launch_bounds__(256) bias_act_kernel(void *D, const void *bias
                 for (int e = 0; e < 8; e += 2) {
                     float x0 = f[e] + (AXIS == AXIS_ROW ? rb : bcol[8 * s + e]);
                     float x1 = f[e + 1] + (AXIS == AXIS_ROW ? rb : bcol[8 * s + e + 1]);
+                    if constexpr (EPI == EPI_DRELU) {
+                        x0 = ((mbits >> (8 * s + e)) & 1u) ? f[e] : 0.0f;
+                        x1 = ((mbits >> (8 * s + e + 1)) & 1u) ? f[e + 1] : 0.0f;
+                    }
                     if constexpr (EPI == EPI_RELU_AUX) {
                         bits |= (x0 > 0.0f ? 1u : 0u) << (8 * s + e);
                         bits |= (x1 > 0.0f ? 1u : 0u) << (8 * s + e + 1);
@@ -76,6 +85,7 @@ __global__ void __launch_bounds__(256) bias_act_kernel(void *D, const void *bias
         } else {
             for (int j = j0; j < n; ++j) {
                 float x = O::load(row, j) + (AXIS == AXIS_ROW ? rb : (bias != nullptr ? O::load(bias, j) : 0.0f));
+                if constexpr (EPI == EPI_DRELU) x = ((mbits >> (j - j0)) & 1u) ? O::load(row, j) : 0.0f;
                 if constexpr (EPI == EPI_RELU_AUX) bits |= (x > 0.0f ? 1u : 0u) << (j - j0);
                 const float y = activate<EPI>(x);
                 if constexpr (DT == DT_F16) row[j] = __float2half_rn(y);

@@ -33,6 +33,7 @@ struct Plan {
     int dtype, epilogue, axis, b_layout;
     int kepi;            // kernel epilogue (EPI_*): the activation
     bool has_bias;       // the public epilogue adds a bias
+    bool bwd, bgrad;     // backward epilogue (DRELU*); with a bias gradient (DRELU_BGRAD)
     gemm_epi_options opts;
     int device, num_sms;
     // kernel choice
@@ -43,11 +44,15 @@ struct Plan {
     int kb_per_cta;
     int grid;
     int group_m;
+    bool pdl;            // programmatic dependent launch (GEMM_EPI_PDL=0 turns it off)
     // split tail (TC kernels): tiles [0, sk_tiles) cut along k into sk_split parts
     int sk_tiles = 0, sk_split = 0;
     float *workspace = nullptr;          // owned: units x CG x 128 x block_n fp32
     unsigned int *flags = nullptr;       // owned: units x CG x 4 words, zero between launches
     size_t flags_bytes = 0;
+    // DRELU_BGRAD: fp32 partial sums [dbias_parts][dbias_len] (owned)
+    float *dbias_ws = nullptr;
+    int64_t dbias_parts = 0, dbias_len = 0;
     TcLauncher tc_launch = nullptr, tc_none_launch = nullptr;
     SkLauncher sk_launch = nullptr, sk_none_launch = nullptr;
     BiasActLauncher ba_launch = nullptr;
@@ -83,6 +88,7 @@ int kernel_epi(int e) {
     case GEMM_EPI_RELU_AUX_BIAS: case GEMM_EPI_RELU_AUX: return EPI_RELU_AUX;
     case GEMM_EPI_GELU_BIAS: case GEMM_EPI_GELU: return EPI_GELU;
     case GEMM_EPI_TANH_BIAS: case GEMM_EPI_TANH: return EPI_TANH;
+    case GEMM_EPI_DRELU: case GEMM_EPI_DRELU_BGRAD: return EPI_DRELU;
     default: return EPI_NONE;
     }
 }
@@ -149,17 +155,25 @@ int round_nm(int64_t m) {
 
 int choose(Plan *P) {
     const int64_t m = P->m, n = P->n;
+    // The GEMM kernels do only on-chip setup before waiting on the previous grid, so they are
+    // launched as programmatic dependents: their launch and setup overlap the previous
+    // kernel's tail.  GEMM_EPI_PDL=0 launches them plainly (for comparison).
+    {
+        const char *e = getenv("GEMM_EPI_PDL");
+        P->pdl = !(e && e[0] == '0');
+    }
     int kernel = P->opts.kernel;
     if (kernel == GEMM_EPI_KERNEL_AUTO) {
         // small m: swapped split-K; enough 256 x 256 tiles for every SM pair: CTA pairs
         // (half the operand traffic per SM); otherwise single CTAs
         const int64_t pair_tiles = ((m + 255) / 256) * ((n + 255) / 256);
         const int sms_auto = P->opts.max_ctas > 0 ? std::min(P->opts.max_ctas, P->num_sms) : P->num_sms;
-        if (m <= 64) kernel = GEMM_EPI_KERNEL_SPLITK;
+        // (the split-K kernel has no backward epilogue)
+        if (m <= 64 && P->kepi != EPI_DRELU) kernel = GEMM_EPI_KERNEL_SPLITK;
         else if (pair_tiles >= sms_auto / 2) kernel = GEMM_EPI_KERNEL_TC2;
         else kernel = GEMM_EPI_KERNEL_TC1;
     }
-    if (kernel == GEMM_EPI_KERNEL_SPLITK && m > 128) return GEMM_EPI_ERR_UNSUPPORTED;
+    if (kernel == GEMM_EPI_KERNEL_SPLITK && (m > 128 || P->kepi == EPI_DRELU)) return GEMM_EPI_ERR_UNSUPPORTED;
     P->kernel = kernel;
     const bool b_mn = P->b_layout == GEMM_EPI_B_KN;
     const int bk = 128 / esize(P->dtype);
@@ -194,6 +208,8 @@ int choose(Plan *P) {
         if (bn == 0) {
             const int64_t tiles256 = ((m + bm - 1) / bm) * ((n + 255) / 256);
             bn = tiles256 >= sms / cg ? 256 : 128;
+            // a pair's e4m3 B half-tile stored (k, n) must be a whole 128-byte box: 128 columns
+            if (cg == 2 && P->dtype == GEMM_EPI_E4M3 && b_mn) bn = 256;
         }
         if (bn != 128 && bn != 256) return GEMM_EPI_ERR_ARG;
         P->block_n = bn;
@@ -257,6 +273,7 @@ unsigned long long *trace_buffer() {
 }
 
 int check_run_args(Plan *P, const void *A, const void *B, const void *bias, void *D, uint32_t *aux) {
+    if (P->bwd) return GEMM_EPI_ERR_ARG;          // backward plans run through gemm_epi_run_bwd
     if (!A || !B || !D) return GEMM_EPI_ERR_NULL;
     if (P->has_bias && !bias) return GEMM_EPI_ERR_NULL;
     if (P->kepi == EPI_RELU_AUX && !aux) return GEMM_EPI_ERR_NULL;
@@ -264,6 +281,16 @@ int check_run_args(Plan *P, const void *A, const void *B, const void *bias, void
     if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return GEMM_EPI_ERR_ALIGN;
     if (P->has_bias && !aligned16(bias)) return GEMM_EPI_ERR_ALIGN;
     if (P->kepi == EPI_RELU_AUX && !aligned16(aux)) return GEMM_EPI_ERR_ALIGN;
+    return GEMM_EPI_OK;
+}
+
+int check_bwd_args(Plan *P, const void *A, const void *B, const uint32_t *aux, void *D, void *dbias) {
+    if (!P->bwd) return GEMM_EPI_ERR_ARG;
+    if (!A || !B || !D || !aux) return GEMM_EPI_ERR_NULL;
+    if (P->bgrad && !dbias) return GEMM_EPI_ERR_NULL;
+    if (P->dtype == GEMM_EPI_E4M3 && (!P->scale_a || !P->scale_b)) return GEMM_EPI_ERR_NULL;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(aux)) return GEMM_EPI_ERR_ALIGN;
+    if (P->bgrad && !aligned16(dbias)) return GEMM_EPI_ERR_ALIGN;
     return GEMM_EPI_OK;
 }
 
@@ -299,7 +326,8 @@ int ensure_maps(Plan *P, const void *A, const void *B, void *D) {
     return GEMM_EPI_OK;
 }
 
-int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, cudaStream_t stream) {
+int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, cudaStream_t stream,
+                float *dbias_ws = nullptr) {
     if (!P->has_bias) bias = nullptr;
     const int bk = 128 / esize(P->dtype);
     const int num_kb = (int)((P->k + bk - 1) / bk);
@@ -323,6 +351,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.status = P->status;
         L.grid = P->grid;
         L.cluster = P->split;
+        L.pdl = P->pdl;
         L.stream = stream;
         e = (fused ? P->sk_launch : P->sk_none_launch)(L);
     } else {
@@ -351,7 +380,9 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.workspace = P->workspace;
         L.p.flags = P->flags;
         L.p.trace = trace_buffer();
+        L.p.dbias_ws = fused ? dbias_ws : nullptr;
         L.grid = P->grid;
+        L.pdl = P->pdl;
         L.stream = stream;
         e = (fused ? P->tc_launch : P->tc_none_launch)(L);
     }
@@ -364,7 +395,7 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     if (m <= 0 || n <= 0 || k <= 0) return GEMM_EPI_ERR_ARG;
     if (m > 0x7fffffffll || n > 0x7fffffffll || k > 0x7fffffffll) return GEMM_EPI_ERR_ARG;
     if (dtype < GEMM_EPI_F16 || dtype > GEMM_EPI_E4M3) return GEMM_EPI_ERR_ARG;
-    if (epilogue < GEMM_EPI_NONE || epilogue > GEMM_EPI_TANH) return GEMM_EPI_ERR_ARG;
+    if (epilogue < GEMM_EPI_NONE || epilogue > GEMM_EPI_DRELU_BGRAD) return GEMM_EPI_ERR_ARG;
     if (bias_axis != GEMM_EPI_BIAS_ROW && bias_axis != GEMM_EPI_BIAS_COL) return GEMM_EPI_ERR_ARG;
     if (b_layout != GEMM_EPI_B_KN && b_layout != GEMM_EPI_B_NK) return GEMM_EPI_ERR_ARG;
     gemm_epi_options o{};
@@ -401,7 +432,9 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     P->epilogue = epilogue;
     P->kepi = kernel_epi(epilogue);
     P->has_bias = epi_has_bias(epilogue);
-    P->axis = P->has_bias ? bias_axis : GEMM_EPI_BIAS_ROW;
+    P->bwd = P->kepi == EPI_DRELU;
+    P->bgrad = epilogue == GEMM_EPI_DRELU_BGRAD;
+    P->axis = (P->has_bias || P->bgrad) ? bias_axis : GEMM_EPI_BIAS_ROW;
     P->b_layout = b_layout;
     P->opts = o;
     P->device = dev;
@@ -425,6 +458,19 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
         P->flags_bytes = fl_bytes;
         if (cudaMalloc(&P->workspace, ws_bytes) != cudaSuccess || cudaMalloc(&P->flags, fl_bytes) != cudaSuccess ||
             cudaMemset(P->flags, 0, fl_bytes) != cudaSuccess) {
+            cudaGetLastError();
+            if (P->workspace) cudaFree(P->workspace);
+            if (P->flags) cudaFree(P->flags);
+            cudaFree(P->status);
+            delete P;
+            return GEMM_EPI_ERR_CUDA;
+        }
+    }
+    if (P->bgrad) {
+        // one fp32 partial per (row, tile column) for ROW, per (32-row block, column) for COL
+        P->dbias_len = P->axis == GEMM_EPI_BIAS_ROW ? m : n;
+        P->dbias_parts = P->axis == GEMM_EPI_BIAS_ROW ? (n + P->block_n - 1) / P->block_n : (m + 31) / 32;
+        if (cudaMalloc(&P->dbias_ws, (size_t)P->dbias_parts * (size_t)P->dbias_len * sizeof(float)) != cudaSuccess) {
             cudaGetLastError();
             if (P->workspace) cudaFree(P->workspace);
             if (P->flags) cudaFree(P->flags);
@@ -537,6 +583,50 @@ int gemm_epi_unfused_run(gemm_epi_plan_t plan, const void *A, const void *B, con
     return e == cudaSuccess ? GEMM_EPI_OK : GEMM_EPI_ERR_CUDA;
 }
 
+int gemm_epi_run_bwd(gemm_epi_plan_t plan, const void *A, const void *B, const uint32_t *aux, void *D,
+                     void *dbias, void *stream) {
+    if (!live(plan)) return GEMM_EPI_ERR_ARG;
+    Plan *P = reinterpret_cast<Plan *>(plan);
+    int rc = check_bwd_args(P, A, B, aux, D, dbias);
+    if (rc != GEMM_EPI_OK) return rc;
+    rc = ensure_maps(P, A, B, D);
+    if (rc != GEMM_EPI_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    rc = launch_main(P, true, nullptr, D, const_cast<uint32_t *>(aux), s, P->bgrad ? P->dbias_ws : nullptr);
+    if (rc != GEMM_EPI_OK || !P->bgrad) return rc;
+    const int out_dt = P->dtype == GEMM_EPI_E4M3 ? DT_BF16 : P->dtype;
+    const cudaError_t e = launch_sum_parts_f32(out_dt, P->dbias_ws, P->dbias_parts, P->dbias_len, dbias, s);
+    return e == cudaSuccess ? GEMM_EPI_OK : GEMM_EPI_ERR_CUDA;
+}
+
+int gemm_epi_unfused_run_bwd(gemm_epi_plan_t plan, const void *A, const void *B, const uint32_t *aux, void *D,
+                             void *dbias, void *stream) {
+    if (!live(plan)) return GEMM_EPI_ERR_ARG;
+    Plan *P = reinterpret_cast<Plan *>(plan);
+    int rc = check_bwd_args(P, A, B, aux, D, dbias);
+    if (rc != GEMM_EPI_OK) return rc;
+    rc = ensure_maps(P, A, B, D);
+    if (rc != GEMM_EPI_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    rc = launch_main(P, false, nullptr, D, nullptr, s);
+    if (rc != GEMM_EPI_OK) return rc;
+    const int64_t pitch_words = ((P->n + 127) / 128) * 4;
+    const int64_t total = P->m * pitch_words;
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, (int64_t)P->num_sms * 16);
+    cudaError_t e = P->ba_launch(D, nullptr, const_cast<uint32_t *>(aux), (int)P->m, (int)P->n, pitch_words,
+                                 (int)blocks, s);
+    if (e != cudaSuccess) return GEMM_EPI_ERR_CUDA;
+    if (!P->bgrad) return GEMM_EPI_OK;
+    const int out_dt = P->dtype == GEMM_EPI_E4M3 ? DT_BF16 : P->dtype;
+    if (P->axis == GEMM_EPI_BIAS_ROW) {
+        const int64_t g = std::min<int64_t>((P->m + 7) / 8, (int64_t)P->num_sms * 16);
+        e = launch_sum_rows(out_dt, D, P->m, P->n, dbias, (int)g, s);
+    } else {
+        e = launch_sum_cols(out_dt, D, P->m, P->n, dbias, s);
+    }
+    return e == cudaSuccess ? GEMM_EPI_OK : GEMM_EPI_ERR_CUDA;
+}
+
 int gemm_epi_check(gemm_epi_plan_t plan, void *stream) {
     if (!live(plan)) return GEMM_EPI_ERR_ARG;
     Plan *P = reinterpret_cast<Plan *>(plan);
@@ -587,6 +677,7 @@ int gemm_epi_free(gemm_epi_plan_t plan) {
     if (P->status) cudaFree(P->status);
     if (P->workspace) cudaFree(P->workspace);
     if (P->flags) cudaFree(P->flags);
+    if (P->dbias_ws) cudaFree(P->dbias_ws);
     P->magic = 0;
     delete P;
     return GEMM_EPI_OK;
@@ -597,7 +688,7 @@ const char *gemm_epi_status_string(int status) {
     case GEMM_EPI_OK: return "ok";
     case GEMM_EPI_ERR_ARG: return "invalid argument (size, enum, option or plan handle)";
     case GEMM_EPI_ERR_ALIGN: return "pointer not 16-byte aligned or row pitch not a multiple of 16 bytes";
-    case GEMM_EPI_ERR_NULL: return "required pointer is NULL (operand, bias, aux or FP8 scales)";
+    case GEMM_EPI_ERR_NULL: return "required pointer is NULL (operand, bias, aux, dbias or FP8 scales)";
     case GEMM_EPI_ERR_UNSUPPORTED: return "combination not supported by this build";
     case GEMM_EPI_ERR_CUDA: return "CUDA runtime or driver call failed";
     case GEMM_EPI_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";

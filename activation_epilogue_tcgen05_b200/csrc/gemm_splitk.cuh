@@ -124,6 +124,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // on-chip setup above; global memory only after the previous kernel has completed
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {

@@ -56,7 +56,10 @@ namespace gemm_epi {
 enum : int { DT_F16 = 0, DT_BF16 = 1, DT_E4M3 = 2 };
 // Kernel epilogues (activation after alpha*A.B + bias).  A bias pointer of
 // NULL means no bias: the bias-free public epilogues run these same kernels.
-enum : int { EPI_NONE = 0, EPI_BIAS = 1, EPI_RELU = 2, EPI_RELU_AUX = 3, EPI_GELU = 4, EPI_TANH = 5 };
+// EPI_DRELU is the ReLU backward: D = mask ? alpha*A.B : 0 with the mask read
+// from aux, plus (when TcParams::dbias_ws is set) per-part bias-gradient sums.
+enum : int { EPI_NONE = 0, EPI_BIAS = 1, EPI_RELU = 2, EPI_RELU_AUX = 3, EPI_GELU = 4, EPI_TANH = 5,
+             EPI_DRELU = 6 };
 enum : int { AXIS_ROW = 0, AXIS_COL = 1 };
 
 // Status-word bits written by kernels that gave up waiting.
@@ -76,7 +79,7 @@ struct TcParams {
     int tiles_m, tiles_n, num_tiles, num_kb;
     int group_m;                 // tile-raster group height (in tiles along m)
     const void *bias;            // length m (ROW) or n (COL), output type
-    uint32_t *aux;               // RELU_AUX only
+    uint32_t *aux;               // RELU_AUX: mask written; DRELU: mask read
     int64_t aux_pitch_words;     // ceil(n/128)*4
     const float *scale_a;        // alpha = *scale_a * *scale_b when set (always for E4M3)
     const float *scale_b;
@@ -87,6 +90,10 @@ struct TcParams {
     float *workspace;            // partial tiles, 128 x BN fp32 per (unit, cta rank); see ws_slot()
     unsigned int *flags;         // [unit][cta rank][4 epilogue warps]: 1 while a partial is unread
     unsigned long long *trace;   // timeline records; used only by builds with GEMM_EPI_TRACE=1
+    // DRELU with a bias gradient: fp32 partial sums of D, written once each per launch.
+    //   ROW: [n-part = column / BN][row]      (m floats per part, ceil(n/BN) parts)
+    //   COL: [m-part = row / 32][column]      (n floats per part, ceil(m/32) parts)
+    float *dbias_ws;
 };
 
 // Timeline tracing (off unless the library is compiled with -DGEMM_EPI_TRACE=1):
@@ -312,6 +319,8 @@ struct TcCfg {
     // quadrant (each taking half the columns) so that the epilogue keeps up with the
     // next tile's mainloop; the cheap epilogues use one warp per quadrant.
     static constexpr bool HEAVY_EPI = EPI == EPI_GELU || EPI == EPI_TANH;
+    static constexpr bool BWD = EPI == EPI_DRELU;             // reads the mask, adds no bias
+    static constexpr bool FWD_BIAS = EPI != EPI_NONE && !BWD;  // may add a bias
     static constexpr int EPI_WARPS = HEAVY_EPI ? 8 : 4;
     static constexpr int THREADS = 64 + 32 * EPI_WARPS;
     static constexpr int COLS_W = BN * 4 / EPI_WARPS;       // columns of a tile one epilogue warp handles
@@ -326,7 +335,7 @@ struct TcCfg {
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_BIAS = OFF_STG + EPI_WARPS * STG_BYTES;
-    static constexpr int BIAS_FLOATS = (EPI != EPI_NONE && AXIS == AXIS_COL) ? COLS_W : 0;
+    static constexpr int BIAS_FLOATS = (FWD_BIAS && AXIS == AXIS_COL) ? COLS_W : 0;
     static constexpr int OFF_BAR = OFF_BIAS + EPI_WARPS * BIAS_FLOATS * 4;
     static constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -336,6 +345,7 @@ struct TcCfg {
     static_assert(B_MN == false || BN_LOCAL % B_BOX_N == 0, "MN-major B tile must be whole boxes");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "stage alignment");
+    static_assert(!BWD || (EPI_WARPS == 4 && CPG == 4), "backward epilogue: one mask uint4 per chunk group");
 };
 
 // Tile index -> (tile_m, tile_n) with a grouped raster: GROUP_M tile-rows are
@@ -401,6 +411,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if constexpr (C::CG == 2) ptx::cluster_sync(); else __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // Everything above touches only on-chip state, so under programmatic dependent launch
+    // it overlaps the previous kernel's tail.  No global memory is read or written before
+    // the previous kernel has completed; the next kernel may be scheduled from here on.
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -517,6 +532,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         float alpha = 1.0f;
         if (p.scale_a != nullptr) alpha = __ldg(p.scale_a) * __ldg(p.scale_b);
         const bool has_bias = p.bias != nullptr;
+        const bool bgrad = C::BWD && p.dbias_ws != nullptr;   // backward: bias-gradient partials
         uint32_t acc = 0, acc_phase = 0;
         bool ok = true;
         WorkIter it(p, unit, units);
@@ -534,9 +550,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const int row = m0 + 32 * q + lane;
             const bool row_ok = row < p.m;
             float rbias = 0.0f;
-            if constexpr (C::EPI != EPI_NONE && C::AXIS == AXIS_ROW) {
+            if constexpr (C::FWD_BIAS && C::AXIS == AXIS_ROW) {
                 if (row_ok && has_bias) rbias = O::load(p.bias, row);
             }
+            // backward: this lane's mask words for columns [nw, nw + COLS_W), one uint4 per
+            // 128 columns, fetched before the accumulator wait so that their latency hides
+            uint4 mk0 = make_uint4(0u, 0u, 0u, 0u), mk1 = mk0;
+            if constexpr (C::BWD) if (!partial_out && row_ok) {
+                const int64_t w0 = nw / 32;
+                const uint32_t *mrow = p.aux + (int64_t)row * p.aux_pitch_words + w0;
+                if (w0 < p.aux_pitch_words) mk0 = __ldg(reinterpret_cast<const uint4 *>(mrow));
+                if constexpr (C::NCH_W == 8)
+                    if (w0 + 4 < p.aux_pitch_words) mk1 = __ldg(reinterpret_cast<const uint4 *>(mrow + 4));
+            }
+            float rsum = 0.0f;                   // backward, ROW axis: this row's sum over the tile
             if constexpr (C::BIAS_FLOATS > 0) if (!partial_out) {
                 // this warp's copy of bias[nw .. nw+COLS_W) as fp32 (read once per tile)
                 __syncwarp();
@@ -573,6 +600,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll 1
             for (int g = 0; g < C::NCH_W / C::CPG; ++g) {    // CPG chunks share a mask store
                 uint32_t words[C::CPG];
+                const uint4 mk = g == 0 ? mk0 : mk1;
 #pragma unroll
                 for (int cc = 0; cc < C::CPG; ++cc) {          // 32 columns per chunk
                     const int c = cbase + C::CPG * g + cc;     // chunk index within the tile
@@ -612,14 +640,28 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const int col0 = n0 + 32 * c;
                     uint32_t packed[16];
                     uint32_t bits = 0;
+                    const uint32_t mbits = cc == 0 ? mk.x : cc == 1 ? mk.y : cc == 2 ? mk.z : mk.w;
+                    (void)mbits;
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
                         float x0 = __uint_as_float(v[j]), x1 = __uint_as_float(v[j + 1]);
                         x0 *= alpha;
                         x1 *= alpha;
-                        if constexpr (C::EPI != EPI_NONE) {
+                        if constexpr (C::FWD_BIAS) {
                             if constexpr (C::AXIS == AXIS_ROW) { x0 += rbias; x1 += rbias; }
                             else { x0 += bsm[32 * cl + j]; x1 += bsm[32 * cl + j + 1]; }
+                        }
+                        if constexpr (C::BWD) {
+                            // ReLU backward: the gradient passes where the forward input was > 0
+                            x0 = ((mbits >> j) & 1u) ? x0 : 0.0f;
+                            x1 = ((mbits >> (j + 1)) & 1u) ? x1 : 0.0f;
+                            if constexpr (C::AXIS == AXIS_ROW) {
+                                rsum += x0;
+                                rsum += x1;
+                            } else {
+                                v[j] = __float_as_uint(x0);
+                                v[j + 1] = __float_as_uint(x1);
+                            }
                         }
                         if constexpr (C::EPI == EPI_RELU_AUX) {
                             bits |= (x0 > 0.0f ? 1u : 0u) << j;
@@ -650,6 +692,26 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         ptx::tma_store_2d(&tmD, stg, col0, m0 + 32 * q);
                         ptx::bulk_commit();
                     }
+                    if constexpr (C::BWD && C::AXIS == AXIS_COL) if (bgrad) {
+                        // column sums over this warp's 32 rows: a butterfly that halves the
+                        // live values at each of 5 exchange steps (31 shuffles for 32 columns);
+                        // afterwards lane l holds the sum of column col0 + l, in a fixed order
+                        float f[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
+#pragma unroll
+                        for (int sh = 16; sh >= 1; sh >>= 1) {
+                            const bool upper = (lane & sh) != 0;
+#pragma unroll
+                            for (int j = 0; j < sh; ++j) {
+                                const float send = upper ? f[j] : f[j + sh];
+                                const float keep = upper ? f[j + sh] : f[j];
+                                f[j] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
+                            }
+                        }
+                        if (m0 + 32 * q < p.m && col0 + lane < p.n)
+                            p.dbias_ws[(size_t)((m0 + 32 * q) >> 5) * p.n + col0 + lane] = f[0];
+                    }
                 }
                 if (partial_out) continue;
                 if constexpr (C::EPI == EPI_RELU_AUX) {
@@ -663,6 +725,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                 }
             }
+            if constexpr (C::BWD && C::AXIS == AXIS_ROW)
+                if (bgrad && !partial_out && row_ok) p.dbias_ws[(size_t)(nw / C::COLS_W) * p.m + row] = rsum;
             if (lane == 0) trace_event(p.trace, warp, 8, w.tile, partial_out ? 1 : 0);
             if (partial_out) {
                 // publish: every lane's stores are ordered before the warp's flag

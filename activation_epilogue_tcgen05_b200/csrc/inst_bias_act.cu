@@ -26,6 +26,7 @@ static BiasActLauncher pick_epi(int epi, int axis) {
     case EPI_RELU_AUX: return pick_axis<DT, EPI_RELU_AUX>(axis);
     case EPI_GELU: return pick_axis<DT, EPI_GELU>(axis);
     case EPI_TANH: return pick_axis<DT, EPI_TANH>(axis);
+    case EPI_DRELU: return &launch_ba<DT, EPI_DRELU, AXIS_ROW>;   // no bias: the axis plays no part
     }
     return nullptr;
 }

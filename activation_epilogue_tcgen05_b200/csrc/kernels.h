@@ -16,6 +16,7 @@ struct TcLaunch {
     CUtensorMap tmA, tmB, tmD;
     TcParams p;
     int grid;
+    bool pdl;            // launch with programmatic stream serialisation
     cudaStream_t stream;
 };
 // One split-K cluster launch.
@@ -24,6 +25,7 @@ struct SkLaunch {
     SkParams p;
     int grid;
     int cluster;
+    bool pdl;            // launch with programmatic stream serialisation
     cudaStream_t stream;
 };
 
@@ -45,6 +47,15 @@ bool find_tc(int cg, int dt, int epi, int axis, bool b_mn, int bn, TcLauncher *l
 bool find_sk(int dt, int epi, int axis, bool w_mn, int nm, SkLauncher *launch, KernelInfo *info);
 bool find_bias_act(int dt, int epi, int axis, BiasActLauncher *launch);
 
+// Bias-gradient reductions (dbias.cuh); out_dt is the bias type (DT_F16 or DT_BF16).
+//   sum_parts_f32: out[i] = sum_p src[p * len + i] over fp32 partials (fused backward)
+//   sum_cols:      out[j] = sum_i D[i, j]  (unfused backward, COL axis)
+//   sum_rows:      out[i] = sum_j D[i, j]  (unfused backward, ROW axis)
+cudaError_t launch_sum_parts_f32(int out_dt, const float *src, int64_t parts, int64_t len, void *out,
+                                 cudaStream_t s);
+cudaError_t launch_sum_cols(int out_dt, const void *D, int64_t m, int64_t n, void *out, cudaStream_t s);
+cudaError_t launch_sum_rows(int out_dt, const void *D, int64_t m, int64_t n, void *out, int grid, cudaStream_t s);
+
 // per-dtype halves of the lookups (one instantiation unit each)
 bool find_tc_f16(int cg, int epi, int axis, bool b_mn, int bn, TcLauncher *, KernelInfo *);
 bool find_tc_bf16(int cg, int epi, int axis, bool b_mn, int bn, TcLauncher *, KernelInfo *);
@@ -53,8 +64,11 @@ bool find_sk_f16(int epi, int axis, bool w_mn, int nm, SkLauncher *, KernelInfo 
 bool find_sk_bf16(int epi, int axis, bool w_mn, int nm, SkLauncher *, KernelInfo *);
 bool find_sk_e4m3(int epi, int axis, bool w_mn, int nm, SkLauncher *, KernelInfo *);
 
-// Ring depth that fills ~192 KB of shared memory with stages.
-constexpr int tc_stages(int stage_bytes) { return (192 * 1024) / stage_bytes; }
+// Ring depth that fills GEMM_EPI_RING_KB (default 192) KB of shared memory with stages.
+#ifndef GEMM_EPI_RING_KB
+#define GEMM_EPI_RING_KB 192
+#endif
+constexpr int tc_stages(int stage_bytes) { return (GEMM_EPI_RING_KB * 1024) / stage_bytes; }
 
 // Shared launch helpers used by the instantiation units.
 template <class C>
@@ -73,15 +87,22 @@ cudaError_t launch_tc(const TcLaunch &L) {
     cfg.blockDim = dim3(C::THREADS, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = L.stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    int na = 0;
     if constexpr (C::CG == 2) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 2;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
     }
+    if (L.pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = na ? attr : nullptr;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, kern, L.tmA, L.tmB, L.tmD, L.p);
 }
 
@@ -114,13 +135,19 @@ cudaError_t launch_sk(const SkLaunch &L) {
     cfg.blockDim = dim3(C::THREADS, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = L.stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = L.cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    int na = 1;
+    if (L.pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, kern, L.tmW, L.tmX, L.p);
 }
 
@@ -177,6 +204,8 @@ KernelInfo sk_info() {
                                    : NAME##_mn<CG, EPI_GELU, AXIS_ROW>(bmn, bn, l, i);                  \
         case EPI_TANH: return axis ? NAME##_mn<CG, EPI_TANH, AXIS_COL>(bmn, bn, l, i)                   \
                                    : NAME##_mn<CG, EPI_TANH, AXIS_ROW>(bmn, bn, l, i);                  \
+        case EPI_DRELU: return axis ? NAME##_mn<CG, EPI_DRELU, AXIS_COL>(bmn, bn, l, i)                 \
+                                    : NAME##_mn<CG, EPI_DRELU, AXIS_ROW>(bmn, bn, l, i);                \
         }                                                                                               \
         return false;                                                                                   \
     }                                                                                                   \

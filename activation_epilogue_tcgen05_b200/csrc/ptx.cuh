@@ -285,6 +285,14 @@ __device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
 }
 
 // Named barrier over `count` threads (multiple of 32).
+// Programmatic dependent launch.  griddep_wait: block until the grid this one
+// depends on (the previous kernel in the stream, when this grid was launched
+// with programmatic stream serialisation) has completed and its memory
+// operations are visible; a no-op otherwise.  griddep_launch_dependents: allow
+// the next grid in the stream to be scheduled before this one completes.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(PKG, "libgemm_epi.so")
 F16, BF16, E4M3 = 0, 1, 2
 NONE, BIAS, RELU_BIAS, RELU_AUX_BIAS, GELU_BIAS = 0, 1, 2, 3, 4
 TANH_BIAS, RELU, RELU_AUX, GELU, TANH = 5, 6, 7, 8, 9
+DRELU, DRELU_BGRAD = 10, 11
 BIAS_ROW, BIAS_COL = 0, 1
 B_KN, B_NK = 0, 1
 KERNEL_AUTO, KERNEL_TC1, KERNEL_TC2, KERNEL_SPLITK = 0, 1, 2, 3
@@ -30,9 +31,10 @@ OK, ERR_ARG, ERR_ALIGN, ERR_NULL, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NO
 DTYPE = {"f16": F16, "bf16": BF16, "e4m3": E4M3}
 EPILOGUE = {"none": NONE, "bias": BIAS, "relu_bias": RELU_BIAS, "relu_aux_bias": RELU_AUX_BIAS,
             "gelu_bias": GELU_BIAS, "tanh_bias": TANH_BIAS, "relu": RELU, "relu_aux": RELU_AUX,
-            "gelu": GELU, "tanh": TANH}
+            "gelu": GELU, "tanh": TANH, "drelu": DRELU, "drelu_bgrad": DRELU_BGRAD}
 HAS_BIAS = {"bias", "relu_bias", "relu_aux_bias", "gelu_bias", "tanh_bias"}
 HAS_AUX = {"relu_aux_bias", "relu_aux"}
+BACKWARD = {"drelu", "drelu_bgrad"}
 AXIS = {"row": BIAS_ROW, "col": BIAS_COL}
 LAYOUT = {"kn": B_KN, "nk": B_NK}
 KERNEL = {"auto": KERNEL_AUTO, "tc1": KERNEL_TC1, "tc2": KERNEL_TC2, "splitk": KERNEL_SPLITK}
@@ -42,7 +44,7 @@ STREAM_K = {"auto": 0, "off": 1, "on": 2}
 EXPORTS = ("gemm_epi_plan", "gemm_epi_plan_ex", "gemm_epi_plan_opts", "gemm_epi_set_scales",
            "gemm_epi_run", "gemm_epi_unfused_run", "gemm_epi_check", "gemm_epi_plan_query",
            "gemm_epi_free", "gemm_epi_status_string", "gemm_epi_aux_pitch_bytes",
-           "gemm_epi_version", "gemm_epi_run_noalloc")
+           "gemm_epi_version", "gemm_epi_run_noalloc", "gemm_epi_run_bwd", "gemm_epi_unfused_run_bwd")
 
 
 class Options(ctypes.Structure):
@@ -89,6 +91,8 @@ def lib():
             L.gemm_epi_set_scales.argtypes = [vp, vp, vp]
             L.gemm_epi_run.argtypes = [vp, vp, vp, vp, vp, vp, vp]
             L.gemm_epi_unfused_run.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+            L.gemm_epi_run_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+            L.gemm_epi_unfused_run_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp]
             L.gemm_epi_check.argtypes = [vp, vp]
             L.gemm_epi_plan_query.argtypes = [vp, ctypes.POINTER(PlanInfo)]
             L.gemm_epi_free.argtypes = [vp]
@@ -102,7 +106,8 @@ def lib():
             for name in ("gemm_epi_plan", "gemm_epi_plan_ex", "gemm_epi_plan_opts",
                          "gemm_epi_set_scales", "gemm_epi_run", "gemm_epi_unfused_run",
                          "gemm_epi_check", "gemm_epi_plan_query", "gemm_epi_free",
-                         "gemm_epi_version", "gemm_epi_run_noalloc"):
+                         "gemm_epi_version", "gemm_epi_run_noalloc", "gemm_epi_run_bwd",
+                         "gemm_epi_unfused_run_bwd"):
                 getattr(L, name).restype = i32
             _lib = L
     return _lib
@@ -140,6 +145,14 @@ def gemm_epi_run(plan, A, B, bias, D, aux, stream) -> None:
 
 def gemm_epi_unfused_run(plan, A, B, bias, D, aux, stream) -> None:
     _check(lib().gemm_epi_unfused_run(plan, A, B, bias, D, aux, stream), "gemm_epi_unfused_run")
+
+
+def gemm_epi_run_bwd(plan, A, B, aux, D, dbias, stream) -> None:
+    _check(lib().gemm_epi_run_bwd(plan, A, B, aux, D, dbias, stream), "gemm_epi_run_bwd")
+
+
+def gemm_epi_unfused_run_bwd(plan, A, B, aux, D, dbias, stream) -> None:
+    _check(lib().gemm_epi_unfused_run_bwd(plan, A, B, aux, D, dbias, stream), "gemm_epi_unfused_run_bwd")
 
 
 def gemm_epi_check(plan, stream) -> None:
@@ -223,6 +236,12 @@ class Plan:
         s = _stream_ptr(stream)
         f = gemm_epi_run if fused else gemm_epi_unfused_run
         f(self.handle, _ptr(A), _ptr(B), _ptr(bias), _ptr(D), _ptr(aux), s)
+
+    def run_bwd(self, A, B, aux, D, dbias=None, stream=None, fused=True):
+        """Backward plans (``drelu``/``drelu_bgrad``): D = mask ? alpha*A.B : 0 (+ dbias)."""
+        s = _stream_ptr(stream)
+        f = gemm_epi_run_bwd if fused else gemm_epi_unfused_run_bwd
+        f(self.handle, _ptr(A), _ptr(B), _ptr(aux), _ptr(D), _ptr(dbias), s)
 
     def check(self, stream=None):
         gemm_epi_check(self.handle, _stream_ptr(stream))

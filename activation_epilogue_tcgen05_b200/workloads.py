@@ -143,6 +143,38 @@ def make_problem(wl: Workload, device="cpu", int_scales: bool = False) -> Proble
     return Problem(wl, a.to(t), b.to(t), bias_t)
 
 
+def make_mask(m: int, n: int, seed: int = 0, kind: str = "bernoulli", p: float = 0.5) -> np.ndarray:
+    """Seeded (m, n) 0/1 uint8 mask for the ReLU backward epilogues.
+
+    kind: "bernoulli" (each bit 1 with probability p, from one seeded
+    ``torch.Generator``), "zeros", "ones", or "checker" (bit = (i + j) odd).
+    """
+    if kind == "bernoulli":
+        gen = torch.Generator(device="cpu")
+        gen.manual_seed(seed)
+        return (torch.rand((m, n), generator=gen) < p).to(torch.uint8).numpy()
+    if kind == "zeros":
+        return np.zeros((m, n), np.uint8)
+    if kind == "ones":
+        return np.ones((m, n), np.uint8)
+    if kind == "checker":
+        return ((np.arange(m)[:, None] + np.arange(n)[None, :]) & 1).astype(np.uint8)
+    raise ValueError(f"unknown mask kind {kind}")
+
+
+def pack_mask(mask: np.ndarray, pad_fill: int = 0) -> np.ndarray:
+    """(m, n) 0/1 array -> the library's aux storage: row-major uint32 words, row
+    pitch ceil(n/128)*4 words, bit b of word w in row i = element (i, 32w + b).
+
+    ``pad_fill`` = 1 sets every bit past column n-1 (which readers ignore).
+    """
+    m, n = mask.shape
+    pitch = ((n + 127) // 128) * 4
+    bits = np.full((m, pitch * 32), 1 if pad_fill else 0, np.uint8)
+    bits[:, :n] = mask
+    return np.packbits(bits, axis=1, bitorder="little").view(np.uint32).reshape(-1).copy()
+
+
 def storage(t: torch.Tensor) -> np.ndarray:
     """Raw bit patterns of a fp16/bf16 (uint16) or e4m3 (uint8) tensor, on the host."""
     t = t.detach().contiguous().cpu()

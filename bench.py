@@ -191,15 +191,23 @@ def oracle_rows_rate(wl, prob, target_s: float, max_rows=None):
     import oracle
     from activation_epilogue_tcgen05_b200.workloads import storage
 
+    from activation_epilogue_tcgen05_b200.workloads import make_mask
+
     Bs = storage(prob.B)
     bias_full = storage(prob.bias)
+    bwd = wl.epilogue in ("drelu", "drelu_bgrad")
 
     def run(rows):
         As = storage(prob.A[:rows])
         bias = bias_full[:rows] if wl.bias_axis == "row" else bias_full
         t0 = time.perf_counter()
-        oracle.gemm_epi(As, Bs, bias, dtype=wl.dtype, epilogue=wl.epilogue, bias_axis=wl.bias_axis,
-                        b_layout=wl.b_layout, scale_a=prob.scale_a, scale_b=prob.scale_b)
+        if bwd:
+            oracle.gemm_epi_bwd(As, Bs, make_mask(rows, wl.n, seed=wl.seed), dtype=wl.dtype,
+                                epilogue=wl.epilogue, bias_axis=wl.bias_axis, b_layout=wl.b_layout,
+                                scale_a=prob.scale_a, scale_b=prob.scale_b)
+        else:
+            oracle.gemm_epi(As, Bs, bias, dtype=wl.dtype, epilogue=wl.epilogue, bias_axis=wl.bias_axis,
+                            b_layout=wl.b_layout, scale_a=prob.scale_a, scale_b=prob.scale_b)
         return time.perf_counter() - t0
 
     threads = oracle.threads()
@@ -233,10 +241,21 @@ def reference_arm(args):
     m_avail = As.shape[0]
     rng = np.random.default_rng(0)
 
+    bwd = wl.epilogue in ("drelu", "drelu_bgrad")
+    if bwd:
+        from activation_epilogue_tcgen05_b200.workloads import make_mask
+        mask_full = make_mask(m_avail, wl.n, seed=wl.seed)
+
     def step(count):
+        t0 = time.perf_counter()
+        if bwd:     # backward: `count` whole output rows (mask, D row and its dbias share)
+            r0 = int(rng.integers(0, max(1, m_avail - count + 1)))
+            oracle.gemm_epi_bwd(As[r0:r0 + count], Bs, mask_full[r0:r0 + count], dtype=wl.dtype,
+                                epilogue=wl.epilogue, bias_axis=wl.bias_axis, b_layout=wl.b_layout,
+                                scale_a=prob.scale_a, scale_b=prob.scale_b)
+            return time.perf_counter() - t0
         rows = rng.integers(0, m_avail, count)
         cols = rng.integers(0, wl.n, count)
-        t0 = time.perf_counter()
         oracle.gemm_epi_sampled(As, Bs, bias if wl.bias_axis == "col" else bias[:m_avail], rows, cols,
                                 dtype=wl.dtype, epilogue=wl.epilogue, bias_axis=wl.bias_axis,
                                 b_layout=wl.b_layout, scale_a=prob.scale_a, scale_b=prob.scale_b)
@@ -244,19 +263,22 @@ def reference_arm(args):
 
     threads = oracle.threads()
     # size one step so that warmup + steps take about a minute in total
-    probe = max(threads * 4, 64)
+    per_unit = wl.n if bwd else 1          # output positions per counted unit (row or position)
+    probe = max(threads, 1) if bwd else max(threads * 4, 64)
     t_probe = step(probe)
     per_pos = t_probe / probe
     budget = 60.0 / max(1, args.steps + args.warmup)
-    count = int(max(threads, min(1 << 20, budget / max(per_pos, 1e-9))))
+    count = int(max(threads if not bwd else 1, min((1 << 20) // per_unit, budget / max(per_pos, 1e-9))))
+    count = min(count, m_avail) if bwd else count
     for _ in range(args.warmup):
         step(count)
     total = 0.0
     for _ in range(args.steps):
         total += step(count)
-    flops = 2.0 * wl.k * count * args.steps
+    flops = 2.0 * wl.k * count * per_unit * args.steps
     value = flops / total / 1e12
-    sample = f"{count} seeded output positions per step (one fp64 dot product of length k each)"
+    sample = (f"{count} consecutive seeded output rows per step (backward oracle, all {wl.n} columns)" if bwd
+              else f"{count} seeded output positions per step (one fp64 dot product of length k each)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps,
@@ -281,7 +303,8 @@ def main(argv=None):
     import torch
     from activation_epilogue_tcgen05_b200 import gemm_epi as g
     from activation_epilogue_tcgen05_b200 import replicas
-    from activation_epilogue_tcgen05_b200.workloads import TORCH_DTYPE, WORKLOADS, make_problem
+    from activation_epilogue_tcgen05_b200.workloads import (TORCH_DTYPE, WORKLOADS, make_mask, make_problem,
+                                                            pack_mask)
 
     rank, world, local_rank = replicas.env_rank()
     if not torch.cuda.is_available():
@@ -295,24 +318,43 @@ def main(argv=None):
     out_t = TORCH_DTYPE[wl.out_dtype]
     big = wl.m * wl.k > (1 << 28)
     prob = make_problem(wl, device="cuda" if big else "cpu")
-    A0, B0, bias0 = prob.A.to(dev), prob.B.to(dev), prob.bias.to(dev)
-    aux_words = wl.m * g.aux_pitch_words(wl.n) if wl.epilogue in g.HAS_AUX else 0
+    A0, B0 = prob.A.to(dev), prob.B.to(dev)
+    # Each step's arguments are (A, B, x, D, y): forward x = bias, y = aux mask (written);
+    # backward x = the packed forward mask (read), y = dbias (written)
+    bwd = wl.epilogue in g.BACKWARD
+    if bwd:
+        import numpy as np
+        x0 = torch.from_numpy(pack_mask(make_mask(wl.m, wl.n, seed=wl.seed)).view(np.int32)).to(dev)
+        y_shape, y_dtype = ((wl.m if wl.bias_axis == "row" else wl.n,), out_t) \
+            if wl.epilogue == "drelu_bgrad" else (None, None)
+    else:
+        x0 = prob.bias.to(dev)
+        aux_words = wl.m * g.aux_pitch_words(wl.n) if wl.epilogue in g.HAS_AUX else 0
+        y_shape, y_dtype = ((aux_words,), torch.int32) if aux_words else (None, None)
+
+    def new_y():
+        return torch.empty(y_shape, dtype=y_dtype, device=dev) if y_shape else None
+
+    y_bytes = (math.prod(y_shape) * torch.empty((), dtype=y_dtype).element_size()) if y_shape else 0
     esz = 1 if wl.dtype == "e4m3" else 2
-    in_bytes = (wl.m * wl.k + wl.k * wl.n) * esz + bias0.numel() * 2
-    out_bytes = wl.m * wl.n * 2 + aux_words * 4
+    in_bytes = (wl.m * wl.k + wl.k * wl.n) * esz + x0.numel() * x0.element_size()
+    out_bytes = wl.m * wl.n * 2 + y_bytes
     set_bytes = in_bytes + out_bytes
     n_sets = 1 if set_bytes > 2 * L2_BYTES else max(2, math.ceil(3 * L2_BYTES / set_bytes))
+    # launches per step: the GEMM (+ the dbias reduction); unfused: + the elementwise pass (+ the sums)
+    launches = 2 if wl.epilogue == "drelu_bgrad" else 1
+    launches_unfused = 3 if wl.epilogue == "drelu_bgrad" else 2
 
     sets = []
     for i in range(n_sets):
         A = A0 if i == 0 else A0.clone()
         B = B0 if i == 0 else B0.clone()
-        bias = bias0 if i == 0 else bias0.clone()
+        x = x0 if i == 0 else x0.clone()
         D = torch.empty((wl.m, wl.n), dtype=out_t, device=dev)
-        aux = torch.empty((aux_words,), dtype=torch.int32, device=dev) if aux_words else None
-        sets.append((A, B, bias, D, aux))
+        sets.append((A, B, x, D, new_y()))
     plan = g.Plan(wl.m, wl.n, wl.k, wl.dtype, wl.epilogue, wl.bias_axis, wl.b_layout,
                   kernel=args.kernel, block_n=args.block_n, stream_k=args.stream_k)
+    run = plan.run_bwd if bwd else plan.run
     if wl.dtype == "e4m3":
         plan.set_scales(torch.tensor([prob.scale_a], dtype=torch.float32, device=dev),
                         torch.tensor([prob.scale_b], dtype=torch.float32, device=dev))
@@ -322,13 +364,13 @@ def main(argv=None):
 
     # first call (tensor-map encode) timed apart from the steady state
     t0 = time.perf_counter()
-    plan.run(*sets[0], stream=stream)
+    run(*sets[0], stream=stream)
     torch.cuda.synchronize(dev)
     first_call_ms = 1000 * (time.perf_counter() - t0)
     plan.check(stream)
 
     for i in range(args.warmup):
-        plan.run(*sets[i % n_sets], stream=stream)
+        run(*sets[i % n_sets], stream=stream)
     torch.cuda.synchronize(dev)
     plan.check(stream)
     if sampler:
@@ -343,7 +385,7 @@ def main(argv=None):
         with torch.cuda.graph(graph):
             cs = torch.cuda.current_stream(dev)
             for i in range(count):
-                plan.run(*sets[i % n_sets], stream=cs, fused=fused)
+                run(*sets[i % n_sets], stream=cs, fused=fused)
         return graph
 
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -374,7 +416,7 @@ def main(argv=None):
         start.record(stream)
         for i in range(K):
             ev[i][0].record(stream)
-            plan.run(*sets[i % n_sets], stream=stream)
+            run(*sets[i % n_sets], stream=stream)
             ev[i][1].record(stream)
         end.record(stream)
         torch.cuda.synchronize(dev)
@@ -407,13 +449,15 @@ def main(argv=None):
                 "peak_source": peak_src + (", bf16 burst x nominal fp8/bf16 ratio 2"
                                            if wl.dtype == "e4m3" else ", bf16 burst")}
     roof["kernel_source"] = khash
+    if launches > 1:
+        roof["note"] = "per-step time: the GEMM launch plus the dbias reduction launch"
 
     # ---- the library's own unfused path (bare GEMM, then the elementwise kernel)
     unfused = None
     if not args.no_unfused and wl.epilogue != "none":
         Ku = min(K, 200)
         for i in range(3):
-            plan.run(*sets[i % n_sets], stream=stream, fused=False)
+            run(*sets[i % n_sets], stream=stream, fused=False)
         torch.cuda.synchronize(dev)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if use_graph:
@@ -426,13 +470,13 @@ def main(argv=None):
         else:
             s0.record(stream)
             for i in range(Ku):
-                plan.run(*sets[i % n_sets], stream=stream, fused=False)
+                run(*sets[i % n_sets], stream=stream, fused=False)
             s1.record(stream)
         torch.cuda.synchronize(dev)
         plan.check(stream)
         ums = replicas.max_over_ranks(s0.elapsed_time(s1), device=dev) / Ku
         unfused = {"ms_per_step": ums, "value": flops * world / (ums / 1000) / 1e12, "unit": "TFLOP/s",
-                   "steps": Ku, "launches_per_step": 2, "fused_speedup": ums / ms_per_step}
+                   "steps": Ku, "launches_per_step": launches_unfused, "fused_speedup": ums / ms_per_step}
 
     # ---- end to end through the public API with host buffers: every step copies its inputs
     # from pinned host memory and reads its result back; copies of neighbouring steps overlap
@@ -442,17 +486,15 @@ def main(argv=None):
         Ke = min(K, 50)
         hA = torch.empty(A0.shape, dtype=A0.dtype, pin_memory=True)
         hB = torch.empty(B0.shape, dtype=B0.dtype, pin_memory=True)
-        hbias = torch.empty(bias0.shape, dtype=bias0.dtype, pin_memory=True)
+        hx = torch.empty(x0.shape, dtype=x0.dtype, pin_memory=True)
         hA.copy_(A0)
         hB.copy_(B0)
-        hbias.copy_(bias0)
+        hx.copy_(x0)
         e_sets = [sets[0], sets[1] if n_sets > 1 else (
-            torch.empty_like(A0), torch.empty_like(B0), torch.empty_like(bias0),
-            torch.empty((wl.m, wl.n), dtype=out_t, device=dev),
-            torch.empty((aux_words,), dtype=torch.int32, device=dev) if aux_words else None)]
+            torch.empty_like(A0), torch.empty_like(B0), torch.empty_like(x0),
+            torch.empty((wl.m, wl.n), dtype=out_t, device=dev), new_y())]
         hD = [torch.empty((wl.m, wl.n), dtype=out_t, pin_memory=True) for _ in range(2)]
-        haux = [torch.empty((aux_words,), dtype=torch.int32, pin_memory=True) if aux_words else None
-                for _ in range(2)]
+        hy = [torch.empty(y_shape, dtype=y_dtype, pin_memory=True) if y_shape else None for _ in range(2)]
         h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_comp = [torch.cuda.Event() for _ in range(2)]
@@ -462,7 +504,7 @@ def main(argv=None):
             used = [False, False]
             for i in range(count):
                 j = i % 2
-                A, B, bias, D, aux = e_sets[j]
+                A, B, x, D, y = e_sets[j]
                 with torch.cuda.stream(h2d_s):
                     if i == 0 and t_start is not None:
                         t_start.record(h2d_s)
@@ -470,18 +512,18 @@ def main(argv=None):
                         h2d_s.wait_event(ev_comp[j])      # step i-2 has finished reading set j
                     A.copy_(hA, non_blocking=True)
                     B.copy_(hB, non_blocking=True)
-                    bias.copy_(hbias, non_blocking=True)
+                    x.copy_(hx, non_blocking=True)
                     ev_in[j].record(h2d_s)
                 stream.wait_event(ev_in[j])
                 if used[j]:
                     stream.wait_event(ev_out[j])          # step i-2's result has been read back
-                plan.run(A, B, bias, D, aux, stream=stream)
+                run(A, B, x, D, y, stream=stream)
                 ev_comp[j].record(stream)
                 with torch.cuda.stream(d2h_s):
                     d2h_s.wait_event(ev_comp[j])
                     hD[j].copy_(D, non_blocking=True)
-                    if aux is not None:
-                        haux[j].copy_(aux, non_blocking=True)
+                    if y is not None:
+                        hy[j].copy_(y, non_blocking=True)
                     ev_out[j].record(d2h_s)
                 used[j] = True
             if t_end is not None:
@@ -498,7 +540,8 @@ def main(argv=None):
         e2e = {"value": flops * world / (ems / 1000) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(out_bytes),
                "ms_per_step": ems, "steps": Ke,
-               "api": "gemm_epi_run (C ABI) with pinned host buffers; H2D, compute and D2H of "
+               "api": f"{'gemm_epi_run_bwd' if bwd else 'gemm_epi_run'} (C ABI) with pinned host buffers; "
+                      "H2D, compute and D2H of "
                       "neighbouring steps overlap on three streams"}
 
     # ---- context only: the vendor library's bare GEMM (no bias, no activation) at this shape
@@ -550,10 +593,11 @@ def main(argv=None):
                               f"one set of {set_bytes / 2**20:.0f} MiB > 126 MB L2"),
                        "plan": info, "first_call_ms": first_call_ms,
                        "launch": "CUDA graph of the K steps (one kernel launch each)" if use_graph
-                       else "direct launches"},
+                       else "direct launches",
+                       "pdl": os.environ.get("GEMM_EPI_PDL", "1")[:1] != "0"},
             "pct_of_peak": 100.0 * roof["frac"],
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "unfused": unfused,
-            "gpu_launches": K, "clocks": clocks,
+            "gpu_launches": K * launches, "clocks": clocks,
         }
         if cublas is not None:
             line["cublas_bare_gemm"] = cublas

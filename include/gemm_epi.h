@@ -31,6 +31,11 @@
  *     16 bytes: k and n multiples of 8 for 16-bit types, of 16 for e4m3.
  *   - Calls are asynchronous on the given stream (a cudaStream_t passed as
  *     void*, NULL = legacy default stream) and never synchronise.
+ *   - The GEMM kernels are launched with programmatic stream serialisation:
+ *     their launch and on-chip setup may overlap the previous kernel on the
+ *     stream, but they read and write no global memory before that kernel has
+ *     completed, so stream order is kept.  GEMM_EPI_PDL=0 in the environment
+ *     (read when a plan is created) launches them plainly.
  *   - On any error nothing is launched and a negative status is returned.
  */
 #ifndef GEMM_EPI_H
@@ -57,7 +62,18 @@ enum gemm_epi_dtype { GEMM_EPI_F16 = 0, GEMM_EPI_BF16 = 1, GEMM_EPI_E4M3 = 2 };
  *   RELU_AUX_BIAS  as RELU_BIAS, plus aux = sign mask of the ReLU input x
  *   GELU_BIAS      D = GELU(x) = 0.5 x (1 + erf(x / sqrt 2))
  *   TANH_BIAS      D = tanh(x)
- *   RELU, RELU_AUX, GELU, TANH: the same without a bias */
+ *   RELU, RELU_AUX, GELU, TANH: the same without a bias
+ * Backward epilogues (run with gemm_epi_run_bwd / gemm_epi_unfused_run_bwd only): the
+ * ReLU backward of a layer z = alpha*A.B + bias, y = relu(z), fed the aux mask that the
+ * forward RELU_AUX(_BIAS) wrote ([nvmath-fusion] paragraph 6: the mask is kept for the
+ * backward pass; paragraph 7: fusing dBias is the next step).  g = alpha*A.B is the
+ * incoming gradient (for example dY . W of the next layer):
+ *   DRELU          D = mask ? g : 0
+ *   DRELU_BGRAD    as DRELU, plus dbias = the sum of D over the axis the forward bias
+ *                  was broadcast along: ROW (bias length m): dbias[i] = sum_j D[i][j];
+ *                  COL (bias length n): dbias[j] = sum_i D[i][j].  The sums are taken in
+ *                  fp32 on the unrounded values of D, in an order fixed by the shapes
+ *                  (identical results from run to run), and rounded once to the bias type. */
 enum gemm_epi_epilogue {
     GEMM_EPI_NONE = 0,
     GEMM_EPI_BIAS = 1,
@@ -68,7 +84,9 @@ enum gemm_epi_epilogue {
     GEMM_EPI_RELU = 6,
     GEMM_EPI_RELU_AUX = 7,
     GEMM_EPI_GELU = 8,
-    GEMM_EPI_TANH = 9
+    GEMM_EPI_TANH = 9,
+    GEMM_EPI_DRELU = 10,
+    GEMM_EPI_DRELU_BGRAD = 11
 };
 
 /* Bias broadcast ([epilog-params] body paragraph 3; [nvmath-fusion] paragraph 5):
@@ -95,7 +113,8 @@ enum gemm_epi_status {
     GEMM_EPI_ERR_ARG = -1,          /* size <= 0, unknown enum, bad option, bad plan handle */
     GEMM_EPI_ERR_ALIGN = -2,        /* pointer not 16-byte aligned, or row pitch not a multiple of 16 B */
     GEMM_EPI_ERR_NULL = -3,         /* required pointer NULL (A, B, D; bias for a bias epilogue;
-                                       aux for RELU_AUX_BIAS; scales unset for E4M3) */
+                                       aux for RELU_AUX(_BIAS) and the backward epilogues; dbias
+                                       for DRELU_BGRAD; scales unset for E4M3) */
     GEMM_EPI_ERR_UNSUPPORTED = -4,  /* valid request this build cannot serve (option combination) */
     GEMM_EPI_ERR_CUDA = -5,         /* a CUDA runtime/driver call failed (launch, tensor map) */
     GEMM_EPI_ERR_TIMEOUT = -6,      /* a kernel gave up on a bounded wait (reported by check()) */
@@ -105,14 +124,17 @@ enum gemm_epi_status {
 /* Opaque plan.  Created by gemm_epi_plan*, owned by the caller until
  * gemm_epi_free; holds host metadata, a tensor-map cache, one 256-byte
  * device status word and, when the plan uses stream-K, a workspace for
- * partial tiles plus their flags.  A plan may be run any number of times, on any stream,
+ * partial tiles plus their flags; a DRELU_BGRAD plan also owns an fp32 workspace for
+ * the bias-gradient partial sums (ROW: m x ceil(n/block_n) floats; COL: n x
+ * ceil(m/32) floats).  A plan may be run any number of times, on any stream,
  * from one host thread at a time. */
 typedef struct gemm_epi_plan_s *gemm_epi_plan_t;
 
 /* Optional tuning knobs; zero-initialise for automatic choices. */
 typedef struct gemm_epi_options {
     int32_t kernel;    /* enum gemm_epi_kernel                                        */
-    int32_t block_n;   /* output tile width (128 or 256; 0 = auto)                    */
+    int32_t block_n;   /* output tile width (128 or 256; 0 = auto).  TC2 with e4m3 and B
+                          stored (k, n) supports 256 only (128 is ERR_UNSUPPORTED)      */
     int32_t split_k;   /* SPLITK: CTAs per cluster along k (1..8; 0 = auto).  TC1/TC2:
                           cap on the parts a tail tile is split into (0 = 2)          */
     int32_t max_ctas;  /* persistent kernels: cap on resident CTAs (0 = one per SM)    */
@@ -192,6 +214,32 @@ int gemm_epi_run(gemm_epi_plan_t plan, const void *A, const void *B, const void 
 int gemm_epi_unfused_run(gemm_epi_plan_t plan, const void *A, const void *B, const void *bias,
                          void *D, uint32_t *aux, void *stream);
 
+/* Enqueue a backward plan (epilogue DRELU or DRELU_BGRAD).
+ *   A, B   operands of g = alpha*A.B (as for gemm_epi_run).
+ *   aux    the forward pass's packed mask for the (m, n) output, read only: row-major
+ *          uint32 words, row pitch gemm_epi_aux_pitch_bytes(n), bit b of word w in row i
+ *          for element (i, 32w + b) -- the layout gemm_epi_run writes.  Bits past
+ *          column n-1 are ignored.
+ *   D      (m, n) output in the output type: D = mask ? alpha*A.B : 0.
+ *   dbias  DRELU_BGRAD: output, length m (ROW plan) or n (COL plan), bias type (fp16 for
+ *          F16, bf16 for BF16 and E4M3).  DRELU: ignored (may be NULL).
+ * Fused: one GEMM launch whose epilogue applies the mask, writes D once and (BGRAD)
+ * writes fp32 partial sums of each tile to the plan's workspace, then one small launch
+ * that adds the partials in a fixed order and writes dbias.  Every pointer is a 16-byte
+ * aligned device pointer.  Returns OK, ERR_ARG (bad handle, or a forward plan),
+ * ERR_NULL, ERR_ALIGN or ERR_CUDA; gemm_epi_run with a backward plan returns ERR_ARG.
+ * The small-m split-K kernel has no backward epilogue: AUTO plans use TC1 there, and a
+ * plan that forces GEMM_EPI_KERNEL_SPLITK fails with ERR_UNSUPPORTED. */
+int gemm_epi_run_bwd(gemm_epi_plan_t plan, const void *A, const void *B, const uint32_t *aux, void *D,
+                     void *dbias, void *stream);
+
+/* The UNFUSED baseline of gemm_epi_run_bwd on the same plan and arguments: the bare
+ * GEMM writes alpha*A.B to D, an elementwise kernel reads D back and zeroes it where
+ * the mask is 0, and (BGRAD) a third kernel reads D again and sums it along the bias
+ * axis (so dbias here adds values already rounded to the output type). */
+int gemm_epi_unfused_run_bwd(gemm_epi_plan_t plan, const void *A, const void *B, const uint32_t *aux,
+                             void *D, void *dbias, void *stream);
+
 /* Synchronise `stream`, read and clear the plan's device status word.
  * Returns OK, ERR_TIMEOUT (some kernel of this plan gave up waiting since the
  * last check), ERR_CUDA (a sticky CUDA error) or ERR_ARG. */
@@ -208,7 +256,8 @@ int gemm_epi_plan_query(gemm_epi_plan_t plan, gemm_epi_plan_info *info);
  * callers cannot create a plan (a plan allocates its status word), so this
  * call takes the problem description and the buffers directly and computes
  * exactly what gemm_epi_plan_ex + gemm_epi_run would (same kernels, same
- * automatic kernel choice, same argument rules and errors).
+ * automatic kernel choice, same argument rules and errors).  Forward epilogues
+ * only (NONE .. TANH); the backward ones return GEMM_EPI_ERR_ARG.
  *
  * Arguments: as gemm_epi_plan_ex and gemm_epi_run; d_scale_a/d_scale_b as in
  * gemm_epi_set_scales (E4M3 only, else ignored).  wait = 0: enqueue and

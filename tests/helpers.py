@@ -68,3 +68,9 @@ def aux_padding_bits(words: np.ndarray, m: int, n: int) -> int:
     w = np.ascontiguousarray(words, dtype=np.uint32).reshape(m, pitch)
     bits = np.unpackbits(w.view(np.uint8).reshape(m, pitch * 4), axis=1, bitorder="little")
     return int(bits[:, n:].sum())
+
+
+def pack_aux(mask: np.ndarray, pad_fill: int = 0) -> np.ndarray:
+    """(m, n) 0/1 array -> library aux layout (the seeded-input module's packer)."""
+    from activation_epilogue_tcgen05_b200.workloads import pack_mask
+    return pack_mask(mask, pad_fill)

@@ -75,7 +75,7 @@ def test_plan_rejects_bad_sizes(g, args):
     assert _plan_rc(g, *args) == g.ERR_ARG
 
 
-@pytest.mark.parametrize("kw", [dict(dt=3), dict(dt=-1), dict(epi=10), dict(epi=-1), dict(axis=2),
+@pytest.mark.parametrize("kw", [dict(dt=3), dict(dt=-1), dict(epi=12), dict(epi=-1), dict(axis=2),
                                 dict(layout=2)])
 def test_plan_rejects_bad_enums(g, kw):
     assert _plan_rc(g, 64, 64, 64, **kw) == g.ERR_ARG
@@ -146,3 +146,22 @@ def test_product_does_not_import_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text
                 assert "gemm_epi_oracle" not in text and "libgemm_epi_oracle" not in text
+
+
+def test_backward_entry_points_reject_bad_handles(g):
+    for fn in (g.lib().gemm_epi_run_bwd, g.lib().gemm_epi_unfused_run_bwd):
+        assert fn(None, None, None, None, None, None, None) == g.ERR_ARG
+        assert fn(ctypes.c_void_p(0x1000), None, None, None, None, None, None) == g.ERR_ARG
+
+
+@pytest.mark.parametrize("epi", [10, 11])
+def test_backward_epilogues_are_valid_enums(g, epi):
+    # accepted as enums: without a device the plan stops at the device check
+    assert _plan_rc(g, 64, 64, 64, epi=epi) == g.ERR_NO_DEVICE
+
+
+@pytest.mark.parametrize("epi", [10, 11])
+def test_noalloc_refuses_backward_epilogues(g, epi):
+    rc = g.lib().gemm_epi_run_noalloc(64, 64, 64, 1, epi, 0, 0, None, None, None, None, None, None, None,
+                                      0, None)
+    assert rc == g.ERR_ARG

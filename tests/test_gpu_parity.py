@@ -304,6 +304,69 @@ def test_non_default_stream():
     compare(wl, D.cpu(), None, ref, pre, mask, *sigmas(prob))
 
 
+@pytest.mark.parametrize("kernel2", ["tc1", "tc2", "splitk"])
+@pytest.mark.parametrize("graph", [False, True])
+def test_dependent_launches_keep_stream_order(kernel2, graph):
+    """Back-to-back launches on one stream, each allowed to start before the previous one
+    ends (programmatic dependent launch): the consumer must read the producer's output
+    (read after write) and the producer's next launch must not overwrite it before the
+    consumer has read it (write after read).  Producer: H = GELU(X.W1 + b1); consumer:
+    Y = A2.H (H as the (k, n) operand).  Expected values: the oracle chain (the oracle's
+    H rounded to f16, fed to the oracle again)."""
+    m1, n1, k1 = 512, 256, 1024
+    m2 = 48 if kernel2 == "splitk" else 384
+    wl1 = Workload("pdl_h", m1, n1, k1, "f16", "gelu_bias", "col", "kn", seed=40)
+    wl1b = wl1.with_(seed=41)
+    wl2 = Workload("pdl_y", m2, n1, m1, "f16", "none", "row", "kn", seed=42)
+    p1, p1b, p2 = make_problem(wl1), make_problem(wl1b), make_problem(wl2)
+    X, W1, b1 = device_inputs(p1)
+    Xb, W1b, b1b = device_inputs(p1b)
+    A2 = p2.A.cuda()
+    H = torch.full((m1, n1), float("nan"), dtype=torch.float16, device="cuda")
+    Y = torch.full((m2, n1), float("nan"), dtype=torch.float16, device="cuda")
+    plan1 = make_plan(wl1, p1, kernel="tc1")
+    plan2 = make_plan(wl2, p2, kernel=kernel2)
+    s = torch.cuda.Stream()
+    try:
+        def chain():
+            plan1.run(X, W1, b1, H, None, stream=s)          # producer
+            plan2.run(A2, H, None, Y, None, stream=s)        # consumer of H
+            plan1.run(Xb, W1b, b1b, H, None, stream=s)       # overwrites H after the read
+        with torch.cuda.stream(s):
+            chain()                                           # also encodes the tensor maps
+            s.synchronize()
+            if graph:
+                g_ = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g_, stream=s):
+                    chain()
+                H.fill_(float("nan"))
+                Y.fill_(float("nan"))
+                s.synchronize()
+                for _ in range(3):
+                    g_.replay()
+            else:
+                for _ in range(3):
+                    H.fill_(float("nan"))
+                    Y.fill_(float("nan"))
+                    chain()
+        s.synchronize()
+        plan1.check(stream=s)
+        plan2.check(stream=s)
+    finally:
+        plan1.close()
+        plan2.close()
+    h_ref, _, _ = oracle_full(wl1, p1)
+    hb_ref, hb_pre, hb_mask = oracle_full(wl1b, p1b)
+    # the consumer saw the first producer's H
+    h16 = torch.tensor(h_ref, dtype=torch.float64).to(torch.float16)
+    y_ref, y_pre, y_mask = oracle.gemm_epi(storage(p2.A), storage(h16), None, dtype="f16", epilogue="none")
+    sa = float(p2.A.double().std(unbiased=False))
+    sb = float(h16.double().std(unbiased=False))
+    compare(wl2, Y.cpu(), None, y_ref, y_pre, y_mask, sa, sb)
+    # and H holds the second producer's result
+    compare(wl1b, H.cpu(), None, hb_ref, hb_pre, hb_mask, *sigmas(p1b))
+
+
 # ------------------------------------------------------------------ errors and failure paths
 def test_run_argument_errors():
     wl = Workload("err", 128, 128, 128, "bf16", "relu_aux_bias", "row", "kn")
