@@ -74,6 +74,14 @@ def _load():
             lib.oracle_gemm_epi_bwd.argtypes = [i64, i64, i64, cp, cp, cp, cp, vp, vp, vp, dp, dp,
                                                 vp, vp]
             lib.oracle_gemm_epi_bwd.restype = ctypes.c_int
+            lib.oracle_encode_e4m3.argtypes = [dp]
+            lib.oracle_encode_e4m3.restype = ctypes.c_uint8
+            lib.oracle_encode_f16.argtypes = [dp]
+            lib.oracle_encode_f16.restype = ctypes.c_uint16
+            lib.oracle_encode_bf16.argtypes = [dp]
+            lib.oracle_encode_bf16.restype = ctypes.c_uint16
+            lib.oracle_encode.argtypes = [i64, cp, vp, dp, vp]
+            lib.oracle_encode.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -208,3 +216,45 @@ def threads() -> int:
     if env and env.isdigit():
         return int(env)
     return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
+def encode(x, dtype: str, scale: float = 1.0):
+    """Storage codes of x / scale in `dtype` (uint8 for e4m3, uint16 bit patterns for fp16 /
+    bf16): round to nearest even from the format definitions, e4m3 saturating at +-448.
+
+    The MLP block's intermediate stored in a narrower type ("nvmath-python cuBLASLt bias
+    fusion for PyTorch inference", paragraphs 1 and 5; "PyTorch 2.14 NVGEMM epilogue
+    fusion", section "why epilogue fusion matters": scaling and type conversion)."""
+    if dtype not in DTYPES:
+        raise ValueError(f"unknown dtype {dtype}")
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape, np.uint8 if dtype == "e4m3" else np.uint16)
+    rc = _load().oracle_encode(x.size, dtype.encode(), _ptr(x), float(scale), _ptr(out))
+    if rc != 0:
+        raise RuntimeError(f"oracle_encode failed with status {rc}")
+    return out
+
+
+def mlp(X, W1, b1, W2, b2, *, dtype: str, act: str = "gelu_bias", w_layout: str = "kn",
+        scale_x: float = 1.0, scale_w1: float = 1.0, scale_h: float = 1.0, scale_w2: float = 1.0):
+    """MLP block ("nvmath-python cuBLASLt bias fusion for PyTorch inference", paragraph 1):
+
+        H = act(scale_x*scale_w1 * X.W1 + b1)          (bias along the d_ff columns)
+        Hs = encode(H / scale_h) in the storage type    (e4m3: the per-tensor requantisation)
+        Y = scale_h*scale_w2 * decode(Hs).W2 + b2       (bias along the d_model columns)
+
+    For fp16 / bf16, scale_h is 1 and Hs is H rounded to that type.  X is (m, d_model); W1
+    is (d_model, d_ff) for w_layout "kn" or (d_ff, d_model) for "nk" (an nn.Linear weight);
+    W2 likewise (d_ff, d_model) or (d_model, d_ff).
+
+    Returns (Y, H, Hs, amax) with Y and H in float64 (H before encoding), Hs the stored
+    codes, and amax = max |H|."""
+    if dtype != "e4m3" and scale_h != 1.0:
+        raise ValueError("scale_h applies to e4m3 only")
+    H, _, _ = gemm_epi(X, W1, b1, dtype=dtype, epilogue=act, bias_axis="col", b_layout=w_layout,
+                       scale_a=scale_x, scale_b=scale_w1)
+    amax = float(np.abs(H).max())
+    Hs = encode(H, dtype, scale_h)
+    Y, _, _ = gemm_epi(Hs, W2, b2, dtype=dtype, epilogue="bias", bias_axis="col", b_layout=w_layout,
+                       scale_a=scale_h, scale_b=scale_w2)
+    return Y, H, Hs, amax

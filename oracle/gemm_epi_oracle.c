@@ -355,3 +355,83 @@ int oracle_gemm_epi_bwd(int64_t m, int64_t n, int64_t k, const char *dtype, cons
     }
     return 0;
 }
+
+/*
+ * Encoding a real value into a storage format (the inverse of the decoders
+ * above), for results that are stored in a narrower type: the intermediate H
+ * of an MLP block (up-projection, then down-projection; "nvmath-python
+ * cuBLASLt bias fusion for PyTorch inference" (blog.hotdry.top), paragraph 1:
+ * the MLP is where the GEMM + bias time goes) and its FP8 form (paragraph 5:
+ * FP8 inputs; "PyTorch 2.14 NVGEMM epilogue fusion" (zdabc.icu), section "why
+ * epilogue fusion matters": scaling and type conversion in the epilogue).
+ *
+ * Written from the formats' definitions only: the non-negative finite codes
+ * 0 .. max_code of each format decode (with the decoders above) to strictly
+ * increasing values, so |x| is located between two neighbouring codes by
+ * bisection and rounded to the nearer; a tie goes to the code whose last
+ * fraction bit is 0 (round to nearest, ties to even).  Beyond the largest
+ * finite value, e4m3 saturates to it (+-448); fp16 and bf16 round to
+ * infinity once |x| reaches the largest finite value plus half its spacing.
+ * The sign bit is copied from x (so -0.0 and tiny negatives give -0).
+ */
+static double decode_code(int dt, uint32_t c) {
+    switch (dt) {
+    case OR_F16: return oracle_decode_f16((uint16_t)c);
+    case OR_BF16: return oracle_decode_bf16((uint16_t)c);
+    case OR_E4M3: return oracle_decode_e4m3((uint8_t)c);
+    }
+    return NAN;
+}
+
+static uint32_t encode_value(int dt, double x) {
+    const uint32_t max_code = dt == OR_E4M3 ? 0x7Eu : dt == OR_F16 ? 0x7BFFu : 0x7F7Fu;
+    const uint32_t inf_code = dt == OR_F16 ? 0x7C00u : 0x7F80u;     /* 16-bit formats only */
+    const uint32_t sign_bit = dt == OR_E4M3 ? 0x80u : 0x8000u;
+    const int neg = signbit(x) != 0;
+    const double a = fabs(x);
+    const double vmax = decode_code(dt, max_code);
+    uint32_t code;
+    if (!(a < vmax)) {
+        if (dt == OR_E4M3) {
+            code = max_code;
+        } else {
+            /* half the spacing below the largest finite value equals half the spacing above it */
+            const double half = 0.5 * (vmax - decode_code(dt, max_code - 1));
+            code = a < vmax + half ? max_code : inf_code;
+        }
+    } else {
+        uint32_t lo = 0, hi = max_code;         /* decode(lo) <= a < decode(hi) */
+        while (hi - lo > 1) {
+            const uint32_t mid = lo + (hi - lo) / 2;
+            if (decode_code(dt, mid) <= a) lo = mid;
+            else hi = mid;
+        }
+        const double dl = a - decode_code(dt, lo), dh = decode_code(dt, hi) - a;
+        if (dl < dh) code = lo;
+        else if (dh < dl) code = hi;
+        else code = (lo & 1u) ? hi : lo;
+    }
+    return neg ? (code | sign_bit) : code;
+}
+
+uint8_t oracle_encode_e4m3(double x) { return (uint8_t)encode_value(OR_E4M3, x); }
+uint16_t oracle_encode_f16(double x) { return (uint16_t)encode_value(OR_F16, x); }
+uint16_t oracle_encode_bf16(double x) { return (uint16_t)encode_value(OR_BF16, x); }
+
+/*
+ * codes[i] = encode(x[i] / scale) in `dtype` storage (uint8 for e4m3, uint16
+ * otherwise): the per-tensor quantisation of the MLP block's intermediate,
+ * scale > 0 (s = amax / 448 is the usual choice for e4m3; 1 stores the values
+ * themselves).  Returns 0, or -1 on a bad argument.
+ */
+int oracle_encode(int64_t count, const char *dtype, const double *x, double scale, void *codes) {
+    const int dt = dtype_code(dtype);
+    if (!dt || count < 0 || !x || !codes || !(scale > 0.0)) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; ++i) {
+        const uint32_t c = encode_value(dt, x[i] / scale);
+        if (dt == OR_E4M3) ((uint8_t *)codes)[i] = (uint8_t)c;
+        else ((uint16_t *)codes)[i] = (uint16_t)c;
+    }
+    return 0;
+}

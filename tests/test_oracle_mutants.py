@@ -47,6 +47,13 @@ MUTANTS = [
      "D_ref[i * n + j] = mask[i * n + j] ? 0.0 : alpha * row[j];", None),
     ("bwd_alpha_dropped", "D_ref[i * n + j] = mask[i * n + j] ? alpha * row[j] : 0.0;",
      "D_ref[i * n + j] = mask[i * n + j] ? row[j] : 0.0;", None),
+    ("encode_ties_up", "else code = (lo & 1u) ? hi : lo;", "else code = hi;", None),
+    ("encode_truncates", "if (dl < dh) code = lo;", "if (1) code = lo;", None),
+    ("encode_no_saturation", "code = max_code;\n        } else {", "code = 0x7Fu;\n        } else {", None),
+    ("encode_sign_dropped", "return neg ? (code | sign_bit) : code;", "return code;", None),
+    ("encode_scale_multiplies", "encode_value(dt, x[i] / scale)", "encode_value(dt, x[i] * scale)", None),
+    ("encode_f16_overflow_early", "code = a < vmax + half ? max_code : inf_code;",
+     "code = a < vmax ? max_code : inf_code;", None),
     ("bwd_bgrad_wrong_axis", "if (axis == OR_ROW) {\n            for (int64_t i = 0; i < m; ++i) {\n                double s",
      "if (axis != OR_ROW) {\n            for (int64_t i = 0; i < m; ++i) {\n                double s", None),
 ]

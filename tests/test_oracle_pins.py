@@ -388,3 +388,122 @@ def test_backward_mask_extremes(oracle_lib):
     D0, db0 = oracle_lib.gemm_epi_bwd(A, B, 0 * ones, dtype="f16", epilogue="drelu_bgrad",
                                       bias_axis="col")
     assert (D0 == 0).all() and (db0 == 0).all()
+
+
+# ----------------------------------------------------------------------------- encoders (MLP block)
+def _all_finite_codes(dtype):
+    if dtype == "e4m3":
+        c = np.arange(256, dtype=np.uint32)
+        return c[(c & 0x7F) != 0x7F]
+    c = np.arange(65536, dtype=np.uint32)
+    exp_all_ones = ((c >> 10) & 0x1F) == 0x1F if dtype == "f16" else ((c >> 7) & 0xFF) == 0xFF
+    return c[~exp_all_ones]
+
+
+@pytest.mark.parametrize("dtype", ["e4m3", "f16", "bf16"])
+def test_encode_inverts_decode_on_every_finite_code(oracle_lib, dtype):
+    codes = _all_finite_codes(dtype)
+    store = codes.astype(np.uint8 if dtype == "e4m3" else np.uint16)
+    vals = oracle_lib.decode(store, dtype)
+    np.testing.assert_array_equal(oracle_lib.encode(vals, dtype), store)
+
+
+@pytest.mark.parametrize("dtype", ["e4m3", "f16", "bf16"])
+def test_encode_midpoints_tie_to_even_and_neighbours_round_to_nearest(oracle_lib, dtype):
+    """Between every pair of neighbouring non-negative codes (e4m3: all of them; 16-bit:
+    a seeded sample plus the subnormal/normal seam and the top of the range)."""
+    top = {"e4m3": 0x7E, "f16": 0x7BFF, "bf16": 0x7F7F}[dtype]
+    if dtype == "e4m3":
+        lo = np.arange(0, top, dtype=np.int64)
+    else:
+        rng = np.random.default_rng(5)
+        seam = {"f16": 0x0400, "bf16": 0x0080}[dtype]
+        lo = np.unique(np.concatenate([rng.integers(0, top, 3000), [0, 1, seam - 1, seam, top - 1]]))
+    st = np.uint8 if dtype == "e4m3" else np.uint16
+    a = oracle_lib.decode(lo.astype(st), dtype)
+    b = oracle_lib.decode((lo + 1).astype(st), dtype)
+    mid = 0.5 * (a + b)
+    even = np.where(lo % 2 == 0, lo, lo + 1)
+    np.testing.assert_array_equal(oracle_lib.encode(mid, dtype), even.astype(st))
+    np.testing.assert_array_equal(oracle_lib.encode(-mid, dtype),
+                                  (even | (0x80 if dtype == "e4m3" else 0x8000)).astype(st))
+    eps = (b - a) * 1e-3
+    np.testing.assert_array_equal(oracle_lib.encode(mid - eps, dtype), lo.astype(st))
+    np.testing.assert_array_equal(oracle_lib.encode(mid + eps, dtype), (lo + 1).astype(st))
+
+
+def test_encode_f16_matches_numpy_rounding(oracle_lib):
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal(20000) * np.exp2(rng.integers(-26, 16, 20000))
+    x = x[np.abs(x) < 65504]
+    np.testing.assert_array_equal(oracle_lib.encode(x, "f16"), x.astype(np.float16).view(np.uint16))
+
+
+def test_encode_bf16_and_e4m3_match_torch_rounding(oracle_lib):
+    """fp32 inputs (so the library casts round once): bf16 everywhere, e4m3 inside +-448."""
+    gen = torch.Generator().manual_seed(7)
+    x = torch.randn(20000, generator=gen) * torch.exp2(torch.randint(-20, 20, (20000,), generator=gen).float())
+    bf = x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(oracle_lib.encode(x.double().numpy(), "bf16"), bf)
+    y = (torch.rand(20000, generator=gen) * 2 - 1) * 448 * torch.exp2(-torch.randint(0, 14, (20000,), generator=gen).float())
+    e = y.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(oracle_lib.encode(y.double().numpy(), "e4m3"), e)
+
+
+def test_encode_saturation_and_overflow(oracle_lib):
+    np.testing.assert_array_equal(oracle_lib.encode([448.0, 464.0, 480.0, 1e6, -1e6, -449.0], "e4m3"),
+                                  np.array([0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE], np.uint8))
+    # fp16: the largest finite value is 65504 with spacing 32, so 65520 rounds to infinity
+    np.testing.assert_array_equal(oracle_lib.encode([65504.0, 65519.0, 65520.0, -70000.0], "f16"),
+                                  np.array([0x7BFF, 0x7BFF, 0x7C00, 0xFC00], np.uint16))
+    np.testing.assert_array_equal(oracle_lib.encode([0.0, -0.0, -1e-9], "e4m3"),
+                                  np.array([0x00, 0x80, 0x80], np.uint8))
+
+
+def test_encode_applies_the_scale(oracle_lib):
+    # 8.5 / 0.25 = 34 -> e4m3 spacing 4 in [32, 64): 34 is halfway between 32 (0x60) and 36 (0x61)
+    np.testing.assert_array_equal(oracle_lib.encode([8.5, 8.0, -9.0], "e4m3", 0.25),
+                                  np.array([0x60, 0x60, 0xE1], np.uint8))
+
+
+MLP = load_golden("tiny_cases.json")["cases_mlp"]
+
+
+@pytest.mark.parametrize("c", MLP, ids=[c["id"] for c in MLP])
+def test_golden_mlp_case(oracle_lib, c):
+    dt = c["dtype"]
+    bdt = "bf16" if dt == "e4m3" else dt
+    args = [to_storage_values(c["x"], dt), to_storage_values(c["w1"], dt), to_storage_values(c["b1"], bdt),
+            to_storage_values(c["w2"], dt), to_storage_values(c["b2"], bdt)]
+    Y, H, Hs, amax = oracle_lib.mlp(*args, dtype=dt, act=c["act"], w_layout=c["w_layout"],
+                                    scale_x=c["scale_x"], scale_w1=c["scale_w1"], scale_h=c["scale_h"],
+                                    scale_w2=c["scale_w2"])
+    np.testing.assert_allclose(H, np.array(c["h"]), rtol=1e-15, atol=0)
+    np.testing.assert_array_equal(Hs, np.array(c["h_codes"]))
+    assert amax == pytest.approx(c["amax"], rel=1e-15, abs=0)
+    np.testing.assert_array_equal(Y, np.array(c["y"]))
+
+
+@pytest.mark.parametrize("layout", ["kn", "nk"])
+def test_mlp_equals_two_numpy_products(oracle_lib, layout):
+    """16-bit MLP: H from the GELU of the first product, rounded to fp16 by numpy, then the
+    second product by numpy matmul (with exactly representable integer weights)."""
+    rng = np.random.default_rng(8)
+    m, d, f = 5, 16, 24
+    X = rng.integers(-2, 3, (m, d)).astype(np.float16)
+    W1 = rng.integers(-2, 3, (d, f)).astype(np.float16)
+    b1 = (rng.integers(-4, 5, f) / 4).astype(np.float16)
+    W2 = rng.integers(-2, 3, (f, d)).astype(np.float16)
+    b2 = (rng.integers(-4, 5, d) / 4).astype(np.float16)
+    w1s = W1 if layout == "kn" else np.ascontiguousarray(W1.T)
+    w2s = W2 if layout == "kn" else np.ascontiguousarray(W2.T)
+    v = lambda a: a.view(np.uint16)
+    Y, H, Hs, amax = oracle_lib.mlp(v(X), v(w1s), v(b1), v(w2s), v(b2), dtype="f16", act="gelu_bias",
+                                    w_layout=layout)
+    p = X.astype(np.float64) @ W1.astype(np.float64) + b1.astype(np.float64)
+    gelu = np.vectorize(lambda t: 0.5 * t * (1 + math.erf(t / math.sqrt(2))))
+    np.testing.assert_allclose(H, gelu(p), rtol=1e-14, atol=1e-15)
+    np.testing.assert_array_equal(Hs, H.astype(np.float16).view(np.uint16))
+    assert amax == np.abs(H).max()
+    want = Hs.view(np.float16).astype(np.float64) @ W2.astype(np.float64) + b2.astype(np.float64)
+    np.testing.assert_allclose(Y, want, rtol=1e-14, atol=1e-14)
