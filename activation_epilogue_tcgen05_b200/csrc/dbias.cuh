@@ -36,18 +36,35 @@ __device__ __forceinline__ void store_out(void *out, int64_t i, float v) {
     else reinterpret_cast<__nv_bfloat16 *>(out)[i] = __float2bfloat16_rn(v);
 }
 
-// Block: 32 consecutive outputs x 8 part-strides.  Thread (x, y) sums parts
-// y, y + 8, y + 16, ... of output x; row y = 0 then adds the 8 strides in order.
-constexpr int SUM_PARTS_Y = 8;
+// Block: 32 consecutive outputs x SUM_PARTS_Y part-strides.  Thread (x, y) sums
+// parts y, y + Y, y + 2Y, ... of output x into four independent accumulators (so
+// four loads are in flight), combines them in a fixed order, and row y = 0 then adds
+// the Y strides in order: the result depends only on (parts, len).
+constexpr int SUM_PARTS_Y = 32;
 
 template <typename IN, int DT>
 __global__ void __launch_bounds__(32 * SUM_PARTS_Y) sum_parts_kernel(const IN *__restrict__ src, int64_t parts,
                                                                   int64_t len, void *out) {
     __shared__ float red[SUM_PARTS_Y][33];
+    // launched as a dependent of the kernel that wrote src: wait for it before reading;
+    // the next kernel (itself waiting before any global access) may then be scheduled
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t i = (int64_t)blockIdx.x * 32 + threadIdx.x;
     float s = 0.0f;
-    if (i < len)
-        for (int64_t p = threadIdx.y; p < parts; p += SUM_PARTS_Y) s += to_f32(__ldg(src + p * len + i));
+    if (i < len) {
+        constexpr int Y = SUM_PARTS_Y;
+        float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+        int64_t p = threadIdx.y;
+        for (; p + 3 * Y < parts; p += 4 * Y) {
+            s0 += to_f32(__ldg(src + p * len + i));
+            s1 += to_f32(__ldg(src + (p + Y) * len + i));
+            s2 += to_f32(__ldg(src + (p + 2 * Y) * len + i));
+            s3 += to_f32(__ldg(src + (p + 3 * Y) * len + i));
+        }
+        for (; p < parts; p += Y) s0 += to_f32(__ldg(src + p * len + i));
+        s = (s0 + s1) + (s2 + s3);
+    }
     red[threadIdx.y][threadIdx.x] = s;
     __syncthreads();
     if (threadIdx.y == 0 && i < len) {

@@ -34,6 +34,7 @@ struct Plan {
     int kepi;            // kernel epilogue (EPI_*): the activation
     bool has_bias;       // the public epilogue adds a bias
     bool bwd, bgrad;     // backward epilogue (DRELU*); with a bias gradient (DRELU_BGRAD)
+    bool qout;           // e4m3 output quantised in the epilogue (options.out_e4m3)
     gemm_epi_options opts;
     int device, num_sms;
     // kernel choice
@@ -59,6 +60,9 @@ struct Plan {
     KernelInfo info{};
     // FP8 scales (device pointers, borrowed)
     const float *scale_a = nullptr, *scale_b = nullptr;
+    // FP8 output: the output scale and the optional amax word (device pointers, borrowed)
+    const float *out_scale = nullptr;
+    float *amax = nullptr;
     // device status word (owned)
     unsigned int *status = nullptr;
     // tensor-map cache, keyed on the operand pointers
@@ -169,11 +173,12 @@ int choose(Plan *P) {
         const int64_t pair_tiles = ((m + 255) / 256) * ((n + 255) / 256);
         const int sms_auto = P->opts.max_ctas > 0 ? std::min(P->opts.max_ctas, P->num_sms) : P->num_sms;
         // (the split-K kernel has no backward epilogue)
-        if (m <= 64 && P->kepi != EPI_DRELU) kernel = GEMM_EPI_KERNEL_SPLITK;
+        if (m <= 64 && P->kepi != EPI_DRELU && !P->qout) kernel = GEMM_EPI_KERNEL_SPLITK;
         else if (pair_tiles >= sms_auto / 2) kernel = GEMM_EPI_KERNEL_TC2;
         else kernel = GEMM_EPI_KERNEL_TC1;
     }
-    if (kernel == GEMM_EPI_KERNEL_SPLITK && (m > 128 || P->kepi == EPI_DRELU)) return GEMM_EPI_ERR_UNSUPPORTED;
+    if (kernel == GEMM_EPI_KERNEL_SPLITK && (m > 128 || P->kepi == EPI_DRELU || P->qout))
+        return GEMM_EPI_ERR_UNSUPPORTED;
     P->kernel = kernel;
     const bool b_mn = P->b_layout == GEMM_EPI_B_KN;
     const int bk = 128 / esize(P->dtype);
@@ -245,13 +250,13 @@ int choose(Plan *P) {
             if (v >= 1 && v <= 64) P->group_m = v;
         }
         KernelInfo none_info;
-        if (!find_tc(cg, P->dtype, GEMM_EPI_NONE, 0, b_mn, bn, &P->tc_none_launch, &none_info))
+        if (!find_tc(cg, P->dtype, GEMM_EPI_NONE, 0, b_mn, bn, false, &P->tc_none_launch, &none_info))
             return GEMM_EPI_ERR_UNSUPPORTED;
-        if (!find_tc(cg, P->dtype, P->kepi, P->axis, b_mn, bn, &P->tc_launch, &P->info))
+        if (!find_tc(cg, P->dtype, P->kepi, P->axis, b_mn, bn, P->qout, &P->tc_launch, &P->info))
             return GEMM_EPI_ERR_UNSUPPORTED;
         P->split = 1;
     }
-    if (P->kepi != EPI_NONE && !find_bias_act(P->dtype, P->kepi, P->axis, &P->ba_launch))
+    if (P->kepi != EPI_NONE && !P->qout && !find_bias_act(P->dtype, P->kepi, P->axis, &P->ba_launch))
         return GEMM_EPI_ERR_UNSUPPORTED;
     return GEMM_EPI_OK;
 }
@@ -278,6 +283,7 @@ int check_run_args(Plan *P, const void *A, const void *B, const void *bias, void
     if (P->has_bias && !bias) return GEMM_EPI_ERR_NULL;
     if (P->kepi == EPI_RELU_AUX && !aux) return GEMM_EPI_ERR_NULL;
     if (P->dtype == GEMM_EPI_E4M3 && (!P->scale_a || !P->scale_b)) return GEMM_EPI_ERR_NULL;
+    if (P->qout && !P->out_scale) return GEMM_EPI_ERR_NULL;
     if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return GEMM_EPI_ERR_ALIGN;
     if (P->has_bias && !aligned16(bias)) return GEMM_EPI_ERR_ALIGN;
     if (P->kepi == EPI_RELU_AUX && !aligned16(aux)) return GEMM_EPI_ERR_ALIGN;
@@ -312,8 +318,10 @@ int ensure_maps(Plan *P, const void *A, const void *B, void *D) {
         ok = ok && make_map(&P->tmA, dt, A, k, m, bk, 128);
         ok = ok && (b_kn ? make_map(&P->tmB, dt, B, n, k, box_n, bk) : make_map(&P->tmB, dt, B, k, n, bk, bn_local));
         const int out_dt = dt == GEMM_EPI_E4M3 ? GEMM_EPI_BF16 : dt;
-        // the epilogue stages 32 rows x 32 outputs (64 bytes a row, 64-byte swizzle) per store
-        ok = ok && make_map(&P->tmD, out_dt, D, n, m, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+        if (P->qout)   // e4m3 output goes out with direct stores; the map is valid but unused
+            ok = ok && make_map(&P->tmD, GEMM_EPI_E4M3, D, n, m, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+        else           // the epilogue stages 32 rows x 32 outputs (64 bytes a row, 64-byte swizzle) per store
+            ok = ok && make_map(&P->tmD, out_dt, D, n, m, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
     }
     if (!ok) {
         P->maps_valid = false;
@@ -381,6 +389,9 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.flags = P->flags;
         L.p.trace = trace_buffer();
         L.p.dbias_ws = fused ? dbias_ws : nullptr;
+        L.p.dq = P->qout ? static_cast<uint8_t *>(D) : nullptr;
+        L.p.out_scale = P->out_scale;
+        L.p.amax = reinterpret_cast<unsigned int *>(P->amax);
         L.grid = P->grid;
         L.pdl = P->pdl;
         L.stream = stream;
@@ -406,6 +417,13 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     if (o.inject_stall != 0 && o.inject_stall != 1) return GEMM_EPI_ERR_ARG;
     if (o.stream_k < 0 || o.stream_k > 2) return GEMM_EPI_ERR_ARG;
     if (o.inject_stall && o.kernel == GEMM_EPI_KERNEL_SPLITK) return GEMM_EPI_ERR_UNSUPPORTED;
+    if (o.out_e4m3 != 0 && o.out_e4m3 != 1) return GEMM_EPI_ERR_ARG;
+    if (o.out_e4m3) {
+        // FP8 output: e4m3 operands, forward epilogues without a mask or tanh, persistent kernels
+        const bool epi_ok = epilogue == GEMM_EPI_NONE || epilogue == GEMM_EPI_BIAS || epilogue == GEMM_EPI_RELU_BIAS ||
+                            epilogue == GEMM_EPI_GELU_BIAS || epilogue == GEMM_EPI_RELU || epilogue == GEMM_EPI_GELU;
+        if (dtype != GEMM_EPI_E4M3 || !epi_ok || o.kernel == GEMM_EPI_KERNEL_SPLITK) return GEMM_EPI_ERR_UNSUPPORTED;
+    }
     // 16-byte row pitches (TMA strides; the pages' 16-byte alignment rule)
     const int es = esize(dtype);
     const int out_es = 2;
@@ -434,6 +452,7 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     P->has_bias = epi_has_bias(epilogue);
     P->bwd = P->kepi == EPI_DRELU;
     P->bgrad = epilogue == GEMM_EPI_DRELU_BGRAD;
+    P->qout = o.out_e4m3 == 1;
     P->axis = (P->has_bias || P->bgrad) ? bias_axis : GEMM_EPI_BIAS_ROW;
     P->b_layout = b_layout;
     P->opts = o;
@@ -498,9 +517,10 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
 
 // ----------------------------------------------------------------- lookups
 namespace gemm_epi {
-bool find_tc(int cg, int dt, int epi, int axis, bool b_mn, int bn, TcLauncher *l, KernelInfo *i) {
+bool find_tc(int cg, int dt, int epi, int axis, bool b_mn, int bn, bool qout, TcLauncher *l, KernelInfo *i) {
     KernelInfo tmp;
     if (!i) i = &tmp;
+    if (qout) return dt == DT_E4M3 && find_tc_e4m3_q(cg, epi, axis, b_mn, bn, l, i);
     switch (dt) {
     case DT_F16: return find_tc_f16(cg, epi, axis, b_mn, bn, l, i);
     case DT_BF16: return find_tc_bf16(cg, epi, axis, b_mn, bn, l, i);
@@ -553,6 +573,18 @@ int gemm_epi_set_scales(gemm_epi_plan_t plan, const float *d_scale_a, const floa
     return GEMM_EPI_OK;
 }
 
+int gemm_epi_set_out_scale(gemm_epi_plan_t plan, const float *d_scale_out, float *d_amax) {
+    if (!live(plan)) return GEMM_EPI_ERR_ARG;
+    Plan *P = reinterpret_cast<Plan *>(plan);
+    if (!P->qout) return GEMM_EPI_ERR_ARG;
+    if (!d_scale_out) return GEMM_EPI_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(d_scale_out) & 3u) || (reinterpret_cast<uintptr_t>(d_amax) & 3u))
+        return GEMM_EPI_ERR_ALIGN;
+    P->out_scale = d_scale_out;
+    P->amax = d_amax;
+    return GEMM_EPI_OK;
+}
+
 int gemm_epi_run(gemm_epi_plan_t plan, const void *A, const void *B, const void *bias, void *D, uint32_t *aux,
                  void *stream) {
     if (!live(plan)) return GEMM_EPI_ERR_ARG;
@@ -561,13 +593,17 @@ int gemm_epi_run(gemm_epi_plan_t plan, const void *A, const void *B, const void 
     if (rc != GEMM_EPI_OK) return rc;
     rc = ensure_maps(P, A, B, D);
     if (rc != GEMM_EPI_OK) return rc;
-    return launch_main(P, true, bias, D, aux, reinterpret_cast<cudaStream_t>(stream));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // the amax word is this run's maximum: start it at 0 (the kernel max-reduces into it)
+    if (P->qout && P->amax && cudaMemsetAsync(P->amax, 0, sizeof(float), s) != cudaSuccess) return GEMM_EPI_ERR_CUDA;
+    return launch_main(P, true, bias, D, aux, s);
 }
 
 int gemm_epi_unfused_run(gemm_epi_plan_t plan, const void *A, const void *B, const void *bias, void *D,
                          uint32_t *aux, void *stream) {
     if (!live(plan)) return GEMM_EPI_ERR_ARG;
     Plan *P = reinterpret_cast<Plan *>(plan);
+    if (P->qout) return GEMM_EPI_ERR_UNSUPPORTED;
     int rc = check_run_args(P, A, B, bias, D, aux);
     if (rc != GEMM_EPI_OK) return rc;
     rc = ensure_maps(P, A, B, D);
@@ -595,7 +631,7 @@ int gemm_epi_run_bwd(gemm_epi_plan_t plan, const void *A, const void *B, const u
     rc = launch_main(P, true, nullptr, D, const_cast<uint32_t *>(aux), s, P->bgrad ? P->dbias_ws : nullptr);
     if (rc != GEMM_EPI_OK || !P->bgrad) return rc;
     const int out_dt = P->dtype == GEMM_EPI_E4M3 ? DT_BF16 : P->dtype;
-    const cudaError_t e = launch_sum_parts_f32(out_dt, P->dbias_ws, P->dbias_parts, P->dbias_len, dbias, s);
+    const cudaError_t e = launch_sum_parts_f32(out_dt, P->dbias_ws, P->dbias_parts, P->dbias_len, dbias, P->pdl, s);
     return e == cudaSuccess ? GEMM_EPI_OK : GEMM_EPI_ERR_CUDA;
 }
 
@@ -700,6 +736,124 @@ const char *gemm_epi_status_string(int status) {
 int64_t gemm_epi_aux_pitch_bytes(int64_t n) { return n <= 0 ? 0 : ((n + 127) / 128) * 16; }
 
 int gemm_epi_version(void) { return 100; }
+
+}  // extern "C"
+
+// ----------------------------------------------------------------- MLP block
+//
+// Up-projection H = act(X.W1 + b1) and down-projection Y = H.W2 + b2 as two plans of
+// the fused kernel ("nvmath-python cuBLASLt bias fusion for PyTorch inference"
+// (blog.hotdry.top), paragraph 1: the MLP is where the GEMM + bias time goes).  For
+// e4m3 the up-projection's epilogue also quantises H to e4m3 with the caller's scale
+// s_H and reports max |H|, so the down-projection reads H in FP8 with no kernel between
+// the two GEMMs.
+namespace {
+
+constexpr uint64_t kMlpMagic = 0x6d6c705f626c6f63ull;   // "mlp_bloc"
+
+struct Mlp {
+    uint64_t magic;
+    int dtype;
+    gemm_epi_plan_t up = nullptr, down = nullptr;
+};
+
+std::mutex g_mlp_mu;
+std::unordered_set<Mlp *> g_mlps;
+
+Mlp *mlp_live(gemm_epi_mlp_t h) {
+    std::lock_guard<std::mutex> lk(g_mlp_mu);
+    Mlp *M = reinterpret_cast<Mlp *>(h);
+    return (h && g_mlps.count(M) && M->magic == kMlpMagic) ? M : nullptr;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gemm_epi_mlp_plan(int64_t m, int64_t d_model, int64_t d_ff, int dtype, int act, int w_layout,
+                      gemm_epi_mlp_t *out) {
+    if (!out) return GEMM_EPI_ERR_ARG;
+    if (act != GEMM_EPI_BIAS && act != GEMM_EPI_RELU_BIAS && act != GEMM_EPI_GELU_BIAS) return GEMM_EPI_ERR_ARG;
+    Mlp *M = new (std::nothrow) Mlp();
+    if (!M) return GEMM_EPI_ERR_CUDA;
+    M->magic = kMlpMagic;
+    M->dtype = dtype;
+    gemm_epi_options up_opts{};
+    up_opts.out_e4m3 = dtype == GEMM_EPI_E4M3 ? 1 : 0;
+    int rc = make_plan(m, d_ff, d_model, dtype, act, GEMM_EPI_BIAS_COL, w_layout, &up_opts, &M->up);
+    if (rc == GEMM_EPI_OK) rc = make_plan(m, d_model, d_ff, dtype, GEMM_EPI_BIAS, GEMM_EPI_BIAS_COL, w_layout, nullptr,
+                                          &M->down);
+    if (rc != GEMM_EPI_OK) {
+        if (M->up) gemm_epi_free(M->up);
+        M->magic = 0;
+        delete M;
+        return rc;
+    }
+    {
+        std::lock_guard<std::mutex> lk(g_mlp_mu);
+        g_mlps.insert(M);
+    }
+    *out = reinterpret_cast<gemm_epi_mlp_t>(M);
+    return GEMM_EPI_OK;
+}
+
+int gemm_epi_mlp_set_scales(gemm_epi_mlp_t mlp, const float *d_scale_x, const float *d_scale_w1,
+                            const float *d_scale_h, float *d_amax_h, const float *d_scale_w2) {
+    Mlp *M = mlp_live(mlp);
+    if (!M || M->dtype != GEMM_EPI_E4M3) return GEMM_EPI_ERR_ARG;
+    if (!d_scale_x || !d_scale_w1 || !d_scale_h || !d_scale_w2) return GEMM_EPI_ERR_NULL;
+    int rc = gemm_epi_set_scales(M->up, d_scale_x, d_scale_w1);
+    if (rc == GEMM_EPI_OK) rc = gemm_epi_set_out_scale(M->up, d_scale_h, d_amax_h);
+    if (rc == GEMM_EPI_OK) rc = gemm_epi_set_scales(M->down, d_scale_h, d_scale_w2);
+    return rc;
+}
+
+int gemm_epi_mlp_run(gemm_epi_mlp_t mlp, const void *X, const void *W1, const void *b1, const void *W2,
+                     const void *b2, void *H, void *Y, void *stream) {
+    Mlp *M = mlp_live(mlp);
+    if (!M) return GEMM_EPI_ERR_ARG;
+    Plan *U = reinterpret_cast<Plan *>(M->up), *Dn = reinterpret_cast<Plan *>(M->down);
+    // every check of both launches before either is enqueued
+    int rc = check_run_args(U, X, W1, b1, H, nullptr);
+    if (rc == GEMM_EPI_OK) rc = check_run_args(Dn, H, W2, b2, Y, nullptr);
+    if (rc == GEMM_EPI_OK) rc = ensure_maps(U, X, W1, H);
+    if (rc == GEMM_EPI_OK) rc = ensure_maps(Dn, H, W2, Y);
+    if (rc != GEMM_EPI_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (U->qout && U->amax && cudaMemsetAsync(U->amax, 0, sizeof(float), s) != cudaSuccess) return GEMM_EPI_ERR_CUDA;
+    rc = launch_main(U, true, b1, H, nullptr, s);
+    if (rc != GEMM_EPI_OK) return rc;
+    return launch_main(Dn, true, b2, Y, nullptr, s);
+}
+
+int gemm_epi_mlp_check(gemm_epi_mlp_t mlp, void *stream) {
+    Mlp *M = mlp_live(mlp);
+    if (!M) return GEMM_EPI_ERR_ARG;
+    const int a = gemm_epi_check(M->up, stream);
+    const int b = gemm_epi_check(M->down, stream);
+    return a != GEMM_EPI_OK ? a : b;
+}
+
+int gemm_epi_mlp_query(gemm_epi_mlp_t mlp, gemm_epi_plan_info *up, gemm_epi_plan_info *down) {
+    Mlp *M = mlp_live(mlp);
+    if (!M || !up || !down) return GEMM_EPI_ERR_ARG;
+    const int rc = gemm_epi_plan_query(M->up, up);
+    return rc != GEMM_EPI_OK ? rc : gemm_epi_plan_query(M->down, down);
+}
+
+int gemm_epi_mlp_free(gemm_epi_mlp_t mlp) {
+    Mlp *M = reinterpret_cast<Mlp *>(mlp);
+    {
+        std::lock_guard<std::mutex> lk(g_mlp_mu);
+        if (!mlp || !g_mlps.count(M)) return GEMM_EPI_ERR_ARG;
+        g_mlps.erase(M);
+    }
+    gemm_epi_free(M->up);
+    gemm_epi_free(M->down);
+    M->magic = 0;
+    delete M;
+    return GEMM_EPI_OK;
+}
 
 }  // extern "C"
 

@@ -124,7 +124,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    // on-chip setup above; global memory only after the previous kernel has completed
+    // This CTA's slice of the weight operand is prefetched into L2 before waiting on the
+    // previous grid, so its DRAM latency overlaps that grid's tail.  A prefetch writes
+    // nothing and L2 is the point of coherence, so the loads below still see any value the
+    // previous kernel stores.  Every other global access waits for the previous grid.
+    if (warp == 0 && lane == 0) {
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
+            if constexpr (C::W_MN) {
+#pragma unroll
+                for (int b = 0; b < C::W_BOXES; ++b) ptx::tma_prefetch_l2_2d(&tmW, n0 + b * C::W_BOX_N, kb * C::BK);
+            } else {
+                ptx::tma_prefetch_l2_2d(&tmW, kb * C::BK, n0);
+            }
+        }
+    }
     ptx::griddep_wait();
     ptx::griddep_launch_dependents();
 

@@ -46,6 +46,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include <cstdint>
 
@@ -94,6 +95,11 @@ struct TcParams {
     //   ROW: [n-part = column / BN][row]      (m floats per part, ceil(n/BN) parts)
     //   COL: [m-part = row / 32][column]      (n floats per part, ceil(m/32) parts)
     float *dbias_ws;
+    // FP8 output (QOUT kernels): D = e4m3(y / *out_scale), stored m x n bytes; amax (optional)
+    // receives max |y| over the launch as float bits (an atomic max: order-independent)
+    uint8_t *dq;
+    const float *out_scale;
+    unsigned int *amax;
 };
 
 // Timeline tracing (off unless the library is compiled with -DGEMM_EPI_TRACE=1):
@@ -298,7 +304,7 @@ __device__ __forceinline__ float activate(float x) {
     }
 }
 
-template <int DT_, int EPI_, int AXIS_, bool B_MN_, int BN_, int CG_, int STAGES_>
+template <int DT_, int EPI_, int AXIS_, bool B_MN_, int BN_, int CG_, int STAGES_, bool QOUT_ = false>
 struct TcCfg {
     static constexpr int DT = DT_, EPI = EPI_, AXIS = AXIS_, BN = BN_, CG = CG_, STAGES = STAGES_;
     static constexpr bool B_MN = B_MN_;             // B stored (k, n): N contiguous
@@ -321,6 +327,9 @@ struct TcCfg {
     static constexpr bool HEAVY_EPI = EPI == EPI_GELU || EPI == EPI_TANH;
     static constexpr bool BWD = EPI == EPI_DRELU;             // reads the mask, adds no bias
     static constexpr bool FWD_BIAS = EPI != EPI_NONE && !BWD;  // may add a bias
+    // e4m3 output quantised with a per-tensor scale (the MLP block's intermediate): written
+    // with direct 16-byte stores from registers, no staging
+    static constexpr bool QOUT = QOUT_;
     static constexpr int EPI_WARPS = HEAVY_EPI ? 8 : 4;
     static constexpr int THREADS = 64 + 32 * EPI_WARPS;
     static constexpr int COLS_W = BN * 4 / EPI_WARPS;       // columns of a tile one epilogue warp handles
@@ -329,7 +338,7 @@ struct TcCfg {
     static_assert(NCH_W % CPG == 0 && (CPG == 2 || CPG == 4), "chunk grouping");
     static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                    : (2 * BN <= 256) ? 256 : 512;
-    static constexpr int STG_BYTES = 32 * 64;       // per epilogue warp: 32 rows x 32 16-bit outputs
+    static constexpr int STG_BYTES = QOUT ? 0 : 32 * 64;   // per epilogue warp: 32 rows x 32 16-bit outputs
     // shared-memory layout (offsets from a 1024-byte aligned base)
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
@@ -346,6 +355,7 @@ struct TcCfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "stage alignment");
     static_assert(!BWD || (EPI_WARPS == 4 && CPG == 4), "backward epilogue: one mask uint4 per chunk group");
+    static_assert(!QOUT || (DT == DT_E4M3 && !BWD && EPI != EPI_RELU_AUX), "FP8 output: e4m3 forward plans");
 };
 
 // Tile index -> (tile_m, tile_n) with a grouped raster: GROUP_M tile-rows are
@@ -390,7 +400,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (warp == 0 && lane == 0) {
         ptx::prefetch_tmap(&tmA);
         ptx::prefetch_tmap(&tmB);
-        ptx::prefetch_tmap(&tmD);
+        if constexpr (!C::QOUT) ptx::prefetch_tmap(&tmD);
         for (int s = 0; s < C::STAGES; ++s) {
             ptx::mbar_init(full_bar(s), 1);
             ptx::mbar_init(empty_bar(s), 1);
@@ -533,6 +543,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (p.scale_a != nullptr) alpha = __ldg(p.scale_a) * __ldg(p.scale_b);
         const bool has_bias = p.bias != nullptr;
         const bool bgrad = C::BWD && p.dbias_ws != nullptr;   // backward: bias-gradient partials
+        float inv_out = 1.0f, amax_l = 0.0f;                  // FP8 output: 1 / scale, running max |y|
+        if constexpr (C::QOUT) inv_out = 1.0f / __ldg(p.out_scale);
         uint32_t acc = 0, acc_phase = 0;
         bool ok = true;
         WorkIter it(p, unit, units);
@@ -667,30 +679,53 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             bits |= (x0 > 0.0f ? 1u : 0u) << j;
                             bits |= (x1 > 0.0f ? 1u : 0u) << (j + 1);
                         }
-                        packed[j / 2] = O::pack(activate<C::EPI>(x0), activate<C::EPI>(x1));
+                        const float y0 = activate<C::EPI>(x0), y1 = activate<C::EPI>(x1);
+                        if constexpr (C::QOUT) {
+                            amax_l = fmaxf(amax_l, fmaxf(fabsf(y0), fabsf(y1)));
+                            // two e4m3 codes, round to nearest even, saturating at +-448; y0 low byte
+                            packed[j / 2] = __nv_cvt_float2_to_fp8x2(make_float2(y0 * inv_out, y1 * inv_out),
+                                                                     __NV_SATFINITE, __NV_E4M3);
+                        } else {
+                            packed[j / 2] = O::pack(y0, y1);
+                        }
                     }
                     if constexpr (C::EPI == EPI_RELU_AUX) {
                         const int valid = p.n - col0;
                         const uint32_t keep = valid >= 32 ? 0xFFFFFFFFu : (valid <= 0 ? 0u : ((1u << valid) - 1u));
                         words[cc] = bits & keep;
                     }
-                    // stage 32 rows x 32 outputs in the 64-byte swizzled layout the TMA store reads:
-                    // 16-byte piece j of row r sits at r*64 + ((j ^ ((r >> 1) & 3)) * 16)
-                    if (lane == 0) ptx::bulk_wait_read<0>();     // previous store has read the buffer
-                    __syncwarp();
-                    uint8_t *stg_row = smem + C::OFF_STG + ew * C::STG_BYTES + lane * 64;
+                    if constexpr (C::QOUT) {
+                        // this lane's 32 codes are 32 contiguous bytes of its row (n is a multiple of 16)
+                        if (row_ok) {
+                            uint8_t *dst = p.dq + (int64_t)row * p.n + col0;
+                            if (col0 + 16 <= p.n)
+                                *reinterpret_cast<uint4 *>(dst) =
+                                    make_uint4(packed[0] | (packed[1] << 16), packed[2] | (packed[3] << 16),
+                                               packed[4] | (packed[5] << 16), packed[6] | (packed[7] << 16));
+                            if (col0 + 32 <= p.n)
+                                *reinterpret_cast<uint4 *>(dst + 16) =
+                                    make_uint4(packed[8] | (packed[9] << 16), packed[10] | (packed[11] << 16),
+                                               packed[12] | (packed[13] << 16), packed[14] | (packed[15] << 16));
+                        }
+                    } else {
+                        // stage 32 rows x 32 outputs in the 64-byte swizzled layout the TMA store reads:
+                        // 16-byte piece j of row r sits at r*64 + ((j ^ ((r >> 1) & 3)) * 16)
+                        if (lane == 0) ptx::bulk_wait_read<0>();     // previous store has read the buffer
+                        __syncwarp();
+                        uint8_t *stg_row = smem + C::OFF_STG + ew * C::STG_BYTES + lane * 64;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int piece = i ^ ((lane >> 1) & 3);
-                        *reinterpret_cast<uint4 *>(stg_row + piece * 16) =
-                            make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-                    }
-                    ptx::fence_proxy_async_smem();
-                    __syncwarp();
-                    // boxes starting past the last row or column hold nothing to store
-                    if (lane == 0 && m0 + 32 * q < p.m && col0 < p.n) {
-                        ptx::tma_store_2d(&tmD, stg, col0, m0 + 32 * q);
-                        ptx::bulk_commit();
+                        for (int i = 0; i < 4; ++i) {
+                            const int piece = i ^ ((lane >> 1) & 3);
+                            *reinterpret_cast<uint4 *>(stg_row + piece * 16) =
+                                make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                        }
+                        ptx::fence_proxy_async_smem();
+                        __syncwarp();
+                        // boxes starting past the last row or column hold nothing to store
+                        if (lane == 0 && m0 + 32 * q < p.m && col0 < p.n) {
+                            ptx::tma_store_2d(&tmD, stg, col0, m0 + 32 * q);
+                            ptx::bulk_commit();
+                        }
                     }
                     if constexpr (C::BWD && C::AXIS == AXIS_COL) if (bgrad) {
                         // column sums over this warp's 32 rows: a butterfly that halves the
@@ -742,6 +777,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         if (lane == 0) ptx::bulk_wait<0>();
         __syncwarp();
+        if constexpr (C::QOUT) {
+            // one atomic per warp: the launch's max |y| (non-negative floats order as their bits)
+            const unsigned int wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax_l));
+            if (ok && lane == 0 && p.amax != nullptr) atomicMax(p.amax, wmax);
+        }
     }
 
     // ---------------------------------------------------------------- teardown

@@ -43,7 +43,8 @@ using BiasActLauncher = cudaError_t (*)(void *D, const void *bias, uint32_t *aux
                                         int64_t pitch_words, int grid, cudaStream_t stream);
 
 // Lookups return false when the combination is not instantiated.
-bool find_tc(int cg, int dt, int epi, int axis, bool b_mn, int bn, TcLauncher *launch, KernelInfo *info);
+// qout: e4m3 output quantised in the epilogue (e4m3 operands only)
+bool find_tc(int cg, int dt, int epi, int axis, bool b_mn, int bn, bool qout, TcLauncher *launch, KernelInfo *info);
 bool find_sk(int dt, int epi, int axis, bool w_mn, int nm, SkLauncher *launch, KernelInfo *info);
 bool find_bias_act(int dt, int epi, int axis, BiasActLauncher *launch);
 
@@ -51,7 +52,7 @@ bool find_bias_act(int dt, int epi, int axis, BiasActLauncher *launch);
 //   sum_parts_f32: out[i] = sum_p src[p * len + i] over fp32 partials (fused backward)
 //   sum_cols:      out[j] = sum_i D[i, j]  (unfused backward, COL axis)
 //   sum_rows:      out[i] = sum_j D[i, j]  (unfused backward, ROW axis)
-cudaError_t launch_sum_parts_f32(int out_dt, const float *src, int64_t parts, int64_t len, void *out,
+cudaError_t launch_sum_parts_f32(int out_dt, const float *src, int64_t parts, int64_t len, void *out, bool pdl,
                                  cudaStream_t s);
 cudaError_t launch_sum_cols(int out_dt, const void *D, int64_t m, int64_t n, void *out, cudaStream_t s);
 cudaError_t launch_sum_rows(int out_dt, const void *D, int64_t m, int64_t n, void *out, int grid, cudaStream_t s);
@@ -60,6 +61,7 @@ cudaError_t launch_sum_rows(int out_dt, const void *D, int64_t m, int64_t n, voi
 bool find_tc_f16(int cg, int epi, int axis, bool b_mn, int bn, TcLauncher *, KernelInfo *);
 bool find_tc_bf16(int cg, int epi, int axis, bool b_mn, int bn, TcLauncher *, KernelInfo *);
 bool find_tc_e4m3(int cg, int epi, int axis, bool b_mn, int bn, TcLauncher *, KernelInfo *);
+bool find_tc_e4m3_q(int cg, int epi, int axis, bool b_mn, int bn, TcLauncher *, KernelInfo *);
 bool find_sk_f16(int epi, int axis, bool w_mn, int nm, SkLauncher *, KernelInfo *);
 bool find_sk_bf16(int epi, int axis, bool w_mn, int nm, SkLauncher *, KernelInfo *);
 bool find_sk_e4m3(int epi, int axis, bool w_mn, int nm, SkLauncher *, KernelInfo *);

@@ -44,13 +44,16 @@ STREAM_K = {"auto": 0, "off": 1, "on": 2}
 EXPORTS = ("gemm_epi_plan", "gemm_epi_plan_ex", "gemm_epi_plan_opts", "gemm_epi_set_scales",
            "gemm_epi_run", "gemm_epi_unfused_run", "gemm_epi_check", "gemm_epi_plan_query",
            "gemm_epi_free", "gemm_epi_status_string", "gemm_epi_aux_pitch_bytes",
-           "gemm_epi_version", "gemm_epi_run_noalloc", "gemm_epi_run_bwd", "gemm_epi_unfused_run_bwd")
+           "gemm_epi_version", "gemm_epi_run_noalloc", "gemm_epi_run_bwd", "gemm_epi_unfused_run_bwd",
+           "gemm_epi_set_out_scale", "gemm_epi_mlp_plan", "gemm_epi_mlp_set_scales", "gemm_epi_mlp_run",
+           "gemm_epi_mlp_check", "gemm_epi_mlp_query", "gemm_epi_mlp_free")
 
 
 class Options(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("block_n", ctypes.c_int32),
                 ("split_k", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
-                ("inject_stall", ctypes.c_int32), ("stream_k", ctypes.c_int32)]
+                ("inject_stall", ctypes.c_int32), ("stream_k", ctypes.c_int32),
+                ("out_e4m3", ctypes.c_int32)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -93,6 +96,13 @@ def lib():
             L.gemm_epi_unfused_run.argtypes = [vp, vp, vp, vp, vp, vp, vp]
             L.gemm_epi_run_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp]
             L.gemm_epi_unfused_run_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+            L.gemm_epi_set_out_scale.argtypes = [vp, vp, vp]
+            L.gemm_epi_mlp_plan.argtypes = [i64, i64, i64, i32, i32, i32, pp]
+            L.gemm_epi_mlp_set_scales.argtypes = [vp, vp, vp, vp, vp, vp]
+            L.gemm_epi_mlp_run.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            L.gemm_epi_mlp_check.argtypes = [vp, vp]
+            L.gemm_epi_mlp_query.argtypes = [vp, ctypes.POINTER(PlanInfo), ctypes.POINTER(PlanInfo)]
+            L.gemm_epi_mlp_free.argtypes = [vp]
             L.gemm_epi_check.argtypes = [vp, vp]
             L.gemm_epi_plan_query.argtypes = [vp, ctypes.POINTER(PlanInfo)]
             L.gemm_epi_free.argtypes = [vp]
@@ -107,7 +117,9 @@ def lib():
                          "gemm_epi_set_scales", "gemm_epi_run", "gemm_epi_unfused_run",
                          "gemm_epi_check", "gemm_epi_plan_query", "gemm_epi_free",
                          "gemm_epi_version", "gemm_epi_run_noalloc", "gemm_epi_run_bwd",
-                         "gemm_epi_unfused_run_bwd"):
+                         "gemm_epi_unfused_run_bwd", "gemm_epi_set_out_scale", "gemm_epi_mlp_plan",
+                         "gemm_epi_mlp_set_scales", "gemm_epi_mlp_run", "gemm_epi_mlp_check",
+                         "gemm_epi_mlp_query", "gemm_epi_mlp_free"):
                 getattr(L, name).restype = i32
             _lib = L
     return _lib
@@ -153,6 +165,40 @@ def gemm_epi_run_bwd(plan, A, B, aux, D, dbias, stream) -> None:
 
 def gemm_epi_unfused_run_bwd(plan, A, B, aux, D, dbias, stream) -> None:
     _check(lib().gemm_epi_unfused_run_bwd(plan, A, B, aux, D, dbias, stream), "gemm_epi_unfused_run_bwd")
+
+
+def gemm_epi_set_out_scale(plan, d_scale_out, d_amax) -> None:
+    _check(lib().gemm_epi_set_out_scale(plan, d_scale_out, d_amax), "gemm_epi_set_out_scale")
+
+
+def gemm_epi_mlp_plan(m, d_model, d_ff, dtype, act, w_layout) -> int:
+    h = ctypes.c_void_p()
+    _check(lib().gemm_epi_mlp_plan(m, d_model, d_ff, dtype, act, w_layout, ctypes.byref(h)),
+           "gemm_epi_mlp_plan")
+    return h.value
+
+
+def gemm_epi_mlp_set_scales(mlp, d_scale_x, d_scale_w1, d_scale_h, d_amax_h, d_scale_w2) -> None:
+    _check(lib().gemm_epi_mlp_set_scales(mlp, d_scale_x, d_scale_w1, d_scale_h, d_amax_h, d_scale_w2),
+           "gemm_epi_mlp_set_scales")
+
+
+def gemm_epi_mlp_run(mlp, X, W1, b1, W2, b2, H, Y, stream) -> None:
+    _check(lib().gemm_epi_mlp_run(mlp, X, W1, b1, W2, b2, H, Y, stream), "gemm_epi_mlp_run")
+
+
+def gemm_epi_mlp_check(mlp, stream) -> None:
+    _check(lib().gemm_epi_mlp_check(mlp, stream), "gemm_epi_mlp_check")
+
+
+def gemm_epi_mlp_query(mlp) -> tuple:
+    up, down = PlanInfo(), PlanInfo()
+    _check(lib().gemm_epi_mlp_query(mlp, ctypes.byref(up), ctypes.byref(down)), "gemm_epi_mlp_query")
+    return up.as_dict(), down.as_dict()
+
+
+def gemm_epi_mlp_free(mlp) -> None:
+    _check(lib().gemm_epi_mlp_free(mlp), "gemm_epi_mlp_free")
 
 
 def gemm_epi_check(plan, stream) -> None:
@@ -214,11 +260,12 @@ class Plan:
     """
 
     def __init__(self, m, n, k, dtype="bf16", epilogue="bias", bias_axis="row", b_layout="kn",
-                 kernel="auto", block_n=0, split_k=0, max_ctas=0, inject_stall=0, stream_k="auto"):
+                 kernel="auto", block_n=0, split_k=0, max_ctas=0, inject_stall=0, stream_k="auto",
+                 out_e4m3=False):
         self.m, self.n, self.k = int(m), int(n), int(k)
         self.dtype, self.epilogue, self.bias_axis, self.b_layout = dtype, epilogue, bias_axis, b_layout
         opts = Options(KERNEL[kernel], int(block_n), int(split_k), int(max_ctas), int(inject_stall),
-                       STREAM_K[stream_k])
+                       STREAM_K[stream_k], 1 if out_e4m3 else 0)
         self.handle = gemm_epi_plan_opts(self.m, self.n, self.k, DTYPE[dtype], EPILOGUE[epilogue],
                                          AXIS[bias_axis], LAYOUT[b_layout], opts)
         self._scales = None
@@ -231,6 +278,11 @@ class Plan:
         """fp32 device scalars (torch tensors); kept alive by the plan object."""
         self._scales = (scale_a, scale_b)
         gemm_epi_set_scales(self.handle, _ptr(scale_a), _ptr(scale_b))
+
+    def set_out_scale(self, scale_out, amax=None):
+        """FP8-output plans: fp32 device scalars (the output scale; the amax word or None)."""
+        self._out = (scale_out, amax)
+        gemm_epi_set_out_scale(self.handle, _ptr(scale_out), _ptr(amax))
 
     def run(self, A, B, bias, D, aux=None, stream=None, fused=True):
         s = _stream_ptr(stream)
@@ -273,3 +325,47 @@ def _stream_ptr(stream):
 
 def aux_pitch_words(n: int) -> int:
     return gemm_epi_aux_pitch_bytes(n) // 4
+
+
+class MlpPlan:
+    """Owns one MLP-block handle (gemm_epi_mlp_*): H = act(X.W1 + b1), Y = H.W2 + b2."""
+
+    def __init__(self, m, d_model, d_ff, dtype="bf16", act="gelu_bias", w_layout="kn"):
+        self.m, self.d_model, self.d_ff = int(m), int(d_model), int(d_ff)
+        self.dtype, self.act, self.w_layout = dtype, act, w_layout
+        self.handle = gemm_epi_mlp_plan(self.m, self.d_model, self.d_ff, DTYPE[dtype], EPILOGUE[act],
+                                        LAYOUT[w_layout])
+        self._scales = None
+
+    @property
+    def info(self) -> tuple:
+        return gemm_epi_mlp_query(self.handle)
+
+    def set_scales(self, scale_x, scale_w1, scale_h, amax_h, scale_w2):
+        self._scales = (scale_x, scale_w1, scale_h, amax_h, scale_w2)
+        gemm_epi_mlp_set_scales(self.handle, _ptr(scale_x), _ptr(scale_w1), _ptr(scale_h), _ptr(amax_h),
+                                _ptr(scale_w2))
+
+    def run(self, X, W1, b1, W2, b2, H, Y, stream=None):
+        gemm_epi_mlp_run(self.handle, _ptr(X), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(H), _ptr(Y),
+                         _stream_ptr(stream))
+
+    def check(self, stream=None):
+        gemm_epi_mlp_check(self.handle, _stream_ptr(stream))
+
+    def close(self):
+        if getattr(self, "handle", None):
+            gemm_epi_mlp_free(self.handle)
+            self.handle = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

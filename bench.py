@@ -25,6 +25,10 @@ elementwise path), ``clocks`` and ``gpu_launches``.
 ``--impl reference`` times the CPU oracle itself, as it stands, on the same
 workload and metric (bounded samples per step); under torchrun only rank 0
 runs it.
+
+``--mlp m,d_model,d_ff,dtype,act,layout`` times the MLP block instead (two
+fused GEMMs per step, 4*m*d_model*d_ff flops; for e4m3 the up-projection's
+epilogue requantises H, with s_H set from a first run's amax).
 """
 from __future__ import annotations
 
@@ -62,6 +66,9 @@ def parse(argv=None):
     ap.add_argument("--kernel", default="auto", choices=["auto", "tc1", "tc2", "splitk"])
     ap.add_argument("--block-n", type=int, default=0)
     ap.add_argument("--stream-k", default="auto", choices=["auto", "off", "on"])
+    ap.add_argument("--split-k", type=int, default=0,
+                    help="split-K kernel: CTAs per cluster along k; TC kernels: parts per tail tile "
+                         "(0 = the plan's choice)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -69,6 +76,8 @@ def parse(argv=None):
     ap.add_argument("--no-unfused", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps directly instead of replaying them from a CUDA graph")
+    ap.add_argument("--mlp", default=None,
+                    help="time the MLP block m,d_model,d_ff,dtype,act,layout instead of one GEMM")
     ap.add_argument("--cublas", action="store_true",
                     help="also time cuBLAS's bare GEMM (torch.matmul, no epilogue) at this shape, "
                          "as context only (16-bit workloads)")
@@ -295,10 +304,116 @@ def reference_arm(args):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+def mlp_arm(args):
+    """The MLP block (gemm_epi_mlp_run): H = act(X.W1 + b1), Y = H.W2 + b2 per step."""
+    import torch
+    from activation_epilogue_tcgen05_b200 import gemm_epi as g
+    from activation_epilogue_tcgen05_b200 import replicas
+    from activation_epilogue_tcgen05_b200.workloads import TORCH_DTYPE, Workload, make_problem
+
+    rank, world, local_rank = replicas.env_rank()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback exists)")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    have_pg = replicas.init("nccl", timeout_s=120, device_id=dev)
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    m, dm, dff, dt, act, lay = args.mlp.split(",")
+    m, dm, dff = int(m), int(dm), int(dff)
+    std = 1.0 if dt == "e4m3" else 1.0 / 64
+    up = Workload("mlp_up", m, dff, dm, dt, act, "col", lay, ("normal", 1.0), ("normal", std), ("normal", 0.1))
+    down = Workload("mlp_down", m, dm, dff, dt, "bias", "col", lay, ("normal", 1.0), ("normal", std),
+                    ("normal", 0.1), seed=1)
+    big = m * dm > (1 << 28)
+    pu, pd = make_problem(up, device="cuda" if big else "cpu"), make_problem(down, device="cuda")
+    X, W1, b1 = pu.A.to(dev), pu.B.to(dev), pu.bias.to(dev)
+    W2, b2 = pd.B.to(dev), pd.bias.to(dev)
+    h_t = torch.uint8 if dt == "e4m3" else TORCH_DTYPE[dt]
+    H = torch.empty((m, dff), dtype=h_t, device=dev)
+    Y = torch.empty((m, dm), dtype=TORCH_DTYPE[up.out_dtype], device=dev)
+    mp = g.MlpPlan(m, dm, dff, dt, act, lay)
+    stream = torch.cuda.current_stream(dev)
+    if dt == "e4m3":
+        f32 = lambda v: torch.tensor([v], dtype=torch.float32, device=dev)
+        s_x, s_w1, s_w2 = f32(pu.scale_a), f32(pu.scale_b), f32(pd.scale_b)
+        s_h, amax = f32(1.0), f32(0.0)
+        mp.set_scales(s_x, s_w1, s_h, amax, s_w2)
+        mp.run(X, W1, b1, W2, b2, H, Y, stream=stream)        # delayed scaling: s_H from this amax
+        torch.cuda.synchronize(dev)
+        s_h.copy_(amax / 448.0)
+    t0 = time.perf_counter()
+    mp.run(X, W1, b1, W2, b2, H, Y, stream=stream)
+    torch.cuda.synchronize(dev)
+    first_call_ms = 1000 * (time.perf_counter() - t0)
+    mp.check(stream)
+    for _ in range(args.warmup):
+        mp.run(X, W1, b1, W2, b2, H, Y, stream=stream)
+    torch.cuda.synchronize(dev)
+    mp.check(stream)
+    if sampler:
+        sampler.wait_first()
+    K = args.steps
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        cs = torch.cuda.current_stream(dev)
+        for _ in range(K):
+            mp.run(X, W1, b1, W2, b2, H, Y, stream=cs)
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    replicas.barrier()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    wall0 = time.time()
+    start.record(stream)
+    graph.replay()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    wall1 = time.time()
+    replicas.barrier()
+    mp.check(stream)
+    del graph
+    elapsed_ms = replicas.max_over_ranks(start.elapsed_time(end), device=dev)
+    clocks = sampler.summary(wall0, wall1) if sampler else None
+    if sampler:
+        sampler.stop()
+    flops = 4.0 * m * dm * dff
+    value = flops * world * K / (elapsed_ms / 1000.0) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = peaks["bf16_tflops"] * (FP8_OVER_BF16 if dt == "e4m3" else 1.0)
+    achieved = flops / (elapsed_ms / K / 1000.0) / 1e12
+    up_info, down_info = mp.info
+    mp.close()
+    if rank == 0:
+        esz = 1 if dt == "e4m3" else 2
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": dt, "data": "synthetic",
+            "config": {"workload": f"mlp_{dt}_{act}_{m}x{dm}x{dff}_{lay}", "m": m, "d_model": dm, "d_ff": dff,
+                       "dtype": dt, "act": act, "w_layout": lay, "parallelism": f"replicas x{world}",
+                       "plans": {"up": up_info, "down": down_info}, "first_call_ms": first_call_ms,
+                       "l2": f"one set: X, W1, W2, H, Y = {((m * dm + 2 * dm * dff) * esz + m * dff * esz + m * dm * 2) / 2**20:.0f} MiB",
+                       "launch": "CUDA graph of the K steps (two kernel launches each)"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": peak_src + (", bf16 burst x nominal fp8/bf16 ratio 2" if dt == "e4m3"
+                                                    else ", bf16 burst"),
+                         "note": "per-step time of both GEMM launches"},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": 2 * K, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if have_pg:
+        replicas.barrier()
+        replicas.finalize()
+    return 0
+
+
 def main(argv=None):
     args = parse(argv)
     if args.impl == "reference":
         return reference_arm(args)
+    if args.mlp:
+        return mlp_arm(args)
 
     import torch
     from activation_epilogue_tcgen05_b200 import gemm_epi as g
@@ -353,7 +468,7 @@ def main(argv=None):
         D = torch.empty((wl.m, wl.n), dtype=out_t, device=dev)
         sets.append((A, B, x, D, new_y()))
     plan = g.Plan(wl.m, wl.n, wl.k, wl.dtype, wl.epilogue, wl.bias_axis, wl.b_layout,
-                  kernel=args.kernel, block_n=args.block_n, stream_k=args.stream_k)
+                  kernel=args.kernel, block_n=args.block_n, stream_k=args.stream_k, split_k=args.split_k)
     run = plan.run_bwd if bwd else plan.run
     if wl.dtype == "e4m3":
         plan.set_scales(torch.tensor([prob.scale_a], dtype=torch.float32, device=dev),

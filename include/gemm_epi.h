@@ -146,6 +146,12 @@ typedef struct gemm_epi_options {
                           incomplete last wave (or all tiles, when there are fewer tiles than
                           SMs) along k over several SMs (stream-K style); partial tiles pass
                           through a workspace the plan allocates (SMs x 128 x block_n fp32). */
+    int32_t out_e4m3;  /* 1 = D is e4m3, quantised in the epilogue: D = e4m3(y / s_out) with
+                          round to nearest even, saturating at +-448, y the epilogue's fp32
+                          result; max |y| is reported (gemm_epi_set_out_scale).  E4M3 plans
+                          with epilogue NONE, BIAS, RELU_BIAS, GELU_BIAS, RELU or GELU, on the
+                          persistent kernels (small m uses TC1); else ERR_UNSUPPORTED.
+                          0 = D in the 16-bit output type.                              */
 } gemm_epi_options;
 
 /* What a plan decided (for logging and tests). */
@@ -183,6 +189,16 @@ int gemm_epi_plan_opts(int64_t m, int64_t n, int64_t k, int dtype, int epilogue,
  * plans, whose alpha is 1 until set (both NULL resets it).  The pointers are
  * borrowed, not owned.  ERR_NULL if only one is given. */
 int gemm_epi_set_scales(gemm_epi_plan_t plan, const float *d_scale_a, const float *d_scale_b);
+
+/* For plans created with options.out_e4m3 = 1: the output scale s_out (DEVICE pointer to
+ * one float, > 0; D = e4m3(y / s_out), the usual choice being amax / 448 from an earlier
+ * run) and, optionally, d_amax (DEVICE pointer to one float): each run sets it to 0 on the
+ * stream before the launch and the kernel max-reduces |y| into it, so after the run it
+ * holds max |y| over D before quantisation (exact: a maximum does not depend on order).
+ * Borrowed, not owned.  ERR_ARG for other plans, ERR_NULL without d_scale_out, ERR_ALIGN
+ * for pointers not 4-byte aligned.  A run of such a plan without a scale is ERR_NULL; its
+ * unfused run is ERR_UNSUPPORTED. */
+int gemm_epi_set_out_scale(gemm_epi_plan_t plan, const float *d_scale_out, float *d_amax);
 
 /* Enqueue the fused kernel: one launch, D (and aux) written once.
  *   A     (m, k) operand, B (k, n) or (n, k) operand, device pointers.
@@ -279,6 +295,43 @@ int gemm_epi_run_noalloc(int64_t m, int64_t n, int64_t k, int dtype, int epilogu
                          int b_layout, const void *A, const void *B, const void *bias,
                          const float *d_scale_a, const float *d_scale_b, void *D, uint32_t *aux,
                          int wait, void *stream);
+
+/* ---- MLP block ------------------------------------------------------------ */
+
+/* Two fused GEMMs of a transformer MLP ([nvmath-fusion] paragraph 1: the MLP layers are
+ * where GEMM + bias time goes):
+ *     H = act(alpha1 * X . W1 + b1)     up-projection, act = BIAS, RELU_BIAS or GELU_BIAS
+ *     Y = alpha2 * H . W2 + b2          down-projection (BIAS)
+ * X is (m, d_model); W1 is (d_model, d_ff) and W2 (d_ff, d_model) for GEMM_EPI_B_KN, or
+ * nn.Linear weights (d_ff, d_model) and (d_model, d_ff) for GEMM_EPI_B_NK; b1 has length
+ * d_ff, b2 length d_model (per output feature); H (m, d_ff) is caller-owned scratch.
+ * fp16 / bf16: alpha1 = alpha2 = 1 and H, Y are in the input type.
+ * e4m3: X, W1, W2 are e4m3 with per-tensor scales; the up-projection's epilogue stores H
+ * in e4m3 as e4m3(h / s_H) and reports max |h| (the per-tensor requantisation), so
+ * alpha1 = s_X * s_W1, alpha2 = s_H * s_W2, and b1, b2, Y are bf16.  Two launches, the
+ * second a programmatic dependent of the first; no kernel between them.
+ * The handle owns two plans (see gemm_epi_plan); errors as there. */
+typedef struct gemm_epi_mlp_s *gemm_epi_mlp_t;
+
+int gemm_epi_mlp_plan(int64_t m, int64_t d_model, int64_t d_ff, int dtype, int act, int w_layout,
+                      gemm_epi_mlp_t *out);
+
+/* E4M3 only (ERR_ARG otherwise); all four scales required (ERR_NULL), d_amax_h optional.
+ * DEVICE pointers to one float each, borrowed. */
+int gemm_epi_mlp_set_scales(gemm_epi_mlp_t mlp, const float *d_scale_x, const float *d_scale_w1,
+                            const float *d_scale_h, float *d_amax_h, const float *d_scale_w2);
+
+/* Enqueue both GEMMs on `stream` (all arguments are checked before either is enqueued). */
+int gemm_epi_mlp_run(gemm_epi_mlp_t mlp, const void *X, const void *W1, const void *b1, const void *W2,
+                     const void *b2, void *H, void *Y, void *stream);
+
+/* gemm_epi_check on both plans (the first non-OK status). */
+int gemm_epi_mlp_check(gemm_epi_mlp_t mlp, void *stream);
+
+/* The two plans' choices. */
+int gemm_epi_mlp_query(gemm_epi_mlp_t mlp, gemm_epi_plan_info *up, gemm_epi_plan_info *down);
+
+int gemm_epi_mlp_free(gemm_epi_mlp_t mlp);
 
 /* Release the plan (host metadata, tensor maps, status word).  Must not
  * overlap a run still executing on the GPU that uses this plan's status word:

@@ -165,3 +165,26 @@ def test_noalloc_refuses_backward_epilogues(g, epi):
     rc = g.lib().gemm_epi_run_noalloc(64, 64, 64, 1, epi, 0, 0, None, None, None, None, None, None, None,
                                       0, None)
     assert rc == g.ERR_ARG
+
+
+def test_fp8_output_option_checks_before_the_device(g):
+    o = g.Options(kernel=0, block_n=0, split_k=0, max_ctas=0, inject_stall=0, stream_k=0, out_e4m3=2)
+    assert _plan_rc(g, 64, 64, 64, dt=2, epi=1, opts=o) == g.ERR_ARG
+    o.out_e4m3 = 1
+    assert _plan_rc(g, 64, 64, 64, dt=1, epi=1, opts=o) == g.ERR_UNSUPPORTED      # bf16 operands
+    assert _plan_rc(g, 64, 64, 64, dt=2, epi=3, opts=o) == g.ERR_UNSUPPORTED      # RELU_AUX_BIAS
+    assert _plan_rc(g, 64, 64, 64, dt=2, epi=4, opts=o) == g.ERR_NO_DEVICE        # GELU_BIAS: valid
+    assert g.lib().gemm_epi_set_out_scale(None, None, None) == g.ERR_ARG
+
+
+def test_mlp_entry_points_reject_bad_handles_and_acts(g):
+    L = g.lib()
+    h = ctypes.c_void_p()
+    assert L.gemm_epi_mlp_plan(64, 64, 128, 1, 5, 0, ctypes.byref(h)) == g.ERR_ARG   # TANH_BIAS
+    assert L.gemm_epi_mlp_plan(64, 64, 128, 1, 4, 0, None) == g.ERR_ARG
+    assert L.gemm_epi_mlp_plan(64, 64, 128, 1, 4, 0, ctypes.byref(h)) == g.ERR_NO_DEVICE
+    for bad in (None, ctypes.c_void_p(0x1000)):
+        assert L.gemm_epi_mlp_set_scales(bad, None, None, None, None, None) == g.ERR_ARG
+        assert L.gemm_epi_mlp_run(bad, None, None, None, None, None, None, None, None) == g.ERR_ARG
+        assert L.gemm_epi_mlp_check(bad, None) == g.ERR_ARG
+        assert L.gemm_epi_mlp_free(bad) == g.ERR_ARG
