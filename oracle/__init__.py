@@ -34,6 +34,7 @@ EPILOGUES = ("none", "bias", "relu_bias", "relu_aux_bias", "gelu_bias", "tanh_bi
              "relu_aux", "gelu", "tanh")
 AXES = ("row", "col")
 LAYOUTS = ("kn", "nk")
+A_LAYOUTS = ("mk", "km")   # A stored (m, k) row-major, or transposed: (k, m) row-major
 
 
 def build(force: bool = False) -> str:
@@ -113,25 +114,36 @@ def gelu(x: float) -> float:
     return _load().oracle_gelu(float(x))
 
 
-def _names(dtype, epilogue, bias_axis, b_layout):
+def _names(dtype, epilogue, bias_axis, b_layout, a_layout="mk"):
     if dtype not in DTYPES or epilogue not in EPILOGUES or bias_axis not in AXES \
-            or b_layout not in LAYOUTS:
-        raise ValueError(f"unknown oracle option {(dtype, epilogue, bias_axis, b_layout)}")
-    return tuple(s.encode() for s in (dtype, epilogue, bias_axis, b_layout))
+            or b_layout not in LAYOUTS or a_layout not in A_LAYOUTS:
+        raise ValueError(f"unknown oracle option {(dtype, epilogue, bias_axis, b_layout, a_layout)}")
+    return tuple(s.encode() for s in (dtype, epilogue, bias_axis, _layout(b_layout, a_layout)))
+
+
+def _layout(b_layout, a_layout):
+    """The C side's layout string: B's layout, prefixed "at_" when A is stored (k, m)."""
+    return ("at_" if a_layout == "km" else "") + b_layout
+
+
+def _a_shape(A, a_layout):
+    """(m, k) of the operand A from its storage array."""
+    return (A.shape[1], A.shape[0]) if a_layout == "km" else A.shape
 
 
 def gemm_epi(A, B, bias, *, dtype: str, epilogue: str, bias_axis: str = "row",
-             b_layout: str = "kn", scale_a: float = 1.0, scale_b: float = 1.0):
+             b_layout: str = "kn", scale_a: float = 1.0, scale_b: float = 1.0, a_layout: str = "mk"):
     """Full fp64 result (D, pre-activation, mask) of act(alpha*A.B + bias).
 
-    A is (m, k) row-major storage; B is (k, n) for ``b_layout="kn"`` or (n, k)
+    A is (m, k) row-major storage (``a_layout="mk"``) or its transpose, (k, m)
+    row-major (``"km"``); B is (k, n) for ``b_layout="kn"`` or (n, k)
     for ``"nk"``; bias has length m (``"row"``: one value per output row,
     added to every column -- the pages' default broadcast) or n (``"col"``).
     Returns float64 D and pre (m, n) and a uint8 0/1 mask (m, n).
     """
     A = _storage(A, dtype)
     B = _storage(B, dtype)
-    m, k = A.shape
+    m, k = _a_shape(A, a_layout)
     n = B.shape[1] if b_layout == "kn" else B.shape[0]
     if (B.shape[0] if b_layout == "kn" else B.shape[1]) != k:
         raise ValueError("inner dimensions differ")
@@ -142,7 +154,7 @@ def gemm_epi(A, B, bias, *, dtype: str, epilogue: str, bias_axis: str = "row",
     D = np.empty((m, n), np.float64)
     pre = np.empty((m, n), np.float64)
     mask = np.empty((m, n), np.uint8)
-    rc = _load().oracle_gemm_epi(m, n, k, *_names(dtype, epilogue, bias_axis, b_layout),
+    rc = _load().oracle_gemm_epi(m, n, k, *_names(dtype, epilogue, bias_axis, b_layout, a_layout),
                                  _ptr(A), _ptr(B), _ptr(bias), float(scale_a), float(scale_b),
                                  _ptr(D), _ptr(pre), _ptr(mask))
     if rc != 0:
@@ -152,7 +164,8 @@ def gemm_epi(A, B, bias, *, dtype: str, epilogue: str, bias_axis: str = "row",
 
 def gemm_epi_sampled(A, B, bias, rows, cols, *, dtype: str, epilogue: str,
                      bias_axis: str = "row", b_layout: str = "kn", scale_a: float = 1.0,
-                     scale_b: float = 1.0, m: int | None = None, k: int | None = None):
+                     scale_b: float = 1.0, m: int | None = None, k: int | None = None,
+                     a_layout: str = "mk"):
     """(D, pre, mask) at positions (rows[s], cols[s]); one fp64 dot product each.
 
     ``A`` may be given as the full (m, k) storage array.  Same conventions as
@@ -160,7 +173,7 @@ def gemm_epi_sampled(A, B, bias, rows, cols, *, dtype: str, epilogue: str,
     """
     A = _storage(A, dtype)
     B = _storage(B, dtype)
-    m_, k_ = A.shape
+    m_, k_ = _a_shape(A, a_layout)
     m = m_ if m is None else m
     k = k_ if k is None else k
     n = B.shape[1] if b_layout == "kn" else B.shape[0]
@@ -174,7 +187,7 @@ def gemm_epi_sampled(A, B, bias, rows, cols, *, dtype: str, epilogue: str,
     D = np.empty(cnt, np.float64)
     pre = np.empty(cnt, np.float64)
     mask = np.empty(cnt, np.uint8)
-    rc = _load().oracle_gemm_epi_sampled(m, n, k, *_names(dtype, epilogue, bias_axis, b_layout),
+    rc = _load().oracle_gemm_epi_sampled(m, n, k, *_names(dtype, epilogue, bias_axis, b_layout, a_layout),
                                          _ptr(A), _ptr(B), _ptr(bias), float(scale_a),
                                          float(scale_b), cnt, _ptr(rows), _ptr(cols), _ptr(D),
                                          _ptr(pre), _ptr(mask))

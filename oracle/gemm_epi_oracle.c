@@ -94,11 +94,21 @@ static int axis_code(const char *s) {
     if (!strcmp(s, "col")) return OR_COL;
     return 0;
 }
+/* Operand storage.  B: "kn" = (k, n) row-major, "nk" = (n, k) row-major.  A is
+ * (m, k) row-major unless the layout string carries the prefix "at_" ("at_kn",
+ * "at_nk"): then A is stored transposed, (k, m) row-major. */
+enum { OR_MK = 40, OR_KM = 41 };
+static int a_layout_of(const char *s) { return (s && !strncmp(s, "at_", 3)) ? OR_KM : OR_MK; }
 static int layout_code(const char *s) {
     if (!s) return 0;
+    if (!strncmp(s, "at_", 3)) s += 3;
     if (!strcmp(s, "kn")) return OR_KN;
     if (!strcmp(s, "nk")) return OR_NK;
     return 0;
+}
+/* Where element (i, t) of the (m, k) operand A is stored. */
+static int64_t a_index(int la, int64_t i, int64_t t, int64_t m, int64_t k) {
+    return la == OR_MK ? i * k + t : t * m + i;
 }
 
 /* ---- format decoding, written from each format's bit-level definition ----- */
@@ -211,7 +221,7 @@ int oracle_gemm_epi(int64_t m, int64_t n, int64_t k, const char *dtype, const ch
                     const void *bias, double scale_a, double scale_b, double *D_ref,
                     double *pre_ref, uint8_t *mask_ref) {
     int dt = dtype_code(dtype), epi = epi_code(epilogue), axis = axis_code(bias_axis);
-    int lay = layout_code(b_layout);
+    int lay = layout_code(b_layout), la = a_layout_of(b_layout);
     if (check_args(m, n, k, dt, epi, axis, lay, A, B, bias) || !D_ref) return -1;
     double alpha = scale_a * scale_b;
     int bdt = bias_dtype(dt);
@@ -235,7 +245,7 @@ int oracle_gemm_epi(int64_t m, int64_t n, int64_t k, const char *dtype, const ch
             if (!row) continue;
             for (int64_t j = 0; j < n; ++j) row[j] = 0.0;
             for (int64_t t = 0; t < k; ++t) {
-                double a = load(A, dt, i * k + t);
+                double a = load(A, dt, a_index(la, i, t, m, k));
                 const double *brow = Bd + t * n;
                 for (int64_t j = 0; j < n; ++j) row[j] += a * brow[j];
             }
@@ -261,7 +271,7 @@ int oracle_gemm_epi_sampled(int64_t m, int64_t n, int64_t k, const char *dtype,
                             const int64_t *cols, double *D_ref, double *pre_ref,
                             uint8_t *mask_ref) {
     int dt = dtype_code(dtype), epi = epi_code(epilogue), axis = axis_code(bias_axis);
-    int lay = layout_code(b_layout);
+    int lay = layout_code(b_layout), la = a_layout_of(b_layout);
     if (check_args(m, n, k, dt, epi, axis, lay, A, B, bias) || !D_ref || !rows || !cols ||
         count < 0)
         return -1;
@@ -274,7 +284,7 @@ int oracle_gemm_epi_sampled(int64_t m, int64_t n, int64_t k, const char *dtype,
         int64_t i = rows[s], j = cols[s];
         double p = 0.0;
         for (int64_t t = 0; t < k; ++t)
-            p += load(A, dt, i * k + t) * load(B, dt, lay == OR_KN ? t * n + j : j * k + t);
+            p += load(A, dt, a_index(la, i, t, m, k)) * load(B, dt, lay == OR_KN ? t * n + j : j * k + t);
         finish(p, epi, axis, bdt, bias, i, j, alpha, &D_ref[s], pre_ref ? &pre_ref[s] : NULL,
                mask_ref ? &mask_ref[s] : NULL);
     }
@@ -302,6 +312,7 @@ int oracle_gemm_epi_bwd(int64_t m, int64_t n, int64_t k, const char *dtype, cons
                         const uint8_t *mask, double scale_a, double scale_b, double *D_ref,
                         double *dbias_ref) {
     int dt = dtype_code(dtype), axis = axis_code(bias_axis), lay = layout_code(b_layout);
+    int la = a_layout_of(b_layout);
     int bgrad;
     if (!epilogue) return -1;
     if (!strcmp(epilogue, "drelu")) bgrad = 0;
@@ -329,7 +340,7 @@ int oracle_gemm_epi_bwd(int64_t m, int64_t n, int64_t k, const char *dtype, cons
             if (!row) continue;
             for (int64_t j = 0; j < n; ++j) row[j] = 0.0;
             for (int64_t t = 0; t < k; ++t) {
-                double a = load(A, dt, i * k + t);
+                double a = load(A, dt, a_index(la, i, t, m, k));
                 const double *brow = Bd + t * n;
                 for (int64_t j = 0; j < n; ++j) row[j] += a * brow[j];
             }

@@ -24,7 +24,9 @@ MUTANTS = [
      "lay == OR_KN ? j * k + t : t * n + j", 0),
     ("b_transposed_sampled", "lay == OR_KN ? t * n + j : j * k + t",
      "lay == OR_KN ? j * k + t : t * n + j", 1),
-    ("a_index_wrong", "load(A, dt, i * k + t)", "load(A, dt, t * m + i)", None),
+    ("a_index_wrong", "return la == OR_MK ? i * k + t : t * m + i;", "return la == OR_MK ? t * m + i : t * m + i;", None),
+    ("a_transposed_index_wrong", "return la == OR_MK ? i * k + t : t * m + i;", "return la == OR_MK ? i * k + t : i * k + t;", None),
+    ("a_layout_ignored", "return (s && !strncmp(s, \"at_\", 3)) ? OR_KM : OR_MK;", "return OR_MK;", None),
     ("gelu_sign", "0.5 * x * (1.0 + erf(", "0.5 * x * (1.0 - erf(", None),
     ("gelu_tanh_form", "0.5 * x * (1.0 + erf(x / sqrt(2.0)))",
      "0.5 * x * (1.0 + tanh(0.7978845608028654 * (x + 0.044715 * x * x * x)))", None),

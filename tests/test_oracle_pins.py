@@ -507,3 +507,31 @@ def test_mlp_equals_two_numpy_products(oracle_lib, layout):
     assert amax == np.abs(H).max()
     want = Hs.view(np.float16).astype(np.float64) @ W2.astype(np.float64) + b2.astype(np.float64)
     np.testing.assert_allclose(Y, want, rtol=1e-14, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- A stored transposed
+@pytest.mark.parametrize("c", [c for c in CASES if c["dtype"] != "e4m3" or "e4m3_codes" not in c],
+                         ids=[c["id"] for c in CASES if c["dtype"] != "e4m3" or "e4m3_codes" not in c])
+def test_golden_cases_with_a_stored_transposed(oracle_lib, c):
+    """Every hand-computed case again, with A handed over as its (k, m) transpose."""
+    a, b, bias = _case_inputs(c)
+    at = np.ascontiguousarray(a.reshape(len(c["a"]), -1).T)
+    kw = dict(dtype=c["dtype"], epilogue=c["epilogue"], bias_axis=c["bias_axis"], b_layout=c["b_layout"],
+              scale_a=c.get("scale_a", 1.0), scale_b=c.get("scale_b", 1.0))
+    D, pre, mask = oracle_lib.gemm_epi(at, b, bias, a_layout="km", **kw)
+    np.testing.assert_allclose(D, np.array(c["d"], dtype=np.float64), rtol=c.get("rtol", 0.0), atol=0.0)
+    np.testing.assert_array_equal(mask, np.array(c["mask"], dtype=np.uint8))
+    rows, cols = np.meshgrid(np.arange(D.shape[0]), np.arange(D.shape[1]), indexing="ij")
+    Ds, _, _ = oracle_lib.gemm_epi_sampled(at, b, bias, rows.ravel(), cols.ravel(), a_layout="km", **kw)
+    np.testing.assert_array_equal(Ds, D.ravel())
+
+
+def test_a_transposed_non_square_matches_numpy(oracle_lib):
+    """m != k, so a swapped index cannot go unnoticed: numpy's product of the decoded values."""
+    rng = np.random.default_rng(9)
+    m, k, n = 5, 7, 3
+    a = rng.integers(-3, 4, (m, k)).astype(np.float16)
+    b = rng.integers(-3, 4, (k, n)).astype(np.float16)
+    at = np.ascontiguousarray(a.T).view(np.uint16)
+    D, _, _ = oracle_lib.gemm_epi(at, b.view(np.uint16), None, dtype="f16", epilogue="none", a_layout="km")
+    np.testing.assert_array_equal(D, a.astype(np.float64) @ b.astype(np.float64))
