@@ -30,7 +30,8 @@ constexpr uint64_t kPlanMagic = 0x67656d6d5f657069ull;   // "gemm_epi"
 struct Plan {
     uint64_t magic;
     int64_t m, n, k;
-    int dtype, epilogue, axis, b_layout;
+    int dtype, epilogue, axis, b_layout;   // b_layout: GEMM_EPI_B_KN or GEMM_EPI_B_NK
+    bool a_km;           // A stored (k, m) row-major (layout flag GEMM_EPI_A_KM)
     int kepi;            // kernel epilogue (EPI_*): the activation
     bool has_bias;       // the public epilogue adds a bias
     bool bwd, bgrad;     // backward epilogue (DRELU*); with a bias gradient (DRELU_BGRAD)
@@ -173,11 +174,11 @@ int choose(Plan *P) {
         const int64_t pair_tiles = ((m + 255) / 256) * ((n + 255) / 256);
         const int sms_auto = P->opts.max_ctas > 0 ? std::min(P->opts.max_ctas, P->num_sms) : P->num_sms;
         // (the split-K kernel has no backward epilogue)
-        if (m <= 64 && P->kepi != EPI_DRELU && !P->qout) kernel = GEMM_EPI_KERNEL_SPLITK;
+        if (m <= 64 && P->kepi != EPI_DRELU && !P->a_km) kernel = GEMM_EPI_KERNEL_SPLITK;
         else if (pair_tiles >= sms_auto / 2) kernel = GEMM_EPI_KERNEL_TC2;
         else kernel = GEMM_EPI_KERNEL_TC1;
     }
-    if (kernel == GEMM_EPI_KERNEL_SPLITK && (m > 128 || P->kepi == EPI_DRELU || P->qout))
+    if (kernel == GEMM_EPI_KERNEL_SPLITK && (m > 128 || P->kepi == EPI_DRELU || P->a_km))
         return GEMM_EPI_ERR_UNSUPPORTED;
     P->kernel = kernel;
     const bool b_mn = P->b_layout == GEMM_EPI_B_KN;
@@ -202,9 +203,9 @@ int choose(Plan *P) {
         P->split = split;
         P->grid = (int)(tiles_n * split);
         KernelInfo none_info;
-        if (!find_sk(P->dtype, GEMM_EPI_NONE, 0, b_mn, P->nm, &P->sk_none_launch, &none_info))
+        if (!find_sk(P->dtype, GEMM_EPI_NONE, 0, b_mn, P->nm, false, &P->sk_none_launch, &none_info))
             return GEMM_EPI_ERR_UNSUPPORTED;
-        if (!find_sk(P->dtype, P->kepi, P->axis, b_mn, P->nm, &P->sk_launch, &P->info))
+        if (!find_sk(P->dtype, P->kepi, P->axis, b_mn, P->nm, P->qout, &P->sk_launch, &P->info))
             return GEMM_EPI_ERR_UNSUPPORTED;
     } else {
         const int cg = kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
@@ -215,6 +216,7 @@ int choose(Plan *P) {
             bn = tiles256 >= sms / cg ? 256 : 128;
             // a pair's e4m3 B half-tile stored (k, n) must be a whole 128-byte box: 128 columns
             if (cg == 2 && P->dtype == GEMM_EPI_E4M3 && b_mn) bn = 256;
+            if (P->a_km) bn = 256;     // A stored (k, m) is built with 256-wide tiles only
         }
         if (bn != 128 && bn != 256) return GEMM_EPI_ERR_ARG;
         P->block_n = bn;
@@ -250,9 +252,9 @@ int choose(Plan *P) {
             if (v >= 1 && v <= 64) P->group_m = v;
         }
         KernelInfo none_info;
-        if (!find_tc(cg, P->dtype, GEMM_EPI_NONE, 0, b_mn, bn, false, &P->tc_none_launch, &none_info))
+        if (!find_tc(cg, P->dtype, GEMM_EPI_NONE, 0, b_mn, bn, false, P->a_km, &P->tc_none_launch, &none_info))
             return GEMM_EPI_ERR_UNSUPPORTED;
-        if (!find_tc(cg, P->dtype, P->kepi, P->axis, b_mn, bn, P->qout, &P->tc_launch, &P->info))
+        if (!find_tc(cg, P->dtype, P->kepi, P->axis, b_mn, bn, P->qout, P->a_km, &P->tc_launch, &P->info))
             return GEMM_EPI_ERR_UNSUPPORTED;
         P->split = 1;
     }
@@ -315,7 +317,7 @@ int ensure_maps(Plan *P, const void *A, const void *B, void *D) {
     } else {
         const int cg = P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
         const int bn_local = P->block_n / cg;
-        ok = ok && make_map(&P->tmA, dt, A, k, m, bk, 128);
+        ok = ok && (P->a_km ? make_map(&P->tmA, dt, A, m, k, box_n, bk) : make_map(&P->tmA, dt, A, k, m, bk, 128));
         ok = ok && (b_kn ? make_map(&P->tmB, dt, B, n, k, box_n, bk) : make_map(&P->tmB, dt, B, k, n, bk, bn_local));
         const int out_dt = dt == GEMM_EPI_E4M3 ? GEMM_EPI_BF16 : dt;
         if (P->qout)   // e4m3 output goes out with direct stores; the map is valid but unused
@@ -357,6 +359,9 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.scale_a = P->scale_a;
         L.p.scale_b = P->scale_b;
         L.p.status = P->status;
+        L.p.dq = P->qout ? static_cast<uint8_t *>(D) : nullptr;
+        L.p.out_scale = P->out_scale;
+        L.p.amax = reinterpret_cast<unsigned int *>(P->amax);
         L.grid = P->grid;
         L.cluster = P->split;
         L.pdl = P->pdl;
@@ -408,7 +413,9 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     if (dtype < GEMM_EPI_F16 || dtype > GEMM_EPI_E4M3) return GEMM_EPI_ERR_ARG;
     if (epilogue < GEMM_EPI_NONE || epilogue > GEMM_EPI_DRELU_BGRAD) return GEMM_EPI_ERR_ARG;
     if (bias_axis != GEMM_EPI_BIAS_ROW && bias_axis != GEMM_EPI_BIAS_COL) return GEMM_EPI_ERR_ARG;
-    if (b_layout != GEMM_EPI_B_KN && b_layout != GEMM_EPI_B_NK) return GEMM_EPI_ERR_ARG;
+    if (b_layout & ~(GEMM_EPI_B_NK | GEMM_EPI_A_KM)) return GEMM_EPI_ERR_ARG;
+    const bool a_km = (b_layout & GEMM_EPI_A_KM) != 0;
+    b_layout &= GEMM_EPI_B_NK;
     gemm_epi_options o{};
     if (opts) o = *opts;
     if (o.kernel < GEMM_EPI_KERNEL_AUTO || o.kernel > GEMM_EPI_KERNEL_SPLITK) return GEMM_EPI_ERR_ARG;
@@ -419,16 +426,17 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     if (o.inject_stall && o.kernel == GEMM_EPI_KERNEL_SPLITK) return GEMM_EPI_ERR_UNSUPPORTED;
     if (o.out_e4m3 != 0 && o.out_e4m3 != 1) return GEMM_EPI_ERR_ARG;
     if (o.out_e4m3) {
-        // FP8 output: e4m3 operands, forward epilogues without a mask or tanh, persistent kernels
+        // FP8 output: e4m3 operands, forward epilogues without a mask or tanh
         const bool epi_ok = epilogue == GEMM_EPI_NONE || epilogue == GEMM_EPI_BIAS || epilogue == GEMM_EPI_RELU_BIAS ||
                             epilogue == GEMM_EPI_GELU_BIAS || epilogue == GEMM_EPI_RELU || epilogue == GEMM_EPI_GELU;
-        if (dtype != GEMM_EPI_E4M3 || !epi_ok || o.kernel == GEMM_EPI_KERNEL_SPLITK) return GEMM_EPI_ERR_UNSUPPORTED;
+        if (dtype != GEMM_EPI_E4M3 || !epi_ok) return GEMM_EPI_ERR_UNSUPPORTED;
     }
     // 16-byte row pitches (TMA strides; the pages' 16-byte alignment rule)
     const int es = esize(dtype);
     const int out_es = 2;
     if ((k * es) % 16 != 0) return GEMM_EPI_ERR_ALIGN;
     if ((n * es) % 16 != 0 || (n * out_es) % 16 != 0) return GEMM_EPI_ERR_ALIGN;
+    if (a_km && (m * es) % 16 != 0) return GEMM_EPI_ERR_ALIGN;     // A (k, m): row pitch m * esize
 
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -455,6 +463,7 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     P->qout = o.out_e4m3 == 1;
     P->axis = (P->has_bias || P->bgrad) ? bias_axis : GEMM_EPI_BIAS_ROW;
     P->b_layout = b_layout;
+    P->a_km = a_km;
     P->opts = o;
     P->device = dev;
     P->num_sms = num_sms_of(dev);
@@ -517,10 +526,19 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
 
 // ----------------------------------------------------------------- lookups
 namespace gemm_epi {
-bool find_tc(int cg, int dt, int epi, int axis, bool b_mn, int bn, bool qout, TcLauncher *l, KernelInfo *i) {
+bool find_tc(int cg, int dt, int epi, int axis, bool b_mn, int bn, bool qout, bool a_mn, TcLauncher *l,
+             KernelInfo *i) {
     KernelInfo tmp;
     if (!i) i = &tmp;
-    if (qout) return dt == DT_E4M3 && find_tc_e4m3_q(cg, epi, axis, b_mn, bn, l, i);
+    if (qout) return !a_mn && dt == DT_E4M3 && find_tc_e4m3_q(cg, epi, axis, b_mn, bn, l, i);
+    if (a_mn) {
+        switch (dt) {
+        case DT_F16: return find_tc_f16_at(cg, epi, axis, b_mn, bn, l, i);
+        case DT_BF16: return find_tc_bf16_at(cg, epi, axis, b_mn, bn, l, i);
+        case DT_E4M3: return find_tc_e4m3_at(cg, epi, axis, b_mn, bn, l, i);
+        }
+        return false;
+    }
     switch (dt) {
     case DT_F16: return find_tc_f16(cg, epi, axis, b_mn, bn, l, i);
     case DT_BF16: return find_tc_bf16(cg, epi, axis, b_mn, bn, l, i);
@@ -528,9 +546,10 @@ bool find_tc(int cg, int dt, int epi, int axis, bool b_mn, int bn, bool qout, Tc
     }
     return false;
 }
-bool find_sk(int dt, int epi, int axis, bool w_mn, int nm, SkLauncher *l, KernelInfo *i) {
+bool find_sk(int dt, int epi, int axis, bool w_mn, int nm, bool qout, SkLauncher *l, KernelInfo *i) {
     KernelInfo tmp;
     if (!i) i = &tmp;
+    if (qout) return dt == DT_E4M3 && find_sk_e4m3_q(epi, axis, w_mn, nm, l, i);
     switch (dt) {
     case DT_F16: return find_sk_f16(epi, axis, w_mn, nm, l, i);
     case DT_BF16: return find_sk_bf16(epi, axis, w_mn, nm, l, i);
@@ -774,6 +793,7 @@ int gemm_epi_mlp_plan(int64_t m, int64_t d_model, int64_t d_ff, int dtype, int a
                       gemm_epi_mlp_t *out) {
     if (!out) return GEMM_EPI_ERR_ARG;
     if (act != GEMM_EPI_BIAS && act != GEMM_EPI_RELU_BIAS && act != GEMM_EPI_GELU_BIAS) return GEMM_EPI_ERR_ARG;
+    if (w_layout != GEMM_EPI_B_KN && w_layout != GEMM_EPI_B_NK) return GEMM_EPI_ERR_ARG;
     Mlp *M = new (std::nothrow) Mlp();
     if (!M) return GEMM_EPI_ERR_CUDA;
     M->magic = kMlpMagic;
@@ -824,6 +844,48 @@ int gemm_epi_mlp_run(gemm_epi_mlp_t mlp, const void *X, const void *W1, const vo
     rc = launch_main(U, true, b1, H, nullptr, s);
     if (rc != GEMM_EPI_OK) return rc;
     return launch_main(Dn, true, b2, Y, nullptr, s);
+}
+
+int gemm_epi_mlp_unfused_run(gemm_epi_mlp_t mlp, const void *X, const void *W1, const void *b1, const void *W2,
+                             const void *b2, void *H, void *Y, void *H_wide, void *stream) {
+    Mlp *M = mlp_live(mlp);
+    if (!M) return GEMM_EPI_ERR_ARG;
+    Plan *U = reinterpret_cast<Plan *>(M->up), *Dn = reinterpret_cast<Plan *>(M->down);
+    const bool fp8 = U->qout;
+    if (fp8 && !H_wide) return GEMM_EPI_ERR_NULL;
+    if (fp8 && !aligned16(H_wide)) return GEMM_EPI_ERR_ALIGN;
+    int rc = check_run_args(U, X, W1, b1, H, nullptr);
+    if (rc == GEMM_EPI_OK) rc = check_run_args(Dn, H, W2, b2, Y, nullptr);
+    if (rc != GEMM_EPI_OK) return rc;
+    // the up-projection as a bare GEMM writing the 16-bit type (bf16 for e4m3 operands):
+    // a copy of its plan without the FP8 output, with its own tensor maps
+    Plan Uc = *U;
+    Uc.qout = false;
+    Uc.maps_valid = false;
+    void *Hout = fp8 ? H_wide : H;
+    BiasActLauncher ba = nullptr;
+    if (!find_bias_act(U->dtype, U->kepi, U->axis, &ba)) return GEMM_EPI_ERR_UNSUPPORTED;
+    rc = ensure_maps(&Uc, X, W1, Hout);
+    if (rc == GEMM_EPI_OK) rc = ensure_maps(Dn, H, W2, Y);
+    if (rc != GEMM_EPI_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    rc = launch_main(&Uc, false, nullptr, Hout, nullptr, s);
+    if (rc != GEMM_EPI_OK) return rc;
+    const int64_t count = U->m * U->n;
+    const int64_t pitch_words = ((U->n + 127) / 128) * 4;
+    const int64_t blocks = std::min<int64_t>((U->m * pitch_words + 255) / 256, (int64_t)U->num_sms * 16);
+    if (ba(Hout, b1, nullptr, (int)U->m, (int)U->n, pitch_words, (int)blocks, s) != cudaSuccess)
+        return GEMM_EPI_ERR_CUDA;
+    if (fp8) {
+        const int grid = (int)std::min<int64_t>((count / 8 + 255) / 256, (int64_t)U->num_sms * 16);
+        if (U->amax && (cudaMemsetAsync(U->amax, 0, sizeof(float), s) != cudaSuccess ||
+                        launch_amax_bf16(H_wide, count, reinterpret_cast<unsigned int *>(U->amax), grid, s) !=
+                            cudaSuccess))
+            return GEMM_EPI_ERR_CUDA;
+        if (launch_quantize_bf16_e4m3(H_wide, count, U->out_scale, static_cast<uint8_t *>(H), grid, s) != cudaSuccess)
+            return GEMM_EPI_ERR_CUDA;
+    }
+    return gemm_epi_unfused_run(M->down, H, W2, b2, Y, nullptr, stream);
 }
 
 int gemm_epi_mlp_check(gemm_epi_mlp_t mlp, void *stream) {
@@ -907,10 +969,11 @@ extern "C" int gemm_epi_run_noalloc(int64_t m, int64_t n, int64_t k, int dtype, 
     if (dtype < GEMM_EPI_F16 || dtype > GEMM_EPI_E4M3) return GEMM_EPI_ERR_ARG;
     if (epilogue < GEMM_EPI_NONE || epilogue > GEMM_EPI_TANH) return GEMM_EPI_ERR_ARG;
     if (bias_axis != GEMM_EPI_BIAS_ROW && bias_axis != GEMM_EPI_BIAS_COL) return GEMM_EPI_ERR_ARG;
-    if (b_layout != GEMM_EPI_B_KN && b_layout != GEMM_EPI_B_NK) return GEMM_EPI_ERR_ARG;
+    if (b_layout & ~(GEMM_EPI_B_NK | GEMM_EPI_A_KM)) return GEMM_EPI_ERR_ARG;
     if (wait != 0 && wait != 1) return GEMM_EPI_ERR_ARG;
     const int es = esize(dtype);
     if ((k * es) % 16 != 0 || (n * es) % 16 != 0 || (n * 2) % 16 != 0) return GEMM_EPI_ERR_ALIGN;
+    if ((b_layout & GEMM_EPI_A_KM) && (m * es) % 16 != 0) return GEMM_EPI_ERR_ALIGN;
     // the call needs kNoallocNeededBytes of scratch; anything larger than the array is refused
     if (kNoallocNeededBytes > kNoallocScratchBytes) return GEMM_EPI_ERR_UNSUPPORTED;
 
@@ -934,7 +997,8 @@ extern "C" int gemm_epi_run_noalloc(int64_t m, int64_t n, int64_t k, int dtype, 
     P.kepi = kernel_epi(epilogue);
     P.has_bias = epi_has_bias(epilogue);
     P.axis = P.has_bias ? bias_axis : GEMM_EPI_BIAS_ROW;
-    P.b_layout = b_layout;
+    P.b_layout = b_layout & GEMM_EPI_B_NK;
+    P.a_km = (b_layout & GEMM_EPI_A_KM) != 0;
     P.device = dev;
     P.num_sms = num_sms_of(dev);
     P.opts.stream_k = 1;                        // stream-K would need a workspace: off

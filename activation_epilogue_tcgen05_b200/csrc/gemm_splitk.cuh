@@ -40,11 +40,17 @@ struct SkParams {
     const float *scale_a;
     const float *scale_b;
     unsigned int *status;
+    // FP8 output (QOUT kernels): D = e4m3(y / *out_scale), one byte per element; amax
+    // (optional) receives max |y| as float bits through an atomic max
+    uint8_t *dq;
+    const float *out_scale;
+    unsigned int *amax;
 };
 
-template <int DT_, int EPI_, int AXIS_, bool W_MN_, int NM_, int STAGES_>
+template <int DT_, int EPI_, int AXIS_, bool W_MN_, int NM_, int STAGES_, bool QOUT_ = false>
 struct SkCfg {
     static constexpr int DT = DT_, EPI = EPI_, AXIS = AXIS_, NM = NM_, STAGES = STAGES_;
+    static constexpr bool QOUT = QOUT_;             // e4m3 output quantised in the epilogue
     static constexpr bool W_MN = W_MN_;             // weight stored (k, n): MMA operand A is MN-major
     static constexpr int ESIZE = DT == DT_E4M3 ? 1 : 2;
     static constexpr int KIND = DT == DT_E4M3 ? 1 : 0;
@@ -72,6 +78,7 @@ struct SkCfg {
     static_assert(NM % 16 == 0 && NM >= 16 && NM <= 128, "MMA N for M = 128");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(X_BYTES % 1024 == 0, "stage alignment");
+    static_assert(!QOUT || (DT == DT_E4M3 && EPI != EPI_RELU_AUX), "FP8 output: e4m3 forward plans");
 };
 
 // grid = tiles_n * S CTAs, cluster (S, 1, 1): cluster c owns output columns
@@ -265,6 +272,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if (col_ok && has_bias) cbias = O::load(p.bias, col);
         }
         T *D = reinterpret_cast<T *>(p.D);
+        float inv_out = 1.0f, amax_l = 0.0f;
+        if constexpr (C::QOUT) inv_out = 1.0f / __ldg(p.out_scale);
         // every word of the mask pitch belongs to exactly one warp of one tile;
         // columns at or past n contribute 0 bits, so padding words come out 0
         const int64_t word = (n0 + 32 * q) / 32;
@@ -283,10 +292,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
                 const float y = activate<C::EPI>(x);
                 if (col_ok) {
-                    if constexpr (C::DT == DT_F16) D[(int64_t)i * p.n + col] = __float2half_rn(y);
-                    else D[(int64_t)i * p.n + col] = __float2bfloat16_rn(y);
+                    if constexpr (C::QOUT) {
+                        // e4m3 code, round to nearest even, saturating at +-448
+                        amax_l = fmaxf(amax_l, fabsf(y));
+                        p.dq[(int64_t)i * p.n + col] = __nv_cvt_float_to_fp8(y * inv_out, __NV_SATFINITE, __NV_E4M3);
+                    } else if constexpr (C::DT == DT_F16) {
+                        D[(int64_t)i * p.n + col] = __float2half_rn(y);
+                    } else {
+                        D[(int64_t)i * p.n + col] = __float2bfloat16_rn(y);
+                    }
                 }
             }
+        }
+        if constexpr (C::QOUT) {
+            // one atomic per warp: the launch's max |y| (non-negative floats order as their bits)
+            const unsigned int wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax_l));
+            if (lane == 0 && p.amax != nullptr) atomicMax(p.amax, wmax);
         }
     }
 

@@ -304,10 +304,12 @@ __device__ __forceinline__ float activate(float x) {
     }
 }
 
-template <int DT_, int EPI_, int AXIS_, bool B_MN_, int BN_, int CG_, int STAGES_, bool QOUT_ = false>
+template <int DT_, int EPI_, int AXIS_, bool B_MN_, int BN_, int CG_, int STAGES_, bool QOUT_ = false,
+          bool A_MN_ = false>
 struct TcCfg {
     static constexpr int DT = DT_, EPI = EPI_, AXIS = AXIS_, BN = BN_, CG = CG_, STAGES = STAGES_;
     static constexpr bool B_MN = B_MN_;             // B stored (k, n): N contiguous
+    static constexpr bool A_MN = A_MN_;             // A stored (k, m): M contiguous
     static constexpr int ESIZE = DT == DT_E4M3 ? 1 : 2;
     static constexpr int KIND = DT == DT_E4M3 ? 1 : 0;
     static constexpr uint32_t FMT = DT == DT_BF16 ? 1u : 0u;
@@ -321,6 +323,9 @@ struct TcCfg {
     static constexpr int B_BOX_N = 128 / ESIZE;     // n per 128-byte MN-major box
     static constexpr int B_BOXES = B_MN ? BN_LOCAL / B_BOX_N : 1;
     static constexpr int B_BOX_BYTES = B_MN ? BK * 128 : B_BYTES;
+    static constexpr int A_BOX_M = 128 / ESIZE;     // m per 128-byte MN-major box
+    static constexpr int A_BOXES = A_MN ? BM / A_BOX_M : 1;
+    static constexpr int A_BOX_BYTES = A_MN ? BK * 128 : A_BYTES;
     // GELU / tanh cost ~20 instructions an element: two epilogue warps per TMEM lane
     // quadrant (each taking half the columns) so that the epilogue keeps up with the
     // next tile's mainloop; the cheap epilogues use one warp per quadrant.
@@ -356,6 +361,7 @@ struct TcCfg {
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "stage alignment");
     static_assert(!BWD || (EPI_WARPS == 4 && CPG == 4), "backward epilogue: one mask uint4 per chunk group");
     static_assert(!QOUT || (DT == DT_E4M3 && !BWD && EPI != EPI_RELU_AUX), "FP8 output: e4m3 forward plans");
+    static_assert(!A_MN || BM % A_BOX_M == 0, "MN-major A tile must be whole boxes");
 };
 
 // Tile index -> (tile_m, tile_n) with a grouped raster: GROUP_M tile-rows are
@@ -463,7 +469,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         else
                             ptx::tma_load_2d(dst, map, fb, c0, c1, 0x1000000000000000ull);
                     };
-                    load(a_dst, &tmA, k0, m0);
+                    if constexpr (C::A_MN) {
+#pragma unroll
+                        for (int b = 0; b < C::A_BOXES; ++b)
+                            load(a_dst + b * C::A_BOX_BYTES, &tmA, m0 + b * C::A_BOX_M, k0);
+                    } else {
+                        load(a_dst, &tmA, k0, m0);
+                    }
                     if constexpr (C::B_MN) {
 #pragma unroll
                         for (int b = 0; b < C::B_BOXES; ++b)
@@ -485,7 +497,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && leader) {
-            constexpr uint32_t idesc = make_idesc(C::FMT, false, C::B_MN, 128 * C::CG, C::BN);
+            constexpr uint32_t idesc = make_idesc(C::FMT, C::A_MN, C::B_MN, 128 * C::CG, C::BN);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             bool ok = true;
             // with inject_stall nothing is issued or committed: the epilogue's
@@ -511,7 +523,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const uint32_t b_base = sB + stage * C::B_BYTES;
 #pragma unroll
                     for (int ks = 0; ks < C::KSTEPS; ++ks) {
-                        const uint64_t ad = make_sdesc(a_base + ks * 32, 16, 1024);
+                        const uint64_t ad = C::A_MN ? make_sdesc(a_base + ks * C::UMMA_K * 128, C::A_BOX_BYTES, 1024)
+                                                    : make_sdesc(a_base + ks * 32, 16, 1024);
                         const uint64_t bd = C::B_MN ? make_sdesc(b_base + ks * C::UMMA_K * 128, C::B_BOX_BYTES, 1024)
                                                     : make_sdesc(b_base + ks * 32, 16, 1024);
                         ptx::mma<C::CG, C::KIND>(d_tmem, ad, bd, idesc, (kb > w.kb0 || ks > 0) ? 1u : 0u);

@@ -24,6 +24,7 @@ TANH_BIAS, RELU, RELU_AUX, GELU, TANH = 5, 6, 7, 8, 9
 DRELU, DRELU_BGRAD = 10, 11
 BIAS_ROW, BIAS_COL = 0, 1
 B_KN, B_NK = 0, 1
+A_KM = 2          # layout flag: A stored (k, m)
 KERNEL_AUTO, KERNEL_TC1, KERNEL_TC2, KERNEL_SPLITK = 0, 1, 2, 3
 OK, ERR_ARG, ERR_ALIGN, ERR_NULL, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NO_DEVICE = \
     0, -1, -2, -3, -4, -5, -6, -7
@@ -46,7 +47,7 @@ EXPORTS = ("gemm_epi_plan", "gemm_epi_plan_ex", "gemm_epi_plan_opts", "gemm_epi_
            "gemm_epi_free", "gemm_epi_status_string", "gemm_epi_aux_pitch_bytes",
            "gemm_epi_version", "gemm_epi_run_noalloc", "gemm_epi_run_bwd", "gemm_epi_unfused_run_bwd",
            "gemm_epi_set_out_scale", "gemm_epi_mlp_plan", "gemm_epi_mlp_set_scales", "gemm_epi_mlp_run",
-           "gemm_epi_mlp_check", "gemm_epi_mlp_query", "gemm_epi_mlp_free")
+           "gemm_epi_mlp_check", "gemm_epi_mlp_query", "gemm_epi_mlp_free", "gemm_epi_mlp_unfused_run")
 
 
 class Options(ctypes.Structure):
@@ -100,6 +101,7 @@ def lib():
             L.gemm_epi_mlp_plan.argtypes = [i64, i64, i64, i32, i32, i32, pp]
             L.gemm_epi_mlp_set_scales.argtypes = [vp, vp, vp, vp, vp, vp]
             L.gemm_epi_mlp_run.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            L.gemm_epi_mlp_unfused_run.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
             L.gemm_epi_mlp_check.argtypes = [vp, vp]
             L.gemm_epi_mlp_query.argtypes = [vp, ctypes.POINTER(PlanInfo), ctypes.POINTER(PlanInfo)]
             L.gemm_epi_mlp_free.argtypes = [vp]
@@ -119,7 +121,7 @@ def lib():
                          "gemm_epi_version", "gemm_epi_run_noalloc", "gemm_epi_run_bwd",
                          "gemm_epi_unfused_run_bwd", "gemm_epi_set_out_scale", "gemm_epi_mlp_plan",
                          "gemm_epi_mlp_set_scales", "gemm_epi_mlp_run", "gemm_epi_mlp_check",
-                         "gemm_epi_mlp_query", "gemm_epi_mlp_free"):
+                         "gemm_epi_mlp_query", "gemm_epi_mlp_free", "gemm_epi_mlp_unfused_run"):
                 getattr(L, name).restype = i32
             _lib = L
     return _lib
@@ -185,6 +187,11 @@ def gemm_epi_mlp_set_scales(mlp, d_scale_x, d_scale_w1, d_scale_h, d_amax_h, d_s
 
 def gemm_epi_mlp_run(mlp, X, W1, b1, W2, b2, H, Y, stream) -> None:
     _check(lib().gemm_epi_mlp_run(mlp, X, W1, b1, W2, b2, H, Y, stream), "gemm_epi_mlp_run")
+
+
+def gemm_epi_mlp_unfused_run(mlp, X, W1, b1, W2, b2, H, Y, H_wide, stream) -> None:
+    _check(lib().gemm_epi_mlp_unfused_run(mlp, X, W1, b1, W2, b2, H, Y, H_wide, stream),
+           "gemm_epi_mlp_unfused_run")
 
 
 def gemm_epi_mlp_check(mlp, stream) -> None:
@@ -261,13 +268,14 @@ class Plan:
 
     def __init__(self, m, n, k, dtype="bf16", epilogue="bias", bias_axis="row", b_layout="kn",
                  kernel="auto", block_n=0, split_k=0, max_ctas=0, inject_stall=0, stream_k="auto",
-                 out_e4m3=False):
+                 out_e4m3=False, a_layout="mk"):
         self.m, self.n, self.k = int(m), int(n), int(k)
         self.dtype, self.epilogue, self.bias_axis, self.b_layout = dtype, epilogue, bias_axis, b_layout
         opts = Options(KERNEL[kernel], int(block_n), int(split_k), int(max_ctas), int(inject_stall),
                        STREAM_K[stream_k], 1 if out_e4m3 else 0)
+        layout = LAYOUT[b_layout] | (A_KM if a_layout == "km" else 0)
         self.handle = gemm_epi_plan_opts(self.m, self.n, self.k, DTYPE[dtype], EPILOGUE[epilogue],
-                                         AXIS[bias_axis], LAYOUT[b_layout], opts)
+                                         AXIS[bias_axis], layout, opts)
         self._scales = None
 
     @property
@@ -346,9 +354,14 @@ class MlpPlan:
         gemm_epi_mlp_set_scales(self.handle, _ptr(scale_x), _ptr(scale_w1), _ptr(scale_h), _ptr(amax_h),
                                 _ptr(scale_w2))
 
-    def run(self, X, W1, b1, W2, b2, H, Y, stream=None):
-        gemm_epi_mlp_run(self.handle, _ptr(X), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(H), _ptr(Y),
-                         _stream_ptr(stream))
+    def run(self, X, W1, b1, W2, b2, H, Y, stream=None, fused=True, H_wide=None):
+        """fused=False: the unfused baseline (H_wide: bf16 (m, d_ff) scratch, e4m3 plans)."""
+        if fused:
+            gemm_epi_mlp_run(self.handle, _ptr(X), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(H), _ptr(Y),
+                             _stream_ptr(stream))
+        else:
+            gemm_epi_mlp_unfused_run(self.handle, _ptr(X), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(H),
+                                     _ptr(Y), _ptr(H_wide), _stream_ptr(stream))
 
     def check(self, stream=None):
         gemm_epi_mlp_check(self.handle, _stream_ptr(stream))

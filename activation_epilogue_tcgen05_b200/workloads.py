@@ -46,6 +46,7 @@ class Workload:
     dist_bias: tuple = ("normal", 1.0)
     seed: int = 0
     extra: dict = field(default_factory=dict, compare=False)
+    a_layout: str = "mk"        # "mk": A stored (m, k) row-major; "km": stored transposed, (k, m)
 
     @property
     def out_dtype(self) -> str:
@@ -133,14 +134,16 @@ def make_problem(wl: Workload, device="cpu", int_scales: bool = False) -> Proble
     blen = wl.m if wl.bias_axis == "row" else wl.n
     bias = _draw((blen,), wl.dist_bias, gen, device)
     bias_t = bias.to(TORCH_DTYPE[wl.out_dtype])
+    # A stored transposed holds the same values, (k, m) row-major
+    lay = (lambda x: x.t().contiguous()) if wl.a_layout == "km" else (lambda x: x)
     if wl.dtype == "e4m3":
         if int_scales:
-            return Problem(wl, a.to(torch.float8_e4m3fn), b.to(torch.float8_e4m3fn), bias_t)
+            return Problem(wl, lay(a.to(torch.float8_e4m3fn)), b.to(torch.float8_e4m3fn), bias_t)
         qa, sa = _to_e4m3(a)
         qb, sb = _to_e4m3(b)
-        return Problem(wl, qa, qb, bias_t, sa, sb)
+        return Problem(wl, lay(qa), qb, bias_t, sa, sb)
     t = TORCH_DTYPE[wl.dtype]
-    return Problem(wl, a.to(t), b.to(t), bias_t)
+    return Problem(wl, lay(a.to(t)), b.to(t), bias_t)
 
 
 def make_mask(m: int, n: int, seed: int = 0, kind: str = "bernoulli", p: float = 0.5) -> np.ndarray:

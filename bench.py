@@ -61,8 +61,8 @@ def parse(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--shape", default=None,
-                    help="custom problem m,n,k,dtype,epilogue,bias_axis,b_layout (overrides --workload; "
-                         "operands N(0,1)/64, bias N(0,1), seed 0)")
+                    help="custom problem m,n,k,dtype,epilogue,bias_axis,b_layout[,km] (overrides --workload; "
+                         "operands N(0,1)/64, bias N(0,1), seed 0; km = A stored (k, m))")
     ap.add_argument("--kernel", default="auto", choices=["auto", "tc1", "tc2", "splitk"])
     ap.add_argument("--block-n", type=int, default=0)
     ap.add_argument("--stream-k", default="auto", choices=["auto", "off", "on"])
@@ -185,10 +185,13 @@ def workload_from_args(args):
     from activation_epilogue_tcgen05_b200.workloads import WORKLOADS, Workload
     if not args.shape:
         return WORKLOADS[args.workload]
-    m, n, k, dt, epi, axis, lay = args.shape.split(",")
+    parts = args.shape.split(",")
+    m, n, k, dt, epi, axis, lay = parts[:7]
+    a_lay = parts[7] if len(parts) > 7 else "mk"
     std = 1.0 if dt == "e4m3" else 1.0 / 64
-    return Workload(f"custom_{dt}_{epi}_{m}x{n}x{k}_{lay}", int(m), int(n), int(k), dt, epi, axis, lay,
-                    ("normal", std), ("normal", std), ("normal", 1.0))
+    name = f"custom_{dt}_{epi}_{m}x{n}x{k}_{lay}" + ("_at" if a_lay == "km" else "")
+    return Workload(name, int(m), int(n), int(k), dt, epi, axis, lay,
+                    ("normal", std), ("normal", std), ("normal", 1.0), a_layout=a_lay)
 
 
 # ----------------------------------------------------------------------------- CPU oracle legs
@@ -206,8 +209,11 @@ def oracle_rows_rate(wl, prob, target_s: float, max_rows=None):
     bias_full = storage(prob.bias)
     bwd = wl.epilogue in ("drelu", "drelu_bgrad")
 
+    # the oracle reads A as (m, k); an A stored (k, m) is handed over row by row of its transpose
+    A_mk = prob.A.t() if wl.a_layout == "km" else prob.A
+
     def run(rows):
-        As = storage(prob.A[:rows])
+        As = storage(A_mk[:rows].contiguous())
         bias = bias_full[:rows] if wl.bias_axis == "row" else bias_full
         t0 = time.perf_counter()
         if bwd:
@@ -246,7 +252,8 @@ def reference_arm(args):
         prob = make_problem(wl_small, device=gen_dev)
     else:
         prob = make_problem(wl, device=gen_dev)
-    As, Bs, bias = storage(prob.A), storage(prob.B), storage(prob.bias)
+    As = storage((prob.A.t() if wl.a_layout == "km" else prob.A).contiguous())      # (m, k) for the oracle
+    Bs, bias = storage(prob.B), storage(prob.bias)
     m_avail = As.shape[0]
     rng = np.random.default_rng(0)
 
@@ -374,6 +381,33 @@ def mlp_arm(args):
     del graph
     elapsed_ms = replicas.max_over_ranks(start.elapsed_time(end), device=dev)
     clocks = sampler.summary(wall0, wall1) if sampler else None
+    # the library's own unfused sequence: bare GEMM, bias + activation kernel, (e4m3) amax and
+    # quantise passes over a bf16 H, bare GEMM, bias kernel
+    unfused = None
+    if not args.no_unfused:
+        Hw = torch.empty((m, dff), dtype=torch.bfloat16, device=dev) if dt == "e4m3" else None
+        for _ in range(3):
+            mp.run(X, W1, b1, W2, b2, H, Y, stream=stream, fused=False, H_wide=Hw)
+        torch.cuda.synchronize(dev)
+        Ku = min(K, 200)
+        ugraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ugraph):
+            cs = torch.cuda.current_stream(dev)
+            for _ in range(Ku):
+                mp.run(X, W1, b1, W2, b2, H, Y, stream=cs, fused=False, H_wide=Hw)
+        ugraph.replay()
+        torch.cuda.synchronize(dev)
+        u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        u0.record(stream)
+        ugraph.replay()
+        u1.record(stream)
+        torch.cuda.synchronize(dev)
+        mp.check(stream)
+        del ugraph
+        ums = replicas.max_over_ranks(u0.elapsed_time(u1), device=dev) / Ku
+        unfused = {"ms_per_step": ums, "value": 4.0 * m * dm * dff * world / (ums / 1000) / 1e12,
+                   "unit": "TFLOP/s", "steps": Ku, "launches_per_step": 6 if dt == "e4m3" else 4,
+                   "fused_speedup": ums / (elapsed_ms / K)}
     if sampler:
         sampler.stop()
     flops = 4.0 * m * dm * dff
@@ -399,7 +433,7 @@ def mlp_arm(args):
                          "peak_source": peak_src + (", bf16 burst x nominal fp8/bf16 ratio 2" if dt == "e4m3"
                                                     else ", bf16 burst"),
                          "note": "per-step time of both GEMM launches"},
-            "cpu_baseline": None, "e2e": None, "gpu_launches": 2 * K, "clocks": clocks,
+            "cpu_baseline": None, "e2e": None, "unfused": unfused, "gpu_launches": 2 * K, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if have_pg:
@@ -468,7 +502,8 @@ def main(argv=None):
         D = torch.empty((wl.m, wl.n), dtype=out_t, device=dev)
         sets.append((A, B, x, D, new_y()))
     plan = g.Plan(wl.m, wl.n, wl.k, wl.dtype, wl.epilogue, wl.bias_axis, wl.b_layout,
-                  kernel=args.kernel, block_n=args.block_n, stream_k=args.stream_k, split_k=args.split_k)
+                  kernel=args.kernel, block_n=args.block_n, stream_k=args.stream_k, split_k=args.split_k,
+                  a_layout=wl.a_layout)
     run = plan.run_bwd if bwd else plan.run
     if wl.dtype == "e4m3":
         plan.set_scales(torch.tensor([prob.scale_a], dtype=torch.float32, device=dev),

@@ -18,7 +18,7 @@
  *   [nvgemm]        "PyTorch 2.14 NVGEMM epilogue fusion" (zdabc.icu/article/2026/9/3/3582.html)
  *
  * Conventions for every entry point
- *   - A is row-major (m, k).  B is row-major (k, n) (GEMM_EPI_B_KN, default)
+ *   - A is row-major (m, k) (or (k, m) with the GEMM_EPI_A_KM layout flag).  B is row-major (k, n) (GEMM_EPI_B_KN, default)
  *     or row-major (n, k) (GEMM_EPI_B_NK: an nn.Linear weight, D = A . B^T).
  *   - D is row-major (m, n), densely packed (row pitch n elements).
  *   - Accumulation and all epilogue arithmetic are fp32; D is rounded to
@@ -96,8 +96,12 @@ enum gemm_epi_epilogue {
  *        (a (1,n) bias). */
 enum gemm_epi_bias_axis { GEMM_EPI_BIAS_ROW = 0, GEMM_EPI_BIAS_COL = 1 };
 
-/* Storage of B. */
-enum gemm_epi_b_layout { GEMM_EPI_B_KN = 0, GEMM_EPI_B_NK = 1 };
+/* Operand storage, passed as `b_layout`: GEMM_EPI_B_KN or GEMM_EPI_B_NK for B, optionally
+ * OR-ed with GEMM_EPI_A_KM for an A stored transposed, (k, m) row-major (m contiguous; its
+ * row pitch m*esize must be a multiple of 16 bytes).  A stored (k, m) runs on the persistent
+ * kernels with 256-wide tiles (block_n 128 is ERR_UNSUPPORTED; small m uses TC1) and the
+ * forward epilogues, not with the backward epilogues or an e4m3 output. */
+enum gemm_epi_b_layout { GEMM_EPI_B_KN = 0, GEMM_EPI_B_NK = 1, GEMM_EPI_A_KM = 2 };
 
 /* Kernel families a plan can use (GEMM_EPI_KERNEL_AUTO lets the plan choose). */
 enum gemm_epi_kernel {
@@ -149,8 +153,8 @@ typedef struct gemm_epi_options {
     int32_t out_e4m3;  /* 1 = D is e4m3, quantised in the epilogue: D = e4m3(y / s_out) with
                           round to nearest even, saturating at +-448, y the epilogue's fp32
                           result; max |y| is reported (gemm_epi_set_out_scale).  E4M3 plans
-                          with epilogue NONE, BIAS, RELU_BIAS, GELU_BIAS, RELU or GELU, on the
-                          persistent kernels (small m uses TC1); else ERR_UNSUPPORTED.
+                          with epilogue NONE, BIAS, RELU_BIAS, GELU_BIAS, RELU or GELU, on every
+                          kernel family; else ERR_UNSUPPORTED.
                           0 = D in the 16-bit output type.                              */
 } gemm_epi_options;
 
@@ -324,6 +328,15 @@ int gemm_epi_mlp_set_scales(gemm_epi_mlp_t mlp, const float *d_scale_x, const fl
 /* Enqueue both GEMMs on `stream` (all arguments are checked before either is enqueued). */
 int gemm_epi_mlp_run(gemm_epi_mlp_t mlp, const void *X, const void *W1, const void *b1, const void *W2,
                      const void *b2, void *H, void *Y, void *stream);
+
+/* The UNFUSED baseline of gemm_epi_mlp_run, same plan and arguments: bare GEMM writing the
+ * up-projection in the 16-bit type, a separate bias + activation kernel, and for e4m3 an amax
+ * pass and a quantisation pass (H_wide: caller-owned bf16 scratch, (m, d_ff); ignored, may be
+ * NULL, for 16-bit plans); then the down-projection as bare GEMM plus bias kernel.  The same
+ * result as the fused run up to the roundings it adds; the sequence the epilogues remove. */
+int gemm_epi_mlp_unfused_run(gemm_epi_mlp_t mlp, const void *X, const void *W1, const void *b1,
+                             const void *W2, const void *b2, void *H, void *Y, void *H_wide,
+                             void *stream);
 
 /* gemm_epi_check on both plans (the first non-OK status). */
 int gemm_epi_mlp_check(gemm_epi_mlp_t mlp, void *stream);

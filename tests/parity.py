@@ -33,7 +33,8 @@ def alloc_outputs(wl: Workload, device="cuda"):
 
 
 def make_plan(wl: Workload, prob: Problem, device="cuda", **opts):
-    plan = g.Plan(wl.m, wl.n, wl.k, wl.dtype, wl.epilogue, wl.bias_axis, wl.b_layout, **opts)
+    plan = g.Plan(wl.m, wl.n, wl.k, wl.dtype, wl.epilogue, wl.bias_axis, wl.b_layout, a_layout=wl.a_layout,
+                  **opts)
     if wl.dtype == "e4m3" or prob.scale_a != 1.0 or prob.scale_b != 1.0:
         sa = torch.tensor([prob.scale_a], dtype=torch.float32, device=device)
         sb = torch.tensor([prob.scale_b], dtype=torch.float32, device=device)
@@ -76,7 +77,7 @@ def sigmas(prob: Problem):
 def oracle_full(wl: Workload, prob: Problem):
     return oracle.gemm_epi(storage(prob.A), storage(prob.B), storage(prob.bias), dtype=wl.dtype,
                            epilogue=wl.epilogue, bias_axis=wl.bias_axis, b_layout=wl.b_layout,
-                           scale_a=prob.scale_a, scale_b=prob.scale_b)
+                           scale_a=prob.scale_a, scale_b=prob.scale_b, a_layout=wl.a_layout)
 
 
 def compare(wl, D_gpu, words, ref, pre, mask, sa, sb, rows=None, cols=None, extra=None):

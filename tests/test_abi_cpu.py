@@ -76,7 +76,7 @@ def test_plan_rejects_bad_sizes(g, args):
 
 
 @pytest.mark.parametrize("kw", [dict(dt=3), dict(dt=-1), dict(epi=12), dict(epi=-1), dict(axis=2),
-                                dict(layout=2)])
+                                dict(layout=4)])
 def test_plan_rejects_bad_enums(g, kw):
     assert _plan_rc(g, 64, 64, 64, **kw) == g.ERR_ARG
 
@@ -186,5 +186,14 @@ def test_mlp_entry_points_reject_bad_handles_and_acts(g):
     for bad in (None, ctypes.c_void_p(0x1000)):
         assert L.gemm_epi_mlp_set_scales(bad, None, None, None, None, None) == g.ERR_ARG
         assert L.gemm_epi_mlp_run(bad, None, None, None, None, None, None, None, None) == g.ERR_ARG
+        assert L.gemm_epi_mlp_unfused_run(bad, None, None, None, None, None, None, None, None, None) == g.ERR_ARG
         assert L.gemm_epi_mlp_check(bad, None) == g.ERR_ARG
         assert L.gemm_epi_mlp_free(bad) == g.ERR_ARG
+
+
+def test_layout_flags_checked_before_the_device(g):
+    assert _plan_rc(g, 64, 64, 64, layout=4) == g.ERR_ARG                   # unknown flag
+    assert _plan_rc(g, 100, 64, 64, dt=0, layout=2) == g.ERR_ALIGN          # A (k, m): m*2 = 200 B
+    assert _plan_rc(g, 104, 64, 64, dt=0, layout=3) == g.ERR_NO_DEVICE      # valid: A (k, m), B (n, k)
+    h = ctypes.c_void_p()
+    assert g.lib().gemm_epi_mlp_plan(64, 64, 128, 1, 4, 2, ctypes.byref(h)) == g.ERR_ARG   # MLP: B layouts only

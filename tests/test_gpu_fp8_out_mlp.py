@@ -130,10 +130,22 @@ def test_fp8_out_stream_k(kernel, max_ctas):
     assert info["sk_tiles"] > 0
 
 
-def test_fp8_out_small_m_uses_tc1():
+def test_fp8_out_small_m_uses_splitk():
     wl = Workload("qsmall", 16, 512, 1024, "e4m3", "gelu_bias", "col", "nk", seed=34)
     _, info = check_qout(wl)
-    assert info["kernel"] == g.KERNEL_TC1
+    assert info["kernel"] == g.KERNEL_SPLITK
+
+
+@pytest.mark.parametrize("layout", ["nk", "kn"])
+@pytest.mark.parametrize("axis", ["col", "row"])
+@pytest.mark.parametrize("epilogue", ["none", "bias", "relu_bias", "gelu_bias"])
+@pytest.mark.parametrize("m", [16, 40, 100])
+def test_fp8_out_splitk_variants(m, epilogue, axis, layout):
+    if epilogue == "none" and axis == "col":
+        pytest.skip("no bias: the axis plays no part")
+    wl = Workload("qsk2", m, 400, 1024, "e4m3", epilogue, axis, layout, seed=38)
+    _, info = check_qout(wl, kernel="splitk")
+    assert info["kernel"] == g.KERNEL_SPLITK
 
 
 def test_fp8_out_argument_errors():
@@ -145,7 +157,6 @@ def test_fp8_out_argument_errors():
     assert status(lambda: g.Plan(256, 256, 256, "bf16", "bias", out_e4m3=True)) == g.ERR_UNSUPPORTED
     assert status(lambda: g.Plan(256, 256, 256, "e4m3", "relu_aux_bias", out_e4m3=True)) == g.ERR_UNSUPPORTED
     assert status(lambda: g.Plan(256, 256, 256, "e4m3", "tanh_bias", out_e4m3=True)) == g.ERR_UNSUPPORTED
-    assert status(lambda: g.Plan(16, 256, 256, "e4m3", "bias", kernel="splitk", out_e4m3=True)) == g.ERR_UNSUPPORTED
     A = torch.zeros((256, 256), dtype=torch.uint8, device="cuda")
     D = torch.zeros((256, 256), dtype=torch.uint8, device="cuda")
     bias = torch.zeros((256,), dtype=torch.bfloat16, device="cuda")
@@ -173,7 +184,7 @@ def mlp_problem(m, d_model, d_ff, dtype, act, layout, seed):
     return up, make_problem(up), down, make_problem(down)
 
 
-def run_mlp(m, d_model, d_ff, dtype, act, layout, seed, rows=None):
+def run_mlp(m, d_model, d_ff, dtype, act, layout, seed, rows=None, fused=True):
     up, pu, down, pd = mlp_problem(m, d_model, d_ff, dtype, act, layout, seed)
     X, W1, b1, W2, b2 = storage(pu.A), storage(pu.B), storage(pu.bias), storage(pd.B), storage(pd.bias)
     # the oracle on all rows (or on the sampled rows: MLP rows are independent)
@@ -197,7 +208,8 @@ def run_mlp(m, d_model, d_ff, dtype, act, layout, seed, rows=None):
     with g.MlpPlan(m, d_model, d_ff, dtype, act, layout) as mp:
         if dtype == "e4m3":
             mp.set_scales(_f32(pu.scale_a), _f32(pu.scale_b), _f32(s_h), amax, _f32(pd.scale_b))
-        mp.run(pu.A.cuda(), pu.B.cuda(), pu.bias.cuda(), pd.B.cuda(), pd.bias.cuda(), H, Y)
+        Hw = torch.empty((m, d_ff), dtype=torch.bfloat16, device="cuda") if not fused else None
+        mp.run(pu.A.cuda(), pu.B.cuda(), pu.bias.cuda(), pd.B.cuda(), pd.bias.cuda(), H, Y, fused=fused, H_wide=Hw)
         mp.check()
         info = mp.info
     torch.cuda.synchronize()
@@ -228,11 +240,19 @@ def test_mlp_block(dtype, act, layout):
     run_mlp(200, 256, 512, dtype, act, layout, seed=35)
 
 
+@pytest.mark.parametrize("m", [48, 200])
+@pytest.mark.parametrize("dtype", ["e4m3", "bf16"])
+def test_mlp_block_unfused_baseline(dtype, m):
+    """The unfused sequence (bare GEMM, bias + activation, amax, quantise, bare GEMM, bias) lands
+    within the same bounds: its extra bf16 rounding of H is far inside the decision band."""
+    run_mlp(m, 256, 512, dtype, "gelu_bias", "kn", seed=39, fused=False)
+
+
 @pytest.mark.parametrize("m", [16, 64, 1000])
 def test_mlp_block_batch_sizes(m):
     up, down = run_mlp(m, 512, 1024, "e4m3", "gelu_bias", "kn", seed=36)
     if m <= 64:
-        assert up["kernel"] == g.KERNEL_TC1 and down["kernel"] == g.KERNEL_SPLITK
+        assert up["kernel"] == g.KERNEL_SPLITK and down["kernel"] == g.KERNEL_SPLITK
 
 
 def test_mlp_block_fp8_full_size_sampled():

@@ -367,6 +367,42 @@ def test_dependent_launches_keep_stream_order(kernel2, graph):
     compare(wl1b, H.cpu(), None, hb_ref, hb_pre, hb_mask, *sigmas(p1b))
 
 
+# ------------------------------------------------------------------ A stored transposed, (k, m)
+@pytest.mark.parametrize("layout", ["kn", "nk"])
+@pytest.mark.parametrize("epilogue", ["none", "bias", "relu_aux_bias", "gelu_bias", "tanh"])
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("kernel", ["tc1", "tc2"])
+def test_a_stored_transposed(kernel, dtype, epilogue, layout):
+    k = 336 if dtype == "e4m3" else 328
+    wl = Workload("at", 208, 272, k, dtype, epilogue, "col", layout, seed=50, a_layout="km")
+    worst, info = check_against_oracle(wl, make_problem(wl), kernel=kernel)
+    assert info["kernel"] == g.KERNEL[kernel] and info["block_n"] == 256
+    assert worst <= 1.0
+
+
+@pytest.mark.parametrize("m", [16, 520])
+def test_a_stored_transposed_auto_split_tail_and_unfused(m):
+    wl = Workload("at2", m, 528, 1000, "bf16", "relu_aux_bias", "row", "kn", seed=51, a_layout="km")
+    prob = make_problem(wl)
+    worst, info = check_against_oracle(wl, prob, stream_k="on", max_ctas=8)
+    assert info["kernel"] in (g.KERNEL_TC1, g.KERNEL_TC2) and worst <= 1.0
+    D, words, _ = gpu_run(wl, prob, fused=False)
+    ref, pre, mask = oracle_full(wl, prob)
+    compare(wl, D, words, ref, pre, mask, *sigmas(prob), extra=unfused_extra(wl, prob, pre))
+
+
+def test_a_stored_transposed_refusals():
+    def status(fn):
+        with pytest.raises(g.GemmEpiError) as e:
+            fn()
+        return e.value.status
+
+    assert status(lambda: g.Plan(256, 256, 256, "bf16", "bias", a_layout="km", block_n=128)) == g.ERR_UNSUPPORTED
+    assert status(lambda: g.Plan(16, 256, 256, "bf16", "bias", a_layout="km", kernel="splitk")) == g.ERR_UNSUPPORTED
+    assert status(lambda: g.Plan(256, 256, 256, "bf16", "drelu", a_layout="km")) == g.ERR_UNSUPPORTED
+    assert status(lambda: g.Plan(256, 256, 256, "e4m3", "bias", a_layout="km", out_e4m3=True)) == g.ERR_UNSUPPORTED
+
+
 # ------------------------------------------------------------------ errors and failure paths
 def test_run_argument_errors():
     wl = Workload("err", 128, 128, 128, "bf16", "relu_aux_bias", "row", "kn")
