@@ -249,7 +249,8 @@ def encode(x, dtype: str, scale: float = 1.0):
 
 
 def mlp(X, W1, b1, W2, b2, *, dtype: str, act: str = "gelu_bias", w_layout: str = "kn",
-        scale_x: float = 1.0, scale_w1: float = 1.0, scale_h: float = 1.0, scale_w2: float = 1.0):
+        scale_x: float = 1.0, scale_w1: float = 1.0, scale_h: float = 1.0, scale_w2: float = 1.0,
+        stepwise: bool = False):
     """MLP block ("nvmath-python cuBLASLt bias fusion for PyTorch inference", paragraph 1):
 
         H = act(scale_x*scale_w1 * X.W1 + b1)          (bias along the d_ff columns)
@@ -260,14 +261,34 @@ def mlp(X, W1, b1, W2, b2, *, dtype: str, act: str = "gelu_bias", w_layout: str 
     is (d_model, d_ff) for w_layout "kn" or (d_ff, d_model) for "nk" (an nn.Linear weight);
     W2 likewise (d_ff, d_model) or (d_model, d_ff).
 
+    ``stepwise=True`` follows the unfused sequence instead ("nvmath-python epilog bias fusion
+    parameters", body paragraph 1: the product is written back in the output type, then a
+    separate kernel adds the bias and applies the activation): every product is rounded to
+    the 16-bit output type (bf16 for e4m3) before its bias is added, H is rounded to that
+    type before it is quantised, and Y's product is rounded before b2 is added.
+
     Returns (Y, H, Hs, amax) with Y and H in float64 (H before encoding), Hs the stored
     codes, and amax = max |H|."""
     if dtype != "e4m3" and scale_h != 1.0:
         raise ValueError("scale_h applies to e4m3 only")
-    H, _, _ = gemm_epi(X, W1, b1, dtype=dtype, epilogue=act, bias_axis="col", b_layout=w_layout,
-                       scale_a=scale_x, scale_b=scale_w1)
+    if not stepwise:
+        H, _, _ = gemm_epi(X, W1, b1, dtype=dtype, epilogue=act, bias_axis="col", b_layout=w_layout,
+                           scale_a=scale_x, scale_b=scale_w1)
+        amax = float(np.abs(H).max())
+        Hs = encode(H, dtype, scale_h)
+        Y, _, _ = gemm_epi(Hs, W2, b2, dtype=dtype, epilogue="bias", bias_axis="col", b_layout=w_layout,
+                           scale_a=scale_h, scale_b=scale_w2)
+        return Y, H, Hs, amax
+    out = "bf16" if dtype == "e4m3" else dtype
+    rnd = lambda v: decode(encode(v, out), out)            # round to the 16-bit output type
+    f = {"bias": lambda z: z, "relu_bias": lambda z: np.where(z > 0.0, z, 0.0),
+         "gelu_bias": np.vectorize(gelu, otypes=[np.float64])}[act]
+    P, _, _ = gemm_epi(X, W1, None, dtype=dtype, epilogue="none", b_layout=w_layout, scale_a=scale_x,
+                       scale_b=scale_w1)
+    H = rnd(f(rnd(P) + decode(_storage(b1, out), out)[None, :]))
     amax = float(np.abs(H).max())
     Hs = encode(H, dtype, scale_h)
-    Y, _, _ = gemm_epi(Hs, W2, b2, dtype=dtype, epilogue="bias", bias_axis="col", b_layout=w_layout,
-                       scale_a=scale_h, scale_b=scale_w2)
+    Q, _, _ = gemm_epi(Hs, W2, None, dtype=dtype, epilogue="none", b_layout=w_layout, scale_a=scale_h,
+                       scale_b=scale_w2)
+    Y = rnd(rnd(Q) + decode(_storage(b2, out), out)[None, :])
     return Y, H, Hs, amax

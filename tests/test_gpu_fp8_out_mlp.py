@@ -191,16 +191,19 @@ def run_mlp(m, d_model, d_ff, dtype, act, layout, seed, rows=None, fused=True):
     Xo = X if rows is None else np.ascontiguousarray(X[rows])
     if dtype == "e4m3":
         _, H0, _, amax0 = oracle.mlp(Xo, W1, b1, W2, b2, dtype="e4m3", act=act, w_layout=layout,
-                                     scale_x=pu.scale_a, scale_w1=pu.scale_b, scale_h=1.0, scale_w2=pd.scale_b)
+                                     scale_x=pu.scale_a, scale_w1=pu.scale_b, scale_h=1.0, scale_w2=pd.scale_b,
+                                     stepwise=not fused)
         s_h = (amax0 if rows is None else float(np.abs(H0).max())) / 448.0
         if rows is not None:
             s_h *= 1.5                 # leave headroom for rows the sample did not see
         s_h = float(np.float32(s_h))   # the fp32 value the GPU reads
     else:
         s_h = 1.0
+    # the unfused sequence is checked against the oracle's stepwise reading (each product
+    # rounded to the 16-bit type before its bias, H rounded before it is quantised)
     Y_ref, H_ref, Hs_ref, amax_ref = oracle.mlp(Xo, W1, b1, W2, b2, dtype=dtype, act=act, w_layout=layout,
                                                 scale_x=pu.scale_a, scale_w1=pu.scale_b, scale_h=s_h,
-                                                scale_w2=pd.scale_b)
+                                                scale_w2=pd.scale_b, stepwise=not fused)
     h_t = torch.uint8 if dtype == "e4m3" else TORCH_DTYPE[dtype]
     H = torch.full((m, d_ff), 0x7F if dtype == "e4m3" else 0, dtype=h_t, device="cuda")
     Y = torch.full((m, d_model), float("nan"), dtype=TORCH_DTYPE[up.out_dtype], device="cuda")
@@ -243,8 +246,8 @@ def test_mlp_block(dtype, act, layout):
 @pytest.mark.parametrize("m", [48, 200])
 @pytest.mark.parametrize("dtype", ["e4m3", "bf16"])
 def test_mlp_block_unfused_baseline(dtype, m):
-    """The unfused sequence (bare GEMM, bias + activation, amax, quantise, bare GEMM, bias) lands
-    within the same bounds: its extra bf16 rounding of H is far inside the decision band."""
+    """The unfused sequence (bare GEMM, bias + activation, amax, quantise, bare GEMM, bias)
+    against the oracle's stepwise reading of that sequence."""
     run_mlp(m, 256, 512, dtype, "gelu_bias", "kn", seed=39, fused=False)
 
 

@@ -484,6 +484,21 @@ def test_golden_mlp_case(oracle_lib, c):
     np.testing.assert_array_equal(Y, np.array(c["y"]))
 
 
+@pytest.mark.parametrize("c", MLP, ids=[c["id"] for c in MLP])
+def test_golden_mlp_case_stepwise(oracle_lib, c):
+    dt = c["dtype"]
+    bdt = "bf16" if dt == "e4m3" else dt
+    args = [to_storage_values(c["x"], dt), to_storage_values(c["w1"], dt), to_storage_values(c["b1"], bdt),
+            to_storage_values(c["w2"], dt), to_storage_values(c["b2"], bdt)]
+    Y, H, Hs, amax = oracle_lib.mlp(*args, dtype=dt, act=c["act"], w_layout=c["w_layout"],
+                                    scale_x=c["scale_x"], scale_w1=c["scale_w1"], scale_h=c["scale_h"],
+                                    scale_w2=c["scale_w2"], stepwise=True)
+    np.testing.assert_array_equal(H, np.array(c["h_stepwise"]))
+    np.testing.assert_array_equal(Hs, np.array(c["h_codes_stepwise"]))
+    assert amax == c["amax_stepwise"]
+    np.testing.assert_array_equal(Y, np.array(c["y_stepwise"]))
+
+
 @pytest.mark.parametrize("layout", ["kn", "nk"])
 def test_mlp_equals_two_numpy_products(oracle_lib, layout):
     """16-bit MLP: H from the GELU of the first product, rounded to fp16 by numpy, then the
