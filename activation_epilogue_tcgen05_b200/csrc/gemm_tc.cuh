@@ -20,12 +20,16 @@
 //               tcgen05.mma (M = 128*CG, N = BN, K = 32 bytes per step) into
 //               one of two fp32 accumulators in tensor memory; tcgen05.commit
 //               frees ring stages and publishes finished accumulators.
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time, then
-//               scale, bias, activation, sign-mask bits, RNE cast, 128-byte
-//               swizzled staging in shared memory and TMA stores of D; the
-//               mask goes out as 16-byte vector stores.  With two
+//   warps 2..    epilogue (4 warps; 8 for GELU and tanh, two per TMEM lane
+//               quadrant): tcgen05.ld 32 lanes x 32 columns at a time, then
+//               scale, bias, activation, sign-mask bits, RNE cast, 64-byte
+//               swizzled staging in shared memory and 32 x 32 TMA stores of D;
+//               the mask goes out as 16-byte vector stores.  With two
 //               accumulators the epilogue of tile t overlaps the mainloop of
-//               tile t+1.
+//               tile t+1.  Variants: an e4m3 output (QOUT) written with direct
+//               16-byte stores plus an amax reduction; the ReLU backward
+//               (EPI_DRELU) reading the mask and writing bias-gradient partials;
+//               A stored (k, m) (A_MN) loaded as MN-major boxes.
 //
 // Split tail (stream-K style): when the tiles do not divide evenly over the
 // units (CTAs, or CTA pairs), the first sk_tiles tiles are not given out
@@ -88,7 +92,7 @@ struct TcParams {
     int inject_stall;            // testing only: 1 = the MMA issuer publishes no accumulator
     int sk_tiles;                // tiles [0, sk_tiles) are split along k over units
     int sk_split;                // parts per split tile (units per split tile)
-    float *workspace;            // partial tiles, 128 x BN fp32 per (unit, cta rank); see ws_slot()
+    float *workspace;            // partial tiles, 128 x BN fp32 per (unit, cta rank); see ws_chunk()
     unsigned int *flags;         // [unit][cta rank][4 epilogue warps]: 1 while a partial is unread
     unsigned long long *trace;   // timeline records; used only by builds with GEMM_EPI_TRACE=1
     // DRELU with a bias gradient: fp32 partial sums of D, written once each per launch.
