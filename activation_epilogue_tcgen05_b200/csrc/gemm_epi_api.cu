@@ -279,7 +279,19 @@ unsigned long long *trace_buffer() {
 #endif
 }
 
+// A plan's status word and workspaces live on the device it was created on: its runs must be
+// issued with that device current.
+bool on_plan_device(const Plan *P) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return dev == P->device;
+}
+
 int check_run_args(Plan *P, const void *A, const void *B, const void *bias, void *D, uint32_t *aux) {
+    if (!on_plan_device(P)) return GEMM_EPI_ERR_ARG;
     if (P->bwd) return GEMM_EPI_ERR_ARG;          // backward plans run through gemm_epi_run_bwd
     if (!A || !B || !D) return GEMM_EPI_ERR_NULL;
     if (P->has_bias && !bias) return GEMM_EPI_ERR_NULL;
@@ -293,6 +305,7 @@ int check_run_args(Plan *P, const void *A, const void *B, const void *bias, void
 }
 
 int check_bwd_args(Plan *P, const void *A, const void *B, const uint32_t *aux, void *D, void *dbias) {
+    if (!on_plan_device(P)) return GEMM_EPI_ERR_ARG;
     if (!P->bwd) return GEMM_EPI_ERR_ARG;
     if (!A || !B || !D || !aux) return GEMM_EPI_ERR_NULL;
     if (P->bgrad && !dbias) return GEMM_EPI_ERR_NULL;
@@ -410,6 +423,7 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     if (!out) return GEMM_EPI_ERR_ARG;
     if (m <= 0 || n <= 0 || k <= 0) return GEMM_EPI_ERR_ARG;
     if (m > 0x7fffffffll || n > 0x7fffffffll || k > 0x7fffffffll) return GEMM_EPI_ERR_ARG;
+    if (((m + 127) / 128) * ((n + 127) / 128) > 0x7fffffffll) return GEMM_EPI_ERR_ARG;   // tile count is an int
     if (dtype < GEMM_EPI_F16 || dtype > GEMM_EPI_E4M3) return GEMM_EPI_ERR_ARG;
     if (epilogue < GEMM_EPI_NONE || epilogue > GEMM_EPI_DRELU_BGRAD) return GEMM_EPI_ERR_ARG;
     if (bias_axis != GEMM_EPI_BIAS_ROW && bias_axis != GEMM_EPI_BIAS_COL) return GEMM_EPI_ERR_ARG;
@@ -966,6 +980,7 @@ extern "C" int gemm_epi_run_noalloc(int64_t m, int64_t n, int64_t k, int dtype, 
     // the same argument rules as a plan (sizes are limited to 2^31 - 1)
     if (m <= 0 || n <= 0 || k <= 0) return GEMM_EPI_ERR_ARG;
     if (m > 0x7fffffffll || n > 0x7fffffffll || k > 0x7fffffffll) return GEMM_EPI_ERR_ARG;
+    if (((m + 127) / 128) * ((n + 127) / 128) > 0x7fffffffll) return GEMM_EPI_ERR_ARG;
     if (dtype < GEMM_EPI_F16 || dtype > GEMM_EPI_E4M3) return GEMM_EPI_ERR_ARG;
     if (epilogue < GEMM_EPI_NONE || epilogue > GEMM_EPI_TANH) return GEMM_EPI_ERR_ARG;
     if (bias_axis != GEMM_EPI_BIAS_ROW && bias_axis != GEMM_EPI_BIAS_COL) return GEMM_EPI_ERR_ARG;

@@ -216,9 +216,11 @@ int gemm_epi_set_out_scale(gemm_epi_plan_t plan, const float *d_scale_out, float
  *         type); bits past column n-1 are 0.  ([epilog-params] body
  *         paragraph 2: the ReLU input's sign mask kept for the backward pass.)
  *   stream  cudaStream_t as void*.
- * Returns OK, ERR_ARG (bad plan), ERR_NULL, ERR_ALIGN or ERR_CUDA.  A kernel
- * that gives up on a bounded internal wait records it in the plan's status
- * word; gemm_epi_check() reports it. */
+ * Returns OK, ERR_ARG (bad plan, or a current device other than the one the
+ * plan was created on), ERR_NULL, ERR_ALIGN or ERR_CUDA.  A kernel that gives
+ * up on a bounded internal wait records it in the plan's status word;
+ * gemm_epi_check() reports it.  The same device rule holds for every run entry
+ * point below. */
 int gemm_epi_run(gemm_epi_plan_t plan, const void *A, const void *B, const void *bias, void *D,
                  uint32_t *aux, void *stream);
 

@@ -197,3 +197,8 @@ def test_layout_flags_checked_before_the_device(g):
     assert _plan_rc(g, 104, 64, 64, dt=0, layout=3) == g.ERR_NO_DEVICE      # valid: A (k, m), B (n, k)
     h = ctypes.c_void_p()
     assert g.lib().gemm_epi_mlp_plan(64, 64, 128, 1, 4, 2, ctypes.byref(h)) == g.ERR_ARG   # MLP: B layouts only
+
+
+def test_plan_rejects_tile_counts_beyond_int(g):
+    # m, n each below 2^31 but (m/128) * (n/128) above it
+    assert _plan_rc(g, (1 << 31) - 1, 1 << 28, 64) == g.ERR_ARG
