@@ -20,8 +20,8 @@
 //               tcgen05.mma (M = 128*CG, N = BN, K = 32 bytes per step) into
 //               one of two fp32 accumulators in tensor memory; tcgen05.commit
 //               frees ring stages and publishes finished accumulators.
-//   warps 2..    epilogue (4 warps; 8 for GELU and tanh, two per TMEM lane
-//               quadrant): tcgen05.ld 32 lanes x 32 columns at a time, then
+//   warps 2..    epilogue (8 warps, two per TMEM lane quadrant; 4 for the ReLU
+//               backward): tcgen05.ld 32 lanes x 32 columns at a time, then
 //               scale, bias, activation, sign-mask bits, RNE cast, 64-byte
 //               swizzled staging in shared memory and 32 x 32 TMA stores of D;
 //               the mask goes out as 16-byte vector stores.  With two
@@ -66,6 +66,7 @@ enum : int { DT_F16 = 0, DT_BF16 = 1, DT_E4M3 = 2 };
 enum : int { EPI_NONE = 0, EPI_BIAS = 1, EPI_RELU = 2, EPI_RELU_AUX = 3, EPI_GELU = 4, EPI_TANH = 5,
              EPI_DRELU = 6 };
 enum : int { AXIS_ROW = 0, AXIS_COL = 1 };
+
 
 // Status-word bits written by kernels that gave up waiting.
 enum : unsigned int {
@@ -330,10 +331,12 @@ struct TcCfg {
     static constexpr int A_BOX_M = 128 / ESIZE;     // m per 128-byte MN-major box
     static constexpr int A_BOXES = A_MN ? BM / A_BOX_M : 1;
     static constexpr int A_BOX_BYTES = A_MN ? BK * 128 : A_BYTES;
-    // GELU / tanh cost ~20 instructions an element: two epilogue warps per TMEM lane
-    // quadrant (each taking half the columns) so that the epilogue keeps up with the
-    // next tile's mainloop; the cheap epilogues use one warp per quadrant.
-    static constexpr bool HEAVY_EPI = EPI == EPI_GELU || EPI == EPI_TANH;
+    // Two epilogue warps per TMEM lane quadrant (each taking half the columns): GELU and
+    // tanh cost ~20 instructions an element and must keep up with the next tile's
+    // mainloop, and for every epilogue the last wave's drain, which nothing overlaps, is
+    // halved (a small launch gains 4.5 %; large ones are unchanged).  The ReLU backward
+    // keeps one warp per quadrant (its mask words are read one 16-byte load per 128 columns).
+    static constexpr bool HEAVY_EPI = EPI != EPI_DRELU;
     static constexpr bool BWD = EPI == EPI_DRELU;             // reads the mask, adds no bias
     static constexpr bool FWD_BIAS = EPI != EPI_NONE && !BWD;  // may add a bias
     // e4m3 output quantised with a per-tensor scale (the MLP block's intermediate): written

@@ -2,6 +2,46 @@
 // quantised in the epilogue.
 #include "kernels.h"
 namespace gemm_epi {
+
+// Split-K kernels for e4m3 operands with an e4m3 output quantised in the epilogue:
+// NONE (ROW), BIAS, RELU, GELU, either bias axis, every batch width.
+struct SkFindQ {
+    template <int EPI, int AXIS, bool WMN, int NM>
+    static bool leaf(SkLauncher *l, KernelInfo *i) {
+        using C = SkCfg<DT_E4M3, EPI, AXIS, WMN, NM, sk_stages(NM), true>;
+        *l = &launch_sk<C>;
+        *i = sk_info<C>();
+        return true;
+    }
+    template <int EPI, int AXIS, bool WMN>
+    static bool nm(int v, SkLauncher *l, KernelInfo *i) {
+        switch (v) {
+        case 16: return leaf<EPI, AXIS, WMN, 16>(l, i);
+        case 32: return leaf<EPI, AXIS, WMN, 32>(l, i);
+        case 64: return leaf<EPI, AXIS, WMN, 64>(l, i);
+        case 128: return leaf<EPI, AXIS, WMN, 128>(l, i);
+        }
+        return false;
+    }
+    template <int EPI, int AXIS>
+    static bool mn(bool wmn, int v, SkLauncher *l, KernelInfo *i) {
+        return wmn ? nm<EPI, AXIS, true>(v, l, i) : nm<EPI, AXIS, false>(v, l, i);
+    }
+    template <int EPI>
+    static bool ax(int axis, bool wmn, int v, SkLauncher *l, KernelInfo *i) {
+        return axis ? mn<EPI, AXIS_COL>(wmn, v, l, i) : mn<EPI, AXIS_ROW>(wmn, v, l, i);
+    }
+    static bool find(int epi, int axis, bool wmn, int v, SkLauncher *l, KernelInfo *i) {
+        switch (epi) {
+        case EPI_NONE: return mn<EPI_NONE, AXIS_ROW>(wmn, v, l, i);
+        case EPI_BIAS: return ax<EPI_BIAS>(axis, wmn, v, l, i);
+        case EPI_RELU: return ax<EPI_RELU>(axis, wmn, v, l, i);
+        case EPI_GELU: return ax<EPI_GELU>(axis, wmn, v, l, i);
+        }
+        return false;
+    }
+};
+
 bool find_sk_e4m3_q(int epi, int axis, bool w_mn, int nm, SkLauncher *l, KernelInfo *i) {
     return SkFindQ::find(epi, axis, w_mn, nm, l, i);
 }

@@ -1,5 +1,5 @@
 // Instantiations of the persistent tcgen05 kernel for e4m3 operands with A stored (k, m).
-#include "kernels.h"
+#include "find_at.cuh"
 namespace gemm_epi {
 bool find_tc_e4m3_at(int cg, int epi, int axis, bool bmn, int bn, TcLauncher *l, KernelInfo *i) {
     return TcFindAT<DT_E4M3>::find(cg, epi, axis, bmn, bn, l, i);
