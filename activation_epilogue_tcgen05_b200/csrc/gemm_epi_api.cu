@@ -217,8 +217,18 @@ int choose(Plan *P) {
             // a pair's e4m3 B half-tile stored (k, n) must be a whole 128-byte box: 128 columns
             if (cg == 2 && P->dtype == GEMM_EPI_E4M3 && b_mn) bn = 256;
             if (P->a_km) bn = 256;     // A stored (k, m) is built with 256-wide tiles only
+            // Many waves of 16-bit work with a light epilogue: 512-wide pair tiles.  They move a
+            // quarter fewer operand bytes per flop into each SM, which under the power cap buys
+            // clock (+7 % at 8192^3 and 65536 x 8192 x 16384), but hold a single accumulator, so
+            // the epilogue is not overlapped: they need >= 4 waves, and they lose with GELU / tanh
+            // or with e4m3's twice-as-short mainloop (-7 % on the FP8 GELU shape).
+            const int64_t tiles512 = ((m + 255) / 256) * ((n + 511) / 512);
+            const bool light = P->kepi == EPI_NONE || P->kepi == EPI_BIAS || P->kepi == EPI_RELU ||
+                               P->kepi == EPI_RELU_AUX;
+            if (cg == 2 && light && P->dtype != GEMM_EPI_E4M3 && !P->a_km && !P->qout && tiles512 >= 4 * (sms / 2))
+                bn = 512;
         }
-        if (bn != 128 && bn != 256) return GEMM_EPI_ERR_ARG;
+        if (bn != 128 && bn != 256 && bn != 512) return GEMM_EPI_ERR_ARG;
         P->block_n = bn;
         const int64_t tiles = ((m + bm - 1) / bm) * ((n + bn - 1) / bn);
         const int64_t units_max = cg == 2 ? sms / 2 : sms;
@@ -329,7 +339,7 @@ int ensure_maps(Plan *P, const void *A, const void *B, void *D) {
         ok = ok && make_map(&P->tmB, dt, A, k, m, bk, P->nm);
     } else {
         const int cg = P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
-        const int bn_local = P->block_n / cg;
+        const int bn_local = std::min(P->block_n, 256) / cg;   // B rows of one MMA in this CTA
         ok = ok && (P->a_km ? make_map(&P->tmA, dt, A, m, k, box_n, bk) : make_map(&P->tmA, dt, A, k, m, bk, 128));
         ok = ok && (b_kn ? make_map(&P->tmB, dt, B, n, k, box_n, bk) : make_map(&P->tmB, dt, B, k, n, bk, bn_local));
         const int out_dt = dt == GEMM_EPI_E4M3 ? GEMM_EPI_BF16 : dt;
@@ -433,7 +443,7 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     gemm_epi_options o{};
     if (opts) o = *opts;
     if (o.kernel < GEMM_EPI_KERNEL_AUTO || o.kernel > GEMM_EPI_KERNEL_SPLITK) return GEMM_EPI_ERR_ARG;
-    if (o.block_n != 0 && o.block_n != 128 && o.block_n != 256) return GEMM_EPI_ERR_ARG;
+    if (o.block_n != 0 && o.block_n != 128 && o.block_n != 256 && o.block_n != 512) return GEMM_EPI_ERR_ARG;
     if (o.split_k < 0 || o.split_k > 8 || o.max_ctas < 0) return GEMM_EPI_ERR_ARG;
     if (o.inject_stall != 0 && o.inject_stall != 1) return GEMM_EPI_ERR_ARG;
     if (o.stream_k < 0 || o.stream_k > 2) return GEMM_EPI_ERR_ARG;

@@ -327,6 +327,14 @@ struct TcCfg {
     static constexpr int B_BYTES = BN_LOCAL * 128;
     static constexpr int B_BOX_N = 128 / ESIZE;     // n per 128-byte MN-major box
     static constexpr int B_BOXES = B_MN ? BN_LOCAL / B_BOX_N : 1;
+    // A 512-wide pair tile is two N = 256 MMAs per k-step, each writing its own 256 TMEM
+    // columns; tensor memory then holds one accumulator, not two.  Each CTA's B tile is the
+    // two MMAs' local halves, 128 rows each, one after the other.
+    static constexpr int MMA_N = BN <= 256 ? BN : 256;      // N of one tcgen05.mma
+    static constexpr int N_MMAS = BN / MMA_N;                // MMAs per k-step
+    static constexpr int MMA_N_LOCAL = MMA_N / CG;           // B rows of one MMA in this CTA
+    static constexpr int HALF_B_BYTES = MMA_N_LOCAL * 128;   // shared-memory bytes of those rows
+    static constexpr int NUM_ACC = BN <= 256 ? 2 : 1;        // accumulators in tensor memory
     static constexpr int B_BOX_BYTES = B_MN ? BK * 128 : B_BYTES;
     static constexpr int A_BOX_M = 128 / ESIZE;     // m per 128-byte MN-major box
     static constexpr int A_BOXES = A_MN ? BM / A_BOX_M : 1;
@@ -348,8 +356,8 @@ struct TcCfg {
     static constexpr int NCH_W = COLS_W / 32;                // its 32-column chunks
     static constexpr int CPG = NCH_W < 4 ? NCH_W : 4;        // chunks per mask-word group
     static_assert(NCH_W % CPG == 0 && (CPG == 2 || CPG == 4), "chunk grouping");
-    static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
-                                   : (2 * BN <= 256) ? 256 : 512;
+    static constexpr int TMEM_COLS = (NUM_ACC * BN <= 32) ? 32 : (NUM_ACC * BN <= 64) ? 64 : (NUM_ACC * BN <= 128) ? 128
+                                   : (NUM_ACC * BN <= 256) ? 256 : 512;
     static constexpr int STG_BYTES = QOUT ? 0 : 32 * 64;   // per epilogue warp: 32 rows x 32 16-bit outputs
     // shared-memory layout (offsets from a 1024-byte aligned base)
     static constexpr int OFF_A = 0;
@@ -361,8 +369,9 @@ struct TcCfg {
     static constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
-    static_assert(BN % 128 == 0 && BN <= 256, "BN must be 128 or 256");
-    static_assert(2 * BN <= 512, "two accumulators must fit in tensor memory");
+    static_assert(BN == 128 || BN == 256 || (BN == 512 && CG == 2), "BN is 128 or 256 (512 for CTA pairs)");
+    static_assert(NUM_ACC * BN <= 512, "the accumulators must fit in tensor memory");
+    static_assert(!B_MN || MMA_N_LOCAL % B_BOX_N == 0, "an MMA's B half must be whole boxes");
     static_assert(B_MN == false || BN_LOCAL % B_BOX_N == 0, "MN-major B tile must be whole boxes");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "stage alignment");
@@ -453,7 +462,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 int tm, tn;
                 tile_coords(p, w.tile, tm, tn);
                 const int m0 = tm * (C::BM * C::CG) + (int)rank * C::BM;
-                const int nb = tn * C::BN + (int)rank * C::BN_LOCAL;
+                // local B row r (MMA half h = r / MMA_N_LOCAL) holds global column
+                // tn*BN + h*MMA_N + rank*MMA_N_LOCAL + r % MMA_N_LOCAL
+                const int nb = tn * C::BN + (int)rank * C::MMA_N_LOCAL;
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!wait_bounded<false>(empty_bar(stage), phase ^ 1u, abort_flag, p.status,
                                              ST_TIMEOUT_PRODUCER)) {
@@ -484,11 +495,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         load(a_dst, &tmA, k0, m0);
                     }
                     if constexpr (C::B_MN) {
+                        constexpr int PER_HALF = C::MMA_N_LOCAL / C::B_BOX_N;
 #pragma unroll
                         for (int b = 0; b < C::B_BOXES; ++b)
-                            load(b_dst + b * C::B_BOX_BYTES, &tmB, nb + b * C::B_BOX_N, k0);
+                            load(b_dst + b * C::B_BOX_BYTES, &tmB,
+                                 nb + (b / PER_HALF) * C::MMA_N + (b % PER_HALF) * C::B_BOX_N, k0);
                     } else {
-                        load(b_dst, &tmB, k0, nb);
+#pragma unroll
+                        for (int h = 0; h < C::N_MMAS; ++h)
+                            load(b_dst + h * C::HALF_B_BYTES, &tmB, k0, nb + h * C::MMA_N);
                     }
                     ++issued;
                     if (++stage == (uint32_t)C::STAGES) { stage = 0; phase ^= 1u; }
@@ -504,7 +519,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && leader) {
-            constexpr uint32_t idesc = make_idesc(C::FMT, C::A_MN, C::B_MN, 128 * C::CG, C::BN);
+            constexpr uint32_t idesc = make_idesc(C::FMT, C::A_MN, C::B_MN, 128 * C::CG, C::MMA_N);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             bool ok = true;
             // with inject_stall nothing is issued or committed: the epilogue's
@@ -532,9 +547,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     for (int ks = 0; ks < C::KSTEPS; ++ks) {
                         const uint64_t ad = C::A_MN ? make_sdesc(a_base + ks * C::UMMA_K * 128, C::A_BOX_BYTES, 1024)
                                                     : make_sdesc(a_base + ks * 32, 16, 1024);
-                        const uint64_t bd = C::B_MN ? make_sdesc(b_base + ks * C::UMMA_K * 128, C::B_BOX_BYTES, 1024)
-                                                    : make_sdesc(b_base + ks * 32, 16, 1024);
-                        ptx::mma<C::CG, C::KIND>(d_tmem, ad, bd, idesc, (kb > w.kb0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+                        for (int h = 0; h < C::N_MMAS; ++h) {
+                            const uint32_t bh = b_base + h * C::HALF_B_BYTES;
+                            const uint64_t bd = C::B_MN ? make_sdesc(bh + ks * C::UMMA_K * 128, C::B_BOX_BYTES, 1024)
+                                                        : make_sdesc(bh + ks * 32, 16, 1024);
+                            ptx::mma<C::CG, C::KIND>(d_tmem + h * C::MMA_N, ad, bd, idesc,
+                                                     (kb > w.kb0 || ks > 0) ? 1u : 0u);
+                        }
                     }
                     if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(empty_bar(stage), 0x3);
                     else ptx::mma_commit(empty_bar(stage));
@@ -544,7 +564,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(tfull_bar(acc), 0x3);
                 else ptx::mma_commit(tfull_bar(acc));
                 trace_event(p.trace, warp, 4, w.tile, w.kb1);
-                if (++acc == 2u) { acc = 0; acc_phase ^= 1u; }
+                if (++acc == (uint32_t)C::NUM_ACC) { acc = 0; acc_phase ^= 1u; }
             }
             // every MMA issued by this thread has completed once done_bar flips
             if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(done_bar, 0x1);
@@ -793,7 +813,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 for (int v = c_first; v < unit; ++v) p.flags[((size_t)v * C::CG + rank) * 4 + q] = 0u;
             }
             if (lane == 0) trace_event(p.trace, warp, 9, w.tile, 0);
-            if (++acc == 2u) { acc = 0; acc_phase ^= 1u; }
+            if (++acc == (uint32_t)C::NUM_ACC) { acc = 0; acc_phase ^= 1u; }
         }
         if (lane == 0) ptx::bulk_wait<0>();
         __syncwarp();

@@ -186,6 +186,8 @@ KernelInfo sk_info() {
         constexpr int STG = tc_stages(128 * 128 + (BN / CG) * 128);                                     \
         if constexpr (BMN && (BN / CG) % (128 / ES) != 0) {                                             \
             return false; /* an MN-major B half-tile narrower than one 128-byte box */                  \
+        } else if constexpr (BN == 512 && (CG != 2 || EPI == EPI_DRELU)) {                              \
+            return false; /* 512-wide tiles: CTA pairs, forward epilogues */                            \
         } else {                                                                                        \
             using C = TcCfg<DTV, EPI, AXIS, BMN, BN, CG, STG>;                                          \
             *l = &launch_tc<C>;                                                                         \
@@ -195,6 +197,7 @@ KernelInfo sk_info() {
     }                                                                                                   \
     template <int CG, int EPI, int AXIS, bool BMN>                                                      \
     static bool NAME##_bn(int bn, TcLauncher *l, KernelInfo *i) {                                       \
+        if (bn == 512) return NAME##_leaf<CG, EPI, AXIS, BMN, 512>(l, i);                               \
         if (bn == 256) return NAME##_leaf<CG, EPI, AXIS, BMN, 256>(l, i);                               \
         if (bn == 128) return NAME##_leaf<CG, EPI, AXIS, BMN, 128>(l, i);                               \
         return false;                                                                                   \

@@ -137,8 +137,10 @@ typedef struct gemm_epi_plan_s *gemm_epi_plan_t;
 /* Optional tuning knobs; zero-initialise for automatic choices. */
 typedef struct gemm_epi_options {
     int32_t kernel;    /* enum gemm_epi_kernel                                        */
-    int32_t block_n;   /* output tile width (128 or 256; 0 = auto).  TC2 with e4m3 and B
-                          stored (k, n) supports 256 only (128 is ERR_UNSUPPORTED)      */
+    int32_t block_n;   /* output tile width (128, 256, or 512 for TC2 forward plans; 0 =
+                          auto, which takes 512 for TC2 with 16-bit operands, an epilogue
+                          without GELU / tanh and at least four waves of 256 x 512 tiles).  TC2 with e4m3 and B stored (k, n) supports
+                          256 and 512 only (128 is ERR_UNSUPPORTED)                       */
     int32_t split_k;   /* SPLITK: CTAs per cluster along k (1..8; 0 = auto).  TC1/TC2:
                           cap on the parts a tail tile is split into (0 = 2)          */
     int32_t max_ctas;  /* persistent kernels: cap on resident CTAs (0 = one per SM)    */

@@ -48,7 +48,7 @@ def _cuda():
 @pytest.mark.parametrize("axis", ["row", "col"])
 @pytest.mark.parametrize("epilogue", EPILOGUES)
 @pytest.mark.parametrize("dtype", DTYPES)
-@pytest.mark.parametrize("kernel,block_n", [("tc1", 128), ("tc1", 256), ("tc2", 256), ("tc2", 128)])
+@pytest.mark.parametrize("kernel,block_n", [("tc1", 128), ("tc1", 256), ("tc2", 256), ("tc2", 128), ("tc2", 512)])
 def test_small_all_variants(kernel, block_n, dtype, epilogue, axis, layout):
     if kernel == "tc2" and block_n == 128 and dtype == "e4m3" and layout == "kn":
         pytest.skip("not instantiated: a 64-column e4m3 half-tile is narrower than one 128-byte box")
@@ -158,6 +158,7 @@ def test_alpha_scaling_16bit(kernel, dtype):
     ("tc1", 16, 256, 256, 4),   # fewer tiles than CTAs: every tile in four parts
     ("tc2", 12, 600, 528, 2),   # pairs: 3 x 5 tiles on 6 pairs
     ("tc2", 8, 256, 256, 2),    # pairs, fewer tiles than pairs (2 tiles on 4 pairs)
+    ("tc2", 8, 600, 1104, 2),   # 512-wide pair tiles (block_n 512): 3 x 3 tiles on 4 pairs
 ])
 @pytest.mark.parametrize("dtype,epilogue,axis,layout", [
     ("bf16", "relu_aux_bias", "row", "kn"), ("f16", "gelu_bias", "col", "nk"),
@@ -168,10 +169,25 @@ def test_stream_k(kernel, max_ctas, m, n, parts, dtype, epilogue, axis, layout):
     wl = Workload("sk_tail", m, n, k, dtype, epilogue, axis, layout, seed=12)
     prob = make_problem(wl)
     bn = 256 if (kernel == "tc2" and dtype == "e4m3") else 128
+    if n == 1104:
+        bn = 512
     worst, info = check_against_oracle(wl, prob, kernel=kernel, block_n=bn, max_ctas=max_ctas,
                                        stream_k="on", split_k=parts)
     assert info["sk_tiles"] > 0 and info["sk_split"] == parts
     assert worst <= 1.0
+
+
+def test_wide_tiles_chosen_for_many_waves():
+    """4096 x 16384: 512 tiles of 256 x 512 for 74 pairs, so the plan takes 512-wide tiles;
+    checked on seeded sampled positions (and element-exact mask outside the band)."""
+    wl = Workload("wide", 4096, 16384, 256, "bf16", "relu_aux_bias", "row", "kn",
+                  ("normal", 1.0 / 16), ("normal", 1.0 / 16), ("normal", 1.0), seed=52)
+    prob = make_problem(wl)
+    D, words, info = gpu_run(wl, prob)
+    assert info["kernel"] == g.KERNEL_TC2 and info["block_n"] == 512
+    rows, cols = sample_positions(wl.m, wl.n, 96, 96, seed=52, tile_n=512)
+    ref, pre, mask = sampled_oracle(wl, prob, rows, cols)
+    compare(wl, D, words, ref, pre, mask, *sigmas(prob), rows=rows, cols=cols)
 
 
 @pytest.mark.parametrize("kernel", ["tc1", "tc2"])
