@@ -170,11 +170,13 @@ int choose(Plan *P) {
     int kernel = P->opts.kernel;
     if (kernel == GEMM_EPI_KERNEL_AUTO) {
         // small m: swapped split-K; enough 256 x 256 tiles for every SM pair: CTA pairs
-        // (half the operand traffic per SM); otherwise single CTAs
+        // (half the operand traffic per SM); otherwise single CTAs.  Split-K up to m = 32:
+        // above, its MMA tile is 64 wide and the single CTAs with a four-part split tail are
+        // as fast or faster (Linear 4096 -> 4096 fp16: m = 48 17.8 vs 17.1 us, m = 64 18.5 vs
+        // 17.1 us).  (The split-K kernel has no backward epilogue.)
         const int64_t pair_tiles = ((m + 255) / 256) * ((n + 255) / 256);
         const int sms_auto = P->opts.max_ctas > 0 ? std::min(P->opts.max_ctas, P->num_sms) : P->num_sms;
-        // (the split-K kernel has no backward epilogue)
-        if (m <= 64 && P->kepi != EPI_DRELU && !P->a_km) kernel = GEMM_EPI_KERNEL_SPLITK;
+        if (m <= 32 && P->kepi != EPI_DRELU && !P->a_km) kernel = GEMM_EPI_KERNEL_SPLITK;
         else if (pair_tiles >= sms_auto / 2) kernel = GEMM_EPI_KERNEL_TC2;
         else kernel = GEMM_EPI_KERNEL_TC1;
     }
@@ -234,15 +236,19 @@ int choose(Plan *P) {
         const int64_t units_max = cg == 2 ? sms / 2 : sms;
         // split tail: the tiles of an incomplete last wave (or all tiles, when there are fewer
         // tiles than units) are cut along k into `split` parts on separate units, so the last
-        // wave costs 1/split of a tile.  Two parts by default: the finishing unit then adds a
-        // single partial, which overlaps its next tile's mainloop.
+        // wave costs 1/split of a tile.  Behind whole waves, two parts: the finishing unit then
+        // adds a single partial, which overlaps its next tile's mainloop.  With fewer tiles than
+        // units nothing follows the parts, so up to four parts (at least 8 k-blocks each) put
+        // more SMs on the operand stream: 128 x 4096 x 4096 fp16 19.7 -> 17.3 us, 128 x 4096 x
+        // 14336 43.5 -> 33.4 us, 1024 x 512 x 2048 12.5 -> 11.9 us.
         int64_t sk_tiles = 0, split = 0;
         const int sk_mode = P->opts.stream_k;          // 0 auto, 1 off, 2 on
         if (sk_mode != 1 && tiles % units_max != 0) {
             const int64_t rem = tiles < units_max ? tiles : tiles % units_max;
             const int64_t waves = (tiles + units_max - 1) / units_max;
             const double loss = 1.0 - (double)tiles / (double)(waves * units_max);
-            split = std::min<int64_t>({units_max / rem, P->opts.split_k > 0 ? P->opts.split_k : 2, num_kb});
+            const int64_t parts = tiles < units_max ? std::max<int64_t>(2, std::min<int64_t>(4, num_kb / 8)) : 2;
+            split = std::min<int64_t>({units_max / rem, P->opts.split_k > 0 ? P->opts.split_k : parts, num_kb});
             const bool worth = tiles < units_max ? num_kb >= 8 : loss > 0.02;
             if (split >= 2 && (sk_mode == 2 || worth)) sk_tiles = rem;
         }

@@ -142,7 +142,9 @@ typedef struct gemm_epi_options {
                           without GELU / tanh and at least four waves of 256 x 512 tiles).  TC2 with e4m3 and B stored (k, n) supports
                           256 and 512 only (128 is ERR_UNSUPPORTED)                       */
     int32_t split_k;   /* SPLITK: CTAs per cluster along k (1..8; 0 = auto).  TC1/TC2:
-                          cap on the parts a tail tile is split into (0 = 2)          */
+                          cap on the parts a tail tile is split into (0 = auto: 2 behind
+                          whole waves; with fewer tiles than SMs up to 4, at least 8
+                          k-blocks a part)                                             */
     int32_t max_ctas;  /* persistent kernels: cap on resident CTAs (0 = one per SM)    */
     int32_t inject_stall; /* testing only (TC1/TC2): 1 = the MMA issuer never publishes an
                              accumulator, so the epilogue's bounded wait runs out after about

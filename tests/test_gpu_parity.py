@@ -158,6 +158,7 @@ def test_alpha_scaling_16bit(kernel, dtype):
     ("tc1", 16, 256, 256, 4),   # fewer tiles than CTAs: every tile in four parts
     ("tc2", 12, 600, 528, 2),   # pairs: 3 x 5 tiles on 6 pairs
     ("tc2", 8, 256, 256, 2),    # pairs, fewer tiles than pairs (2 tiles on 4 pairs)
+    ("tc2", 16, 256, 256, 4),   # pairs, fewer tiles than pairs, every tile in four parts
     ("tc2", 8, 600, 1104, 2),   # 512-wide pair tiles (block_n 512): 3 x 3 tiles on 4 pairs
 ])
 @pytest.mark.parametrize("dtype,epilogue,axis,layout", [
@@ -175,6 +176,21 @@ def test_stream_k(kernel, max_ctas, m, n, parts, dtype, epilogue, axis, layout):
                                        stream_k="on", split_k=parts)
     assert info["sk_tiles"] > 0 and info["sk_split"] == parts
     assert worst <= 1.0
+
+
+@pytest.mark.parametrize("kernel", ["tc1", "tc2"])
+def test_auto_split_depth_for_few_tiles(kernel):
+    """Fewer tiles than units and a long k: the automatic plan cuts every tile into four
+    parts; behind whole waves it keeps two."""
+    wl = Workload("sk_auto", 256, 1024, 4096, "f16", "gelu_bias", "col", "nk", seed=15,
+                  dist_b=("uniform", 1 / 64), dist_bias=("uniform", 1 / 64))
+    prob = make_problem(wl)
+    worst, info = check_against_oracle(wl, prob, kernel=kernel)
+    assert info["sk_tiles"] > 0 and info["sk_split"] == 4
+    assert worst <= 1.0
+    big = g.Plan(4096, 4096, 4096, "bf16", "relu_aux_bias", "row", "kn", kernel=kernel, block_n=256)
+    assert big.info["sk_tiles"] > 0 and big.info["sk_split"] == 2
+    big.close()
 
 
 def test_wide_tiles_chosen_for_many_waves():

@@ -54,5 +54,5 @@ def test_random_problem_matches_oracle(wl):
     worst, info = check_against_oracle(wl, make_problem(wl))
     assert worst <= 1.0
     # the automatic choice: split-K for small m where it applies, else a persistent kernel
-    small = wl.m <= 64 and wl.a_layout == "mk"
+    small = wl.m <= 32 and wl.a_layout == "mk"
     assert (info["kernel"] == g.KERNEL_SPLITK) == small
