@@ -283,17 +283,31 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
 // Mathematical Functions, formula 7.1.26:
 //     erfc(z) ~= t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2),  t = 1 / (1 + p z),
 // with p = 0.3275911, a1..a5 = 0.254829592, -0.284496736, 1.421413741,
-// -1.453152027, 1.061405429 and |error| <= 1.5e-7.  1 + erf(x/sqrt 2) is erfc(z)
-// for x < 0 (no cancellation on the negative tail) and 2 - erfc(z) for x >= 0.
-// Branch-free: one reciprocal, one exponential, five FMAs.
+// -1.453152027, 1.061405429 and |error| <= 1.5e-7.  Since Phi(x) = erfc(z)/2 for
+// x < 0 and 1 - erfc(z)/2 for x >= 0, both sides are one expression:
+//     GELU(x) = max(x, 0) - |x| erfc(z) / 2,
+// with no cancellation on the negative tail.  The halves are folded into the
+// coefficients (h_i = a_i / 2), p / sqrt 2 into the reciprocal's argument, and
+// exp(-z^2) = 2^(-(c |x|)^2) with c = sqrt(log2(e) / 2).  Branch-free: 10 fp32
+// operations and two hardware approximations (rcp.approx, ex2.approx of the PTX ISA).
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ float gelu_erf(float x) {
-    const float z = fabsf(x) * 0.70710678118654752f;
-    const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
-    const float poly =
-        t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f), -0.284496736f),
-                 0.254829592f);
-    const float ec = poly * __expf(-z * z);
-    return 0.5f * x * (x >= 0.0f ? 2.0f - ec : ec);
+    const float ax = fabsf(x);
+    const float t = rcp_approx(fmaf(0.3275911f * 0.70710678118654752f, ax, 1.0f));
+    const float half_poly =
+        t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 0.5307027145f, -0.7265760135f), 0.7107068705f), -0.142248368f),
+                 0.127414796f);
+    const float s = ax * 0.84932180028801907f;
+    return fmaf(-ax, half_poly * ex2_approx(-s * s), fmaxf(x, 0.0f));
 }
 
 template <int EPI>
