@@ -434,9 +434,9 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
     return e == cudaSuccess ? GEMM_EPI_OK : GEMM_EPI_ERR_CUDA;
 }
 
-int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis, int b_layout,
-              const gemm_epi_options *opts, gemm_epi_plan_t *out) {
-    if (!out) return GEMM_EPI_ERR_ARG;
+// Argument checks that need no device, and the plan's problem fields.
+int plan_fields(Plan *P, int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis, int b_layout,
+                const gemm_epi_options *opts) {
     if (m <= 0 || n <= 0 || k <= 0) return GEMM_EPI_ERR_ARG;
     if (m > 0x7fffffffll || n > 0x7fffffffll || k > 0x7fffffffll) return GEMM_EPI_ERR_ARG;
     if (((m + 127) / 128) * ((n + 127) / 128) > 0x7fffffffll) return GEMM_EPI_ERR_ARG;   // tile count is an int
@@ -468,19 +468,6 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     if ((n * es) % 16 != 0 || (n * out_es) % 16 != 0) return GEMM_EPI_ERR_ALIGN;
     if (a_km && (m * es) % 16 != 0) return GEMM_EPI_ERR_ALIGN;     // A (k, m): row pitch m * esize
 
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) {
-        cudaGetLastError();
-        return GEMM_EPI_ERR_NO_DEVICE;
-    }
-    int major = 0, minor = 0;
-    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-    if (major != 10 || minor != 0) return GEMM_EPI_ERR_NO_DEVICE;
-
-    Plan *P = new (std::nothrow) Plan();
-    if (!P) return GEMM_EPI_ERR_CUDA;
-    P->magic = kPlanMagic;
     P->m = m;
     P->n = n;
     P->k = k;
@@ -495,9 +482,36 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     P->b_layout = b_layout;
     P->a_km = a_km;
     P->opts = o;
+    return GEMM_EPI_OK;
+}
+
+int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis, int b_layout,
+              const gemm_epi_options *opts, gemm_epi_plan_t *out) {
+    if (!out) return GEMM_EPI_ERR_ARG;
+    Plan *P = new (std::nothrow) Plan();
+    if (!P) return GEMM_EPI_ERR_CUDA;
+    int rc = plan_fields(P, m, n, k, dtype, epilogue, bias_axis, b_layout, opts);
+    if (rc != GEMM_EPI_OK) {
+        delete P;
+        return rc;
+    }
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        delete P;
+        return GEMM_EPI_ERR_NO_DEVICE;
+    }
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0) {
+        delete P;
+        return GEMM_EPI_ERR_NO_DEVICE;
+    }
+    P->magic = kPlanMagic;
     P->device = dev;
     P->num_sms = num_sms_of(dev);
-    int rc = choose(P);
+    rc = choose(P);
     if (rc != GEMM_EPI_OK) {
         delete P;
         return rc;
@@ -728,9 +742,8 @@ int gemm_epi_check(gemm_epi_plan_t plan, void *stream) {
     return GEMM_EPI_OK;
 }
 
-int gemm_epi_plan_query(gemm_epi_plan_t plan, gemm_epi_plan_info *info) {
-    if (!live(plan) || !info) return GEMM_EPI_ERR_ARG;
-    Plan *P = reinterpret_cast<Plan *>(plan);
+namespace {
+void fill_info(const Plan *P, gemm_epi_plan_info *info) {
     info->kernel = P->kernel;
     info->block_m = P->kernel == GEMM_EPI_KERNEL_SPLITK ? P->nm : P->info.block_m;
     info->block_n = P->block_n;
@@ -749,6 +762,26 @@ int gemm_epi_plan_query(gemm_epi_plan_t plan, gemm_epi_plan_info *info) {
         const int bm = P->kernel == GEMM_EPI_KERNEL_TC2 ? 256 : 128;
         info->tiles = (int)(((P->m + bm - 1) / bm) * ((P->n + P->block_n - 1) / P->block_n));
     }
+}
+}  // namespace
+
+int gemm_epi_plan_query(gemm_epi_plan_t plan, gemm_epi_plan_info *info) {
+    if (!live(plan) || !info) return GEMM_EPI_ERR_ARG;
+    fill_info(reinterpret_cast<Plan *>(plan), info);
+    return GEMM_EPI_OK;
+}
+
+int gemm_epi_plan_preview(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis, int b_layout,
+                          const gemm_epi_options *opts, int num_sms, gemm_epi_plan_info *info) {
+    if (!info || num_sms < 2 || num_sms > 1024) return GEMM_EPI_ERR_ARG;
+    Plan P;
+    int rc = plan_fields(&P, m, n, k, dtype, epilogue, bias_axis, b_layout, opts);
+    if (rc != GEMM_EPI_OK) return rc;
+    P.device = -1;
+    P.num_sms = num_sms;
+    rc = choose(&P);
+    if (rc != GEMM_EPI_OK) return rc;
+    fill_info(&P, info);
     return GEMM_EPI_OK;
 }
 

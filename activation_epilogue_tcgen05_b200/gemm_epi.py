@@ -47,7 +47,8 @@ EXPORTS = ("gemm_epi_plan", "gemm_epi_plan_ex", "gemm_epi_plan_opts", "gemm_epi_
            "gemm_epi_free", "gemm_epi_status_string", "gemm_epi_aux_pitch_bytes",
            "gemm_epi_version", "gemm_epi_run_noalloc", "gemm_epi_run_bwd", "gemm_epi_unfused_run_bwd",
            "gemm_epi_set_out_scale", "gemm_epi_mlp_plan", "gemm_epi_mlp_set_scales", "gemm_epi_mlp_run",
-           "gemm_epi_mlp_check", "gemm_epi_mlp_query", "gemm_epi_mlp_free", "gemm_epi_mlp_unfused_run")
+           "gemm_epi_mlp_check", "gemm_epi_mlp_query", "gemm_epi_mlp_free", "gemm_epi_mlp_unfused_run",
+           "gemm_epi_plan_preview")
 
 
 class Options(ctypes.Structure):
@@ -107,6 +108,8 @@ def lib():
             L.gemm_epi_mlp_free.argtypes = [vp]
             L.gemm_epi_check.argtypes = [vp, vp]
             L.gemm_epi_plan_query.argtypes = [vp, ctypes.POINTER(PlanInfo)]
+            L.gemm_epi_plan_preview.argtypes = [i64, i64, i64, i32, i32, i32, i32,
+                                                ctypes.POINTER(Options), i32, ctypes.POINTER(PlanInfo)]
             L.gemm_epi_free.argtypes = [vp]
             L.gemm_epi_status_string.argtypes = [i32]
             L.gemm_epi_status_string.restype = ctypes.c_char_p
@@ -216,6 +219,27 @@ def gemm_epi_plan_query(plan) -> dict:
     info = PlanInfo()
     _check(lib().gemm_epi_plan_query(plan, ctypes.byref(info)), "gemm_epi_plan_query")
     return info.as_dict()
+
+
+def gemm_epi_plan_preview(m, n, k, dtype, epilogue, bias_axis, b_layout, opts: Options | None,
+                          num_sms: int) -> dict:
+    info = PlanInfo()
+    _check(lib().gemm_epi_plan_preview(m, n, k, dtype, epilogue, bias_axis, b_layout,
+                                       ctypes.byref(opts) if opts is not None else None, num_sms,
+                                       ctypes.byref(info)), "gemm_epi_plan_preview")
+    return info.as_dict()
+
+
+def plan_preview(m, n, k, dtype="bf16", epilogue="bias", bias_axis="row", b_layout="kn", num_sms=148,
+                 kernel="auto", block_n=0, split_k=0, max_ctas=0, stream_k="auto", out_e4m3=False,
+                 a_layout="mk") -> dict:
+    """The kernel choice a plan would make on a device with ``num_sms`` SMs, computed on the
+    host (no device needed); the same names as :class:`Plan`, the same keys as ``Plan.info``."""
+    opts = Options(KERNEL[kernel], int(block_n), int(split_k), int(max_ctas), 0, STREAM_K[stream_k],
+                   1 if out_e4m3 else 0)
+    layout = LAYOUT[b_layout] | (A_KM if a_layout == "km" else 0)
+    return gemm_epi_plan_preview(int(m), int(n), int(k), DTYPE[dtype], EPILOGUE[epilogue], AXIS[bias_axis],
+                                 layout, opts, int(num_sms))
 
 
 def gemm_epi_free(plan) -> None:

@@ -274,6 +274,18 @@ int gemm_epi_check(gemm_epi_plan_t plan, void *stream);
 /* Fill *info with the plan's kernel choice.  ERR_ARG on a bad handle. */
 int gemm_epi_plan_query(gemm_epi_plan_t plan, gemm_epi_plan_info *info);
 
+/* The kernel choice gemm_epi_plan_opts would make on a compute-capability 10.0 device
+ * with num_sms SMs, computed on the host alone: no device is needed or touched, nothing is
+ * allocated or launched.  Arguments as gemm_epi_plan_opts (opts may be NULL); num_sms in
+ * 2..1024 (148 on a B200); info is a HOST pointer, filled as by gemm_epi_plan_query.
+ * Returns OK, or the status gemm_epi_plan_opts returns for these arguments before it
+ * looks at the device (ERR_ARG / ERR_ALIGN / ERR_UNSUPPORTED); ERR_ARG for a NULL info
+ * or num_sms out of range.  *info is untouched on error.  (A service of this library;
+ * the pages have no counterpart.) */
+int gemm_epi_plan_preview(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis,
+                          int b_layout, const gemm_epi_options *opts, int num_sms,
+                          gemm_epi_plan_info *info);
+
 /* Fused run that allocates nothing (the pages have no counterpart; this is a
  * service of this library).  For callers that must not allocate device memory:
  * code inside a host framework that hands out all device memory from its own

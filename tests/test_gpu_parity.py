@@ -193,6 +193,25 @@ def test_auto_split_depth_for_few_tiles(kernel):
     big.close()
 
 
+@pytest.mark.parametrize("shape", [
+    (4096, 4096, 4096, "bf16", "relu_aux_bias", "row", "kn", {}),
+    (1024, 512, 2048, "f16", "bias", "row", "kn", {}),
+    (16, 4096, 4096, "f16", "gelu_bias", "col", "nk", {}),
+    (33, 4096, 4096, "f16", "gelu_bias", "col", "nk", {}),
+    (65536, 8192, 16384, "bf16", "relu_bias", "row", "kn", {}),
+    (8192, 14336, 4096, "e4m3", "gelu_bias", "col", "kn", {}),
+    (4096, 4096, 4096, "bf16", "drelu_bgrad", "col", "kn", {}),
+    (600, 528, 1000, "bf16", "relu_aux_bias", "row", "kn", {"max_ctas": 12, "kernel": "tc2"}),
+    (256, 1024, 4096, "f16", "gelu_bias", "col", "nk", {"kernel": "tc1"}),
+])
+def test_preview_matches_plans(shape):
+    """The host-only preview makes the choice a real plan makes on this device."""
+    m, n, k, dt, epi, axis, layout, kw = shape
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    with g.Plan(m, n, k, dt, epi, axis, layout, **kw) as plan:
+        assert g.plan_preview(m, n, k, dt, epi, axis, layout, num_sms=sms, **kw) == plan.info
+
+
 def test_wide_tiles_chosen_for_many_waves():
     """4096 x 16384: 512 tiles of 256 x 512 for 74 pairs, so the plan takes 512-wide tiles;
     checked on seeded sampled positions (and element-exact mask outside the band)."""

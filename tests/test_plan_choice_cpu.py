@@ -1,0 +1,144 @@
+"""The kernel choice (family, tile width, K split, split tail, grid) on the host, without a GPU,
+through gemm_epi_plan_preview: the rules a plan follows for the workloads the library is measured
+on and at the boundaries between the rules.  The GPU suite checks that a real plan makes the same
+choice (test_gpu_parity.py::test_preview_matches_plans)."""
+import pytest
+
+SMS = 148   # a B200
+
+
+@pytest.fixture(scope="module")
+def g():
+    from activation_epilogue_tcgen05_b200 import build, gemm_epi
+    build.build()
+    return gemm_epi
+
+
+def pv(g, m, n, k, dtype="bf16", epilogue="bias", axis="row", layout="kn", sms=SMS, **kw):
+    return g.plan_preview(m, n, k, dtype, epilogue, axis, layout, num_sms=sms, **kw)
+
+
+# ------------------------------------------------------------------ the measured workloads
+def test_headline_relu_aux_bias_4096(g):
+    p = pv(g, 4096, 4096, 4096, "bf16", "relu_aux_bias")
+    # 256 tiles of 256 x 256 on 74 pairs: 3 whole waves, the 34 tiles of the last one in two parts
+    assert (p["kernel"], p["block_m"], p["block_n"], p["cluster"]) == (g.KERNEL_TC2, 256, 256, 2)
+    assert (p["tiles"], p["grid"], p["sk_tiles"], p["sk_split"]) == (256, 148, 34, 2)
+    assert p["threads"] == 320 and p["stages"] == 6
+
+
+def test_small_gemm_bias_1024x512x2048(g):
+    p = pv(g, 1024, 512, 2048, "f16", "bias")
+    # 32 tiles of 128 x 128, fewer than the SMs: every tile in four k-parts on 128 CTAs
+    assert (p["kernel"], p["block_n"], p["tiles"]) == (g.KERNEL_TC1, 128, 32)
+    assert (p["sk_tiles"], p["sk_split"], p["grid"]) == (32, 4, 128)
+
+
+def test_linear_gelu_batch16_splitk(g):
+    p = pv(g, 16, 4096, 4096, "f16", "gelu_bias", "col", "nk")
+    # swapped roles: 32 weight tiles of 128 rows, K split over clusters of 4 CTAs
+    assert (p["kernel"], p["block_m"], p["split_k"], p["cluster"], p["grid"]) == (g.KERNEL_SPLITK, 16, 4, 4, 128)
+
+
+def test_large_relu_bias_wide_tiles(g):
+    p = pv(g, 65536, 8192, 16384, "bf16", "relu_bias")
+    assert (p["kernel"], p["block_n"], p["tiles"], p["grid"]) == (g.KERNEL_TC2, 512, 4096, 148)
+    assert p["sk_tiles"] == 0       # 4096 tiles on 74 pairs: under 2 % lost to the last wave
+
+
+def test_fp8_gelu_bias(g):
+    p = pv(g, 8192, 14336, 4096, "e4m3", "gelu_bias", "col", "kn")
+    assert (p["kernel"], p["block_n"], p["block_k"], p["tiles"]) == (g.KERNEL_TC2, 256, 128, 1792)
+    assert (p["sk_tiles"], p["sk_split"]) == (16, 2)
+
+
+# ------------------------------------------------------------------ family boundaries
+@pytest.mark.parametrize("m,kernel", [(1, "splitk"), (16, "splitk"), (32, "splitk"), (33, "tc1"),
+                                      (64, "tc1"), (128, "tc1"), (256, "tc1")])
+def test_batch_boundary(g, m, kernel):
+    p = pv(g, m, 4096, 4096, "f16", "gelu_bias", "col", "nk")
+    assert p["kernel"] == {"splitk": g.KERNEL_SPLITK, "tc1": g.KERNEL_TC1}[kernel]
+
+
+@pytest.mark.parametrize("m,nm", [(1, 16), (16, 16), (17, 32), (32, 32)])
+def test_splitk_batch_tile(g, m, nm):
+    assert pv(g, m, 4096, 4096, "f16", "gelu_bias", "col", "nk")["block_m"] == nm
+
+
+def test_pairs_need_a_tile_per_pair(g):
+    # 256 x 256 tiles: 73 of them leave a pair idle (single CTAs), 74 fill every pair
+    assert pv(g, 256 * 73, 256, 1024)["kernel"] == g.KERNEL_TC1
+    assert pv(g, 256 * 74, 256, 1024)["kernel"] == g.KERNEL_TC2
+
+
+def test_backward_and_transposed_a_never_take_splitk(g):
+    assert pv(g, 16, 4096, 4096, "bf16", "drelu", "row", "kn")["kernel"] != g.KERNEL_SPLITK
+    assert pv(g, 16, 4096, 4096, "bf16", "bias", "row", "kn", a_layout="km")["kernel"] != g.KERNEL_SPLITK
+
+
+# ------------------------------------------------------------------ tile width
+def test_wide_tiles_only_for_many_waves_of_light_16bit_work(g):
+    big = (8192, 8192, 4096)             # 512 tiles of 256 x 512: 6.9 waves of pairs
+    assert pv(g, *big, "bf16", "relu_bias")["block_n"] == 512
+    assert pv(g, *big, "f16", "relu_aux_bias")["block_n"] == 512
+    assert pv(g, *big, "bf16", "gelu_bias")["block_n"] == 256     # heavy epilogue
+    assert pv(g, *big, "bf16", "tanh_bias")["block_n"] == 256
+    assert pv(g, *big, "e4m3", "bias")["block_n"] == 256         # short fp8 mainloop
+    assert pv(g, *big, "bf16", "drelu")["block_n"] == 256        # backward
+    assert pv(g, 4096, 4096, 4096, "bf16", "bias")["block_n"] == 256   # 1.7 waves of wide tiles
+    assert pv(g, 8192, 4096, 4096, "bf16", "bias")["block_n"] == 256   # 3.5 waves
+
+
+def test_e4m3_pairs_with_b_kn_take_256(g):
+    p = pv(g, 512, 256, 1024, "e4m3", "bias", "row", "kn", kernel="tc2")
+    assert p["block_n"] == 256
+
+
+def test_explicit_tile_width_is_kept(g):
+    assert pv(g, 4096, 4096, 4096, "bf16", "bias", kernel="tc2", block_n=512)["block_n"] == 512
+    assert pv(g, 4096, 4096, 4096, "bf16", "bias", kernel="tc1", block_n=128)["block_n"] == 128
+
+
+# ------------------------------------------------------------------ split tail
+def test_split_tail_parts(g):
+    # fewer tiles than units: up to four parts of at least 8 k-blocks
+    assert pv(g, 1024, 512, 4096, "f16", "bias")["sk_split"] == 4        # 64 k-blocks
+    assert pv(g, 1024, 512, 1024, "f16", "bias")["sk_split"] == 2        # 16 k-blocks
+    assert pv(g, 1024, 512, 256, "f16", "bias")["sk_tiles"] == 0         # 4 k-blocks: not worth it
+    # 64 tiles on 148 SMs: only two parts fit
+    assert pv(g, 256, 4096, 4096, "f16", "gelu_bias", "col", "nk")["sk_split"] == 2
+    # behind whole waves: two parts for the last wave's tiles
+    p = pv(g, 4096, 4096, 4096, "bf16", "relu_aux_bias", kernel="tc1", block_n=256)
+    assert (p["tiles"], p["sk_tiles"], p["sk_split"]) == (512, 512 % 148, 2)
+
+
+def test_split_tail_options(g):
+    assert pv(g, 4096, 4096, 4096, "bf16", "bias", stream_k="off")["sk_tiles"] == 0
+    assert pv(g, 4096, 4096, 4096, "bf16", "bias", split_k=3)["sk_split"] == 2   # 74 // 34 = 2 fit
+    p = pv(g, 1024, 512, 4096, "f16", "bias", split_k=2)
+    assert p["sk_split"] == 2 and p["grid"] == 64
+
+
+def test_units_follow_the_sm_count(g):
+    # a smaller part (or max_ctas) changes the waves, not the rules
+    p = pv(g, 4096, 4096, 4096, "bf16", "relu_aux_bias", sms=100)
+    assert p["kernel"] == g.KERNEL_TC2 and p["grid"] == 100
+    assert (p["sk_tiles"], p["sk_split"]) == (256 % 50, 2)          # 6 tiles left on 50 pairs
+    # 132 SMs: the last wave's 58 tiles on 66 pairs cannot be cut in two, so no split tail
+    assert pv(g, 4096, 4096, 4096, "bf16", "relu_aux_bias", sms=132)["sk_tiles"] == 0
+    q = pv(g, 4096, 4096, 4096, "bf16", "relu_aux_bias", max_ctas=64)
+    assert q["grid"] == 64 and q["sk_tiles"] == 0                   # 256 tiles on 32 pairs: 8 waves
+
+
+# ------------------------------------------------------------------ argument checks
+def test_preview_checks_arguments_like_a_plan(g):
+    def status(**kw):
+        with pytest.raises(g.GemmEpiError) as e:
+            pv(g, **kw)
+        return e.value.status
+    assert status(m=0, n=128, k=128) == g.ERR_ARG
+    assert status(m=128, n=128, k=100, dtype="f16") == g.ERR_ALIGN        # 200-byte rows
+    assert status(m=128, n=128, k=128, dtype="e4m3", epilogue="tanh_bias", out_e4m3=True) == g.ERR_UNSUPPORTED
+    assert status(m=200, n=128, k=128, kernel="splitk") == g.ERR_UNSUPPORTED   # m > 128
+    assert status(m=128, n=128, k=128, sms=1) == g.ERR_ARG
+    assert status(m=128, n=128, k=128, sms=4096) == g.ERR_ARG
