@@ -807,7 +807,7 @@ const char *gemm_epi_status_string(int status) {
     case GEMM_EPI_ERR_ARG: return "invalid argument (size, enum, option or plan handle)";
     case GEMM_EPI_ERR_ALIGN: return "pointer not 16-byte aligned or row pitch not a multiple of 16 bytes";
     case GEMM_EPI_ERR_NULL: return "required pointer is NULL (operand, bias, aux, dbias or FP8 scales)";
-    case GEMM_EPI_ERR_UNSUPPORTED: return "combination not supported by this build";
+    case GEMM_EPI_ERR_UNSUPPORTED: return "combination not supported by this library";
     case GEMM_EPI_ERR_CUDA: return "CUDA runtime or driver call failed";
     case GEMM_EPI_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
     case GEMM_EPI_ERR_NO_DEVICE: return "no current sm_100 (B200-class) CUDA device";

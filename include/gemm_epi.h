@@ -119,7 +119,7 @@ enum gemm_epi_status {
     GEMM_EPI_ERR_NULL = -3,         /* required pointer NULL (A, B, D; bias for a bias epilogue;
                                        aux for RELU_AUX(_BIAS) and the backward epilogues; dbias
                                        for DRELU_BGRAD; scales unset for E4M3) */
-    GEMM_EPI_ERR_UNSUPPORTED = -4,  /* valid request this build cannot serve (option combination) */
+    GEMM_EPI_ERR_UNSUPPORTED = -4,  /* valid request this library cannot serve (option combination) */
     GEMM_EPI_ERR_CUDA = -5,         /* a CUDA runtime/driver call failed (launch, tensor map) */
     GEMM_EPI_ERR_TIMEOUT = -6,      /* a kernel gave up on a bounded wait (reported by check()) */
     GEMM_EPI_ERR_NO_DEVICE = -7     /* current device is not sm_100 (B200 class) */
