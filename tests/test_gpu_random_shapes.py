@@ -45,7 +45,21 @@ def draw_case(i):
     return Workload(f"rand{i}", m, n, k, dtype, epi, axis, b_layout, seed=2000 + i, a_layout=a_layout)
 
 
-CASES = [draw_case(i) for i in range(64)]
+def draw_long_k_case(i):
+    """Few tiles and a long k: the automatic plan splits every tile into three or four parts."""
+    rng = np.random.default_rng(5000 + i)
+    dtype = ["f16", "bf16", "e4m3"][rng.integers(3)]
+    step = 16 if dtype == "e4m3" else 8
+    m = int(rng.integers(33, 520))
+    n = int(step * rng.integers(1, 640 // step + 1))
+    k = int(step * rng.integers(2048 // step, 4096 // step + 1))
+    epi = FORWARD[rng.integers(len(FORWARD))]
+    axis = ["row", "col"][rng.integers(2)]
+    b_layout = ["kn", "nk"][rng.integers(2)]
+    return Workload(f"randk{i}", m, n, k, dtype, epi, axis, b_layout, seed=6000 + i)
+
+
+CASES = [draw_case(i) for i in range(64)] + [draw_long_k_case(i) for i in range(16)]
 
 
 @pytest.mark.parametrize("wl", CASES, ids=[f"{w.name}-{w.m}x{w.n}x{w.k}-{w.dtype}-{w.epilogue}-{w.bias_axis}-"
