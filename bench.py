@@ -71,6 +71,8 @@ def parse(argv=None):
                          "(0 = the plan's choice)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--ref-seconds", type=float, default=60.0,
+                    help="--impl reference: target CPU time of the whole warm-up + timed run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-unfused", action="store_true")
@@ -280,12 +282,12 @@ def reference_arm(args):
         return time.perf_counter() - t0
 
     threads = oracle.threads()
-    # size one step so that warmup + steps take about a minute in total
+    # size one step so that warmup + steps take about --ref-seconds (a minute) in total
     per_unit = wl.n if bwd else 1          # output positions per counted unit (row or position)
     probe = max(threads, 1) if bwd else max(threads * 4, 64)
     t_probe = step(probe)
     per_pos = t_probe / probe
-    budget = 60.0 / max(1, args.steps + args.warmup)
+    budget = args.ref_seconds / max(1, args.steps + args.warmup)
     count = int(max(threads if not bwd else 1, min((1 << 20) // per_unit, budget / max(per_pos, 1e-9))))
     count = min(count, m_avail) if bwd else count
     for _ in range(args.warmup):

@@ -1,0 +1,42 @@
+"""bench.py's reference arm (the fp64 CPU oracle, timed) runs on a machine without a GPU: its one
+JSON line carries the keys and units the benchmark contract asks for."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def reference_line(*extra):
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "2",
+                        "--warmup", "1", "--ref-seconds", "3", *extra], env=env, cwd=ROOT,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1, r.stdout
+    return json.loads(lines[0])
+
+
+@pytest.mark.parametrize("extra,workload", [
+    ((), "relu_aux_bias_bf16_4096x4096x4096"),
+    (("--workload", "gemm_bias_f16_1024x512x2048"), "gemm_bias_f16_1024x512x2048"),
+    (("--shape", "256,256,512,bf16,drelu_bgrad,col,kn"), "custom_bf16_drelu_bgrad_256x256x512_kn"),
+])
+def test_reference_arm_json_line(extra, workload):
+    d = reference_line(*extra)
+    assert d["impl"] == "reference"
+    assert d["metric"].startswith("fused GEMM+bias(+act) TFLOP/s")
+    assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["ms_per_step"] > 0
+    assert (d["n_gpus"], d["steps"], d["warmup"]) == (1, 2, 1)
+    assert d["scaling"] == "weak" and d["vs_baseline"] is None and d["data"] == "synthetic"
+    assert d["config"]["workload"] == workload
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    e = d["e2e"]
+    assert (e["value"], e["unit"]) == (d["value"], d["unit"])
+    assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
