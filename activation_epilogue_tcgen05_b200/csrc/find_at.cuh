@@ -11,7 +11,7 @@ struct TcFindAT {
     template <int CG, int EPI, int AXIS, bool BMN>
     static bool leaf(TcLauncher *l, KernelInfo *i) {
         constexpr int ES = DTV == DT_E4M3 ? 1 : 2;
-        constexpr int STG = tc_stages(128 * 128 + (256 / CG) * 128);
+        constexpr int STG = tc_stages(tc_katoms(128 * 128 + (256 / CG) * 128) * (128 * 128 + (256 / CG) * 128));
         if constexpr (BMN && (256 / CG) % (128 / ES) != 0) {
             return false;
         } else {

@@ -44,6 +44,7 @@ struct Plan {
     int nm;              // SPLITK: MMA N (batch rows rounded up)
     int split;           // SPLITK: cluster size along k
     int kb_per_cta;
+    int katoms = 1;      // TC: 128-byte k-atoms per ring stage (the kernel's KATOMS)
     int grid;
     int group_m;
     bool pdl;            // programmatic dependent launch (GEMM_EPI_PDL=0 turns it off)
@@ -232,6 +233,9 @@ int choose(Plan *P) {
         }
         if (bn != 128 && bn != 256 && bn != 512) return GEMM_EPI_ERR_ARG;
         P->block_n = bn;
+        // the kernel's ring stages hold katoms k-atoms; its k-blocks are stages
+        P->katoms = tc_katoms(128 * 128 + (bn / cg) * 128);
+        const int64_t num_kb_tc = (P->k + (int64_t)bk * P->katoms - 1) / ((int64_t)bk * P->katoms);
         const int64_t tiles = ((m + bm - 1) / bm) * ((n + bn - 1) / bn);
         const int64_t units_max = cg == 2 ? sms / 2 : sms;
         // split tail: the tiles of an incomplete last wave (or all tiles, when there are fewer
@@ -247,8 +251,9 @@ int choose(Plan *P) {
             const int64_t rem = tiles < units_max ? tiles : tiles % units_max;
             const int64_t waves = (tiles + units_max - 1) / units_max;
             const double loss = 1.0 - (double)tiles / (double)(waves * units_max);
+            // (part sizes in 128-byte k-atoms, so that the rule does not depend on the stage size)
             const int64_t parts = tiles < units_max ? std::max<int64_t>(2, std::min<int64_t>(4, num_kb / 8)) : 2;
-            split = std::min<int64_t>({units_max / rem, P->opts.split_k > 0 ? P->opts.split_k : parts, num_kb});
+            split = std::min<int64_t>({units_max / rem, P->opts.split_k > 0 ? P->opts.split_k : parts, num_kb_tc});
             const bool worth = tiles < units_max ? num_kb >= 8 : loss > 0.02;
             if (split >= 2 && (sk_mode == 2 || worth)) sk_tiles = rem;
         }
@@ -272,6 +277,7 @@ int choose(Plan *P) {
             return GEMM_EPI_ERR_UNSUPPORTED;
         if (!find_tc(cg, P->dtype, P->kepi, P->axis, b_mn, bn, P->qout, P->a_km, &P->tc_launch, &P->info))
             return GEMM_EPI_ERR_UNSUPPORTED;
+        if (P->info.katoms != P->katoms || none_info.katoms != P->katoms) return GEMM_EPI_ERR_UNSUPPORTED;
         P->split = 1;
     }
     if (P->kepi != EPI_NONE && !P->qout && !find_bias_act(P->dtype, P->kepi, P->axis, &P->ba_launch))
@@ -408,7 +414,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.tiles_m = (int)((P->m + 128 * cg - 1) / (128 * cg));
         L.p.tiles_n = (int)((P->n + P->block_n - 1) / P->block_n);
         L.p.num_tiles = L.p.tiles_m * L.p.tiles_n;
-        L.p.num_kb = num_kb;
+        L.p.num_kb = (int)((P->k + (int64_t)bk * P->katoms - 1) / ((int64_t)bk * P->katoms));   // ring stages
         L.p.group_m = P->group_m;
         L.p.bias = bias;
         L.p.aux = aux;

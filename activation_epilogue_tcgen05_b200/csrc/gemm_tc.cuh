@@ -323,6 +323,13 @@ __device__ __forceinline__ float activate(float x) {
     }
 }
 
+// 128-byte k-atoms per ring stage.  A stage is turned over (loaded, multiplied, released) in
+// roughly the same time whatever its size, so where one atom's A and B tiles are at most 32 KB
+// per CTA a stage holds two atoms: twice the MMA work per turnover (pair 256 x 256 tiles: 64 KB
+// and 1024 MMA clocks a stage, three stages).  48 KB atoms (the 512-wide pair tile, the
+// single-CTA 256-wide tile) stay at one atom, keeping enough stages in flight.
+constexpr int tc_katoms(int atom_bytes) { return atom_bytes <= 32768 ? 2 : 1; }
+
 template <int DT_, int EPI_, int AXIS_, bool B_MN_, int BN_, int CG_, int STAGES_, bool QOUT_ = false,
           bool A_MN_ = false>
 struct TcCfg {
@@ -337,8 +344,10 @@ struct TcCfg {
     static constexpr int UMMA_K = 32 / ESIZE;       // k per tcgen05.mma
     static constexpr int KSTEPS = BK / UMMA_K;      // 4
     static constexpr int BN_LOCAL = BN / CG;        // B rows (n) this CTA loads
-    static constexpr int A_BYTES = BM * 128;
-    static constexpr int B_BYTES = BN_LOCAL * 128;
+    static constexpr int A_BYTES = BM * 128;                 // one k-atom of A (128 bytes of k a row)
+    static constexpr int B_BYTES = BN_LOCAL * 128;           // one k-atom of this CTA's B rows
+    static constexpr int KATOMS = tc_katoms(A_BYTES + B_BYTES);
+    static constexpr int A_STAGE = KATOMS * A_BYTES, B_STAGE = KATOMS * B_BYTES;
     static constexpr int B_BOX_N = 128 / ESIZE;     // n per 128-byte MN-major box
     static constexpr int B_BOXES = B_MN ? BN_LOCAL / B_BOX_N : 1;
     // A 512-wide pair tile is two N = 256 MMAs per k-step, each writing its own 256 TMEM
@@ -375,8 +384,8 @@ struct TcCfg {
     static constexpr int STG_BYTES = QOUT ? 0 : 32 * 64;   // per epilogue warp: 32 rows x 32 16-bit outputs
     // shared-memory layout (offsets from a 1024-byte aligned base)
     static constexpr int OFF_A = 0;
-    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-    static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
+    static constexpr int OFF_STG = OFF_B + STAGES * B_STAGE;
     static constexpr int OFF_BIAS = OFF_STG + EPI_WARPS * STG_BYTES;
     static constexpr int BIAS_FLOATS = (FWD_BIAS && AXIS == AXIS_COL) ? COLS_W : 0;
     static constexpr int OFF_BAR = OFF_BIAS + EPI_WARPS * BIAS_FLOATS * 4;
@@ -488,13 +497,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     uint32_t fb = full_bar(stage);
                     if constexpr (C::CG == 2) {
                         fb = ptx::mapa(fb, 0);      // the pair's leader counts both CTAs' bytes
-                        if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * (C::A_BYTES + C::B_BYTES));
+                        if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * (C::A_STAGE + C::B_STAGE));
                     } else {
-                        ptx::mbar_arrive_expect_tx(fb, C::A_BYTES + C::B_BYTES);
+                        ptx::mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE);
                     }
-                    const int k0 = kb * C::BK;
-                    const uint32_t a_dst = sA + stage * C::A_BYTES;
-                    const uint32_t b_dst = sB + stage * C::B_BYTES;
+                    for (int at = 0; at < C::KATOMS; ++at) {    // the stage's k-atoms
+                    const int k0 = (kb * C::KATOMS + at) * C::BK;
+                    const uint32_t a_dst = sA + stage * C::A_STAGE + at * C::A_BYTES;
+                    const uint32_t b_dst = sB + stage * C::B_STAGE + at * C::B_BYTES;
                     auto load = [&](uint32_t dst, const CUtensorMap *map, int c0, int c1) {
                         if constexpr (C::CG == 2)
                             ptx::tma_load_2d_pair(dst, map, fb, c0, c1, 0x1000000000000000ull);
@@ -518,6 +528,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
                         for (int h = 0; h < C::N_MMAS; ++h)
                             load(b_dst + h * C::HALF_B_BYTES, &tmB, k0, nb + h * C::MMA_N);
+                    }
                     }
                     ++issued;
                     if (++stage == (uint32_t)C::STAGES) { stage = 0; phase ^= 1u; }
@@ -555,8 +566,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         break;
                     }
                     ptx::tc_fence_after();
-                    const uint32_t a_base = sA + stage * C::A_BYTES;
-                    const uint32_t b_base = sB + stage * C::B_BYTES;
+#pragma unroll
+                    for (int at = 0; at < C::KATOMS; ++at) {
+                    const uint32_t a_base = sA + stage * C::A_STAGE + at * C::A_BYTES;
+                    const uint32_t b_base = sB + stage * C::B_STAGE + at * C::B_BYTES;
 #pragma unroll
                     for (int ks = 0; ks < C::KSTEPS; ++ks) {
                         const uint64_t ad = C::A_MN ? make_sdesc(a_base + ks * C::UMMA_K * 128, C::A_BOX_BYTES, 1024)
@@ -567,8 +580,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             const uint64_t bd = C::B_MN ? make_sdesc(bh + ks * C::UMMA_K * 128, C::B_BOX_BYTES, 1024)
                                                         : make_sdesc(bh + ks * 32, 16, 1024);
                             ptx::mma<C::CG, C::KIND>(d_tmem + h * C::MMA_N, ad, bd, idesc,
-                                                     (kb > w.kb0 || ks > 0) ? 1u : 0u);
+                                                     (kb > w.kb0 || at > 0 || ks > 0) ? 1u : 0u);
                         }
+                    }
                     }
                     if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(empty_bar(stage), 0x3);
                     else ptx::mma_commit(empty_bar(stage));

@@ -7,7 +7,7 @@ namespace gemm_epi {
 
 template <int CG, int EPI, int AXIS, bool BMN, int BN>
 static bool q_leaf(TcLauncher *l, KernelInfo *i) {
-    constexpr int STG = tc_stages(128 * 128 + (BN / CG) * 128);
+    constexpr int STG = tc_stages(tc_katoms(128 * 128 + (BN / CG) * 128) * (128 * 128 + (BN / CG) * 128));
     if constexpr (BMN && (BN / CG) % 128 != 0) {
         return false;   // an MN-major B half-tile narrower than one 128-byte box
     } else {

@@ -34,7 +34,8 @@ struct KernelInfo {
     int threads;
     int smem_bytes;
     int stages;
-    int block_m, block_n, block_k;
+    int block_m, block_n, block_k;   // block_k: k per ring stage
+    int katoms = 1;                  // 128-byte k-atoms per ring stage
 };
 
 using TcLauncher = cudaError_t (*)(const TcLaunch &);
@@ -128,7 +129,8 @@ KernelInfo tc_info() {
     k.stages = C::STAGES;
     k.block_m = C::BM * C::CG;
     k.block_n = C::BN;
-    k.block_k = C::BK;
+    k.block_k = C::BK * C::KATOMS;
+    k.katoms = C::KATOMS;
     return k;
 }
 
@@ -183,7 +185,7 @@ KernelInfo sk_info() {
     template <int CG, int EPI, int AXIS, bool BMN, int BN>                                              \
     static bool NAME##_leaf(TcLauncher *l, KernelInfo *i) {                                             \
         constexpr int ES = (DTV) == DT_E4M3 ? 1 : 2;                                                    \
-        constexpr int STG = tc_stages(128 * 128 + (BN / CG) * 128);                                     \
+        constexpr int STG = tc_stages(tc_katoms(128 * 128 + (BN / CG) * 128) * (128 * 128 + (BN / CG) * 128));                                     \
         if constexpr (BMN && (BN / CG) % (128 / ES) != 0) {                                             \
             return false; /* an MN-major B half-tile narrower than one 128-byte box */                  \
         } else if constexpr (BN == 512 && (CG != 2 || EPI == EPI_DRELU)) {                              \

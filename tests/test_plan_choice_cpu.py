@@ -24,7 +24,8 @@ def test_headline_relu_aux_bias_4096(g):
     # 256 tiles of 256 x 256 on 74 pairs: 3 whole waves, the 34 tiles of the last one in two parts
     assert (p["kernel"], p["block_m"], p["block_n"], p["cluster"]) == (g.KERNEL_TC2, 256, 256, 2)
     assert (p["tiles"], p["grid"], p["sk_tiles"], p["sk_split"]) == (256, 148, 34, 2)
-    assert p["threads"] == 320 and p["stages"] == 6
+    # ring stages of two 128-byte k-atoms (64 KB per CTA): three of them
+    assert p["threads"] == 320 and (p["stages"], p["block_k"]) == (3, 128)
 
 
 def test_small_gemm_bias_1024x512x2048(g):
@@ -48,7 +49,7 @@ def test_large_relu_bias_wide_tiles(g):
 
 def test_fp8_gelu_bias(g):
     p = pv(g, 8192, 14336, 4096, "e4m3", "gelu_bias", "col", "kn")
-    assert (p["kernel"], p["block_n"], p["block_k"], p["tiles"]) == (g.KERNEL_TC2, 256, 128, 1792)
+    assert (p["kernel"], p["block_n"], p["block_k"], p["tiles"]) == (g.KERNEL_TC2, 256, 256, 1792)
     assert (p["sk_tiles"], p["sk_split"]) == (16, 2)
 
 
@@ -87,6 +88,18 @@ def test_wide_tiles_only_for_many_waves_of_light_16bit_work(g):
     assert pv(g, *big, "bf16", "drelu")["block_n"] == 256        # backward
     assert pv(g, 4096, 4096, 4096, "bf16", "bias")["block_n"] == 256   # 1.7 waves of wide tiles
     assert pv(g, 8192, 4096, 4096, "bf16", "bias")["block_n"] == 256   # 3.5 waves
+
+
+def test_ring_stage_atoms(g):
+    # two k-atoms per stage where one atom is at most 32 KB per CTA, one where it is 48 KB
+    big = pv(g, 8192, 8192, 4096, "bf16", "relu_bias")                       # pair 256 x 512
+    assert (big["block_n"], big["block_k"], big["stages"]) == (512, 64, 4)
+    tc1 = pv(g, 4096, 4096, 4096, "bf16", "bias", kernel="tc1", block_n=256)   # single 128 x 256
+    assert (tc1["block_k"], tc1["stages"]) == (64, 4)
+    small = pv(g, 1024, 512, 2048, "f16", "bias")                             # single 128 x 128
+    assert (small["block_k"], small["stages"]) == (128, 3)
+    narrow = pv(g, 4096, 4096, 4096, "bf16", "bias", kernel="tc2", block_n=128)  # pair 256 x 128
+    assert (narrow["block_k"], narrow["stages"]) == (128, 4)
 
 
 def test_e4m3_pairs_with_b_kn_take_256(g):
