@@ -397,6 +397,7 @@ struct TcCfg {
     static_assert(!B_MN || MMA_N_LOCAL % B_BOX_N == 0, "an MMA's B half must be whole boxes");
     static_assert(B_MN == false || BN_LOCAL % B_BOX_N == 0, "MN-major B tile must be whole boxes");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static_assert(STAGES >= 2, "the ring needs two stages: one loading while one is multiplied");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "stage alignment");
     static_assert(!BWD || (EPI_WARPS == 4 && CPG == 4), "backward epilogue: one mask uint4 per chunk group");
     static_assert(!QOUT || (DT == DT_E4M3 && !BWD && EPI != EPI_RELU_AUX), "FP8 output: e4m3 forward plans");

@@ -51,6 +51,8 @@ DEFAULT_WORKLOAD = "relu_aux_bias_bf16_4096x4096x4096"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0        # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+FP8_PEAK_NOTE = (", NOMINAL e4m3 peak: the measured bf16 burst x 2 (the dense fp8/bf16 ratio of the "
+                 "spec); no e4m3 peak is measured")
 
 
 def parse(argv=None):
@@ -82,6 +84,9 @@ def parse(argv=None):
                     help="time the MLP block m,d_model,d_ff,dtype,act,layout instead of one GEMM")
     ap.add_argument("--warm-l2", action="store_true",
                     help="one input set reused every step (L2-warm); the default rotates sets beyond L2")
+    ap.add_argument("--clock-window", type=float, default=0.5,
+                    help="seconds of back-to-back replays of the timed steps, right after the timed "
+                         "region, over which the SM clock is sampled (0 = the timed region only)")
     ap.add_argument("--cublas", action="store_true",
                     help="also time cuBLAS's bare GEMM (torch.matmul, no epilogue) at this shape, "
                          "as context only (16-bit workloads)")
@@ -183,6 +188,42 @@ class ClockSampler:
         reasons = sorted({names[i] for p in win for i in range(4) if p[6 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "power_w_max": max(power) if power else None, "samples": len(win)}
+
+
+def hold_clock_window(replay, region_s: float, hold_s: float, stream, device):
+    """Repeat ``replay`` (the timed region's work) back to back for about ``hold_s`` seconds.
+
+    The timed region of a short workload lasts a few milliseconds, shorter than the clock
+    sampler's period, so its clock is read over this longer window of the same launches
+    instead.  Returns (replays, device seconds, wall-clock end)."""
+    import torch
+    reps = max(1, min(100000, math.ceil(hold_s / max(region_s, 1e-6))))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        replay()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    return reps, a.elapsed_time(b) / 1000.0, time.time()
+
+
+def clock_record(sampler, wall0, wall1, window, flops_per_region, value):
+    """The clock block of the JSON line: samples over the timed region and the window after it."""
+    if sampler is None:
+        return None
+    if window is None:
+        return sampler.summary(wall0, wall1)
+    reps, secs, wall2 = window
+    rec = sampler.summary(wall0, wall2)
+    rec["timed_region_samples"] = sum(1 for (t, _) in sampler.samples if wall0 <= t <= wall1)
+    rec["window"] = {"seconds": secs, "replays_of_timed_region": reps,
+                     "value": flops_per_region * reps / secs / 1e12, "unit": "TFLOP/s",
+                     "what": "the timed region's launches replayed back to back right after it; "
+                             "sm_mhz is the median over the timed region and this window"}
+    if rec.get("sm_mhz"):
+        rec["value_per_ghz"] = value / (rec["sm_mhz"] / 1000.0)
+        rec["window"]["value_per_ghz"] = rec["window"]["value"] / (rec["sm_mhz"] / 1000.0)
+    return rec
 
 
 def workload_from_args(args):
@@ -380,11 +421,16 @@ def mlp_arm(args):
     end.record(stream)
     torch.cuda.synchronize(dev)
     wall1 = time.time()
+    region_ms = start.elapsed_time(end)
+    window = (hold_clock_window(graph.replay, region_ms / 1000.0, args.clock_window, stream, dev)
+              if args.clock_window > 0 else None)
     replicas.barrier()
     mp.check(stream)
     del graph
-    elapsed_ms = replicas.max_over_ranks(start.elapsed_time(end), device=dev)
-    clocks = sampler.summary(wall0, wall1) if sampler else None
+    elapsed_ms = replicas.max_over_ranks(region_ms, device=dev)
+    flops = 4.0 * m * dm * dff
+    value = flops * world * K / (elapsed_ms / 1000.0) / 1e12
+    clocks = clock_record(sampler, wall0, wall1, window, flops * K, value / world)
     # the library's own unfused sequence: bare GEMM, bias + activation kernel, (e4m3) amax and
     # quantise passes over a bf16 H, bare GEMM, bias kernel
     unfused = None
@@ -408,10 +454,13 @@ def mlp_arm(args):
         u1.record(stream)
         torch.cuda.synchronize(dev)
         uw1 = time.time()
+        u_region_ms = u0.elapsed_time(u1)
+        uwin = (hold_clock_window(ugraph.replay, u_region_ms / 1000.0, args.clock_window, stream, dev)
+                if args.clock_window > 0 else None)
         mp.check(stream)
         del ugraph
-        ums = replicas.max_over_ranks(u0.elapsed_time(u1), device=dev) / Ku
-        uclk = sampler.summary(uw0, uw1) if sampler else None
+        ums = replicas.max_over_ranks(u_region_ms, device=dev) / Ku
+        uclk = clock_record(sampler, uw0, uw1, uwin, flops * Ku, flops / (ums / 1000) / 1e12)
         unfused = {"ms_per_step": ums, "value": 4.0 * m * dm * dff * world / (ums / 1000) / 1e12,
                    "unit": "TFLOP/s", "steps": Ku, "launches_per_step": 6 if dt == "e4m3" else 4,
                    "fused_speedup": ums / (elapsed_ms / K), "clocks": uclk}
@@ -420,8 +469,6 @@ def mlp_arm(args):
             unfused["fused_speedup_equal_clock"] = (ums * u_mhz) / ((elapsed_ms / K) * f_mhz)
     if sampler:
         sampler.stop()
-    flops = 4.0 * m * dm * dff
-    value = flops * world * K / (elapsed_ms / 1000.0) / 1e12
     peaks, peak_src = load_peaks()
     peak = peaks["bf16_tflops"] * (FP8_OVER_BF16 if dt == "e4m3" else 1.0)
     achieved = flops / (elapsed_ms / K / 1000.0) / 1e12
@@ -440,8 +487,7 @@ def mlp_arm(args):
                        "launch": "CUDA graph of the K steps (two kernel launches each)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": None,
-                         "peak_source": peak_src + (", bf16 burst x nominal fp8/bf16 ratio 2" if dt == "e4m3"
-                                                    else ", bf16 burst"),
+                         "peak_source": peak_src + (FP8_PEAK_NOTE if dt == "e4m3" else ", bf16 burst"),
                          "note": "per-step time of both GEMM launches"},
             "cpu_baseline": None, "e2e": None, "unfused": unfused, "gpu_launches": 2 * K, "clocks": clocks,
         }
@@ -562,9 +608,11 @@ def main(argv=None):
         end.record(stream)
         torch.cuda.synchronize(dev)
         wall1 = time.time()
+        elapsed_ms = start.elapsed_time(end)
+        window = (hold_clock_window(graph.replay, elapsed_ms / 1000.0, args.clock_window, stream, dev)
+                  if args.clock_window > 0 else None)
         replicas.barrier()
         plan.check(stream)
-        elapsed_ms = start.elapsed_time(end)
         # launches replay back to back: the average launch lasts the region over K
         avg_launch_s = elapsed_ms / K / 1000.0
         del graph
@@ -581,15 +629,21 @@ def main(argv=None):
         end.record(stream)
         torch.cuda.synchronize(dev)
         wall1 = time.time()
+        elapsed_ms = start.elapsed_time(end)
+
+        def direct_steps():
+            for i in range(K):
+                run(*sets[i % n_sets], stream=stream)
+        window = (hold_clock_window(direct_steps, elapsed_ms / 1000.0, args.clock_window, stream, dev)
+                  if args.clock_window > 0 else None)
         replicas.barrier()
         plan.check(stream)
-        elapsed_ms = start.elapsed_time(end)
         avg_launch_s = statistics.fmean(a.elapsed_time(b) for a, b in ev) / 1000.0
     elapsed_ms_max = replicas.max_over_ranks(elapsed_ms, device=dev)
-    clocks = sampler.summary(wall0, wall1) if sampler else None
 
     value = flops * world * K / (elapsed_ms_max / 1000.0) / 1e12
     ms_per_step = elapsed_ms_max / K
+    clocks = clock_record(sampler, wall0, wall1, window, flops * K, value / world)
 
     # ---- roofline of the dominant (only) kernel: one launch per step
     peaks, peak_src = load_peaks()
@@ -606,8 +660,7 @@ def main(argv=None):
         achieved = flops / avg_launch_s / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": in_bytes + out_bytes,
-                "peak_source": peak_src + (", bf16 burst x nominal fp8/bf16 ratio 2"
-                                           if wl.dtype == "e4m3" else ", bf16 burst")}
+                "peak_source": peak_src + (FP8_PEAK_NOTE if wl.dtype == "e4m3" else ", bf16 burst")}
     roof["kernel_source"] = khash
     if launches > 1:
         roof["note"] = "per-step time: the GEMM launch plus the dbias reduction launch"
@@ -622,6 +675,9 @@ def main(argv=None):
             run(*sets[i % n_sets], stream=stream, fused=False)
         torch.cuda.synchronize(dev)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        def unfused_steps():
+            for i in range(Ku):
+                run(*sets[i % n_sets], stream=stream, fused=False)
         if use_graph:
             ugraph = capture(False, Ku)
             ugraph.replay()
@@ -633,14 +689,18 @@ def main(argv=None):
         else:
             uw0 = time.time()
             s0.record(stream)
-            for i in range(Ku):
-                run(*sets[i % n_sets], stream=stream, fused=False)
+            unfused_steps()
             s1.record(stream)
         torch.cuda.synchronize(dev)
         uw1 = time.time()
+        u_region_ms = s0.elapsed_time(s1)
+        uwin = (hold_clock_window(ugraph.replay if use_graph else unfused_steps, u_region_ms / 1000.0,
+                                  args.clock_window, stream, dev) if args.clock_window > 0 else None)
+        if use_graph:
+            del ugraph
         plan.check(stream)
-        ums = replicas.max_over_ranks(s0.elapsed_time(s1), device=dev) / Ku
-        uclk = sampler.summary(uw0, uw1) if sampler else None
+        ums = replicas.max_over_ranks(u_region_ms, device=dev) / Ku
+        uclk = clock_record(sampler, uw0, uw1, uwin, flops * Ku, flops / (ums / 1000) / 1e12)
         unfused = {"ms_per_step": ums, "value": flops * world / (ums / 1000) / 1e12, "unit": "TFLOP/s",
                    "steps": Ku, "launches_per_step": launches_unfused, "fused_speedup": ums / ms_per_step,
                    "clocks": uclk}

@@ -144,7 +144,10 @@ typedef struct gemm_epi_options {
     int32_t split_k;   /* SPLITK: CTAs per cluster along k (1..8; 0 = auto).  TC1/TC2:
                           cap on the parts a tail tile is split into (0 = auto: 2 behind
                           whole waves; with fewer tiles than SMs up to 4, at least 8
-                          k-blocks a part)                                             */
+                          128-byte k-atoms a part).  The parts are whole ring stages
+                          (gemm_epi_plan_info.block_k of k each), so a value above the
+                          number of stages k makes, or above the idle units, is lowered
+                          to that number (gemm_epi_plan_info.sk_split reports it)      */
     int32_t max_ctas;  /* persistent kernels: cap on resident CTAs (0 = one per SM)    */
     int32_t inject_stall; /* testing only (TC1/TC2): 1 = the MMA issuer never publishes an
                              accumulator, so the epilogue's bounded wait runs out after about
@@ -293,9 +296,13 @@ int gemm_epi_plan_preview(int64_t m, int64_t n, int64_t k, int dtype, int epilog
  * cannot afford cudaMalloc/cudaFree and their implicit synchronisation.  Such
  * callers cannot create a plan (a plan allocates its status word), so this
  * call takes the problem description and the buffers directly and computes
- * exactly what gemm_epi_plan_ex + gemm_epi_run would (same kernels, same
- * automatic kernel choice, same argument rules and errors).  Forward epilogues
- * only (NONE .. TANH); the backward ones return GEMM_EPI_ERR_ARG.
+ * what gemm_epi_plan_ex + gemm_epi_run would (same kernels, same automatic
+ * kernel choice, same argument rules and errors), except that the split tail
+ * (options.stream_k), which needs a workspace, is off: where a plan would
+ * split its last wave's tiles along k, the sums are taken in another order and
+ * the results agree with gemm_epi_run within the library's tolerance rather
+ * than bit for bit.  Forward epilogues only (NONE .. TANH); the backward ones
+ * return GEMM_EPI_ERR_ARG.
  *
  * Arguments: as gemm_epi_plan_ex and gemm_epi_run; d_scale_a/d_scale_b as in
  * gemm_epi_set_scales (E4M3 only, else ignored).  wait = 0: enqueue and
@@ -311,7 +318,9 @@ int gemm_epi_plan_preview(int64_t m, int64_t n, int64_t k, int dtype, int epilog
  * that overlap on the GPU (other streams, other host threads) race on it: one
  * call's timeout may be reported by another, or lost.  The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress) with that
- * device current; make that first call before any stream capture.  No
+ * device current and keeps it for the life of the process; make that first
+ * call before any stream capture.  A cudaDeviceReset between calls is not
+ * supported (it unloads the module, and the kept address would go stale).  No
  * cudaMalloc, cudaFree or allocating library routine is called. */
 int gemm_epi_run_noalloc(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias_axis,
                          int b_layout, const void *A, const void *B, const void *bias,

@@ -40,3 +40,24 @@ def test_reference_arm_json_line(extra, workload):
     e = d["e2e"]
     assert (e["value"], e["unit"]) == (d["value"], d["unit"])
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_clock_record_covers_the_window_after_a_short_timed_region():
+    """A timed region shorter than the sampler's period: the clock block is read over the timed
+    region plus the back-to-back window that follows it, and says how many samples each holds."""
+    sys.path.insert(0, ROOT)
+    import bench
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    # samples every 50 ms from t = 0 to 1 s: idle (1965 MHz) before t = 0.1, loaded (1400 MHz) after
+    s.samples = [(0.05 * i, ["ts", "0", "1965" if 0.05 * i < 0.1 else "1400", "1965", "900", "0x4",
+                             "Not Active", "Not Active", "Not Active", "Active"]) for i in range(21)]
+    flops = 2.0 * 4096 ** 3
+    rec = bench.clock_record(s, 0.21, 0.212, (300, 0.6, 0.8), flops * 20, 1500.0)
+    assert rec["timed_region_samples"] == 0          # 2 ms between two samples
+    assert rec["samples"] >= 10 and rec["sm_mhz"] == 1400.0 and rec["sm_max_mhz"] == 1965.0
+    assert rec["reasons"] == ["sw_power_cap"]
+    assert abs(rec["value_per_ghz"] - 1500.0 / 1.4) < 1e-9
+    w = rec["window"]
+    assert w["replays_of_timed_region"] == 300 and abs(w["value"] - flops * 20 * 300 / 0.6 / 1e12) < 1e-6
+    # without a window the timed region alone is summarised
+    assert "window" not in bench.clock_record(s, 0.2, 0.5, None, flops, 1500.0)

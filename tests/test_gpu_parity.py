@@ -579,6 +579,28 @@ def test_workload_fp8_gelu_bias():
     _sampled_check(wl, prob, D, words)
 
 
+@pytest.mark.slow
+def test_workload_fp8_gelu_bias_full_oracle():
+    """Every output of the 8192 x 14336 x 4096 e4m3 GELU_BIAS workload against the oracle.
+
+    Rows of D are independent, so the oracle runs on blocks of 1024 rows of A (all of B and
+    the per-column bias each time), which bounds the host memory its fp64 results take."""
+    wl = _named("fp8_gelu_bias_8192x14336x4096")
+    prob = make_problem(wl)
+    D, words, info = gpu_run(wl, prob)
+    assert info["kernel"] == g.KERNEL_TC2
+    sa, sb = sigmas(prob)
+    Bs, bias = storage(prob.B), storage(prob.bias)
+    worst = 0.0
+    for r0 in range(0, wl.m, 1024):
+        r1 = min(wl.m, r0 + 1024)
+        ref, pre, mask = oracle.gemm_epi(storage(prob.A[r0:r1].contiguous()), Bs, bias, dtype=wl.dtype,
+                                         epilogue=wl.epilogue, bias_axis=wl.bias_axis, b_layout=wl.b_layout,
+                                         scale_a=prob.scale_a, scale_b=prob.scale_b)
+        worst = max(worst, compare(wl.with_(m=r1 - r0), D[r0:r1], None, ref, pre, mask, sa, sb))
+    assert worst <= 1.0
+
+
 def test_workload_large_relu_bias_sampled():
     wl = _named("relu_bias_bf16_65536x8192x16384")
     prob = make_problem(wl, device="cuda")

@@ -132,6 +132,17 @@ def test_split_tail_options(g):
     assert p["sk_split"] == 2 and p["grid"] == 64
 
 
+@pytest.mark.parametrize("k,stages", [(192, 2), (320, 3), (448, 4)])
+def test_split_k_capped_at_ring_stages(g, k, stages):
+    # 4 tiles of 128 x 128 (fewer than the SMs); k is an odd number of 128-byte k-atoms, and the
+    # single-CTA 128-wide tile holds two atoms per ring stage, so k makes ceil(atoms / 2) stages.
+    # A split_k above that is lowered to the stage count: a part is whole stages.
+    p = pv(g, 256, 256, k, "bf16", "bias", kernel="tc1", block_n=128, stream_k="on", split_k=8)
+    assert p["block_k"] == 128 and p["tiles"] == 4
+    assert (p["sk_tiles"], p["sk_split"]) == (4, stages)
+    assert p["grid"] == 4 * stages
+
+
 def test_units_follow_the_sm_count(g):
     # a smaller part (or max_ctas) changes the waves, not the rules
     p = pv(g, 4096, 4096, 4096, "bf16", "relu_aux_bias", sms=100)

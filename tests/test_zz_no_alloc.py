@@ -9,9 +9,13 @@ scratch -- the kernels' timeout status word -- in a static device array.
 
 This file checks, through the C ABI, that two calls in a row of that entry
 point give the same results as the plan-based gemm_epi_run on the same inputs,
-within the tolerance the parity tests use.  It is collected last and builds
-everything it needs itself, so it passes alone in a fresh process as well as
-after the rest of the suite.
+within the tolerance the parity tests use, and that each call also matches the
+fp64 oracle element by element.  The mask is compared bit for bit wherever the
+oracle's pre-activation lies outside the tolerance band (inside it, several
+roundings are correct: the no-alloc call runs without the split tail, so its
+sums may be taken in another order than the plan's).  It is collected last and
+builds everything it needs itself, so it passes alone in a fresh process as
+well as after the rest of the suite.
 """
 import ctypes
 
@@ -19,13 +23,13 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
+from helpers import aux_padding_bits, band, tolerance, unpack_aux
+
 from activation_epilogue_tcgen05_b200 import gemm_epi as g
-from activation_epilogue_tcgen05_b200.workloads import TORCH_DTYPE, Workload, make_problem
+from activation_epilogue_tcgen05_b200.workloads import TORCH_DTYPE, Workload, make_problem, storage
 
 pytestmark = pytest.mark.gpu
-
-# the acceptance bound of the parity tests: RTOL*|ref| + ATOL*sqrt(k)*sigma_A*sigma_B
-TOL = {"f16": (4e-3, 2e-3), "bf16": (4e-3, 2e-3), "e4m3": (6e-2, 2e-2)}
 
 CASES = [
     # persistent tensor-core kernel, ragged edges, mask output
@@ -44,6 +48,7 @@ def _device():
         pytest.skip("needs an sm_100 GPU")
     from activation_epilogue_tcgen05_b200 import build
     build.build()
+    oracle.build()
     g.lib()
 
 
@@ -76,22 +81,37 @@ def test_noalloc_matches_plan_run_twice(wl):
             plan.set_scales(sa, sb)
         plan.run(A, B, bias, D_ref, aux_ref, stream=stream)
         plan.check(stream)
-    ref = D_ref.double().cpu()
+    d_plan = D_ref.double().cpu().numpy()
 
+    # the fp64 oracle on the same stored inputs
+    o_ref, o_pre, o_mask = oracle.gemm_epi(storage(p.A), storage(p.B), storage(p.bias), dtype=wl.dtype,
+                                           epilogue=wl.epilogue, bias_axis=wl.bias_axis,
+                                           b_layout=wl.b_layout, scale_a=p.scale_a, scale_b=p.scale_b)
     sigma_a = float(p.A.double().std(unbiased=False)) * p.scale_a
     sigma_b = float(p.B.double().std(unbiased=False)) * p.scale_b
-    rt, at = TOL[wl.dtype]
-    tol = rt * ref.abs() + at * np.sqrt(wl.k) * sigma_a * sigma_b
+    tol_oracle = tolerance(o_ref, wl.dtype, wl.k, sigma_a, sigma_b)
+    tol_plan = tolerance(d_plan, wl.dtype, wl.k, sigma_a, sigma_b)
+    exact = band(o_pre, wl.dtype, wl.k, sigma_a, sigma_b)     # mask bits that must be exact
+    assert bool((np.abs(d_plan - o_ref) <= tol_oracle).all()), "gemm_epi_run disagrees with the oracle"
 
     for call in range(2):                       # two calls in a row share the static scratch
         D, aux = _outputs(wl)
         rc = g.lib().gemm_epi_run_noalloc(wl.m, wl.n, wl.k, *codes, _ptr(A), _ptr(B), _ptr(bias),
                                           _ptr(sa), _ptr(sb), _ptr(D), _ptr(aux), 1, s)
         assert rc == g.OK, f"call {call}: {g.gemm_epi_status_string(rc)}"
-        err = (D.double().cpu() - ref).abs()
-        assert bool((err <= tol).all()), f"call {call}: {int((~(err <= tol)).sum())} outputs differ"
+        d = D.double().cpu().numpy()            # NaN (an unwritten output) fails both checks
+        bad_plan = ~(np.abs(d - d_plan) <= tol_plan)
+        assert not bad_plan.any(), f"call {call}: {int(bad_plan.sum())} outputs differ from gemm_epi_run"
+        bad_oracle = ~(np.abs(d - o_ref) <= tol_oracle)
+        assert not bad_oracle.any(), f"call {call}: {int(bad_oracle.sum())} outputs outside the oracle's tolerance"
         if aux is not None:
-            assert torch.equal(aux.cpu(), aux_ref.cpu()), f"call {call}: mask words differ"
+            words = aux.cpu().numpy().view(np.uint32)
+            words_plan = aux_ref.cpu().numpy().view(np.uint32)
+            bits = unpack_aux(words, wl.m, wl.n)
+            assert not (exact & (bits != o_mask)).any(), f"call {call}: mask bits differ from the oracle"
+            assert not (exact & (bits != unpack_aux(words_plan, wl.m, wl.n))).any(), \
+                f"call {call}: mask bits differ from gemm_epi_run"
+            assert aux_padding_bits(words, wl.m, wl.n) == 0, f"call {call}: mask padding bits set"
 
 
 def test_noalloc_rejects_bad_requests():
