@@ -287,7 +287,7 @@ int choose(Plan *P) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Timeline buffer of a tracing build (GEMM_EPI_TRACE=1); NULL in a normal build.
+// Timeline buffer of a tracing build (GEMM_EPI_TRACE=1 or 2); NULL in a normal build.
 unsigned long long *trace_buffer() {
 #if GEMM_EPI_TRACE
     static unsigned long long *buf = nullptr;
@@ -299,6 +299,16 @@ unsigned long long *trace_buffer() {
 #else
     return nullptr;
 #endif
+}
+// The trace pointer a launch is given: the whole buffer (level 1), or the next of its
+// per-launch slots (level 2).
+unsigned long long *trace_for_launch() {
+    unsigned long long *buf = trace_buffer();
+#if GEMM_EPI_TRACE == 2
+    static unsigned int next = 0;
+    if (buf) buf += 2 + 2 * (size_t)TRACE_LAUNCH_RECS * (next++ % (TRACE_CAP / TRACE_LAUNCH_RECS));
+#endif
+    return buf;
 }
 
 // A plan's status word and workspaces live on the device it was created on: its runs must be
@@ -397,6 +407,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.dq = P->qout ? static_cast<uint8_t *>(D) : nullptr;
         L.p.out_scale = P->out_scale;
         L.p.amax = reinterpret_cast<unsigned int *>(P->amax);
+        L.p.trace = trace_for_launch();
         L.grid = P->grid;
         L.cluster = P->split;
         L.pdl = P->pdl;
@@ -427,7 +438,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.sk_split = P->sk_split;
         L.p.workspace = P->workspace;
         L.p.flags = P->flags;
-        L.p.trace = trace_buffer();
+        L.p.trace = trace_for_launch();
         L.p.dbias_ws = fused ? dbias_ws : nullptr;
         L.p.dq = P->qout ? static_cast<uint8_t *>(D) : nullptr;
         L.p.out_scale = P->out_scale;
@@ -1106,6 +1117,6 @@ extern "C" int gemm_epi_trace_read(void *host, size_t bytes) {
     if (cudaDeviceSynchronize() != cudaSuccess) return GEMM_EPI_ERR_CUDA;
     const size_t cap = (2 + 2 * (size_t)TRACE_CAP) * sizeof(unsigned long long);
     if (cudaMemcpy(host, buf, bytes < cap ? bytes : cap, cudaMemcpyDeviceToHost) != cudaSuccess) return GEMM_EPI_ERR_CUDA;
-    return cudaMemset(buf, 0, sizeof(unsigned long long)) == cudaSuccess ? GEMM_EPI_OK : GEMM_EPI_ERR_CUDA;
+    return cudaMemset(buf, 0, cap) == cudaSuccess ? GEMM_EPI_OK : GEMM_EPI_ERR_CUDA;
 }
 #endif

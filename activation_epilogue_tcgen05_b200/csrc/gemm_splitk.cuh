@@ -45,6 +45,7 @@ struct SkParams {
     uint8_t *dq;
     const float *out_scale;
     unsigned int *amax;
+    unsigned long long *trace;   // timeline records; used only by builds with GEMM_EPI_TRACE=2
 };
 
 template <int DT_, int EPI_, int AXIS_, bool W_MN_, int NM_, int STAGES_, bool QOUT_ = false>
@@ -111,7 +112,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int kb_end = min(p.num_kb, kb_begin + p.kb_per_cta);
     const int my_kb = kb_end > kb_begin ? kb_end - kb_begin : 0;
 
+    uint32_t tr_i = 0;
     if (warp == 0 && lane == 0) {
+        trace_stage(p.trace, 0, tr_i, 10, tile_n, (int)rank);
         ptx::prefetch_tmap(&tmW);
         ptx::prefetch_tmap(&tmX);
         for (int s = 0; s < C::STAGES; ++s) {
@@ -150,6 +153,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
+            trace_stage(p.trace, 0, tr_i, 11, tile_n, (int)rank);
             uint32_t stage = 0, phase = 0, issued = 0;
             bool ok = true;
             for (int kb = kb_begin; kb < kb_end; ++kb) {
@@ -157,6 +161,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     ok = false;
                     break;
                 }
+                trace_stage(p.trace, 0, tr_i, 20, tile_n, kb);
                 const uint32_t fb = full_bar(stage);
                 ptx::mbar_arrive_expect_tx(fb, C::W_BYTES + C::X_BYTES);
                 const int k0 = kb * C::BK;
@@ -189,6 +194,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     ok = false;
                     break;
                 }
+                trace_stage(p.trace, 1, tr_i, 22, tile_n, kb_begin + i);
                 ptx::tc_fence_after();
                 const uint32_t w_base = sW + stage * C::W_BYTES;
                 const uint32_t x_base = sX + stage * C::X_BYTES;
@@ -203,6 +209,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 if (++stage == (uint32_t)C::STAGES) { stage = 0; phase ^= 1u; }
             }
             if (ok) ptx::mma_commit(tfull);
+            trace_stage(p.trace, 1, tr_i, 23, tile_n, kb_end);
             ptx::mma_commit(done_bar);
             wait_drain(done_bar, 0, p.status);
         }
@@ -216,6 +223,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     bool have = false;
     if (epi) {
         if (my_kb > 0 && wait_bounded<false>(tfull, 0, abort_flag, p.status, ST_TIMEOUT_SPLITK)) {
+            if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 26, tile_n, (int)rank);
             ptx::tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16);
 #pragma unroll
@@ -245,6 +253,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncwarp();
     ptx::tc_fence_before();
     ptx::cluster_sync();     // partials visible in the leader's shared memory
+    if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 28, tile_n, (int)rank);
 
     if (epi && rank == 0) {
         using O = OutT<C::DT>;
@@ -311,12 +320,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
     }
 
+    if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 27, tile_n, (int)rank);
     __syncwarp();
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc<1>(tmem_base, C::TMEM_COLS);
+        if (lane == 0) trace_stage(p.trace, 3, tr_i, 29, tile_n, (int)rank);
     }
 }
 

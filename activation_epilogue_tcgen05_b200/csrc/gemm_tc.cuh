@@ -107,17 +107,41 @@ struct TcParams {
     unsigned int *amax;
 };
 
-// Timeline tracing (off unless the library is compiled with -DGEMM_EPI_TRACE=1):
-// each record is two 64-bit words, %globaltimer and (cta << 40 | warp << 32 |
+// Timeline tracing (off unless the library is compiled with -DGEMM_EPI_TRACE=1 or 2).
+// Level 1: each record is two 64-bit words, %globaltimer and (cta << 40 | warp << 32 |
 // event << 24 | tile << 8 | k-block), appended at trace[2 + 2*i] with i from an
 // atomic counter in trace[0].
+// Level 2 (per ring stage, no atomics): each launch gets its own slot of TRACE_LAUNCH_RECS
+// records (the host rotates over TRACE_CAP / TRACE_LAUNCH_RECS slots and passes the slot's
+// base); in it every (CTA, role) owns TRACE_ROLE_CAP records at
+// base[2 * ((cta * 4 + role) * TRACE_ROLE_CAP + i)], i counted by the caller; a record is
+// %globaltimer and (clock low 32 bits << 32 | event << 24 | tile & 0xFF << 16 | kb & 0xFFFF).
+// The SM clock orders one CTA's roles exactly; %globaltimer relates CTAs.
 #ifndef GEMM_EPI_TRACE
 #define GEMM_EPI_TRACE 0
 #endif
-constexpr unsigned int TRACE_CAP = 1u << 21;
+constexpr unsigned int TRACE_CAP = 1u << 22;
+constexpr unsigned int TRACE_ROLE_CAP = 256;
+constexpr unsigned int TRACE_LAUNCH_RECS = 256u * 4u * TRACE_ROLE_CAP;   // up to 256 CTAs a launch
+__device__ __forceinline__ void trace_stage(unsigned long long *trace, int role, uint32_t &i, unsigned int ev,
+                                            int tile, int kb) {
+    if constexpr (GEMM_EPI_TRACE == 2) {
+        if (trace == nullptr || i >= TRACE_ROLE_CAP || (blockIdx.x * 4u + role + 1u) * TRACE_ROLE_CAP > TRACE_LAUNCH_RECS)
+            return;
+        unsigned long long *r = trace + 2 * ((size_t)(blockIdx.x * 4u + role) * TRACE_ROLE_CAP + i);
+        uint32_t clk;
+        asm volatile("mov.u32 %0, %%clock;" : "=r"(clk));
+        r[0] = ptx::globaltimer();
+        r[1] = ((unsigned long long)clk << 32) | ((unsigned long long)(ev & 0xFFu) << 24) |
+               ((unsigned long long)(tile & 0xFF) << 16) | (unsigned long long)(kb & 0xFFFF);
+        ++i;
+    } else {
+        (void)trace; (void)role; (void)i; (void)ev; (void)tile; (void)kb;
+    }
+}
 __device__ __forceinline__ void trace_event(unsigned long long *trace, int warp, unsigned int ev, int tile,
                                             int kb) {
-    if constexpr (GEMM_EPI_TRACE != 0) {
+    if constexpr (GEMM_EPI_TRACE == 1) {
         if (trace == nullptr) return;
         const unsigned long long i = atomicAdd(trace, 1ull);
         if (i < TRACE_CAP) {
@@ -477,8 +501,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             uint32_t stage = 0, phase = 0;
-            uint32_t issued = 0;
+            uint32_t issued = 0, tr_i = 0;
             bool ok = true;
+            trace_stage(p.trace, 0, tr_i, 10, 0, 0);
             WorkIter it(p, unit, units);
             WorkItem w;
             while (ok && it.next(p, units, w)) {
@@ -495,6 +520,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         ok = false;
                         break;
                     }
+                    trace_stage(p.trace, 0, tr_i, 20, w.tile, kb);
                     uint32_t fb = full_bar(stage);
                     if constexpr (C::CG == 2) {
                         fb = ptx::mapa(fb, 0);      // the pair's leader counts both CTAs' bytes
@@ -546,13 +572,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && leader) {
             constexpr uint32_t idesc = make_idesc(C::FMT, C::A_MN, C::B_MN, 128 * C::CG, C::MMA_N);
-            uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+            uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0, tr_i = 0;
             bool ok = true;
             // with inject_stall nothing is issued or committed: the epilogue's
             // bounded wait for the first accumulator runs out (failure-path test)
             WorkIter it(p, unit, units);
             WorkItem w;
             while (ok && !p.inject_stall && it.next(p, units, w)) {
+                trace_stage(p.trace, 1, tr_i, 24, w.tile, w.kb0);
                 if (!wait_bounded<C::CG == 2>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status,
                                               ST_TIMEOUT_MMA)) {
                     ok = false;
@@ -560,12 +587,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
                 ptx::tc_fence_after();
                 trace_event(p.trace, warp, 3, w.tile, w.kb0);
+                trace_stage(p.trace, 1, tr_i, 25, w.tile, w.kb0);
                 const uint32_t d_tmem = tmem_base + acc * C::BN;
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!wait_bounded<false>(full_bar(stage), phase, abort_flag, p.status, ST_TIMEOUT_MMA)) {
                         ok = false;
                         break;
                     }
+                    trace_stage(p.trace, 1, tr_i, 22, w.tile, kb);
                     ptx::tc_fence_after();
 #pragma unroll
                     for (int at = 0; at < C::KATOMS; ++at) {
@@ -614,7 +643,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const bool bgrad = C::BWD && p.dbias_ws != nullptr;   // backward: bias-gradient partials
         float inv_out = 1.0f, amax_l = 0.0f;                  // FP8 output: 1 / scale, running max |y|
         if constexpr (C::QOUT) inv_out = 1.0f / __ldg(p.out_scale);
-        uint32_t acc = 0, acc_phase = 0;
+        uint32_t acc = 0, acc_phase = 0, tr_i = 0;
         bool ok = true;
         WorkIter it(p, unit, units);
         WorkItem w;
@@ -672,6 +701,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             }
             ptx::tc_fence_after();
             if (lane == 0) trace_event(p.trace, warp, 6, w.tile, w.kb0);
+            if (lane == 0 && ew == 0) trace_stage(p.trace, 2, tr_i, 26, w.tile, w.kb0);
             // this warp's rows of each earlier slice are published by the same warp quadrant
             for (int v = c_first; ok && v < unit && !partial_out; ++v)
                 ok = wait_flag(p.flags + ((size_t)v * C::CG + rank) * 4 + q, abort_flag, p.status);
@@ -842,6 +872,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 for (int v = c_first; v < unit; ++v) p.flags[((size_t)v * C::CG + rank) * 4 + q] = 0u;
             }
             if (lane == 0) trace_event(p.trace, warp, 9, w.tile, 0);
+            if (lane == 0 && ew == 0) trace_stage(p.trace, 2, tr_i, 27, w.tile, w.kb1);
             if (++acc == (uint32_t)C::NUM_ACC) { acc = 0; acc_phase ^= 1u; }
         }
         if (lane == 0) ptx::bulk_wait<0>();
