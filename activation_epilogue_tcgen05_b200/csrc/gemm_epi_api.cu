@@ -47,6 +47,7 @@ struct Plan {
     int katoms = 1;      // TC: 128-byte k-atoms per ring stage (the kernel's KATOMS)
     int grid;
     int group_m;
+    int l2_mode = 1;     // TcParams::l2_mode (GEMM_EPI_L2=0/1/2 overrides)
     bool pdl;            // programmatic dependent launch (GEMM_EPI_PDL=0 turns it off)
     // split tail (TC kernels): tiles [0, sk_tiles) cut along k into sk_split parts
     int sk_tiles = 0, sk_split = 0;
@@ -272,6 +273,11 @@ int choose(Plan *P) {
             const int v = atoi(g);
             if (v >= 1 && v <= 64) P->group_m = v;
         }
+        P->l2_mode = 1;
+        if (const char *g = getenv("GEMM_EPI_L2")) {        // tuning knob: L2 cache policy (TcParams)
+            const int v = atoi(g);
+            if (v >= 0 && v <= 2) P->l2_mode = v;
+        }
         KernelInfo none_info;
         if (!find_tc(cg, P->dtype, GEMM_EPI_NONE, 0, b_mn, bn, false, P->a_km, &P->tc_none_launch, &none_info))
             return GEMM_EPI_ERR_UNSUPPORTED;
@@ -443,6 +449,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.dq = P->qout ? static_cast<uint8_t *>(D) : nullptr;
         L.p.out_scale = P->out_scale;
         L.p.amax = reinterpret_cast<unsigned int *>(P->amax);
+        L.p.l2_mode = P->l2_mode;
         L.grid = P->grid;
         L.pdl = P->pdl;
         L.stream = stream;

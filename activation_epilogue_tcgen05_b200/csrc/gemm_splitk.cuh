@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             trace_stage(p.trace, 0, tr_i, 11, tile_n, (int)rank);
             uint32_t stage = 0, phase = 0, issued = 0;
             bool ok = true;
+            const uint64_t pol = ptx::policy_evict_normal();
             for (int kb = kb_begin; kb < kb_end; ++kb) {
                 if (!wait_bounded<false>(empty_bar(stage), phase ^ 1u, abort_flag, p.status, ST_TIMEOUT_SPLITK)) {
                     ok = false;
@@ -170,11 +171,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
                     for (int b = 0; b < C::W_BOXES; ++b)
                         ptx::tma_load_2d(w_dst + b * C::W_BOX_BYTES, &tmW, fb, n0 + b * C::W_BOX_N, k0,
-                                         0x1000000000000000ull);
+                                         pol);
                 } else {
-                    ptx::tma_load_2d(w_dst, &tmW, fb, k0, n0, 0x1000000000000000ull);
+                    ptx::tma_load_2d(w_dst, &tmW, fb, k0, n0, pol);
                 }
-                ptx::tma_load_2d(sX + stage * C::X_BYTES, &tmX, fb, k0, 0, 0x1000000000000000ull);
+                ptx::tma_load_2d(sX + stage * C::X_BYTES, &tmX, fb, k0, 0, pol);
                 ++issued;
                 if (++stage == (uint32_t)C::STAGES) { stage = 0; phase ^= 1u; }
             }

@@ -105,6 +105,10 @@ struct TcParams {
     uint8_t *dq;
     const float *out_scale;
     unsigned int *amax;
+    // L2 cache policy: 0 = normal for every access; 1 = the outputs (D, mask) are written
+    // evict-first, so that streaming them out does not push the operands out of L2; 2 = as 1,
+    // and the operands are loaded evict-last
+    int l2_mode;
 };
 
 // Timeline tracing (off unless the library is compiled with -DGEMM_EPI_TRACE=1 or 2).
@@ -503,6 +507,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             uint32_t stage = 0, phase = 0;
             uint32_t issued = 0, tr_i = 0;
             bool ok = true;
+            const uint64_t pol_ab = p.l2_mode == 2 ? ptx::policy_evict_last() : ptx::policy_evict_normal();
             trace_stage(p.trace, 0, tr_i, 10, 0, 0);
             WorkIter it(p, unit, units);
             WorkItem w;
@@ -534,9 +539,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const uint32_t b_dst = sB + stage * C::B_STAGE + at * C::B_BYTES;
                     auto load = [&](uint32_t dst, const CUtensorMap *map, int c0, int c1) {
                         if constexpr (C::CG == 2)
-                            ptx::tma_load_2d_pair(dst, map, fb, c0, c1, 0x1000000000000000ull);
+                            ptx::tma_load_2d_pair(dst, map, fb, c0, c1, pol_ab);
                         else
-                            ptx::tma_load_2d(dst, map, fb, c0, c1, 0x1000000000000000ull);
+                            ptx::tma_load_2d(dst, map, fb, c0, c1, pol_ab);
                     };
                     if constexpr (C::A_MN) {
 #pragma unroll
@@ -642,6 +647,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const bool has_bias = p.bias != nullptr;
         const bool bgrad = C::BWD && p.dbias_ws != nullptr;   // backward: bias-gradient partials
         float inv_out = 1.0f, amax_l = 0.0f;                  // FP8 output: 1 / scale, running max |y|
+        const uint64_t pol_d = p.l2_mode >= 1 ? ptx::policy_evict_first() : ptx::policy_evict_normal();
         if constexpr (C::QOUT) inv_out = 1.0f / __ldg(p.out_scale);
         uint32_t acc = 0, acc_phase = 0, tr_i = 0;
         bool ok = true;
@@ -822,7 +828,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         __syncwarp();
                         // boxes starting past the last row or column hold nothing to store
                         if (lane == 0 && m0 + 32 * q < p.m && col0 < p.n) {
-                            ptx::tma_store_2d(&tmD, stg, col0, m0 + 32 * q);
+                            ptx::tma_store_2d_hint(&tmD, stg, col0, m0 + 32 * q, pol_d);
                             ptx::bulk_commit();
                         }
                     }
@@ -853,7 +859,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     if (row_ok && wcol < p.aux_pitch_words * 32) {      // padding words too (zero bits)
                         uint32_t *dst = p.aux + (int64_t)row * p.aux_pitch_words + wcol / 32;
                         if constexpr (C::CPG == 4)
-                            *reinterpret_cast<uint4 *>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
+                            ptx::st_global_v4_hint(dst, make_uint4(words[0], words[1], words[2], words[3]), pol_d);
                         else
                             *reinterpret_cast<uint2 *>(dst) = make_uint2(words[0], words[1]);
                     }
