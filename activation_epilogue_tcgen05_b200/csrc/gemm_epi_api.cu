@@ -42,7 +42,9 @@ struct Plan {
     int kernel;          // GEMM_EPI_KERNEL_TC1 / TC2 / SPLITK
     int block_n;         // TC: tile width; SPLITK: 128
     int nm;              // SPLITK: MMA N (batch rows rounded up)
-    int split;           // SPLITK: cluster size along k
+    int split;           // SPLITK: cluster size along k (cluster form); k-parts per tile, rounded up (grid form)
+    bool sk_grid = false;      // SPLITK: the grid-wide form (workspace reduction) rather than clusters
+    bool no_workspace = false; // the plan may not own device memory beyond its status word (no-alloc runs)
     int kb_per_cta;
     int katoms = 1;      // TC: 128-byte k-atoms per ring stage (the kernel's KATOMS)
     int grid;
@@ -59,6 +61,7 @@ struct Plan {
     int64_t dbias_parts = 0, dbias_len = 0;
     TcLauncher tc_launch = nullptr, tc_none_launch = nullptr;
     SkLauncher sk_launch = nullptr, sk_none_launch = nullptr;
+    SgLauncher sg_launch = nullptr, sg_none_launch = nullptr;
     BiasActLauncher ba_launch = nullptr;
     KernelInfo info{};
     // FP8 scales (device pointers, borrowed)
@@ -160,6 +163,11 @@ int round_nm(int64_t m) {
     return 128;
 }
 
+bool getenv_flag(const char *name) {
+    const char *e = getenv(name);
+    return e && e[0] == '1';
+}
+
 int choose(Plan *P) {
     const int64_t m = P->m, n = P->n;
     // The GEMM kernels do only on-chip setup before waiting on the previous grid, so they are
@@ -190,7 +198,26 @@ int choose(Plan *P) {
     const int64_t num_kb = (P->k + bk - 1) / bk;
     const int sms = P->opts.max_ctas > 0 ? std::min(P->opts.max_ctas, P->num_sms) : P->num_sms;
 
-    if (kernel == GEMM_EPI_KERNEL_SPLITK) {
+    if (kernel == GEMM_EPI_KERNEL_SPLITK && !P->no_workspace && !getenv_flag("GEMM_EPI_SK_CLUSTER")) {
+        // grid-wide form: every SM takes an equal share of the (tile, k-block) units; split
+        // tiles are reduced through a plan-owned workspace by the last of their pieces
+        P->sk_grid = true;
+        P->nm = round_nm(m);
+        P->block_n = 128;
+        const int64_t tiles_n = (n + 127) / 128;
+        const int64_t units = tiles_n * num_kb;
+        int64_t g = sms;
+        if (P->opts.split_k > 0) g = std::min<int64_t>(g, tiles_n * P->opts.split_k);   // k-parts per tile
+        g = std::max<int64_t>(1, std::min<int64_t>(g, units));
+        P->grid = (int)g;
+        P->split = (int)((g + tiles_n - 1) / tiles_n);
+        P->kb_per_cta = (int)((units + g - 1) / g);
+        KernelInfo none_info;
+        if (!find_sg(P->dtype, GEMM_EPI_NONE, 0, b_mn, P->nm, false, &P->sg_none_launch, &none_info))
+            return GEMM_EPI_ERR_UNSUPPORTED;
+        if (!find_sg(P->dtype, P->kepi, P->axis, b_mn, P->nm, P->qout, &P->sg_launch, &P->info))
+            return GEMM_EPI_ERR_UNSUPPORTED;
+    } else if (kernel == GEMM_EPI_KERNEL_SPLITK) {
         P->nm = round_nm(m);
         P->block_n = 128;
         const int64_t tiles_n = (n + 127) / 128;
@@ -394,7 +421,33 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
     const int num_kb = (int)((P->k + bk - 1) / bk);
     const int64_t pitch_words = ((P->n + 127) / 128) * 4;
     cudaError_t e;
-    if (P->kernel == GEMM_EPI_KERNEL_SPLITK) {
+    if (P->kernel == GEMM_EPI_KERNEL_SPLITK && P->sk_grid) {
+        SgLaunch L;
+        L.tmW = P->tmA;
+        L.tmX = P->tmB;
+        L.p.m = (int)P->m;
+        L.p.n = (int)P->n;
+        L.p.k = (int)P->k;
+        L.p.num_kb = num_kb;
+        L.p.tiles_n = (int)((P->n + 127) / 128);
+        L.p.grid = P->grid;
+        L.p.bias = bias;
+        L.p.D = D;
+        L.p.aux = aux;
+        L.p.aux_pitch_words = pitch_words;
+        L.p.scale_a = P->scale_a;
+        L.p.scale_b = P->scale_b;
+        L.p.status = P->status;
+        L.p.dq = P->qout ? static_cast<uint8_t *>(D) : nullptr;
+        L.p.out_scale = P->out_scale;
+        L.p.amax = reinterpret_cast<unsigned int *>(P->amax);
+        L.p.workspace = P->workspace;
+        L.p.counters = P->flags;
+        L.p.trace = trace_for_launch();
+        L.pdl = P->pdl;
+        L.stream = stream;
+        e = (fused ? P->sg_launch : P->sg_none_launch)(L);
+    } else if (P->kernel == GEMM_EPI_KERNEL_SPLITK) {
         SkLaunch L;
         L.tmW = P->tmA;
         L.tmX = P->tmB;
@@ -546,11 +599,20 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
         delete P;
         return GEMM_EPI_ERR_CUDA;
     }
-    if (P->sk_tiles > 0) {
-        const int cg = P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
-        const size_t units = (size_t)P->grid / cg;
-        const size_t ws_bytes = units * cg * 128 * (size_t)P->block_n * sizeof(float);
-        const size_t fl_bytes = units * cg * 4 * sizeof(unsigned int);
+    const int64_t sg_tiles = (n + 127) / 128;
+    if (P->sk_tiles > 0 || (P->sk_grid && P->grid != sg_tiles)) {
+        size_t ws_bytes, fl_bytes;
+        if (P->sk_grid) {
+            // per CTA two partial tiles (its first and last piece) of NM x 128 fp32; one
+            // arrival counter per tile and TMEM lane quadrant
+            ws_bytes = (size_t)P->grid * 2 * 128 * (size_t)P->nm * sizeof(float);
+            fl_bytes = (size_t)sg_tiles * 4 * sizeof(unsigned int);
+        } else {
+            const int cg = P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
+            const size_t units = (size_t)P->grid / cg;
+            ws_bytes = units * cg * 128 * (size_t)P->block_n * sizeof(float);
+            fl_bytes = units * cg * 4 * sizeof(unsigned int);
+        }
         P->flags_bytes = fl_bytes;
         if (cudaMalloc(&P->workspace, ws_bytes) != cudaSuccess || cudaMalloc(&P->flags, fl_bytes) != cudaSuccess ||
             cudaMemset(P->flags, 0, fl_bytes) != cudaSuccess) {
@@ -611,6 +673,17 @@ bool find_tc(int cg, int dt, int epi, int axis, bool b_mn, int bn, bool qout, bo
     case DT_F16: return find_tc_f16(cg, epi, axis, b_mn, bn, l, i);
     case DT_BF16: return find_tc_bf16(cg, epi, axis, b_mn, bn, l, i);
     case DT_E4M3: return find_tc_e4m3(cg, epi, axis, b_mn, bn, l, i);
+    }
+    return false;
+}
+bool find_sg(int dt, int epi, int axis, bool w_mn, int nm, bool qout, SgLauncher *l, KernelInfo *i) {
+    KernelInfo tmp;
+    if (!i) i = &tmp;
+    if (qout) return dt == DT_E4M3 && find_sg_e4m3_q(epi, axis, w_mn, nm, l, i);
+    switch (dt) {
+    case DT_F16: return find_sg_f16(epi, axis, w_mn, nm, l, i);
+    case DT_BF16: return find_sg_bf16(epi, axis, w_mn, nm, l, i);
+    case DT_E4M3: return find_sg_e4m3(epi, axis, w_mn, nm, l, i);
     }
     return false;
 }
@@ -775,7 +848,8 @@ void fill_info(const Plan *P, gemm_epi_plan_info *info) {
     info->stages = P->info.stages;
     info->split_k = P->split;
     info->grid = P->grid;
-    info->cluster = P->kernel == GEMM_EPI_KERNEL_SPLITK ? P->split : (P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1);
+    info->cluster = P->kernel == GEMM_EPI_KERNEL_SPLITK ? (P->sk_grid ? 1 : P->split)
+                                                         : (P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1);
     info->threads = P->info.threads;
     info->smem_bytes = P->info.smem_bytes;
     info->sk_tiles = P->sk_tiles;
@@ -1090,6 +1164,7 @@ extern "C" int gemm_epi_run_noalloc(int64_t m, int64_t n, int64_t k, int dtype, 
     P.device = dev;
     P.num_sms = num_sms_of(dev);
     P.opts.stream_k = 1;                        // stream-K would need a workspace: off
+    P.no_workspace = true;                      // small m: the cluster split-K (no workspace)
     int rc = choose(&P);
     if (rc != GEMM_EPI_OK) return rc;
     if (dtype == GEMM_EPI_E4M3 || d_scale_a || d_scale_b) {      // 16-bit: optional alpha

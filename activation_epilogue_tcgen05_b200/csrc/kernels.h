@@ -7,6 +7,7 @@
 #include <cstdint>
 
 #include "gemm_splitk.cuh"
+#include "gemm_splitk_grid.cuh"
 #include "gemm_tc.cuh"
 
 namespace gemm_epi {
@@ -29,6 +30,14 @@ struct SkLaunch {
     cudaStream_t stream;
 };
 
+// One grid-wide split-K launch (no cluster).
+struct SgLaunch {
+    CUtensorMap tmW, tmX;
+    SgParams p;
+    bool pdl;            // launch with programmatic stream serialisation
+    cudaStream_t stream;
+};
+
 struct KernelInfo {
     const void *func;   // the __global__ symbol (for attributes / occupancy queries)
     int threads;
@@ -40,6 +49,7 @@ struct KernelInfo {
 
 using TcLauncher = cudaError_t (*)(const TcLaunch &);
 using SkLauncher = cudaError_t (*)(const SkLaunch &);
+using SgLauncher = cudaError_t (*)(const SgLaunch &);
 using BiasActLauncher = cudaError_t (*)(void *D, const void *bias, uint32_t *aux, int m, int n,
                                         int64_t pitch_words, int grid, cudaStream_t stream);
 
@@ -48,6 +58,7 @@ using BiasActLauncher = cudaError_t (*)(void *D, const void *bias, uint32_t *aux
 bool find_tc(int cg, int dt, int epi, int axis, bool b_mn, int bn, bool qout, bool a_mn, TcLauncher *launch,
              KernelInfo *info);
 bool find_sk(int dt, int epi, int axis, bool w_mn, int nm, bool qout, SkLauncher *launch, KernelInfo *info);
+bool find_sg(int dt, int epi, int axis, bool w_mn, int nm, bool qout, SgLauncher *launch, KernelInfo *info);
 bool find_bias_act(int dt, int epi, int axis, BiasActLauncher *launch);
 
 // Bias-gradient reductions (dbias.cuh); out_dt is the bias type (DT_F16 or DT_BF16).
@@ -77,6 +88,10 @@ bool find_sk_f16(int epi, int axis, bool w_mn, int nm, SkLauncher *, KernelInfo 
 bool find_sk_bf16(int epi, int axis, bool w_mn, int nm, SkLauncher *, KernelInfo *);
 bool find_sk_e4m3(int epi, int axis, bool w_mn, int nm, SkLauncher *, KernelInfo *);
 bool find_sk_e4m3_q(int epi, int axis, bool w_mn, int nm, SkLauncher *, KernelInfo *);
+bool find_sg_f16(int epi, int axis, bool w_mn, int nm, SgLauncher *, KernelInfo *);
+bool find_sg_bf16(int epi, int axis, bool w_mn, int nm, SgLauncher *, KernelInfo *);
+bool find_sg_e4m3(int epi, int axis, bool w_mn, int nm, SgLauncher *, KernelInfo *);
+bool find_sg_e4m3_q(int epi, int axis, bool w_mn, int nm, SgLauncher *, KernelInfo *);
 
 // Ring depth that fills GEMM_EPI_RING_KB (default 192) KB of shared memory with stages.
 #ifndef GEMM_EPI_RING_KB
@@ -179,6 +194,47 @@ KernelInfo sk_info() {
     return k;
 }
 
+template <class C>
+cudaError_t launch_sg(const SgLaunch &L) {
+    auto kern = splitk_grid_kernel<C>;
+    static int attr_done[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = 1;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(L.p.grid, 1, 1);
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1];
+    int na = 0;
+    if (L.pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = na ? attr : nullptr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, kern, L.tmW, L.tmX, L.p);
+}
+
+template <class C>
+KernelInfo sg_info() {
+    KernelInfo k;
+    k.func = reinterpret_cast<const void *>(splitk_grid_kernel<C>);
+    k.threads = C::THREADS;
+    k.smem_bytes = C::SMEM_BYTES;
+    k.stages = C::STAGES;
+    k.block_m = C::NM;
+    k.block_n = 128;
+    k.block_k = C::BK;
+    return k;
+}
+
 // Instantiate and look up every (epilogue, axis, layout, tile) combination of
 // one dtype.  NONE ignores the bias, so it exists for the ROW axis only.
 #define GEMM_EPI_TC_FIND(NAME, DTV)                                                                     \
@@ -256,6 +312,45 @@ KernelInfo sk_info() {
         return wmn ? NAME##_nm<EPI, AXIS, true>(nm, l, i) : NAME##_nm<EPI, AXIS, false>(nm, l, i);      \
     }                                                                                                   \
     bool NAME(int epi, int axis, bool wmn, int nm, SkLauncher *l, KernelInfo *i) {                      \
+        switch (epi) {                                                                                  \
+        case EPI_NONE: return NAME##_mn<EPI_NONE, AXIS_ROW>(wmn, nm, l, i);                             \
+        case EPI_BIAS: return axis ? NAME##_mn<EPI_BIAS, AXIS_COL>(wmn, nm, l, i)                       \
+                                   : NAME##_mn<EPI_BIAS, AXIS_ROW>(wmn, nm, l, i);                      \
+        case EPI_RELU: return axis ? NAME##_mn<EPI_RELU, AXIS_COL>(wmn, nm, l, i)                       \
+                                   : NAME##_mn<EPI_RELU, AXIS_ROW>(wmn, nm, l, i);                      \
+        case EPI_RELU_AUX: return axis ? NAME##_mn<EPI_RELU_AUX, AXIS_COL>(wmn, nm, l, i)               \
+                                       : NAME##_mn<EPI_RELU_AUX, AXIS_ROW>(wmn, nm, l, i);              \
+        case EPI_GELU: return axis ? NAME##_mn<EPI_GELU, AXIS_COL>(wmn, nm, l, i)                       \
+                                   : NAME##_mn<EPI_GELU, AXIS_ROW>(wmn, nm, l, i);                      \
+        case EPI_TANH: return axis ? NAME##_mn<EPI_TANH, AXIS_COL>(wmn, nm, l, i)                       \
+                                   : NAME##_mn<EPI_TANH, AXIS_ROW>(wmn, nm, l, i);                      \
+        }                                                                                               \
+        return false;                                                                                   \
+    }
+
+#define GEMM_EPI_SG_FIND(NAME, DTV)                                                                     \
+    template <int EPI, int AXIS, bool WMN, int NM>                                                      \
+    static bool NAME##_leaf(SgLauncher *l, KernelInfo *i) {                                             \
+        using C = SgCfg<DTV, EPI, AXIS, WMN, NM, sg_stages(NM)>;                                        \
+        *l = &launch_sg<C>;                                                                             \
+        *i = sg_info<C>();                                                                              \
+        return true;                                                                                    \
+    }                                                                                                   \
+    template <int EPI, int AXIS, bool WMN>                                                              \
+    static bool NAME##_nm(int nm, SgLauncher *l, KernelInfo *i) {                                       \
+        switch (nm) {                                                                                   \
+        case 16: return NAME##_leaf<EPI, AXIS, WMN, 16>(l, i);                                          \
+        case 32: return NAME##_leaf<EPI, AXIS, WMN, 32>(l, i);                                          \
+        case 64: return NAME##_leaf<EPI, AXIS, WMN, 64>(l, i);                                          \
+        case 128: return NAME##_leaf<EPI, AXIS, WMN, 128>(l, i);                                        \
+        }                                                                                               \
+        return false;                                                                                   \
+    }                                                                                                   \
+    template <int EPI, int AXIS>                                                                        \
+    static bool NAME##_mn(bool wmn, int nm, SgLauncher *l, KernelInfo *i) {                             \
+        return wmn ? NAME##_nm<EPI, AXIS, true>(nm, l, i) : NAME##_nm<EPI, AXIS, false>(nm, l, i);      \
+    }                                                                                                   \
+    bool NAME(int epi, int axis, bool wmn, int nm, SgLauncher *l, KernelInfo *i) {                      \
         switch (epi) {                                                                                  \
         case EPI_NONE: return NAME##_mn<EPI_NONE, AXIS_ROW>(wmn, nm, l, i);                             \
         case EPI_BIAS: return axis ? NAME##_mn<EPI_BIAS, AXIS_COL>(wmn, nm, l, i)                       \

@@ -275,12 +275,39 @@ def test_splitk_variants(m, dtype, epilogue, axis, layout):
 
 
 @pytest.mark.parametrize("split", [1, 2, 3, 8])
-def test_splitk_cluster_sizes(split):
+def test_splitk_parts_per_tile(split):
+    """The grid-wide split-K form with split_k parts per tile (1 = whole tiles, no reduction)."""
     wl = Workload("sk_split", 16, 512, 2048, "f16", "gelu_bias", "col", "nk", seed=6,
                   dist_b=("uniform", 1 / 64), dist_bias=("uniform", 1 / 64))
     prob = make_problem(wl)
     worst, info = check_against_oracle(wl, prob, kernel="splitk", split_k=split)
-    assert info["split_k"] == split
+    assert info["split_k"] == split and info["grid"] == 4 * split and info["cluster"] == 1
+    assert worst <= 1.0
+
+
+@pytest.mark.parametrize("ctas", [1, 3, 5, 7, 37, 100])
+@pytest.mark.parametrize("epilogue", ["relu_aux_bias", "gelu_bias"])
+def test_splitk_uneven_ranges(ctas, epilogue):
+    """Ranges of units that cut tiles at arbitrary k-blocks, and (few CTAs) ranges that span
+    several whole and partial tiles: every piece's partial must be added exactly once."""
+    wl = Workload("sk_ranges", 24, 656, 1000, "bf16", epilogue, "col", "kn", seed=16)
+    prob = make_problem(wl)
+    worst, info = check_against_oracle(wl, prob, kernel="splitk", max_ctas=ctas)
+    assert info["grid"] == min(ctas, 6 * 16)          # 6 tiles x 16 k-blocks of units
+    assert worst <= 1.0
+
+
+@pytest.mark.parametrize("split", [1, 2, 3, 8])
+def test_splitk_cluster_form(split, monkeypatch):
+    """The cluster form (partials reduced through distributed shared memory, no workspace):
+    what the allocation-free entry point runs for small m; GEMM_EPI_SK_CLUSTER=1 selects it
+    for a plan."""
+    monkeypatch.setenv("GEMM_EPI_SK_CLUSTER", "1")
+    wl = Workload("sk_cluster", 16, 512, 2048, "f16", "gelu_bias", "col", "nk", seed=6,
+                  dist_b=("uniform", 1 / 64), dist_bias=("uniform", 1 / 64))
+    prob = make_problem(wl)
+    worst, info = check_against_oracle(wl, prob, kernel="splitk", split_k=split)
+    assert info["split_k"] == split and info["cluster"] == split
     assert worst <= 1.0
 
 

@@ -37,8 +37,22 @@ def test_small_gemm_bias_1024x512x2048(g):
 
 def test_linear_gelu_batch16_splitk(g):
     p = pv(g, 16, 4096, 4096, "f16", "gelu_bias", "col", "nk")
-    # swapped roles: 32 weight tiles of 128 rows, K split over clusters of 4 CTAs
-    assert (p["kernel"], p["block_m"], p["split_k"], p["cluster"], p["grid"]) == (g.KERNEL_SPLITK, 16, 4, 4, 128)
+    # swapped roles: 32 weight tiles of 128 rows x 64 k-blocks; every SM takes an equal range
+    # of the 2048 (tile, k-block) units (13 or 14), so a tile is cut into 5 or 6 pieces
+    assert (p["kernel"], p["block_m"], p["cluster"], p["grid"]) == (g.KERNEL_SPLITK, 16, 1, 148)
+    assert p["split_k"] == 5 and p["stages"] == 11
+
+
+def test_splitk_grid_follows_split_k_and_max_ctas(g):
+    # split_k caps the k-parts per tile: the grid is tiles x split_k
+    p = pv(g, 16, 4096, 4096, "f16", "gelu_bias", "col", "nk", split_k=2)
+    assert (p["grid"], p["split_k"]) == (64, 2)
+    # one part per tile: whole tiles, no reduction
+    assert pv(g, 16, 4096, 4096, "f16", "gelu_bias", "col", "nk", split_k=1)["grid"] == 32
+    # fewer units than SMs: one CTA per (tile, k-block) unit
+    q = pv(g, 8, 256, 256, "bf16", "bias", "col", "kn")
+    assert q["kernel"] == g.KERNEL_SPLITK and q["grid"] == 2 * 4
+    assert pv(g, 16, 4096, 4096, "f16", "bias", "col", "nk", max_ctas=100)["grid"] == 100
 
 
 def test_large_relu_bias_wide_tiles(g):
