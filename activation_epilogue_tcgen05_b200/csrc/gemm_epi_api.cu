@@ -48,7 +48,7 @@ struct Plan {
     int kb_per_cta;
     int katoms = 1;      // TC: 128-byte k-atoms per ring stage (the kernel's KATOMS)
     int grid;
-    int group_m;
+    int group_m, group_n = 0;   // TC raster (TcParams::group_m / group_n)
     int l2_mode = 1;     // TcParams::l2_mode (GEMM_EPI_L2=0/1/2 overrides)
     bool pdl;            // programmatic dependent launch (GEMM_EPI_PDL=0 turns it off)
     // split tail (TC kernels): tiles [0, sk_tiles) cut along k into sk_split parts
@@ -199,8 +199,9 @@ int choose(Plan *P) {
     const int sms = P->opts.max_ctas > 0 ? std::min(P->opts.max_ctas, P->num_sms) : P->num_sms;
 
     if (kernel == GEMM_EPI_KERNEL_SPLITK && !P->no_workspace && !getenv_flag("GEMM_EPI_SK_CLUSTER")) {
-        // grid-wide form: every SM takes an equal share of the (tile, k-block) units; split
-        // tiles are reduced through a plan-owned workspace by the last of their pieces
+        // grid-wide form: every SM takes an equal share of the (tile, k-block) units; a split
+        // tile is finished by the CTA holding its first k-block, from partials the others
+        // publish in a plan-owned workspace
         P->sk_grid = true;
         P->nm = round_nm(m);
         P->block_n = 128;
@@ -295,10 +296,28 @@ int choose(Plan *P) {
             const int64_t units = std::min<int64_t>(tiles, units_max);
             P->grid = (int)(units * cg);
         }
-        P->group_m = 8;
+        // Raster from the L2 capacity.  If all of A's panels (or all of B's) fit in a budget
+        // of about 40 % of the 126 MB L2, the whole matrix is walked with that operand resident
+        // and the other streamed once: column by column over every tile-row when A is the
+        // smaller, row by row over every tile-column when B is.  Otherwise groups of 8
+        // tile-rows: with panels this long (large k) the resident tiles only share panels within
+        // a wave.  (FP8 8192 x 14336 x 4096: A 32 MB resident, DRAM reads 3.0x the operands with
+        // groups of 8, where B was re-read by each of the four groups.)
+        {
+            const int64_t kb_bytes = P->k * esize(P->dtype);
+            const int64_t tiles_m = (m + bm - 1) / bm, tiles_n = (n + bn - 1) / bn;
+            const int64_t total_a = tiles_m * bm * kb_bytes, total_b = tiles_n * bn * kb_bytes;
+            const int64_t budget = 50ll << 20;
+            P->group_m = 8;
+            P->group_n = 0;
+            if (std::min(total_a, total_b) <= budget) {
+                if (total_a <= total_b) P->group_m = (int)std::min<int64_t>(tiles_m, 1 << 30);
+                else P->group_n = (int)std::min<int64_t>(tiles_n, 1 << 30);
+            }
+        }
         if (const char *g = getenv("GEMM_EPI_GROUP_M")) {   // tuning knob: tile-raster group height
             const int v = atoi(g);
-            if (v >= 1 && v <= 64) P->group_m = v;
+            if (v >= 1 && v <= 1 << 20) { P->group_m = v; P->group_n = 0; }
         }
         P->l2_mode = 1;
         if (const char *g = getenv("GEMM_EPI_L2")) {        // tuning knob: L2 cache policy (TcParams)
@@ -442,7 +461,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.out_scale = P->out_scale;
         L.p.amax = reinterpret_cast<unsigned int *>(P->amax);
         L.p.workspace = P->workspace;
-        L.p.counters = P->flags;
+        L.p.flags = P->flags;
         L.p.trace = trace_for_launch();
         L.pdl = P->pdl;
         L.stream = stream;
@@ -486,6 +505,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.num_tiles = L.p.tiles_m * L.p.tiles_n;
         L.p.num_kb = (int)((P->k + (int64_t)bk * P->katoms - 1) / ((int64_t)bk * P->katoms));   // ring stages
         L.p.group_m = P->group_m;
+        L.p.group_n = P->group_n;
         L.p.bias = bias;
         L.p.aux = aux;
         L.p.aux_pitch_words = pitch_words;
@@ -603,10 +623,10 @@ int make_plan(int64_t m, int64_t n, int64_t k, int dtype, int epilogue, int bias
     if (P->sk_tiles > 0 || (P->sk_grid && P->grid != sg_tiles)) {
         size_t ws_bytes, fl_bytes;
         if (P->sk_grid) {
-            // per CTA two partial tiles (its first and last piece) of NM x 128 fp32; one
-            // arrival counter per tile and TMEM lane quadrant
-            ws_bytes = (size_t)P->grid * 2 * 128 * (size_t)P->nm * sizeof(float);
-            fl_bytes = (size_t)sg_tiles * 4 * sizeof(unsigned int);
+            // per CTA one partial tile (of its first piece) of NM x 128 fp32 and one flag per
+            // TMEM lane quadrant
+            ws_bytes = (size_t)P->grid * 128 * (size_t)P->nm * sizeof(float);
+            fl_bytes = (size_t)P->grid * 4 * sizeof(unsigned int);
         } else {
             const int cg = P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
             const size_t units = (size_t)P->grid / cg;
@@ -854,6 +874,8 @@ void fill_info(const Plan *P, gemm_epi_plan_info *info) {
     info->smem_bytes = P->info.smem_bytes;
     info->sk_tiles = P->sk_tiles;
     info->sk_split = P->sk_split;
+    info->group_m = P->kernel == GEMM_EPI_KERNEL_SPLITK ? 0 : (P->group_n > 0 ? 0 : P->group_m);
+    info->group_n = P->kernel == GEMM_EPI_KERNEL_SPLITK ? 0 : P->group_n;
     if (P->kernel == GEMM_EPI_KERNEL_SPLITK) {
         info->tiles = (int)((P->n + 127) / 128);
     } else {

@@ -9,14 +9,16 @@
 // The work is the list of (tile, k-block) units, tile-major.  Every CTA of the grid (one
 // per SM) takes an equal contiguous range of it, so all SMs stream the weight whatever
 // the number of tiles; a range is cut at tile boundaries into pieces.  A piece that covers
-// a whole tile is finished in place.  Otherwise each epilogue warp publishes its 32
-// columns' fp32 partial tile to a workspace slot and counts itself on the tile's
-// per-quadrant arrival counter; the warp that arrives last adds every piece's partial in
-// piece order (so the sum does not depend on which CTA finished last) and runs the fused
-// epilogue (scale, bias, ReLU/GELU, sign mask, cast).  Nobody waits for anybody: the last
-// arriver finds every partial already published.  The last arriver also clears the
-// counter, so a launch leaves the counters as it found them (zero) and launches can be
-// replayed from CUDA graphs.
+// a whole tile is finished in place.  A tile cut into pieces is finished by the CTA that
+// holds its first k-block: each other piece is, by construction, the first piece of its
+// CTA's range, so it is multiplied first and published early (each epilogue warp writes its
+// 32 columns' fp32 partial to the CTA's workspace slot and raises a flag).  The finishing
+// warp keeps its own partial in registers, waits (bounded) for the flags, adds the other
+// pieces in piece order (a fixed order: run-to-run identical results), clears the flags and
+// runs the fused epilogue (scale, bias, ReLU/GELU, sign mask, cast).  Waits only ever point
+// to higher-numbered CTAs' first pieces, which wait on nothing lower, so they always end.
+// Every flag is cleared by its one reader, so a launch leaves the flags as it found them
+// (zero) and launches can be replayed from CUDA graphs.
 #pragma once
 #include "gemm_tc.cuh"
 
@@ -42,10 +44,10 @@ struct SgParams {
     uint8_t *dq;                 // FP8 output (QOUT kernels), as SkParams
     const float *out_scale;
     unsigned int *amax;
-    // Partial tiles: [cta][slot 0 = first piece, 1 = last piece][quadrant][NM][32] fp32.
-    // NULL: the grid has one CTA per tile and nothing is split.
+    // Partial tiles of the pieces that do not start a tile (always their CTA's first piece):
+    // [cta][quadrant][NM][32] fp32.  NULL: one CTA per tile, nothing is split.
     float *workspace;
-    unsigned int *counters;      // [tile][quadrant] warps that published a partial; 0 between launches
+    unsigned int *flags;         // [cta][quadrant]: 1 while a published partial is unread; 0 between launches
     unsigned long long *trace;   // timeline records; used only by builds with GEMM_EPI_TRACE=2
 };
 
@@ -73,7 +75,8 @@ struct SgCfg {
     static constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-    static constexpr int WS_FLOATS = 2 * 4 * NM * 32;   // workspace floats per CTA
+    static constexpr int WS_FLOATS = 4 * NM * 32;       // workspace floats per CTA
+    static constexpr int PB = NM <= 32 ? 8 : (NM <= 64 ? 4 : 2);   // partials loaded at once
     static_assert(NM % 16 == 0 && NM >= 16 && NM <= 128, "MMA N for M = 128");
     static_assert(STAGES >= 2, "the ring needs two stages");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -107,8 +110,8 @@ struct SgRange {
 };
 
 template <class C>
-__device__ __forceinline__ float *sg_slot(const SgParams &p, int cta, int slot, int q) {
-    return p.workspace + ((size_t)cta * C::WS_FLOATS) + (size_t)(slot * 4 + q) * C::NM * 32;
+__device__ __forceinline__ float *sg_slot(const SgParams &p, int cta, int q) {
+    return p.workspace + ((size_t)cta * C::WS_FLOATS) + (size_t)q * C::NM * 32;
 }
 
 // grid = p.grid CTAs, no cluster.
@@ -307,33 +310,51 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
             if (++acc == 2u) { acc = 0; acc_phase ^= 1u; }
 
-            if (!(kb0 == 0 && kb1 == p.num_kb)) {
-                // a piece of a split tile: publish this warp's partial, count it, and let the
-                // last of the tile's warps of this quadrant finish the tile
-                const int slot = first ? 0 : 1;
-                float *mine = sg_slot<C>(p, cta, slot, q);
+            if (kb0 > 0) {
+                // a piece after a tile's first k-block (its CTA's first piece): publish this
+                // warp's partial for the CTA that finishes the tile
+                float *mine = sg_slot<C>(p, cta, q);
 #pragma unroll
                 for (int i = 0; i < C::NM; ++i) __stcg(mine + i * 32 + lane, v[i]);
                 __threadfence();
                 __syncwarp();
-                const int64_t t0 = (int64_t)tile * p.num_kb;
-                const int c_lo = r.owner(t0), c_hi = r.owner(t0 + p.num_kb - 1);
-                unsigned int arrived = 0;
-                if (lane == 0) arrived = atomicAdd(p.counters + tile * 4 + q, 1u);
-                arrived = __shfl_sync(0xffffffffu, arrived, 0);
-                if (arrived != (unsigned int)(c_hi - c_lo)) continue;     // not the last
-                __threadfence();
-                if (lane == 0) p.counters[tile * 4 + q] = 0u;          // for the next launch
-                // every piece's partial, this warp's own included, in piece order (so the sum
-                // does not depend on the arrival order)
+                if (lane == 0) ptx::st_release_gpu(p.flags + cta * 4 + q, 1u);
+                if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 27, tile, kb1);
+                continue;
+            }
+            if (kb1 < p.num_kb) {
+                // this CTA holds the tile's first k-block and finishes it: wait for the other
+                // pieces (the first pieces of CTAs cta + 1 .. c_hi), then add them in order
+                const int c_hi = r.owner((int64_t)tile * p.num_kb + p.num_kb - 1);
+                for (int cc = cta + 1; ok && cc <= c_hi; ++cc)
+                    ok = wait_flag(p.flags + cc * 4 + q, abort_flag, p.status);
+                if (!ok) break;
+                __syncwarp();
 #pragma unroll
-                for (int i = 0; i < C::NM; ++i) v[i] = 0.0f;
-                for (int cc = c_lo; cc <= c_hi; ++cc) {
-                    const int sl = (cc == c_lo && r.start_of(cc) != t0) ? 1 : 0;
-                    const float *src = sg_slot<C>(p, cc, sl, q);
+                for (int i0 = 0; i0 < C::NM; i0 += 16) {
+                    for (int cc0 = cta + 1; cc0 <= c_hi; cc0 += C::PB) {
+                        float buf[C::PB][16];
 #pragma unroll
-                    for (int i = 0; i < C::NM; ++i) v[i] += __ldcg(src + i * 32 + lane);
+                        for (int j = 0; j < C::PB; ++j) {
+                            if (cc0 + j <= c_hi) {
+                                const float *src = sg_slot<C>(p, cc0 + j, q) + i0 * 32 + lane;
+#pragma unroll
+                                for (int ii = 0; ii < 16; ++ii) buf[j][ii] = __ldcg(src + ii * 32);
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < C::PB; ++j) {
+                            if (cc0 + j <= c_hi) {
+#pragma unroll
+                                for (int ii = 0; ii < 16; ++ii) v[i0 + ii] += buf[j][ii];
+                            }
+                        }
+                    }
                 }
+                // the partials have been read: clear their flags for the next launch
+                __syncwarp();
+                if (lane == 0)
+                    for (int cc = cta + 1; cc <= c_hi; ++cc) p.flags[cc * 4 + q] = 0u;
             }
 
             // fused epilogue for output column `col`, rows 0..m-1

@@ -83,7 +83,8 @@ constexpr uint64_t DRAIN_TIMEOUT_NS = 100000000ull;  // 100 ms for the wind-down
 struct TcParams {
     int m, n, k;
     int tiles_m, tiles_n, num_tiles, num_kb;
-    int group_m;                 // tile-raster group height (in tiles along m)
+    int group_m;                 // tile raster: groups of group_m tile-rows walked column by column,
+    int group_n;                 // or (group_n > 0) groups of group_n tile-columns walked row by row
     const void *bias;            // length m (ROW) or n (COL), output type
     uint32_t *aux;               // RELU_AUX: mask written; DRELU: mask read
     int64_t aux_pitch_words;     // ceil(n/128)*4
@@ -417,7 +418,9 @@ struct TcCfg {
     static constexpr int OFF_BIAS = OFF_STG + EPI_WARPS * STG_BYTES;
     static constexpr int BIAS_FLOATS = (FWD_BIAS && AXIS == AXIS_COL) ? COLS_W : 0;
     static constexpr int OFF_BAR = OFF_BIAS + EPI_WARPS * BIAS_FLOATS * 4;
-    static constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
+    // a full barrier per (stage, k-atom): the MMA starts on a stage's first atom while the
+    // second is still landing; an empty barrier per stage; two accumulator pairs; done
+    static constexpr int NUM_BARS = (KATOMS + 1) * STAGES + 4 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
     static_assert(BN == 128 || BN == 256 || (BN == 512 && CG == 2), "BN is 128 or 256 (512 for CTA pairs)");
@@ -432,10 +435,21 @@ struct TcCfg {
     static_assert(!A_MN || BM % A_BOX_M == 0, "MN-major A tile must be whole boxes");
 };
 
-// Tile index -> (tile_m, tile_n) with a grouped raster: GROUP_M tile-rows are
-// walked column by column so that concurrently resident CTAs share A and B
-// panels in L2.
+// Tile index -> (tile_m, tile_n) with a grouped raster.  group_n == 0: groups of group_m
+// tile-rows, each walked column by column, so the group's A panels are reused by every
+// column while B panels stream through; group_n > 0: groups of group_n tile-columns walked
+// row by row (B panels reused, A streamed).  The plan sizes the group from the L2 capacity.
 __device__ __forceinline__ void tile_coords(const TcParams &p, int t, int &tm, int &tn) {
+    if (p.group_n > 0) {
+        const int per_group = p.group_n * p.tiles_m;
+        const int g = t / per_group;
+        const int first = g * p.group_n;
+        const int cols = min(p.group_n, p.tiles_n - first);
+        const int r = t - g * per_group;
+        tn = first + r % cols;
+        tm = r / cols;
+        return;
+    }
     const int per_group = p.group_m * p.tiles_n;
     const int g = t / per_group;
     const int first = g * p.group_m;
@@ -456,11 +470,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const uint32_t sA = sb + C::OFF_A, sB = sb + C::OFF_B, sStg = sb + C::OFF_STG;
     float *bias_smem = reinterpret_cast<float *>(smem + C::OFF_BIAS);
     const uint32_t bar0 = sb + C::OFF_BAR;
-    auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
-    auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
-    auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
-    const uint32_t done_bar = bar0 + 8u * (2 * C::STAGES + 4);
+    auto full_bar = [&](int s, int at) { return bar0 + 8u * (s * C::KATOMS + at); };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (C::KATOMS * C::STAGES + s); };
+    auto tfull_bar = [&](int a) { return bar0 + 8u * ((C::KATOMS + 1) * C::STAGES + a); };
+    auto tempty_bar = [&](int a) { return bar0 + 8u * ((C::KATOMS + 1) * C::STAGES + 2 + a); };
+    const uint32_t done_bar = bar0 + 8u * ((C::KATOMS + 1) * C::STAGES + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -476,7 +490,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         ptx::prefetch_tmap(&tmB);
         if constexpr (!C::QOUT) ptx::prefetch_tmap(&tmD);
         for (int s = 0; s < C::STAGES; ++s) {
-            ptx::mbar_init(full_bar(s), 1);
+            for (int at = 0; at < C::KATOMS; ++at) ptx::mbar_init(full_bar(s, at), 1);
             ptx::mbar_init(empty_bar(s), 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -526,14 +540,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         break;
                     }
                     trace_stage(p.trace, 0, tr_i, 20, w.tile, kb);
-                    uint32_t fb = full_bar(stage);
+                    for (int at = 0; at < C::KATOMS; ++at) {    // the stage's k-atoms
+                    uint32_t fb = full_bar(stage, at);
                     if constexpr (C::CG == 2) {
                         fb = ptx::mapa(fb, 0);      // the pair's leader counts both CTAs' bytes
-                        if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * (C::A_STAGE + C::B_STAGE));
+                        if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage, at), 2 * (C::A_BYTES + C::B_BYTES));
                     } else {
-                        ptx::mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE);
+                        ptx::mbar_arrive_expect_tx(fb, C::A_BYTES + C::B_BYTES);
                     }
-                    for (int at = 0; at < C::KATOMS; ++at) {    // the stage's k-atoms
                     const int k0 = (kb * C::KATOMS + at) * C::BK;
                     const uint32_t a_dst = sA + stage * C::A_STAGE + at * C::A_BYTES;
                     const uint32_t b_dst = sB + stage * C::B_STAGE + at * C::B_BYTES;
@@ -570,7 +584,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 // wind down: wait (bounded) until the loads still in flight have landed
                 const uint32_t back = issued < (uint32_t)C::STAGES ? issued : (uint32_t)C::STAGES;
                 for (uint32_t j = issued - back; j < issued; ++j)
-                    wait_drain(full_bar(j % C::STAGES), (j / C::STAGES) & 1u, p.status);
+                    for (int at = 0; at < C::KATOMS; ++at)
+                        wait_drain(full_bar(j % C::STAGES, at), (j / C::STAGES) & 1u, p.status);
             }
         }
     } else if (warp == 1) {
@@ -595,14 +610,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 trace_stage(p.trace, 1, tr_i, 25, w.tile, w.kb0);
                 const uint32_t d_tmem = tmem_base + acc * C::BN;
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
-                    if (!wait_bounded<false>(full_bar(stage), phase, abort_flag, p.status, ST_TIMEOUT_MMA)) {
+#pragma unroll
+                    for (int at = 0; at < C::KATOMS; ++at) {
+                    if (!wait_bounded<false>(full_bar(stage, at), phase, abort_flag, p.status, ST_TIMEOUT_MMA)) {
                         ok = false;
                         break;
                     }
-                    trace_stage(p.trace, 1, tr_i, 22, w.tile, kb);
+                    if (at == 0) trace_stage(p.trace, 1, tr_i, 22, w.tile, kb);
                     ptx::tc_fence_after();
-#pragma unroll
-                    for (int at = 0; at < C::KATOMS; ++at) {
                     const uint32_t a_base = sA + stage * C::A_STAGE + at * C::A_BYTES;
                     const uint32_t b_base = sB + stage * C::B_STAGE + at * C::B_BYTES;
 #pragma unroll
@@ -619,6 +634,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         }
                     }
                     }
+                    if (!ok) break;
                     if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(empty_bar(stage), 0x3);
                     else ptx::mma_commit(empty_bar(stage));
                     if (++stage == (uint32_t)C::STAGES) { stage = 0; phase ^= 1u; }

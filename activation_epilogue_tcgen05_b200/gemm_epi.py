@@ -61,7 +61,7 @@ class Options(ctypes.Structure):
 class PlanInfo(ctypes.Structure):
     _fields_ = [(f, ctypes.c_int32) for f in
                 ("kernel", "block_m", "block_n", "block_k", "stages", "split_k", "grid", "cluster",
-                 "threads", "smem_bytes", "tiles", "sk_tiles", "sk_split")]
+                 "threads", "smem_bytes", "tiles", "sk_tiles", "sk_split", "group_m", "group_n")]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

@@ -208,21 +208,35 @@ def hold_clock_window(replay, region_s: float, hold_s: float, stream, device):
 
 
 def clock_record(sampler, wall0, wall1, window, flops_per_region, value):
-    """The clock block of the JSON line: samples over the timed region and the window after it."""
+    """The clock block of the JSON line.
+
+    ``sm_mhz`` etc. summarise the samples over the timed region and the back-to-back window
+    after it (``hold_clock_window``).  A timed region of a few milliseconds holds at most one
+    sampler period, so ``timed_region`` gives its own samples (often none) and ``window`` the
+    window's throughput, its own median clock and their ratio (work per clock cycle at the
+    clock the power cap settles to)."""
     if sampler is None:
         return None
     if window is None:
         return sampler.summary(wall0, wall1)
     reps, secs, wall2 = window
     rec = sampler.summary(wall0, wall2)
-    rec["timed_region_samples"] = sum(1 for (t, _) in sampler.samples if wall0 <= t <= wall1)
-    rec["window"] = {"seconds": secs, "replays_of_timed_region": reps,
-                     "value": flops_per_region * reps / secs / 1e12, "unit": "TFLOP/s",
-                     "what": "the timed region's launches replayed back to back right after it; "
-                             "sm_mhz is the median over the timed region and this window"}
-    if rec.get("sm_mhz"):
-        rec["value_per_ghz"] = value / (rec["sm_mhz"] / 1000.0)
-        rec["window"]["value_per_ghz"] = rec["window"]["value"] / (rec["sm_mhz"] / 1000.0)
+    inside = [p for (t, p) in sampler.samples if wall0 <= t <= wall1]
+    rec["timed_region"] = {"samples": len(inside), "value": value}
+    if inside:
+        mhz = [float(p[2]) for p in inside if p[2].replace(".", "", 1).isdigit()]
+        if mhz:
+            rec["timed_region"]["sm_mhz"] = statistics.median(mhz)
+    w = {"seconds": secs, "replays_of_timed_region": reps,
+         "value": flops_per_region * reps / secs / 1e12, "unit": "TFLOP/s",
+         "what": "the timed region's launches replayed back to back right after it"}
+    ws = [p for (t, p) in sampler.samples if wall1 <= t <= wall2]
+    wm = [float(p[2]) for p in ws if p[2].replace(".", "", 1).isdigit()]
+    w["samples"] = len(wm)
+    if wm:
+        w["sm_mhz"] = statistics.median(wm)
+        w["value_per_ghz"] = w["value"] / (w["sm_mhz"] / 1000.0)
+    rec["window"] = w
     return rec
 
 

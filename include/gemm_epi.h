@@ -170,6 +170,9 @@ typedef struct gemm_epi_plan_info {
     int32_t kernel, block_m, block_n, block_k, stages, split_k;
     int32_t grid, cluster, threads, smem_bytes, tiles;
     int32_t sk_tiles, sk_split;   /* split tail: tiles split along k, parts per split tile */
+    int32_t group_m, group_n;     /* TC tile raster: groups of group_m tile-rows walked column by
+                                     column, or (group_m == 0) groups of group_n tile-columns
+                                     walked row by row; 0, 0 for SPLITK */
 } gemm_epi_plan_info;
 
 /* ---- entry points -------------------------------------------------------- */

@@ -180,3 +180,22 @@ def test_preview_checks_arguments_like_a_plan(g):
     assert status(m=200, n=128, k=128, kernel="splitk") == g.ERR_UNSUPPORTED   # m > 128
     assert status(m=128, n=128, k=128, sms=1) == g.ERR_ARG
     assert status(m=128, n=128, k=128, sms=4096) == g.ERR_ARG
+
+
+# ------------------------------------------------------------------ tile raster from the L2 budget
+def test_raster_from_l2_budget(g):
+    # 4096^3 bf16, 256 x 256 pair tiles: A and B are 32 MB each; A resident, one column walk
+    p = pv(g, 4096, 4096, 4096, "bf16", "relu_aux_bias")
+    assert (p["group_m"], p["group_n"]) == (16, 0)
+    # FP8 8192 x 14336 x 4096: A 32 MB < B 56 MB: A resident over all 32 tile-rows
+    p = pv(g, 8192, 14336, 4096, "e4m3", "gelu_bias", "col", "kn")
+    assert (p["group_m"], p["group_n"]) == (32, 0)
+    # B the smaller and within the budget (16 MB against A's 64 MB): row walk, B resident
+    p = pv(g, 8192, 2048, 4096, "bf16", "bias")
+    assert (p["group_m"], p["group_n"]) == (0, p["tiles"] // 32)
+    # neither fits (65536 x 8192 x 16384: A 2 GB, B 256 MB): groups of 8 tile-rows
+    p = pv(g, 65536, 8192, 16384, "bf16", "relu_bias")
+    assert (p["group_m"], p["group_n"]) == (8, 0)
+    # the small-m kernel has no raster
+    p = pv(g, 16, 4096, 4096, "f16", "gelu_bias", "col", "nk")
+    assert (p["group_m"], p["group_n"]) == (0, 0)
