@@ -50,6 +50,7 @@ struct Plan {
     int grid;
     int group_m, group_n = 0;   // TC raster (TcParams::group_m / group_n)
     int l2_mode = 1;     // TcParams::l2_mode (GEMM_EPI_L2=0/1/2 overrides)
+    int prefetch = 0;    // TcParams::prefetch (GEMM_EPI_PREFETCH=n overrides)
     bool pdl;            // programmatic dependent launch (GEMM_EPI_PDL=0 turns it off)
     // split tail (TC kernels): tiles [0, sk_tiles) cut along k into sk_split parts
     int sk_tiles = 0, sk_split = 0;
@@ -324,6 +325,11 @@ int choose(Plan *P) {
             const int v = atoi(g);
             if (v >= 0 && v <= 2) P->l2_mode = v;
         }
+        P->prefetch = 0;
+        if (const char *g = getenv("GEMM_EPI_PREFETCH")) {
+            const int v = atoi(g);
+            if (v >= 0 && v <= 64) P->prefetch = v;
+        }
         KernelInfo none_info;
         if (!find_tc(cg, P->dtype, GEMM_EPI_NONE, 0, b_mn, bn, false, P->a_km, &P->tc_none_launch, &none_info))
             return GEMM_EPI_ERR_UNSUPPORTED;
@@ -451,7 +457,6 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.tiles_n = (int)((P->n + 127) / 128);
         L.p.grid = P->grid;
         L.p.bias = bias;
-        L.p.D = D;
         L.p.aux = aux;
         L.p.aux_pitch_words = pitch_words;
         L.p.scale_a = P->scale_a;
@@ -476,7 +481,6 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.num_kb = num_kb;
         L.p.kb_per_cta = P->kb_per_cta;
         L.p.bias = bias;
-        L.p.D = D;
         L.p.aux = aux;
         L.p.aux_pitch_words = pitch_words;
         L.p.scale_a = P->scale_a;
@@ -523,6 +527,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.out_scale = P->out_scale;
         L.p.amax = reinterpret_cast<unsigned int *>(P->amax);
         L.p.l2_mode = P->l2_mode;
+        L.p.prefetch = P->prefetch;
         L.grid = P->grid;
         L.pdl = P->pdl;
         L.stream = stream;

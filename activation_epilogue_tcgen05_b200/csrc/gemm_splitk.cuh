@@ -251,6 +251,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 ptx::st_cluster_v4(remote + j * 4, acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
         }
     }
+    // the leader's column bias, read before the cluster barrier so that its latency hides
+    float cbias = 0.0f;
+    if constexpr (C::EPI != EPI_NONE && C::AXIS == AXIS_COL) {
+        const int col = n0 + 32 * q + lane;
+        if (epi && rank == 0 && col < p.n && p.bias != nullptr) cbias = OutT<C::DT>::load(p.bias, col);
+    }
     __syncwarp();
     ptx::tc_fence_before();
     ptx::cluster_sync();     // partials visible in the leader's shared memory
@@ -277,10 +283,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         float alpha = 1.0f;
         if (p.scale_a != nullptr) alpha = __ldg(p.scale_a) * __ldg(p.scale_b);
         const bool has_bias = p.bias != nullptr;
-        float cbias = 0.0f;
-        if constexpr (C::EPI != EPI_NONE && C::AXIS == AXIS_COL) {
-            if (col_ok && has_bias) cbias = O::load(p.bias, col);
-        }
         T *D = reinterpret_cast<T *>(p.D);
         float inv_out = 1.0f, amax_l = 0.0f;
         if constexpr (C::QOUT) inv_out = 1.0f / __ldg(p.out_scale);

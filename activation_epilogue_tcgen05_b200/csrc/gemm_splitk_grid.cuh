@@ -316,6 +316,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         int tile, kb0, kb1;
         bool first;
         while (ok && r.next(tile, kb0, kb1, first, u_first)) {
+            // this lane's output column and its bias, read before the accumulator is waited for
+            const int n0 = tile * 128;
+            const int col = n0 + 32 * q + lane;
+            const bool col_ok = col < p.n;
+            float cbias = 0.0f;
+            if constexpr (C::EPI != EPI_NONE && C::AXIS == AXIS_COL) {
+                if (kb0 == 0 && col_ok && has_bias) cbias = O::load(p.bias, col);
+            }
             if (!wait_bounded<false>(tfull_bar(acc), acc_phase, abort_flag, p.status, ST_TIMEOUT_SPLITK)) {
                 ok = false;
                 break;
@@ -347,7 +355,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 ptx::fence_acq_rel_gpu();       // this lane's partial before the warp's flag
                 __syncwarp();
                 if (lane == 0) ptx::st_release_gpu(p.flags + cta * 4 + q, 1u);
-                if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 27, tile, kb1);
+                if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 32, tile, kb1);
                 continue;
             }
             if (kb1 < p.num_kb) {
@@ -356,6 +364,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const int c_hi = r.owner((int64_t)tile * p.num_kb + p.num_kb - 1);
                 ok = wait_flags_warp(p.flags + (cta + 1) * 4 + q, 4, c_hi - cta, lane, abort_flag, p.status);
                 if (!ok) break;
+                if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 30, tile, c_hi - cta);
 #pragma unroll
                 for (int i0 = 0; i0 < C::NM; i0 += 16) {
                     for (int cc0 = cta + 1; cc0 <= c_hi; cc0 += C::PB) {
@@ -377,6 +386,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         }
                     }
                 }
+                if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 31, tile, kb1);
                 // the partials have been read: clear their flags for the next launch
                 __syncwarp();
                 if (lane == 0)
@@ -384,13 +394,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             }
 
             // fused epilogue for output column `col`, rows 0..m-1
-            const int n0 = tile * 128;
-            const int col = n0 + 32 * q + lane;
-            const bool col_ok = col < p.n;
-            float cbias = 0.0f;
-            if constexpr (C::EPI != EPI_NONE && C::AXIS == AXIS_COL) {
-                if (col_ok && has_bias) cbias = O::load(p.bias, col);
-            }
             // every word of the mask pitch belongs to exactly one warp of one tile; columns at
             // or past n contribute 0 bits, so padding words come out 0
             const int64_t word = (n0 + 32 * q) / 32;

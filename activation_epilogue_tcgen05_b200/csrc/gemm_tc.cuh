@@ -106,6 +106,7 @@ struct TcParams {
     uint8_t *dq;
     const float *out_scale;
     unsigned int *amax;
+    int prefetch;                // producer: L2 prefetch of the stage this many stages ahead (0: none)
     // L2 cache policy: 0 = normal for every access; 1 = the outputs (D, mask) are written
     // evict-first, so that streaming them out does not push the operands out of L2; 2 = as 1,
     // and the operands are loaded evict-last
@@ -523,16 +524,49 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             bool ok = true;
             const uint64_t pol_ab = p.l2_mode == 2 ? ptx::policy_evict_last() : ptx::policy_evict_normal();
             trace_stage(p.trace, 0, tr_i, 10, 0, 0);
+            // L2 prefetch of stage kb of the tile at (m0_, nb_): the same boxes as its loads, no
+            // shared-memory destination, no barrier (only a hint to L2)
+            auto prefetch_stage = [&](int m0_, int nb_, int kb_) {
+#pragma unroll
+                for (int at = 0; at < C::KATOMS; ++at) {
+                    const int k0 = (kb_ * C::KATOMS + at) * C::BK;
+                    if constexpr (C::A_MN) {
+#pragma unroll
+                        for (int b = 0; b < C::A_BOXES; ++b) ptx::tma_prefetch_l2_2d(&tmA, m0_ + b * C::A_BOX_M, k0);
+                    } else {
+                        ptx::tma_prefetch_l2_2d(&tmA, k0, m0_);
+                    }
+                    if constexpr (C::B_MN) {
+                        constexpr int PER_HALF = C::MMA_N_LOCAL / C::B_BOX_N;
+#pragma unroll
+                        for (int b = 0; b < C::B_BOXES; ++b)
+                            ptx::tma_prefetch_l2_2d(&tmB, nb_ + (b / PER_HALF) * C::MMA_N + (b % PER_HALF) * C::B_BOX_N, k0);
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < C::N_MMAS; ++h) ptx::tma_prefetch_l2_2d(&tmB, k0, nb_ + h * C::MMA_N);
+                    }
+                }
+            };
+            auto origin = [&](int tile, int &m0_, int &nb_) {
+                int tm, tn;
+                tile_coords(p, tile, tm, tn);
+                m0_ = tm * (C::BM * C::CG) + (int)rank * C::BM;
+                // local B row r (MMA half h = r / MMA_N_LOCAL) holds global column
+                // tn*BN + h*MMA_N + rank*MMA_N_LOCAL + r % MMA_N_LOCAL
+                nb_ = tn * C::BN + (int)rank * C::MMA_N_LOCAL;
+            };
             WorkIter it(p, unit, units);
             WorkItem w;
             while (ok && it.next(p, units, w)) {
                 trace_event(p.trace, warp, 1, w.tile, w.kb0);
-                int tm, tn;
-                tile_coords(p, w.tile, tm, tn);
-                const int m0 = tm * (C::BM * C::CG) + (int)rank * C::BM;
-                // local B row r (MMA half h = r / MMA_N_LOCAL) holds global column
-                // tn*BN + h*MMA_N + rank*MMA_N_LOCAL + r % MMA_N_LOCAL
-                const int nb = tn * C::BN + (int)rank * C::MMA_N_LOCAL;
+                int m0, nb;
+                origin(w.tile, m0, nb);
+                // the next work item, for prefetches that run past this one's last stage
+                WorkIter peek = it;
+                WorkItem w2;
+                const bool has_next = peek.next(p, units, w2);
+                int m0n = 0, nbn = 0;
+                if (has_next) origin(w2.tile, m0n, nbn);
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!wait_bounded<false>(empty_bar(stage), phase ^ 1u, abort_flag, p.status,
                                              ST_TIMEOUT_PRODUCER)) {
@@ -575,6 +609,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         for (int h = 0; h < C::N_MMAS; ++h)
                             load(b_dst + h * C::HALF_B_BYTES, &tmB, k0, nb + h * C::MMA_N);
                     }
+                    }
+                    if (p.prefetch > 0) {
+                        // warm L2 for the stage p.prefetch ahead (in this work item or the next), so
+                        // that its load, issued once a ring slot frees, finds the data in L2
+                        const int ahead = kb + p.prefetch;
+                        if (ahead < w.kb1) prefetch_stage(m0, nb, ahead);
+                        else if (has_next && w2.kb0 + (ahead - w.kb1) < w2.kb1)
+                            prefetch_stage(m0n, nbn, w2.kb0 + (ahead - w.kb1));
                     }
                     ++issued;
                     if (++stage == (uint32_t)C::STAGES) { stage = 0; phase ^= 1u; }

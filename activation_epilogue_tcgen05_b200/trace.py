@@ -37,7 +37,8 @@ LAUNCH_RECS = 256 * 4 * ROLE_CAP
 TRACE_CAP = 1 << 22
 EV = {10: "CTA start", 11: "after the dependency wait", 20: "stage load issued", 22: "stage ready (MMA)",
       23: "last MMA issued", 24: "accumulator wait", 25: "accumulator free", 26: "accumulator ready",
-      27: "epilogue piece done", 28: "after cluster barrier", 29: "CTA end"}
+      27: "epilogue piece done", 28: "after cluster barrier", 29: "CTA end", 30: "finisher: flags seen",
+      31: "finisher: partials added", 32: "publisher: flag raised"}
 
 
 def build(force: bool = False) -> str:
@@ -127,6 +128,14 @@ def summarise_small_m(launches):
         rows.append((pick(11).min(), pick(22).min(), pick(23).max(), pick(29).max(), len(np.unique(L["cta"]))))
     rows.sort()
     lines = []
+    # the chain of the last launch's latest events, against its dependency release
+    if launches:
+        Lz = max(launches, key=lambda L: L["gt"].min())
+        rel = Lz["gt"][Lz["ev"] == 11].min() if (Lz["ev"] == 11).any() else Lz["gt"].min()
+        for e in sorted(set(Lz["ev"].tolist())):
+            x = (Lz["gt"][Lz["ev"] == e] - rel) / 1e3
+            lines.append(f"  ev{e:2d} {EV.get(e, ''):28s} min {x.min():7.2f}  p50 {np.median(x):7.2f}  "
+                         f"max {x.max():7.2f} us (from the release)")
     for i in range(1, len(rows)):
         r0, r1 = rows[i - 1], rows[i]
         lines.append(f"launch {i} ({r1[4]} CTAs): release-to-release {(r1[0] - r0[0]) / 1e3:.2f} us | previous end -> "
