@@ -447,7 +447,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
     const int64_t pitch_words = ((P->n + 127) / 128) * 4;
     cudaError_t e;
     if (P->kernel == GEMM_EPI_KERNEL_SPLITK && P->sk_grid) {
-        SgLaunch L;
+        SgLaunch L{};
         L.tmW = P->tmA;
         L.tmX = P->tmB;
         L.p.m = (int)P->m;
@@ -457,6 +457,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.tiles_n = (int)((P->n + 127) / 128);
         L.p.grid = P->grid;
         L.p.bias = bias;
+        L.p.D = D;
         L.p.aux = aux;
         L.p.aux_pitch_words = pitch_words;
         L.p.scale_a = P->scale_a;
@@ -472,7 +473,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.stream = stream;
         e = (fused ? P->sg_launch : P->sg_none_launch)(L);
     } else if (P->kernel == GEMM_EPI_KERNEL_SPLITK) {
-        SkLaunch L;
+        SkLaunch L{};
         L.tmW = P->tmA;
         L.tmX = P->tmB;
         L.p.m = (int)P->m;
@@ -481,6 +482,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.num_kb = num_kb;
         L.p.kb_per_cta = P->kb_per_cta;
         L.p.bias = bias;
+        L.p.D = D;
         L.p.aux = aux;
         L.p.aux_pitch_words = pitch_words;
         L.p.scale_a = P->scale_a;
@@ -497,7 +499,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         e = (fused ? P->sk_launch : P->sk_none_launch)(L);
     } else {
         const int cg = P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
-        TcLaunch L;
+        TcLaunch L{};
         L.tmA = P->tmA;
         L.tmB = P->tmB;
         L.tmD = P->tmD;
@@ -533,6 +535,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.stream = stream;
         e = (fused ? P->tc_launch : P->tc_none_launch)(L);
     }
+    if (e != cudaSuccess && getenv("GEMM_EPI_LOG")) fprintf(stderr, "gemm_epi launch: %s (%d)\n", cudaGetErrorString(e), (int)e);
     return e == cudaSuccess ? GEMM_EPI_OK : GEMM_EPI_ERR_CUDA;
 }
 
@@ -851,7 +854,11 @@ int gemm_epi_unfused_run_bwd(gemm_epi_plan_t plan, const void *A, const void *B,
 int gemm_epi_check(gemm_epi_plan_t plan, void *stream) {
     if (!live(plan)) return GEMM_EPI_ERR_ARG;
     Plan *P = reinterpret_cast<Plan *>(plan);
-    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GEMM_EPI_ERR_CUDA;
+    const cudaError_t se = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (se != cudaSuccess) {
+        if (getenv("GEMM_EPI_LOG")) fprintf(stderr, "gemm_epi_check: %s (%d)\n", cudaGetErrorString(se), (int)se);
+        return GEMM_EPI_ERR_CUDA;
+    }
     unsigned int word = 0;
     if (cudaMemcpy(&word, P->status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
         return GEMM_EPI_ERR_CUDA;
