@@ -434,6 +434,8 @@ struct TcCfg {
     static_assert(!BWD || (EPI_WARPS == 4 && CPG == 4), "backward epilogue: one mask uint4 per chunk group");
     static_assert(!QOUT || (DT == DT_E4M3 && !BWD && EPI != EPI_RELU_AUX), "FP8 output: e4m3 forward plans");
     static_assert(!A_MN || BM % A_BOX_M == 0, "MN-major A tile must be whole boxes");
+    static_assert(EPI_WARPS * NCH_W * 2048 <= STAGES * (A_STAGE + B_STAGE),
+                  "the last tile's output staging fits in the operand ring");
 };
 
 // Tile index -> (tile_m, tile_n) with a grouped raster.  group_n == 0: groups of group_m
@@ -510,9 +512,54 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if constexpr (C::CG == 2) ptx::cluster_sync(); else __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // L2 prefetch of stage kb of the tile at (m0_, nb_): the same boxes as its loads, no
+    // shared-memory destination, no barrier (only a hint to L2)
+    auto prefetch_stage = [&](int m0_, int nb_, int kb_) {
+#pragma unroll
+        for (int at = 0; at < C::KATOMS; ++at) {
+            const int k0 = (kb_ * C::KATOMS + at) * C::BK;
+            if constexpr (C::A_MN) {
+#pragma unroll
+                for (int b = 0; b < C::A_BOXES; ++b) ptx::tma_prefetch_l2_2d(&tmA, m0_ + b * C::A_BOX_M, k0);
+            } else {
+                ptx::tma_prefetch_l2_2d(&tmA, k0, m0_);
+            }
+            if constexpr (C::B_MN) {
+                constexpr int PER_HALF = C::MMA_N_LOCAL / C::B_BOX_N;
+#pragma unroll
+                for (int b = 0; b < C::B_BOXES; ++b)
+                    ptx::tma_prefetch_l2_2d(&tmB, nb_ + (b / PER_HALF) * C::MMA_N + (b % PER_HALF) * C::B_BOX_N, k0);
+            } else {
+#pragma unroll
+                for (int h = 0; h < C::N_MMAS; ++h) ptx::tma_prefetch_l2_2d(&tmB, k0, nb_ + h * C::MMA_N);
+            }
+        }
+    };
+    auto origin = [&](int tile, int &m0_, int &nb_) {
+        int tm, tn;
+        tile_coords(p, tile, tm, tn);
+        m0_ = tm * (C::BM * C::CG) + (int)rank * C::BM;
+        // local B row r (MMA half h = r / MMA_N_LOCAL) holds global column
+        // tn*BN + h*MMA_N + rank*MMA_N_LOCAL + r % MMA_N_LOCAL
+        nb_ = tn * C::BN + (int)rank * C::MMA_N_LOCAL;
+    };
     // Everything above touches only on-chip state, so under programmatic dependent launch
-    // it overlaps the previous kernel's tail.  No global memory is read or written before
-    // the previous kernel has completed; the next kernel may be scheduled from here on.
+    // it overlaps the previous kernel's tail.  Before waiting for that kernel, the producer
+    // asks L2 for the first ring's worth of this unit's operand boxes: a prefetch writes
+    // nothing and brings nothing into the SM, and L2 is the point of coherence, so the loads
+    // below still see every value the previous kernel stores.  No other global memory is read
+    // or written before the previous kernel has completed; the next kernel may be scheduled
+    // from here on.
+    if (warp == 0 && lane == 0) {
+        WorkIter it0(p, unit, units);
+        WorkItem w0;
+        if (it0.next(p, units, w0)) {
+            int m0, nb;
+            origin(w0.tile, m0, nb);
+            const int last = min(w0.kb1, w0.kb0 + C::STAGES);
+            for (int kb = w0.kb0; kb < last; ++kb) prefetch_stage(m0, nb, kb);
+        }
+    }
     ptx::griddep_wait();
     ptx::griddep_launch_dependents();
 
@@ -524,37 +571,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             bool ok = true;
             const uint64_t pol_ab = p.l2_mode == 2 ? ptx::policy_evict_last() : ptx::policy_evict_normal();
             trace_stage(p.trace, 0, tr_i, 10, 0, 0);
-            // L2 prefetch of stage kb of the tile at (m0_, nb_): the same boxes as its loads, no
-            // shared-memory destination, no barrier (only a hint to L2)
-            auto prefetch_stage = [&](int m0_, int nb_, int kb_) {
-#pragma unroll
-                for (int at = 0; at < C::KATOMS; ++at) {
-                    const int k0 = (kb_ * C::KATOMS + at) * C::BK;
-                    if constexpr (C::A_MN) {
-#pragma unroll
-                        for (int b = 0; b < C::A_BOXES; ++b) ptx::tma_prefetch_l2_2d(&tmA, m0_ + b * C::A_BOX_M, k0);
-                    } else {
-                        ptx::tma_prefetch_l2_2d(&tmA, k0, m0_);
-                    }
-                    if constexpr (C::B_MN) {
-                        constexpr int PER_HALF = C::MMA_N_LOCAL / C::B_BOX_N;
-#pragma unroll
-                        for (int b = 0; b < C::B_BOXES; ++b)
-                            ptx::tma_prefetch_l2_2d(&tmB, nb_ + (b / PER_HALF) * C::MMA_N + (b % PER_HALF) * C::B_BOX_N, k0);
-                    } else {
-#pragma unroll
-                        for (int h = 0; h < C::N_MMAS; ++h) ptx::tma_prefetch_l2_2d(&tmB, k0, nb_ + h * C::MMA_N);
-                    }
-                }
-            };
-            auto origin = [&](int tile, int &m0_, int &nb_) {
-                int tm, tn;
-                tile_coords(p, tile, tm, tn);
-                m0_ = tm * (C::BM * C::CG) + (int)rank * C::BM;
-                // local B row r (MMA half h = r / MMA_N_LOCAL) holds global column
-                // tn*BN + h*MMA_N + rank*MMA_N_LOCAL + r % MMA_N_LOCAL
-                nb_ = tn * C::BN + (int)rank * C::MMA_N_LOCAL;
-            };
             WorkIter it(p, unit, units);
             WorkItem w;
             while (ok && it.next(p, units, w)) {
@@ -712,6 +728,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         WorkIter it(p, unit, units);
         WorkItem w;
         while (ok && it.next(p, units, w)) {
+            // the unit's last work item: its MMAs are the last to read the operand ring, so once
+            // its accumulator is complete the ring can hold the output staging
+            WorkIter peek = it;
+            WorkItem wn;
+            const bool last_item = !peek.next(p, units, wn);
             // partial_out: this unit holds a non-final slice of the tile -> publish a partial.
             // Otherwise units [c_first, unit) published the slices before ours.
             const bool partial_out = w.kb1 < p.num_kb;
@@ -872,10 +893,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         }
                     } else {
                         // stage 32 rows x 32 outputs in the 64-byte swizzled layout the TMA store reads:
-                        // 16-byte piece j of row r sits at r*64 + ((j ^ ((r >> 1) & 3)) * 16)
-                        if (lane == 0) ptx::bulk_wait_read<0>();     // previous store has read the buffer
-                        __syncwarp();
+                        // 16-byte piece j of row r sits at r*64 + ((j ^ ((r >> 1) & 3)) * 16).  The
+                        // unit's last tile stages every chunk in its own 2 KB of the (by then idle)
+                        // operand ring, so no chunk waits for the previous one's store to be read;
+                        // otherwise the warp's single staging buffer is reused.
+                        uint32_t stg_c = stg;
                         uint8_t *stg_row = smem + C::OFF_STG + ew * C::STG_BYTES + lane * 64;
+                        if (last_item) {
+                            const int slot = ew * C::NCH_W + cl;
+                            stg_c = sA + slot * 2048;
+                            stg_row = smem + C::OFF_A + slot * 2048 + lane * 64;
+                        } else if (lane == 0) {
+                            ptx::bulk_wait_read<0>();     // previous store has read the buffer
+                        }
+                        __syncwarp();
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const int piece = i ^ ((lane >> 1) & 3);
@@ -886,7 +917,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         __syncwarp();
                         // boxes starting past the last row or column hold nothing to store
                         if (lane == 0 && m0 + 32 * q < p.m && col0 < p.n) {
-                            ptx::tma_store_2d_hint(&tmD, stg, col0, m0 + 32 * q, pol_d);
+                            ptx::tma_store_2d_hint(&tmD, stg_c, col0, m0 + 32 * q, pol_d);
                             ptx::bulk_commit();
                         }
                     }
