@@ -51,6 +51,7 @@ struct Plan {
     int group_m, group_n = 0;   // TC raster (TcParams::group_m / group_n)
     int l2_mode = 1;     // TcParams::l2_mode (GEMM_EPI_L2=0/1/2 overrides)
     int prefetch = 0;    // TcParams::prefetch (GEMM_EPI_PREFETCH=n overrides)
+    bool fused = false;  // TcParams::fused: stage-wide 3-D / 4-D operand copies (GEMM_EPI_FUSED_COPIES=0 disables)
     bool pdl;            // programmatic dependent launch (GEMM_EPI_PDL=0 turns it off)
     // split tail (TC kernels): tiles [0, sk_tiles) cut along k into sk_split parts
     int sk_tiles = 0, sk_split = 0;
@@ -147,6 +148,19 @@ bool make_map(CUtensorMap *map, int dt, const void *ptr, int64_t inner, int64_t 
     CUresult r = fn(map, tmap_type(dt), 2, const_cast<void *>(ptr), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// N-D view (rank 3 or 4) of a row-major tensor, 128-byte swizzle: dims[0] is contiguous,
+// strides_bytes[i] is the byte distance between consecutive indices of dims[i + 1].
+bool make_map_nd(CUtensorMap *map, int dt, const void *ptr, uint32_t rank, const cuuint64_t *dims,
+                 const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, tmap_type(dt), rank, const_cast<void *>(ptr), dims, strides_bytes, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -330,6 +344,18 @@ int choose(Plan *P) {
             const int v = atoi(g);
             if (v >= 0 && v <= 64) P->prefetch = v;
         }
+        // Stage-wide copies: a ring stage of A (all its k-atoms) and of each MMA half of B lands
+        // with one 3-D / 4-D copy instead of one copy per 128-byte box.  The N-D views split k
+        // into atoms (and n or m into 128-byte blocks for an MN-major operand), so those extents
+        // must divide exactly; otherwise the 2-D maps are used.
+        {
+            const int64_t box_el = 128 / esize(P->dtype);
+            const bool ok_k = P->k % bk == 0;
+            const bool ok_b = !b_mn || n % box_el == 0;
+            const bool ok_a = !P->a_km || m % box_el == 0;
+            const char *g = getenv("GEMM_EPI_FUSED_COPIES");
+            P->fused = ok_k && ok_b && ok_a && !(g && g[0] == '0');
+        }
         KernelInfo none_info;
         if (!find_tc(cg, P->dtype, GEMM_EPI_NONE, 0, b_mn, bn, false, P->a_km, &P->tc_none_launch, &none_info))
             return GEMM_EPI_ERR_UNSUPPORTED;
@@ -420,8 +446,37 @@ int ensure_maps(Plan *P, const void *A, const void *B, void *D) {
     } else {
         const int cg = P->kernel == GEMM_EPI_KERNEL_TC2 ? 2 : 1;
         const int bn_local = std::min(P->block_n, 256) / cg;   // B rows of one MMA in this CTA
-        ok = ok && (P->a_km ? make_map(&P->tmA, dt, A, m, k, box_n, bk) : make_map(&P->tmA, dt, A, k, m, bk, 128));
-        ok = ok && (b_kn ? make_map(&P->tmB, dt, B, n, k, box_n, bk) : make_map(&P->tmB, dt, B, k, n, bk, bn_local));
+        if (P->fused) {
+            // stage-wide views: [atom][row][128 B] for a K-major operand, [atom][block][k row][128 B]
+            // for an MN-major one -- the shared-memory layout of the 2-D copies, in one copy
+            const int es = esize(dt);
+            const cuuint32_t ka = (cuuint32_t)P->katoms;
+            if (P->a_km) {
+                const cuuint64_t d[4] = {(cuuint64_t)box_n, (cuuint64_t)bk, (cuuint64_t)(m / box_n), (cuuint64_t)(k / bk)};
+                const cuuint64_t st[3] = {(cuuint64_t)(m * es), 128, (cuuint64_t)(bk * m * es)};
+                const cuuint32_t bx[4] = {(cuuint32_t)box_n, (cuuint32_t)bk, (cuuint32_t)(128 / box_n), ka};
+                ok = ok && make_map_nd(&P->tmA, dt, A, 4, d, st, bx);
+            } else {
+                const cuuint64_t d[3] = {(cuuint64_t)bk, (cuuint64_t)m, (cuuint64_t)(k / bk)};
+                const cuuint64_t st[2] = {(cuuint64_t)(k * es), (cuuint64_t)(bk * es)};
+                const cuuint32_t bx[3] = {(cuuint32_t)bk, 128, ka};
+                ok = ok && make_map_nd(&P->tmA, dt, A, 3, d, st, bx);
+            }
+            if (b_kn) {
+                const cuuint64_t d[4] = {(cuuint64_t)box_n, (cuuint64_t)bk, (cuuint64_t)(n / box_n), (cuuint64_t)(k / bk)};
+                const cuuint64_t st[3] = {(cuuint64_t)(n * es), 128, (cuuint64_t)(bk * n * es)};
+                const cuuint32_t bx[4] = {(cuuint32_t)box_n, (cuuint32_t)bk, (cuuint32_t)(bn_local / box_n), ka};
+                ok = ok && make_map_nd(&P->tmB, dt, B, 4, d, st, bx);
+            } else {
+                const cuuint64_t d[3] = {(cuuint64_t)bk, (cuuint64_t)n, (cuuint64_t)(k / bk)};
+                const cuuint64_t st[2] = {(cuuint64_t)(k * es), (cuuint64_t)(bk * es)};
+                const cuuint32_t bx[3] = {(cuuint32_t)bk, (cuuint32_t)bn_local, ka};
+                ok = ok && make_map_nd(&P->tmB, dt, B, 3, d, st, bx);
+            }
+        } else {
+            ok = ok && (P->a_km ? make_map(&P->tmA, dt, A, m, k, box_n, bk) : make_map(&P->tmA, dt, A, k, m, bk, 128));
+            ok = ok && (b_kn ? make_map(&P->tmB, dt, B, n, k, box_n, bk) : make_map(&P->tmB, dt, B, k, n, bk, bn_local));
+        }
         const int out_dt = dt == GEMM_EPI_E4M3 ? GEMM_EPI_BF16 : dt;
         if (P->qout)   // e4m3 output goes out with direct stores; the map is valid but unused
             ok = ok && make_map(&P->tmD, GEMM_EPI_E4M3, D, n, m, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -530,6 +585,7 @@ int launch_main(Plan *P, bool fused, const void *bias, void *D, uint32_t *aux, c
         L.p.amax = reinterpret_cast<unsigned int *>(P->amax);
         L.p.l2_mode = P->l2_mode;
         L.p.prefetch = P->prefetch;
+        L.p.fused = P->fused ? 1 : 0;
         L.grid = P->grid;
         L.pdl = P->pdl;
         L.stream = stream;

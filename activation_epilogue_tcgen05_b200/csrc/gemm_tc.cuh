@@ -107,6 +107,9 @@ struct TcParams {
     const float *out_scale;
     unsigned int *amax;
     int prefetch;                // producer: L2 prefetch of the stage this many stages ahead (0: none)
+    // 1: tmA / tmB are 3-D / 4-D views that land a whole ring stage of an operand (all its
+    // k-atoms and 128-byte boxes) with one copy; 0: 2-D maps, one copy per box
+    int fused;
     // L2 cache policy: 0 = normal for every access; 1 = the outputs (D, mask) are written
     // evict-first, so that streaming them out does not push the operands out of L2; 2 = as 1,
     // and the operands are loaded evict-last
@@ -436,6 +439,7 @@ struct TcCfg {
     static_assert(!A_MN || BM % A_BOX_M == 0, "MN-major A tile must be whole boxes");
     static_assert(EPI_WARPS * NCH_W * 2048 <= STAGES * (A_STAGE + B_STAGE),
                   "the last tile's output staging fits in the operand ring");
+    static_assert(KATOMS == 1 || N_MMAS == 1, "a stage-wide copy of B lands its atoms one after another");
 };
 
 // Tile index -> (tile_m, tile_n) with a grouped raster.  group_n == 0: groups of group_m
@@ -515,6 +519,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // L2 prefetch of stage kb of the tile at (m0_, nb_): the same boxes as its loads, no
     // shared-memory destination, no barrier (only a hint to L2)
     auto prefetch_stage = [&](int m0_, int nb_, int kb_) {
+        if (p.fused) {
+            if constexpr (C::A_MN) ptx::tma_prefetch_l2_4d(&tmA, 0, 0, m0_ / C::A_BOX_M, kb_ * C::KATOMS);
+            else ptx::tma_prefetch_l2_3d(&tmA, 0, m0_, kb_ * C::KATOMS);
+#pragma unroll
+            for (int h = 0; h < C::N_MMAS; ++h) {
+                if constexpr (C::B_MN) ptx::tma_prefetch_l2_4d(&tmB, 0, 0, (nb_ + h * C::MMA_N) / C::B_BOX_N, kb_ * C::KATOMS);
+                else ptx::tma_prefetch_l2_3d(&tmB, 0, nb_ + h * C::MMA_N, kb_ * C::KATOMS);
+            }
+            return;
+        }
 #pragma unroll
         for (int at = 0; at < C::KATOMS; ++at) {
             const int k0 = (kb_ * C::KATOMS + at) * C::BK;
@@ -590,6 +604,43 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         break;
                     }
                     trace_stage(p.trace, 0, tr_i, 20, w.tile, kb);
+                    if (p.fused) {
+                        // one copy per operand (per MMA half of B) for the whole stage, counted on
+                        // the stage's first full barrier; the other atoms' barriers get a plain arrive
+                        uint32_t fb = full_bar(stage, 0);
+                        if constexpr (C::CG == 2) {
+                            fb = ptx::mapa(fb, 0);
+                            if (leader) {
+                                ptx::mbar_arrive_expect_tx(full_bar(stage, 0), 2 * (C::A_STAGE + C::B_STAGE));
+                                for (int at = 1; at < C::KATOMS; ++at) ptx::mbar_arrive(full_bar(stage, at));
+                            }
+                        } else {
+                            ptx::mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE);
+                            for (int at = 1; at < C::KATOMS; ++at) ptx::mbar_arrive(full_bar(stage, at));
+                        }
+                        const uint32_t a_dst = sA + stage * C::A_STAGE;
+                        const uint32_t b_dst = sB + stage * C::B_STAGE;
+                        const int a0 = kb * C::KATOMS;          // first k-atom of the stage
+                        if constexpr (C::CG == 2) {
+                            if constexpr (C::A_MN) ptx::tma_load_4d_pair(a_dst, &tmA, fb, 0, 0, m0 / C::A_BOX_M, a0, pol_ab);
+                            else ptx::tma_load_3d_pair(a_dst, &tmA, fb, 0, m0, a0, pol_ab);
+                        } else {
+                            if constexpr (C::A_MN) ptx::tma_load_4d(a_dst, &tmA, fb, 0, 0, m0 / C::A_BOX_M, a0, pol_ab);
+                            else ptx::tma_load_3d(a_dst, &tmA, fb, 0, m0, a0, pol_ab);
+                        }
+#pragma unroll
+                        for (int h = 0; h < C::N_MMAS; ++h) {
+                            const uint32_t bd = b_dst + h * C::HALF_B_BYTES;
+                            const int n1 = nb + h * C::MMA_N;
+                            if constexpr (C::CG == 2) {
+                                if constexpr (C::B_MN) ptx::tma_load_4d_pair(bd, &tmB, fb, 0, 0, n1 / C::B_BOX_N, a0, pol_ab);
+                                else ptx::tma_load_3d_pair(bd, &tmB, fb, 0, n1, a0, pol_ab);
+                            } else {
+                                if constexpr (C::B_MN) ptx::tma_load_4d(bd, &tmB, fb, 0, 0, n1 / C::B_BOX_N, a0, pol_ab);
+                                else ptx::tma_load_3d(bd, &tmB, fb, 0, n1, a0, pol_ab);
+                            }
+                        }
+                    } else
                     for (int at = 0; at < C::KATOMS; ++at) {    // the stage's k-atoms
                     uint32_t fb = full_bar(stage, at);
                     if constexpr (C::CG == 2) {
