@@ -51,7 +51,7 @@ struct Plan {
     int group_m, group_n = 0;   // TC raster (TcParams::group_m / group_n)
     int l2_mode = 1;     // TcParams::l2_mode (GEMM_EPI_L2=0/1/2 overrides)
     int prefetch = 0;    // TcParams::prefetch (GEMM_EPI_PREFETCH=n overrides)
-    bool fused = false;  // TcParams::fused: stage-wide 3-D / 4-D operand copies (GEMM_EPI_FUSED_COPIES=0 disables)
+    bool fused = false;  // TcParams::fused: stage-wide 3-D / 4-D operand copies (GEMM_EPI_FUSED_COPIES=1 enables)
     bool pdl;            // programmatic dependent launch (GEMM_EPI_PDL=0 turns it off)
     // split tail (TC kernels): tiles [0, sk_tiles) cut along k into sk_split parts
     int sk_tiles = 0, sk_split = 0;
@@ -213,7 +213,7 @@ int choose(Plan *P) {
     const int64_t num_kb = (P->k + bk - 1) / bk;
     const int sms = P->opts.max_ctas > 0 ? std::min(P->opts.max_ctas, P->num_sms) : P->num_sms;
 
-    if (kernel == GEMM_EPI_KERNEL_SPLITK && !P->no_workspace && !getenv_flag("GEMM_EPI_SK_CLUSTER")) {
+    if (kernel == GEMM_EPI_KERNEL_SPLITK && !P->no_workspace && getenv_flag("GEMM_EPI_SK_GRID")) {
         // grid-wide form: every SM takes an equal share of the (tile, k-block) units; a split
         // tile is finished by the CTA holding its first k-block, from partials the others
         // publish in a plan-owned workspace
@@ -353,8 +353,10 @@ int choose(Plan *P) {
             const bool ok_k = P->k % bk == 0;
             const bool ok_b = !b_mn || n % box_el == 0;
             const bool ok_a = !P->a_km || m % box_el == 0;
+            // Off unless GEMM_EPI_FUSED_COPIES=1: at 4096^3 the per-atom full barriers of the 2-D
+            // copies turn a stage over faster (1110 against 1160 SM clocks on average).
             const char *g = getenv("GEMM_EPI_FUSED_COPIES");
-            P->fused = ok_k && ok_b && ok_a && !(g && g[0] == '0');
+            P->fused = ok_k && ok_b && ok_a && g && g[0] == '1';
         }
         KernelInfo none_info;
         if (!find_tc(cg, P->dtype, GEMM_EPI_NONE, 0, b_mn, bn, false, P->a_km, &P->tc_none_launch, &none_info))

@@ -275,8 +275,10 @@ def test_splitk_variants(m, dtype, epilogue, axis, layout):
 
 
 @pytest.mark.parametrize("split", [1, 2, 3, 8])
-def test_splitk_parts_per_tile(split):
-    """The grid-wide split-K form with split_k parts per tile (1 = whole tiles, no reduction)."""
+def test_splitk_grid_parts_per_tile(split, monkeypatch):
+    """The grid-wide split-K form (GEMM_EPI_SK_GRID=1) with split_k parts per tile (1 = whole
+    tiles, no reduction)."""
+    monkeypatch.setenv("GEMM_EPI_SK_GRID", "1")
     wl = Workload("sk_split", 16, 512, 2048, "f16", "gelu_bias", "col", "nk", seed=6,
                   dist_b=("uniform", 1 / 64), dist_bias=("uniform", 1 / 64))
     prob = make_problem(wl)
@@ -287,9 +289,10 @@ def test_splitk_parts_per_tile(split):
 
 @pytest.mark.parametrize("ctas", [1, 3, 5, 7, 37, 100])
 @pytest.mark.parametrize("epilogue", ["relu_aux_bias", "gelu_bias"])
-def test_splitk_uneven_ranges(ctas, epilogue):
-    """Ranges of units that cut tiles at arbitrary k-blocks, and (few CTAs) ranges that span
-    several whole and partial tiles: every piece's partial must be added exactly once."""
+def test_splitk_grid_uneven_ranges(ctas, epilogue, monkeypatch):
+    """Grid-wide form: ranges of units that cut tiles at arbitrary k-blocks, and (few CTAs)
+    ranges that span several whole and partial tiles: every piece's partial is added once."""
+    monkeypatch.setenv("GEMM_EPI_SK_GRID", "1")
     wl = Workload("sk_ranges", 24, 656, 1000, "bf16", epilogue, "col", "kn", seed=16)
     prob = make_problem(wl)
     worst, info = check_against_oracle(wl, prob, kernel="splitk", max_ctas=ctas)
@@ -298,16 +301,35 @@ def test_splitk_uneven_ranges(ctas, epilogue):
 
 
 @pytest.mark.parametrize("split", [1, 2, 3, 8])
-def test_splitk_cluster_form(split, monkeypatch):
-    """The cluster form (partials reduced through distributed shared memory, no workspace):
-    what the allocation-free entry point runs for small m; GEMM_EPI_SK_CLUSTER=1 selects it
-    for a plan."""
-    monkeypatch.setenv("GEMM_EPI_SK_CLUSTER", "1")
+def test_splitk_cluster_sizes(split):
+    """The cluster form (partials reduced through distributed shared memory, no workspace),
+    the default for small m and what the allocation-free entry point runs."""
     wl = Workload("sk_cluster", 16, 512, 2048, "f16", "gelu_bias", "col", "nk", seed=6,
                   dist_b=("uniform", 1 / 64), dist_bias=("uniform", 1 / 64))
     prob = make_problem(wl)
     worst, info = check_against_oracle(wl, prob, kernel="splitk", split_k=split)
     assert info["split_k"] == split and info["cluster"] == split
+    assert worst <= 1.0
+
+
+@pytest.mark.parametrize("kernel,block_n", [("tc1", 128), ("tc1", 256), ("tc2", 256), ("tc2", 512)])
+@pytest.mark.parametrize("dtype,b_layout,a_layout", [("bf16", "kn", "mk"), ("f16", "nk", "mk"), ("bf16", "kn", "km"),
+                                                     ("e4m3", "kn", "mk"), ("e4m3", "nk", "km")])
+def test_stage_wide_copies(kernel, block_n, dtype, b_layout, a_layout, monkeypatch):
+    """GEMM_EPI_FUSED_COPIES=1: one 3-D / 4-D copy per operand and ring stage (k a multiple of the
+    128-byte atom, n and m of 128-byte blocks), several tiles and an odd k-atom count so that the
+    last stage's second atom lies past k."""
+    if block_n == 512 and (dtype == "e4m3" or a_layout == "km"):
+        pytest.skip("512-wide tiles: 16-bit operands, A stored (m, k)")
+    if a_layout == "km" and block_n != 256:
+        pytest.skip("A stored (k, m): 256-wide tiles")
+    monkeypatch.setenv("GEMM_EPI_FUSED_COPIES", "1")
+    k = 640 if dtype == "e4m3" else 320          # 5 k-atoms of 128 bytes
+    wl = Workload("fused", 512, 640 if block_n == 512 else 384, k, dtype, "relu_aux_bias", "row", b_layout,
+                  seed=26, a_layout=a_layout)
+    prob = make_problem(wl)
+    worst, info = check_against_oracle(wl, prob, kernel=kernel, block_n=block_n)
+    assert info["block_n"] == block_n
     assert worst <= 1.0
 
 

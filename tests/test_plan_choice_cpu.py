@@ -37,13 +37,21 @@ def test_small_gemm_bias_1024x512x2048(g):
 
 def test_linear_gelu_batch16_splitk(g):
     p = pv(g, 16, 4096, 4096, "f16", "gelu_bias", "col", "nk")
-    # swapped roles: 32 weight tiles of 128 rows x 64 k-blocks; every SM takes an equal range
-    # of the 2048 (tile, k-block) units (13 or 14), so a tile is cut into 5 or 6 pieces
+    # swapped roles: 32 weight tiles of 128 rows, K split over clusters of 4 CTAs
+    assert (p["kernel"], p["block_m"], p["split_k"], p["cluster"], p["grid"]) == (g.KERNEL_SPLITK, 16, 4, 4, 128)
+
+
+def test_linear_gelu_batch16_splitk_grid_form(g, monkeypatch):
+    monkeypatch.setenv("GEMM_EPI_SK_GRID", "1")
+    p = pv(g, 16, 4096, 4096, "f16", "gelu_bias", "col", "nk")
+    # every SM takes an equal range of the 2048 (tile, k-block) units (13 or 14), so a tile is
+    # cut into 5 or 6 pieces
     assert (p["kernel"], p["block_m"], p["cluster"], p["grid"]) == (g.KERNEL_SPLITK, 16, 1, 148)
     assert p["split_k"] == 5 and p["stages"] == 11
 
 
-def test_splitk_grid_follows_split_k_and_max_ctas(g):
+def test_splitk_grid_follows_split_k_and_max_ctas(g, monkeypatch):
+    monkeypatch.setenv("GEMM_EPI_SK_GRID", "1")
     # split_k caps the k-parts per tile: the grid is tiles x split_k
     p = pv(g, 16, 4096, 4096, "f16", "gelu_bias", "col", "nk", split_k=2)
     assert (p["grid"], p["split_k"]) == (64, 2)
