@@ -391,6 +391,11 @@ struct TcCfg {
     static constexpr int MMA_N_LOCAL = MMA_N / CG;           // B rows of one MMA in this CTA
     static constexpr int HALF_B_BYTES = MMA_N_LOCAL * 128;   // shared-memory bytes of those rows
     static constexpr int NUM_ACC = BN <= 256 ? 2 : 1;        // accumulators in tensor memory
+    // One accumulator in two halves (a 512-wide pair tile, forward epilogues): the epilogue
+    // drains columns 0-255 first and hands them back (tempty barrier 0), then 256-511 (barrier 1).
+    // The next tile's MMAs start on the first half and keep each stage's shared memory until
+    // the second half is free, then issue the deferred second-half MMAs in order.
+    static constexpr bool SPLIT_HALVES = NUM_ACC == 1 && N_MMAS == 2;
     static constexpr int B_BOX_BYTES = B_MN ? BK * 128 : B_BYTES;
     static constexpr int A_BOX_M = 128 / ESIZE;     // m per 128-byte MN-major box
     static constexpr int A_BOXES = A_MN ? BM / A_BOX_M : 1;
@@ -441,6 +446,20 @@ struct TcCfg {
                   "the last tile's output staging fits in the operand ring");
     static_assert(KATOMS == 1 || N_MMAS == 1, "a stage-wide copy of B lands its atoms one after another");
 };
+
+// The tile's 32-column chunk that chunk cl of epilogue warp ew covers.  Two warps share each TMEM
+// lane quadrant and split its columns; with SPLIT_HALVES each takes a quarter of either half,
+// first-half chunks first, so the first half is read out before the second.
+template <class C>
+__device__ __forceinline__ int chunk_of(int ew, int cl) {
+    if constexpr (C::SPLIT_HALVES) {
+        constexpr int H = C::NCH_W / 2;            // chunks a warp takes from each half
+        constexpr int HALF = C::MMA_N / 32;        // chunks in a half
+        return cl < H ? (ew >> 2) * H + cl : HALF + (ew >> 2) * H + (cl - H);
+    } else {
+        return (ew >> 2) * C::NCH_W + cl;
+    }
+}
 
 // Tile index -> (tile_m, tile_n) with a grouped raster.  group_n == 0: groups of group_m
 // tile-rows, each walked column by column, so the group's A panels are reused by every
@@ -718,6 +737,47 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 trace_event(p.trace, warp, 3, w.tile, w.kb0);
                 trace_stage(p.trace, 1, tr_i, 25, w.tile, w.kb0);
                 const uint32_t d_tmem = tmem_base + acc * C::BN;
+                // the MMAs of k-atom `at` of ring stage `st` (this tile's stage kb_) into halves [h_lo, h_hi)
+                auto issue_atom = [&](uint32_t st, int kb_, int at, int h_lo, int h_hi) {
+                    const uint32_t a_base = sA + st * C::A_STAGE + at * C::A_BYTES;
+                    const uint32_t b_base = sB + st * C::B_STAGE + at * C::B_BYTES;
+#pragma unroll
+                    for (int ks = 0; ks < C::KSTEPS; ++ks) {
+                        const uint64_t ad = C::A_MN ? make_sdesc(a_base + ks * C::UMMA_K * 128, C::A_BOX_BYTES, 1024)
+                                                    : make_sdesc(a_base + ks * 32, 16, 1024);
+#pragma unroll
+                        for (int h = 0; h < C::N_MMAS; ++h) {
+                            if (h < h_lo || h >= h_hi) continue;
+                            const uint32_t bh = b_base + h * C::HALF_B_BYTES;
+                            const uint64_t bd = C::B_MN ? make_sdesc(bh + ks * C::UMMA_K * 128, C::B_BOX_BYTES, 1024)
+                                                        : make_sdesc(bh + ks * 32, 16, 1024);
+                            ptx::mma<C::CG, C::KIND>(d_tmem + h * C::MMA_N, ad, bd, idesc,
+                                                     (kb_ > w.kb0 || at > 0 || ks > 0) ? 1u : 0u);
+                        }
+                    }
+                };
+                auto release = [&](uint32_t st) {
+                    if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(empty_bar(st), 0x3);
+                    else ptx::mma_commit(empty_bar(st));
+                };
+                // SPLIT_HALVES: is the accumulator's second half free yet?  Stages whose second-half
+                // MMAs wait for it (in order; their ring slots are not released meanwhile).
+                bool h1_free = !C::SPLIT_HALVES;
+                uint32_t def_st[C::STAGES];
+                int def_kb[C::STAGES];
+                int ndef = 0;
+                auto flush = [&]() {
+                    for (int i = 0; i < ndef; ++i) {
+#pragma unroll
+                        for (int at = 0; at < C::KATOMS; ++at) issue_atom(def_st[i], def_kb[i], at, 1, 2);
+                        release(def_st[i]);
+                    }
+                    ndef = 0;
+                };
+                auto h1_probe = [&]() {
+                    return C::CG == 2 ? ptx::mbar_test_wait_cluster(tempty_bar(1), acc_phase ^ 1u)
+                                      : ptx::mbar_test_wait(tempty_bar(1), acc_phase ^ 1u);
+                };
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
 #pragma unroll
                     for (int at = 0; at < C::KATOMS; ++at) {
@@ -727,26 +787,47 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                     if (at == 0) trace_stage(p.trace, 1, tr_i, 22, w.tile, kb);
                     ptx::tc_fence_after();
-                    const uint32_t a_base = sA + stage * C::A_STAGE + at * C::A_BYTES;
-                    const uint32_t b_base = sB + stage * C::B_STAGE + at * C::B_BYTES;
-#pragma unroll
-                    for (int ks = 0; ks < C::KSTEPS; ++ks) {
-                        const uint64_t ad = C::A_MN ? make_sdesc(a_base + ks * C::UMMA_K * 128, C::A_BOX_BYTES, 1024)
-                                                    : make_sdesc(a_base + ks * 32, 16, 1024);
-#pragma unroll
-                        for (int h = 0; h < C::N_MMAS; ++h) {
-                            const uint32_t bh = b_base + h * C::HALF_B_BYTES;
-                            const uint64_t bd = C::B_MN ? make_sdesc(bh + ks * C::UMMA_K * 128, C::B_BOX_BYTES, 1024)
-                                                        : make_sdesc(bh + ks * 32, 16, 1024);
-                            ptx::mma<C::CG, C::KIND>(d_tmem + h * C::MMA_N, ad, bd, idesc,
-                                                     (kb > w.kb0 || at > 0 || ks > 0) ? 1u : 0u);
-                        }
-                    }
+                    issue_atom(stage, kb, at, 0, h1_free ? C::N_MMAS : 1);
                     }
                     if (!ok) break;
-                    if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(empty_bar(stage), 0x3);
-                    else ptx::mma_commit(empty_bar(stage));
+                    if constexpr (C::SPLIT_HALVES) {
+                        if (!h1_free && h1_probe()) {
+                            h1_free = true;
+                            ptx::tc_fence_after();
+                            flush();
+                            // this stage's first half went out above; now its second half
+#pragma unroll
+                            for (int at = 0; at < C::KATOMS; ++at) issue_atom(stage, kb, at, 1, 2);
+                            release(stage);
+                        } else if (!h1_free) {
+                            def_st[ndef] = stage;
+                            def_kb[ndef] = kb;
+                            if (++ndef == C::STAGES) {
+                                // every ring slot is held: wait for the second half
+                                if (!wait_bounded<C::CG == 2>(tempty_bar(1), acc_phase ^ 1u, abort_flag, p.status,
+                                                              ST_TIMEOUT_MMA)) {
+                                    ok = false;
+                                    break;
+                                }
+                                ptx::tc_fence_after();
+                                h1_free = true;
+                                flush();
+                            }
+                        } else {
+                            release(stage);
+                        }
+                    } else {
+                        release(stage);
+                    }
                     if (++stage == (uint32_t)C::STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (ok && ndef > 0) {
+                    if (!wait_bounded<C::CG == 2>(tempty_bar(1), acc_phase ^ 1u, abort_flag, p.status, ST_TIMEOUT_MMA)) {
+                        ok = false;
+                    } else {
+                        ptx::tc_fence_after();
+                        flush();
+                    }
                 }
                 if (!ok) break;
                 if constexpr (C::CG == 2) ptx::mma_commit_pair_mc(tfull_bar(acc), 0x3);
@@ -813,20 +894,25 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if constexpr (C::BIAS_FLOATS > 0) if (!partial_out) {
                 // this warp's copy of bias[nw .. nw+COLS_W) as fp32 (read once per tile)
                 __syncwarp();
+                // (bsm[j] holds the bias of the warp's j-th column: chunk j / 32, column j % 32)
                 if (!has_bias) {
                     for (int j = lane; j < C::COLS_W; j += 32) bsm[j] = 0.0f;
-                } else if (nw + C::COLS_W <= p.n) {
+                } else {
 #pragma unroll
                     for (int j = lane * 8; j < C::COLS_W; j += 256) {
-                        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
-                            reinterpret_cast<const typename O::type *>(p.bias) + nw + j));
-                        float f[8];
-                        unpack8<C::DT == DT_F16 ? DT_F16 : DT_BF16>(u, f);
+                        const int col = n0 + 32 * chunk_of<C>(ew, j >> 5) + (j & 31);
+                        if (col + 8 <= p.n) {
+                            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
+                                reinterpret_cast<const typename O::type *>(p.bias) + col));
+                            float f[8];
+                            unpack8<C::DT == DT_F16 ? DT_F16 : DT_BF16>(u, f);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) bsm[j + e] = f[e];
+                            for (int e = 0; e < 8; ++e) bsm[j + e] = f[e];
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) bsm[j + e] = col + e < p.n ? O::load(p.bias, col + e) : 0.0f;
+                        }
                     }
-                } else {
-                    for (int j = lane; j < C::COLS_W; j += 32) bsm[j] = nw + j < p.n ? O::load(p.bias, nw + j) : 0.0f;
                 }
                 __syncwarp();
             }
@@ -850,18 +936,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const uint4 mk = g == 0 ? mk0 : mk1;
 #pragma unroll
                 for (int cc = 0; cc < C::CPG; ++cc) {          // 32 columns per chunk
-                    const int c = cbase + C::CPG * g + cc;     // chunk index within the tile
-                    const int cl = c - cbase;                  // chunk index within this warp
+                    const int cl = C::CPG * g + cc;            // chunk index within this warp
+                    const int c = chunk_of<C>(ew, cl);         // chunk index within the tile
                     uint32_t v[32];
                     ptx::tmem_ld_32x32b_x32(tbase + c * 32, v);
                     ptx::tmem_wait_ld(v);
-                    if (cc == C::CPG - 1 && g == C::NCH_W / C::CPG - 1) {
-                        // accumulator fully read by this warp: hand it back to the MMA issuer
+                    // accumulator (or, SPLIT_HALVES, one half of it) fully read by this warp: hand
+                    // it back to the MMA issuer
+                    const bool last_chunk = cc == C::CPG - 1 && g == C::NCH_W / C::CPG - 1;
+                    const bool half_done = C::SPLIT_HALVES && cl == C::NCH_W / 2 - 1;
+                    if (last_chunk || half_done) {
+                        const uint32_t tb = tempty_bar(C::SPLIT_HALVES ? (last_chunk ? 1 : 0) : (int)acc);
                         ptx::tc_fence_before();
                         __syncwarp();
                         if (lane == 0) {
-                            if constexpr (C::CG == 2) ptx::mbar_arrive_cluster(ptx::mapa(tempty_bar(acc), 0));
-                            else ptx::mbar_arrive(tempty_bar(acc));
+                            if constexpr (C::CG == 2) ptx::mbar_arrive_cluster(ptx::mapa(tb, 0));
+                            else ptx::mbar_arrive(tb);
                         }
                     }
                     if (partial_out) {
@@ -995,7 +1085,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
                 if (partial_out) continue;
                 if constexpr (C::EPI == EPI_RELU_AUX) {
-                    const int wcol = nw + 32 * C::CPG * g;
+                    const int wcol = n0 + 32 * chunk_of<C>(ew, C::CPG * g);
                     if (row_ok && wcol < p.aux_pitch_words * 32) {      // padding words too (zero bits)
                         uint32_t *dst = p.aux + (int64_t)row * p.aux_pitch_words + wcol / 32;
                         if constexpr (C::CPG == 4)
