@@ -930,6 +930,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if (!ok) break;
             if (lane == 0) trace_event(p.trace, warp, 7, w.tile, c_first);
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + acc * C::BN;
+            // two register buffers: the next chunk's TMEM load is in flight while this one is
+            // processed (CPG is even, so a chunk's buffer is fixed by its position in its group)
+            uint32_t vb[2][32];
+            ptx::tmem_ld_32x32b_x32(tbase + chunk_of<C>(ew, 0) * 32, vb[0]);
 #pragma unroll 1
             for (int g = 0; g < C::NCH_W / C::CPG; ++g) {    // CPG chunks share a mask store
                 uint32_t words[C::CPG];
@@ -938,9 +942,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 for (int cc = 0; cc < C::CPG; ++cc) {          // 32 columns per chunk
                     const int cl = C::CPG * g + cc;            // chunk index within this warp
                     const int c = chunk_of<C>(ew, cl);         // chunk index within the tile
-                    uint32_t v[32];
-                    ptx::tmem_ld_32x32b_x32(tbase + c * 32, v);
-                    ptx::tmem_wait_ld(v);
+                    uint32_t(&v)[32] = vb[cc & 1];
+                    ptx::tmem_wait_ld(v);                      // the only load in flight: this chunk's
+                    if (cl + 1 < C::NCH_W) ptx::tmem_ld_32x32b_x32(tbase + chunk_of<C>(ew, cl + 1) * 32, vb[(cc + 1) & 1]);
                     // accumulator (or, SPLIT_HALVES, one half of it) fully read by this warp: hand
                     // it back to the MMA issuer
                     const bool last_chunk = cc == C::CPG - 1 && g == C::NCH_W / C::CPG - 1;
