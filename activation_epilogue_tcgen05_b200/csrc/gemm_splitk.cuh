@@ -9,19 +9,32 @@
 // batch rows, and the accumulator lane of a thread is one output column.
 // To put enough SMs on the weight stream, K is split over a thread-block
 // cluster of S CTAs: each CTA accumulates its k-range in its own tensor
-// memory, the S-1 partner CTAs push their fp32 partial tiles into the leader
-// CTA's shared memory (distributed shared memory, st.shared::cluster), and
-// after one cluster barrier the leader sums them in rank order and runs the
-// same fused epilogue (scale, bias, ReLU/GELU, sign mask, RNE cast).
-// No global scratch memory is used.
+// memory.  The tile's 128 columns form four groups of 32 (one per epilogue
+// warp); group q is finished by CTA q mod S.  Every CTA sends each group's fp32
+// partial to that group's owner with asynchronous remote stores
+// (st.async into distributed shared memory, counted on the owner's mbarrier),
+// and each owner sums the S partials of its groups in rank order and runs the
+// fused epilogue (scale, bias, ReLU/GELU, sign mask, RNE cast) with all four of
+// its epilogue warps.  No global scratch memory is used.
 #pragma once
 #include "gemm_tc.cuh"
 
 namespace gemm_epi {
 
-// Largest K split the leader's reduction buffer is sized for, and that buffer's size.
+// Largest K split the reduction buffer is sized for.
 constexpr int sk_max_split(int nm) { return nm <= 16 ? 8 : (nm <= 64 ? 4 : 2); }
-constexpr int sk_red_bytes(int nm) { return (sk_max_split(nm) - 1) * 128 * (nm + 4) * 4; }
+// Receive slots a CTA needs: it owns ceil(4/S) column groups (at most) and takes S partials
+// of each; the most over the allowed splits.
+constexpr int sk_red_slots(int nm) {
+    int most = 0;
+    for (int s = 1; s <= sk_max_split(nm); ++s) {
+        const int slots = (4 + s - 1) / s * s;
+        if (slots > most) most = slots;
+    }
+    return most;
+}
+// One slot: a 32-column group's partial, NM rows, as NM/4 blocks of [32 lanes][4 rows] floats.
+constexpr int sk_red_bytes(int nm) { return sk_red_slots(nm) * nm * 128; }
 // Ring depth: fill ~200 KB of shared memory with the reduction buffer and stages, at most 8.
 constexpr int sk_stages(int nm) {
     return (200 * 1024 - sk_red_bytes(nm)) / (128 * 128 + nm * 128) > 8
@@ -46,6 +59,8 @@ struct SkParams {
     const float *out_scale;
     unsigned int *amax;
     unsigned long long *trace;   // timeline records; used only by builds with GEMM_EPI_TRACE=2
+    int pre_kb;                  // k-blocks of this CTA's weight slice asked of L2 before the dependency wait (< 0: all)
+    int pre_x;                   // nonzero: also ask L2 for this CTA's activation slice before that wait
 };
 
 template <int DT_, int EPI_, int AXIS_, bool W_MN_, int NM_, int STAGES_, bool QOUT_ = false>
@@ -66,14 +81,13 @@ struct SkCfg {
     static constexpr int W_BOX_BYTES = W_MN ? BK * 128 : W_BYTES;
     static constexpr int THREADS = 64 + 128;
     static constexpr int TMEM_COLS = NM <= 32 ? 32 : (NM <= 64 ? 64 : 128);
-    static constexpr int RED_STRIDE = NM + 4;       // floats per partial row (padded)
     static constexpr int MAX_SPLIT = sk_max_split(NM);
+    static constexpr int SLOT_BYTES = NM * 128;     // one column group's partial
     static constexpr int OFF_W = 0;
     static constexpr int OFF_X = OFF_W + STAGES * W_BYTES;
     static constexpr int OFF_RED = OFF_X + STAGES * X_BYTES;
-    static constexpr int RED_BYTES_PER_RANK = 128 * RED_STRIDE * 4;
     static constexpr int OFF_BAR = OFF_RED + sk_red_bytes(NM);
-    static constexpr int NUM_BARS = 2 * STAGES + 2;
+    static constexpr int NUM_BARS = 2 * STAGES + 3;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
     static_assert(NM % 16 == 0 && NM >= 16 && NM <= 128, "MMA N for M = 128");
@@ -83,7 +97,8 @@ struct SkCfg {
 };
 
 // grid = tiles_n * S CTAs, cluster (S, 1, 1): cluster c owns output columns
-// [128c, 128c + 128), CTA rank r of it owns k-blocks [r*kb_per_cta, ...).
+// [128c, 128c + 128), CTA rank r of it owns k-blocks [r*kb_per_cta, ...) and finishes the
+// column groups q (32 columns each) with q mod S = r.
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     splitk_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -98,6 +113,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
     const uint32_t tfull = bar0 + 8u * (2 * C::STAGES);
     const uint32_t done_bar = bar0 + 8u * (2 * C::STAGES + 1);
+    const uint32_t red_bar = bar0 + 8u * (2 * C::STAGES + 2);   // partials of this CTA's groups in
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -111,6 +127,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int kb_begin = (int)rank * p.kb_per_cta;
     const int kb_end = min(p.num_kb, kb_begin + p.kb_per_cta);
     const int my_kb = kb_end > kb_begin ? kb_end - kb_begin : 0;
+    // column groups q < 4 with q mod S == rank
+    const int groups = rank < 4u ? (int)((4u - rank + csize - 1u) / csize) : 0;
 
     uint32_t tr_i = 0;
     if (warp == 0 && lane == 0) {
@@ -123,8 +141,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         ptx::mbar_init(tfull, 1);
         ptx::mbar_init(done_bar, 1);
+        ptx::mbar_init(red_bar, 1);
         *abort_flag = 0;
         ptx::fence_mbarrier_init();
+        // the one arrival of red_bar's phase, with the bytes every CTA of the cluster will send
+        if (groups > 0) ptx::mbar_arrive_expect_tx(red_bar, (uint32_t)(groups * (int)csize * C::SLOT_BYTES));
     }
     if (warp == 1) {
         ptx::tmem_alloc<1>(ptx::smem_addr(tmem_slot), C::TMEM_COLS);
@@ -134,12 +155,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    // This CTA's slice of the weight operand is prefetched into L2 before waiting on the
-    // previous grid, so its DRAM latency overlaps that grid's tail.  A prefetch writes
-    // nothing and L2 is the point of coherence, so the loads below still see any value the
-    // previous kernel stores.  Every other global access waits for the previous grid.
+    // peers may send into this CTA's red_bar once they are past the matching wait
+    ptx::cluster_arrive();
+    // This CTA's slice of the weight operand (the first p.pre_kb k-blocks of it, or all) and
+    // optionally of the activations is prefetched into L2 before waiting on the previous
+    // grid, so its DRAM latency overlaps that grid's tail.  A prefetch writes nothing and L2
+    // is the point of coherence, so the loads below still see any value the previous kernel
+    // stores.  Every other global access waits for the previous grid.
     if (warp == 0 && lane == 0) {
-        for (int kb = kb_begin; kb < kb_end; ++kb) {
+        if (p.pre_x)
+            for (int kb = kb_begin; kb < kb_end; ++kb) ptx::tma_prefetch_l2_2d(&tmX, kb * C::BK, 0);
+        const int pre_end = p.pre_kb < 0 ? kb_end : min(kb_end, kb_begin + p.pre_kb);
+        for (int kb = kb_begin; kb < pre_end; ++kb) {
             if constexpr (C::W_MN) {
 #pragma unroll
                 for (int b = 0; b < C::W_BOXES; ++b) ptx::tma_prefetch_l2_2d(&tmW, n0 + b * C::W_BOX_N, kb * C::BK);
@@ -150,6 +177,24 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     ptx::griddep_wait();
     ptx::griddep_launch_dependents();
+
+    // The epilogue's operands other than the partials (column bias of each column group this
+    // CTA finishes, FP8 scales), read now by the epilogue warps, idle until the accumulator is
+    // ready, so that their latency is off the reduction's path.
+    const bool epi = warp >= 2;
+    float cbias[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float alpha = 1.0f, inv_out = 1.0f;
+    if (epi && groups > 0) {
+        if constexpr (C::EPI != EPI_NONE && C::AXIS == AXIS_COL) {
+#pragma unroll
+            for (int gl = 0; gl < 4; ++gl) {
+                const int col = n0 + 32 * ((int)rank + gl * (int)csize) + lane;
+                if (gl < groups && col < p.n && p.bias != nullptr) cbias[gl] = OutT<C::DT>::load(p.bias, col);
+            }
+        }
+        if (p.scale_a != nullptr) alpha = __ldg(p.scale_a) * __ldg(p.scale_b);
+        if constexpr (C::QOUT) inv_out = 1.0f / __ldg(p.out_scale);
+    }
 
     if (warp == 0) {
         if (lane == 0) {
@@ -218,11 +263,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
     // -------------------------------------------------------------- epilogue
     // warps 2..5: thread (q, lane) owns accumulator lane 32q + lane = output column n0 + 32q + lane.
-    const bool epi = warp >= 2;
     const int q = warp & 3;
-    float acc[C::NM];
-    bool have = false;
+    __syncwarp();
+    ptx::cluster_wait();     // every CTA's red_bar is initialised
     if (epi) {
+        float acc[C::NM];
+        bool have = false;
         if (my_kb > 0 && wait_bounded<false>(tfull, 0, abort_flag, p.status, ST_TIMEOUT_SPLITK)) {
             if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 26, tile_n, (int)rank);
             ptx::tc_fence_after();
@@ -241,77 +287,77 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < C::NM; ++j) acc[j] = 0.0f;
         }
-        if (rank != 0) {
-            // push this CTA's partial row into the leader's reduction slot rank-1
-            const uint32_t local = sb + C::OFF_RED + (rank - 1) * C::RED_BYTES_PER_RANK +
-                                   (uint32_t)((32 * q + lane) * C::RED_STRIDE * 4);
-            const uint32_t remote = ptx::mapa(local, 0);
+        // this CTA's partial of group q goes to slot (q / S) * S + rank of the group's owner;
+        // a CTA without work (or after an abort) sends zeros, so every owner's count completes
+        const uint32_t owner = (uint32_t)q % csize;
+        const uint32_t slot = ((uint32_t)q / csize) * csize + rank;
+        const uint32_t dst = ptx::mapa(sb + C::OFF_RED + slot * C::SLOT_BYTES + (uint32_t)lane * 16u, owner);
+        const uint32_t dbar = ptx::mapa(red_bar, owner);
 #pragma unroll
-            for (int j = 0; j < C::NM; j += 4)
-                ptx::st_cluster_v4(remote + j * 4, acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-        }
+        for (int u = 0; u < C::NM / 4; ++u)
+            ptx::st_async_v4(dst + (uint32_t)u * 512u, acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3], dbar);
     }
-    // the leader's column bias, read before the cluster barrier so that its latency hides
-    float cbias = 0.0f;
-    if constexpr (C::EPI != EPI_NONE && C::AXIS == AXIS_COL) {
-        const int col = n0 + 32 * q + lane;
-        if (epi && rank == 0 && col < p.n && p.bias != nullptr) cbias = OutT<C::DT>::load(p.bias, col);
-    }
-    __syncwarp();
-    ptx::tc_fence_before();
-    ptx::cluster_sync();     // partials visible in the leader's shared memory
-    if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 28, tile_n, (int)rank);
 
-    if (epi && rank == 0) {
+    if (epi && groups > 0) {
         using O = OutT<C::DT>;
         using T = typename O::type;
-        const float *red = reinterpret_cast<const float *>(smem + C::OFF_RED);
-        const int row_in_tile = 32 * q + lane;
-        for (uint32_t r = 1; r < csize; ++r) {
-            const float *src = red + (r - 1) * (C::RED_BYTES_PER_RANK / 4) + row_in_tile * C::RED_STRIDE;
-#pragma unroll
-            for (int j = 0; j < C::NM; j += 4) {
-                const float4 f = *reinterpret_cast<const float4 *>(src + j);
-                acc[j] += f.x;
-                acc[j + 1] += f.y;
-                acc[j + 2] += f.z;
-                acc[j + 3] += f.w;
-            }
-        }
-        const int col = n0 + row_in_tile;
-        const bool col_ok = col < p.n;
-        float alpha = 1.0f;
-        if (p.scale_a != nullptr) alpha = __ldg(p.scale_a) * __ldg(p.scale_b);
-        const bool has_bias = p.bias != nullptr;
-        T *D = reinterpret_cast<T *>(p.D);
-        float inv_out = 1.0f, amax_l = 0.0f;
-        if constexpr (C::QOUT) inv_out = 1.0f / __ldg(p.out_scale);
-        // every word of the mask pitch belongs to exactly one warp of one tile;
-        // columns at or past n contribute 0 bits, so padding words come out 0
-        const int64_t word = (n0 + 32 * q) / 32;
-#pragma unroll
-        for (int i = 0; i < C::NM; ++i) {
-            if (i < p.m) {
-                float x = acc[i];
-                x *= alpha;
-                if constexpr (C::EPI != EPI_NONE) {
-                    if constexpr (C::AXIS == AXIS_COL) x += cbias;
-                    else if (has_bias) x += O::load(p.bias, i);
+        const int ew = warp - 2;
+        float amax_l = 0.0f;
+        if (wait_bounded<true>(red_bar, 0, abort_flag, p.status, ST_TIMEOUT_SPLITK)) {
+            if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 28, tile_n, (int)rank);
+            const bool has_bias = p.bias != nullptr;
+            T *D = reinterpret_cast<T *>(p.D);
+            constexpr int QUADS = C::NM / 4;
+            // work units (owned group, block of 4 rows), dealt round-robin to the 4 epilogue warps
+            for (int unit = ew; unit < groups * QUADS; unit += 4) {
+                const int gl = unit / QUADS, u = unit - gl * QUADS;
+                const int col = n0 + 32 * ((int)rank + gl * (int)csize) + lane;
+                const bool col_ok = col < p.n;
+                // the S partials, added in rank order
+                const float *src = reinterpret_cast<const float *>(smem + C::OFF_RED) +
+                                   ((gl * (int)csize) * C::SLOT_BYTES + u * 512 + lane * 16) / 4;
+                float4 sum = *reinterpret_cast<const float4 *>(src);
+                for (uint32_t r = 1; r < csize; ++r) {
+                    const float4 f = *reinterpret_cast<const float4 *>(src + r * (C::SLOT_BYTES / 4));
+                    sum.x += f.x;
+                    sum.y += f.y;
+                    sum.z += f.z;
+                    sum.w += f.w;
                 }
-                if constexpr (C::EPI == EPI_RELU_AUX) {
-                    const uint32_t bits = __ballot_sync(0xFFFFFFFFu, col_ok && x > 0.0f);
-                    if (lane == 0) p.aux[(int64_t)i * p.aux_pitch_words + word] = bits;
-                }
-                const float y = activate<C::EPI>(x);
-                if (col_ok) {
-                    if constexpr (C::QOUT) {
-                        // e4m3 code, round to nearest even, saturating at +-448
-                        amax_l = fmaxf(amax_l, fabsf(y));
-                        p.dq[(int64_t)i * p.n + col] = __nv_cvt_float_to_fp8(y * inv_out, __NV_SATFINITE, __NV_E4M3);
-                    } else if constexpr (C::DT == DT_F16) {
-                        D[(int64_t)i * p.n + col] = __float2half_rn(y);
-                    } else {
-                        D[(int64_t)i * p.n + col] = __float2bfloat16_rn(y);
+                const float part[4] = {sum.x, sum.y, sum.z, sum.w};
+                // every word of the mask pitch belongs to exactly one group of one tile;
+                // columns at or past n contribute 0 bits, so padding words come out 0
+                const int64_t word = (col - lane) / 32;
+                float cb = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (j == gl) cb = cbias[j];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int i = 4 * u + c;
+                    if (i < p.m) {
+                        float x = part[c] * alpha;
+                        if constexpr (C::EPI != EPI_NONE) {
+                            if constexpr (C::AXIS == AXIS_COL) x += cb;
+                            else if (has_bias) x += O::load(p.bias, i);
+                        }
+                        if constexpr (C::EPI == EPI_RELU_AUX) {
+                            const uint32_t bits = __ballot_sync(0xFFFFFFFFu, col_ok && x > 0.0f);
+                            if (lane == 0) p.aux[(int64_t)i * p.aux_pitch_words + word] = bits;
+                        }
+                        const float y = activate<C::EPI>(x);
+                        if (col_ok) {
+                            if constexpr (C::QOUT) {
+                                // e4m3 code, round to nearest even, saturating at +-448
+                                amax_l = fmaxf(amax_l, fabsf(y));
+                                p.dq[(int64_t)i * p.n + col] =
+                                    __nv_cvt_float_to_fp8(y * inv_out, __NV_SATFINITE, __NV_E4M3);
+                            } else if constexpr (C::DT == DT_F16) {
+                                D[(int64_t)i * p.n + col] = __float2half_rn(y);
+                            } else {
+                                D[(int64_t)i * p.n + col] = __float2bfloat16_rn(y);
+                            }
+                        }
                     }
                 }
             }
@@ -319,7 +365,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if constexpr (C::QOUT) {
             // one atomic per warp: the launch's max |y| (non-negative floats order as their bits)
             const unsigned int wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax_l));
-            if (lane == 0 && p.amax != nullptr) atomicMax(p.amax, wmax);
+            if (lane == 0 && p.amax != nullptr && wmax != 0u) atomicMax(p.amax, wmax);
         }
     }
 
@@ -327,6 +373,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncwarp();
     ptx::tc_fence_before();
     __syncthreads();
+    // The cluster's CTAs leave together.  (Each one has already received every byte sent to
+    // it, so nothing is in flight towards its shared memory; the relaxed arrival does not wait
+    // for this thread's global stores.)
+    ptx::cluster_arrive_relaxed();
+    ptx::cluster_wait();
     if (warp == 1) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc<1>(tmem_base, C::TMEM_COLS);

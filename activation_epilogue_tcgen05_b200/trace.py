@@ -37,7 +37,7 @@ LAUNCH_RECS = 256 * 4 * ROLE_CAP
 TRACE_CAP = 1 << 22
 EV = {10: "CTA start", 11: "after the dependency wait", 20: "stage load issued", 22: "stage ready (MMA)",
       23: "last MMA issued", 24: "accumulator wait", 25: "accumulator free", 26: "accumulator ready",
-      27: "epilogue piece done", 28: "after cluster barrier", 29: "CTA end", 30: "finisher: flags seen",
+      27: "epilogue piece done", 28: "partials received", 29: "CTA end", 30: "finisher: flags seen",
       31: "finisher: partials added", 32: "publisher: flag raised"}
 
 
@@ -117,6 +117,46 @@ def summarise_persistent(launches, last=3):
     return lines
 
 
+def _cluster_phases(L):
+    """Per-CTA phase durations of one launch of the cluster form, rank 0 and the rest apart:
+    last MMA issued -> accumulator ready -> the partials of its column groups received ->
+    epilogue done -> end, and the spread of the last-MMA times inside each cluster (what the
+    reduction waits for).  CTAs that finish no column group (ranks >= 4) record no receipt."""
+    import numpy as np
+    at, ck = {}, {}
+    for c, e, t, kb, k in zip(L["cta"].tolist(), L["ev"].tolist(), L["gt"].tolist(), L["kb"].tolist(),
+                              L["clk"].tolist()):
+        d = at.setdefault(c, {})
+        if e in (23, 26, 27, 28, 29, 11):
+            d[e] = t
+            ck.setdefault(c, {})[e] = k
+        if e in (26, 28, 27, 29):
+            d["rank"] = kb
+    ctas = [c for c, d in at.items() if all(e in d for e in (11, 23, 26, 27, 28, 29)) and "rank" in d]
+    if not ctas:
+        return []
+    ranks = sorted({at[c]["rank"] for c in ctas})
+    size = len(ranks)
+    out = [f"  per-CTA phases of that launch (us), p10 / p50 / p90 over CTAs, cluster size {size}:"]
+    for name, e0, e1 in (("release -> last MMA issued", 11, 23), ("last MMA -> accumulator ready", 23, 26),
+                         ("accumulator ready -> partials received", 26, 28),
+                         ("partials received -> epilogue done", 28, 27), ("epilogue done -> CTA end", 27, 29)):
+        for who, sel in (("rank 0", lambda c: at[c]["rank"] == 0), ("others", lambda c: at[c]["rank"] != 0)):
+            x = [(at[c][e1] - at[c][e0]) / 1e3 for c in ctas if sel(c)]
+            # the same phase in SM clocks (both events on the CTA's own SM)
+            y = [(ck[c][e1] - ck[c][e0]) & 0xFFFFFFFF for c in ctas if sel(c)]
+            if x:
+                out.append(f"    {name:42s} {who:6s} {_pct(x)}   clocks {_pct(y)}")
+    spread = []
+    for cl in {c // size for c in ctas}:
+        t = [at[c][23] for c in ctas if c // size == cl]
+        if len(t) == size:
+            spread.append((max(t) - min(t)) / 1e3)
+    if spread:
+        out.append(f"    {'last-MMA spread inside a cluster':42s} {'':6s} {_pct(spread)}")
+    return out
+
+
 def summarise_small_m(launches):
     import numpy as np
     rows = []
@@ -136,6 +176,8 @@ def summarise_small_m(launches):
             x = (Lz["gt"][Lz["ev"] == e] - rel) / 1e3
             lines.append(f"  ev{e:2d} {EV.get(e, ''):28s} min {x.min():7.2f}  p50 {np.median(x):7.2f}  "
                          f"max {x.max():7.2f} us (from the release)")
+    if launches and (Lz["ev"] == 28).any():
+        lines += _cluster_phases(Lz)
     for i in range(1, len(rows)):
         r0, r1 = rows[i - 1], rows[i]
         lines.append(f"launch {i} ({r1[4]} CTAs): release-to-release {(r1[0] - r0[0]) / 1e3:.2f} us | previous end -> "
@@ -167,7 +209,7 @@ def run(args) -> int:
                if wl.epilogue in g.HAS_AUX else None)
         sets.append((prob.A.to(dev), prob.B.to(dev), prob.bias.to(dev), D, aux))
     plan = g.Plan(wl.m, wl.n, wl.k, wl.dtype, wl.epilogue, wl.bias_axis, wl.b_layout, kernel=args.kernel,
-                  block_n=args.block_n)
+                  block_n=args.block_n, split_k=args.split_k)
     if wl.dtype == "e4m3":
         plan.set_scales(torch.tensor([prob.scale_a], device=dev), torch.tensor([prob.scale_b], device=dev))
     info = plan.info
@@ -218,6 +260,7 @@ def main(argv=None) -> int:
     r.add_argument("--graph", action="store_true", help="replay the launches from a CUDA graph")
     r.add_argument("--kernel", default="auto", choices=["auto", "tc1", "tc2", "splitk"])
     r.add_argument("--block-n", type=int, default=0)
+    r.add_argument("--split-k", type=int, default=0)
     a = ap.parse_args(argv)
     if a.cmd == "build":
         print(build(a.force))
