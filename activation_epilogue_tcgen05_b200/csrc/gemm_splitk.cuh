@@ -313,18 +313,25 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const int gl = unit / QUADS, u = unit - gl * QUADS;
                 const int col = n0 + 32 * ((int)rank + gl * (int)csize) + lane;
                 const bool col_ok = col < p.n;
-                // the S partials, added in rank order
+                // the S partials, all loaded first, then added in rank order
                 const float *src = reinterpret_cast<const float *>(smem + C::OFF_RED) +
                                    ((gl * (int)csize) * C::SLOT_BYTES + u * 512 + lane * 16) / 4;
-                float4 sum = *reinterpret_cast<const float4 *>(src);
-                for (uint32_t r = 1; r < csize; ++r) {
-                    const float4 f = *reinterpret_cast<const float4 *>(src + r * (C::SLOT_BYTES / 4));
-                    sum.x += f.x;
-                    sum.y += f.y;
-                    sum.z += f.z;
-                    sum.w += f.w;
+                float4 pv[C::MAX_SPLIT];
+#pragma unroll
+                for (int r = 0; r < C::MAX_SPLIT; ++r)
+                    if (r < (int)csize) pv[r] = *reinterpret_cast<const float4 *>(src + r * (C::SLOT_BYTES / 4));
+                float4 sum = pv[0];
+#pragma unroll
+                for (int r = 1; r < C::MAX_SPLIT; ++r) {
+                    if (r < (int)csize) {
+                        sum.x += pv[r].x;
+                        sum.y += pv[r].y;
+                        sum.z += pv[r].z;
+                        sum.w += pv[r].w;
+                    }
                 }
                 const float part[4] = {sum.x, sum.y, sum.z, sum.w};
+                if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 33, tile_n, unit);
                 // every word of the mask pitch belongs to exactly one group of one tile;
                 // columns at or past n contribute 0 bits, so padding words come out 0
                 const int64_t word = (col - lane) / 32;
@@ -332,34 +339,39 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     if (j == gl) cb = cbias[j];
+                // the four rows' values first, without branches, then their stores
+                float y[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const int i = 4 * u + c;
-                    if (i < p.m) {
-                        float x = part[c] * alpha;
-                        if constexpr (C::EPI != EPI_NONE) {
-                            if constexpr (C::AXIS == AXIS_COL) x += cb;
-                            else if (has_bias) x += O::load(p.bias, i);
-                        }
-                        if constexpr (C::EPI == EPI_RELU_AUX) {
-                            const uint32_t bits = __ballot_sync(0xFFFFFFFFu, col_ok && x > 0.0f);
-                            if (lane == 0) p.aux[(int64_t)i * p.aux_pitch_words + word] = bits;
-                        }
-                        const float y = activate<C::EPI>(x);
-                        if (col_ok) {
-                            if constexpr (C::QOUT) {
-                                // e4m3 code, round to nearest even, saturating at +-448
-                                amax_l = fmaxf(amax_l, fabsf(y));
-                                p.dq[(int64_t)i * p.n + col] =
-                                    __nv_cvt_float_to_fp8(y * inv_out, __NV_SATFINITE, __NV_E4M3);
-                            } else if constexpr (C::DT == DT_F16) {
-                                D[(int64_t)i * p.n + col] = __float2half_rn(y);
-                            } else {
-                                D[(int64_t)i * p.n + col] = __float2bfloat16_rn(y);
-                            }
+                    float x = part[c] * alpha;
+                    if constexpr (C::EPI != EPI_NONE) {
+                        if constexpr (C::AXIS == AXIS_COL) x += cb;
+                        else if (has_bias && i < p.m) x += O::load(p.bias, i);
+                    }
+                    if constexpr (C::EPI == EPI_RELU_AUX) {
+                        const uint32_t bits = __ballot_sync(0xFFFFFFFFu, col_ok && x > 0.0f);
+                        if (lane == 0 && i < p.m) p.aux[(int64_t)i * p.aux_pitch_words + word] = bits;
+                    }
+                    y[c] = activate<C::EPI>(x);
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int i = 4 * u + c;
+                    if (col_ok && i < p.m) {
+                        if constexpr (C::QOUT) {
+                            // e4m3 code, round to nearest even, saturating at +-448
+                            amax_l = fmaxf(amax_l, fabsf(y[c]));
+                            p.dq[(int64_t)i * p.n + col] =
+                                __nv_cvt_float_to_fp8(y[c] * inv_out, __NV_SATFINITE, __NV_E4M3);
+                        } else if constexpr (C::DT == DT_F16) {
+                            D[(int64_t)i * p.n + col] = __float2half_rn(y[c]);
+                        } else {
+                            D[(int64_t)i * p.n + col] = __float2bfloat16_rn(y[c]);
                         }
                     }
                 }
+                if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 34, tile_n, unit);
             }
         }
         if constexpr (C::QOUT) {
@@ -373,16 +385,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncwarp();
     ptx::tc_fence_before();
     __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc<1>(tmem_base, C::TMEM_COLS);
+    }
     // The cluster's CTAs leave together.  (Each one has already received every byte sent to
     // it, so nothing is in flight towards its shared memory; the relaxed arrival does not wait
     // for this thread's global stores.)
     ptx::cluster_arrive_relaxed();
     ptx::cluster_wait();
-    if (warp == 1) {
-        ptx::tc_fence_after();
-        ptx::tmem_dealloc<1>(tmem_base, C::TMEM_COLS);
-        if (lane == 0) trace_stage(p.trace, 3, tr_i, 29, tile_n, (int)rank);
-    }
+    if (warp == 1 && lane == 0) trace_stage(p.trace, 3, tr_i, 29, tile_n, (int)rank);
 }
 
 }  // namespace gemm_epi

@@ -38,7 +38,8 @@ TRACE_CAP = 1 << 22
 EV = {10: "CTA start", 11: "after the dependency wait", 20: "stage load issued", 22: "stage ready (MMA)",
       23: "last MMA issued", 24: "accumulator wait", 25: "accumulator free", 26: "accumulator ready",
       27: "epilogue piece done", 28: "partials received", 29: "CTA end", 30: "finisher: flags seen",
-      31: "finisher: partials added", 32: "publisher: flag raised"}
+      31: "finisher: partials added", 32: "publisher: flag raised", 33: "unit's partials added",
+      34: "unit's outputs stored"}
 
 
 def build(force: bool = False) -> str:
@@ -127,7 +128,7 @@ def _cluster_phases(L):
     for c, e, t, kb, k in zip(L["cta"].tolist(), L["ev"].tolist(), L["gt"].tolist(), L["kb"].tolist(),
                               L["clk"].tolist()):
         d = at.setdefault(c, {})
-        if e in (23, 26, 27, 28, 29, 11):
+        if e in (23, 26, 27, 28, 29, 11) or (e in (33, 34) and e not in d):
             d[e] = t
             ck.setdefault(c, {})[e] = k
         if e in (26, 28, 27, 29):
@@ -140,11 +141,12 @@ def _cluster_phases(L):
     out = [f"  per-CTA phases of that launch (us), p10 / p50 / p90 over CTAs, cluster size {size}:"]
     for name, e0, e1 in (("release -> last MMA issued", 11, 23), ("last MMA -> accumulator ready", 23, 26),
                          ("accumulator ready -> partials received", 26, 28),
-                         ("partials received -> epilogue done", 28, 27), ("epilogue done -> CTA end", 27, 29)):
+                         ("partials received -> epilogue done", 28, 27), ("epilogue done -> CTA end", 27, 29),
+                         ("  received -> first unit's sum", 28, 33), ("  first unit: sum -> stored", 33, 34)):
         for who, sel in (("rank 0", lambda c: at[c]["rank"] == 0), ("others", lambda c: at[c]["rank"] != 0)):
-            x = [(at[c][e1] - at[c][e0]) / 1e3 for c in ctas if sel(c)]
+            x = [(at[c][e1] - at[c][e0]) / 1e3 for c in ctas if sel(c) and e0 in at[c] and e1 in at[c]]
             # the same phase in SM clocks (both events on the CTA's own SM)
-            y = [(ck[c][e1] - ck[c][e0]) & 0xFFFFFFFF for c in ctas if sel(c)]
+            y = [(ck[c][e1] - ck[c][e0]) & 0xFFFFFFFF for c in ctas if sel(c) and e0 in ck[c] and e1 in ck[c]]
             if x:
                 out.append(f"    {name:42s} {who:6s} {_pct(x)}   clocks {_pct(y)}")
     spread = []
