@@ -197,13 +197,15 @@ int choose(Plan *P) {
     int kernel = P->opts.kernel;
     if (kernel == GEMM_EPI_KERNEL_AUTO) {
         // small m: swapped split-K; enough 256 x 256 tiles for every SM pair: CTA pairs
-        // (half the operand traffic per SM); otherwise single CTAs.  Split-K up to m = 32:
-        // above, its MMA tile is 64 wide and the single CTAs with a four-part split tail are
-        // as fast or faster (Linear 4096 -> 4096 fp16: m = 48 17.8 vs 17.1 us, m = 64 18.5 vs
-        // 17.1 us).  (The split-K kernel has no backward epilogue.)
+        // (half the operand traffic per SM); otherwise single CTAs.  Split-K up to m = 64,
+        // where it streams the weight faster than the single CTAs with a four-part split tail
+        // (m = 64, fp16 GELU: 10.3 vs 17.1 us at 4096 x 4096, 23.5 vs 31.4 us at n = 4096,
+        // k = 14336, 28.3 vs 29.1 us at n = 14336, k = 4096; e4m3 7.5 vs 14.2 us); above, its
+        // ring holds too few stages (m = 96: 17.5 vs 16.7 us).  (The split-K kernel has no
+        // backward epilogue.)
         const int64_t pair_tiles = ((m + 255) / 256) * ((n + 255) / 256);
         const int sms_auto = P->opts.max_ctas > 0 ? std::min(P->opts.max_ctas, P->num_sms) : P->num_sms;
-        if (m <= 32 && P->kepi != EPI_DRELU && !P->a_km) kernel = GEMM_EPI_KERNEL_SPLITK;
+        if (m <= 64 && P->kepi != EPI_DRELU && !P->a_km) kernel = GEMM_EPI_KERNEL_SPLITK;
         else if (pair_tiles >= sms_auto / 2) kernel = GEMM_EPI_KERNEL_TC2;
         else kernel = GEMM_EPI_KERNEL_TC1;
     }
@@ -242,8 +244,18 @@ int choose(Plan *P) {
         const int max_split = sk_max_split(P->nm);
         int split = P->opts.split_k;
         if (split <= 0) {
-            split = (int)std::max<int64_t>(1, sms / std::max<int64_t>(1, tiles_n));
-            if (split > max_split) split = max_split;
+            // Every cluster of the launch must be resident at once, or the last ones wait for a
+            // second wave.  Measured (m = 16, k = 4096, fp16): clusters of up to 4 CTAs, at most
+            // 128 CTAs, all fit (n = 2048: 4 x 16 CTAs 7.9 us against 8 x 16 11.1 us; n = 3072:
+            // 4 x 24 8.1 against 6 x 24 13.1; n = 6144: 2 x 48 12.8 against 3 x 48 20.1), and
+            // so do 8 clusters of 8 (n = 1024: 5.1 us).
+            const int64_t cap = std::min<int64_t>(128, sms);
+            if (tiles_n * 8 <= 64 && max_split >= 8 && 64 <= cap) {
+                split = 8;
+            } else {
+                split = std::min(4, max_split);
+                while (split > 1 && tiles_n * split > cap) --split;
+            }
         }
         if (split > max_split || split < 1) return GEMM_EPI_ERR_ARG;
         if (split > num_kb) split = (int)num_kb;

@@ -278,7 +278,7 @@ def test_mlp_block_unfused_baseline(dtype, m):
 @pytest.mark.parametrize("m", [16, 32, 64, 1000])
 def test_mlp_block_batch_sizes(m):
     up, down = run_mlp(m, 512, 1024, "e4m3", "gelu_bias", "kn", seed=36)
-    if m <= 32:
+    if m <= 64:
         assert up["kernel"] == g.KERNEL_SPLITK and down["kernel"] == g.KERNEL_SPLITK
     else:
         assert up["kernel"] != g.KERNEL_SPLITK and down["kernel"] != g.KERNEL_SPLITK

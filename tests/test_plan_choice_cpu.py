@@ -76,14 +76,14 @@ def test_fp8_gelu_bias(g):
 
 
 # ------------------------------------------------------------------ family boundaries
-@pytest.mark.parametrize("m,kernel", [(1, "splitk"), (16, "splitk"), (32, "splitk"), (33, "tc1"),
-                                      (64, "tc1"), (128, "tc1"), (256, "tc1")])
+@pytest.mark.parametrize("m,kernel", [(1, "splitk"), (16, "splitk"), (32, "splitk"), (33, "splitk"),
+                                      (64, "splitk"), (65, "tc1"), (128, "tc1"), (256, "tc1")])
 def test_batch_boundary(g, m, kernel):
     p = pv(g, m, 4096, 4096, "f16", "gelu_bias", "col", "nk")
     assert p["kernel"] == {"splitk": g.KERNEL_SPLITK, "tc1": g.KERNEL_TC1}[kernel]
 
 
-@pytest.mark.parametrize("m,nm", [(1, 16), (16, 16), (17, 32), (32, 32)])
+@pytest.mark.parametrize("m,nm", [(1, 16), (16, 16), (17, 32), (32, 32), (33, 64), (64, 64)])
 def test_splitk_batch_tile(g, m, nm):
     assert pv(g, m, 4096, 4096, "f16", "gelu_bias", "col", "nk")["block_m"] == nm
 
@@ -207,3 +207,20 @@ def test_raster_from_l2_budget(g):
     # the small-m kernel has no raster
     p = pv(g, 16, 4096, 4096, "f16", "gelu_bias", "col", "nk")
     assert (p["group_m"], p["group_n"]) == (0, 0)
+
+
+# clusters that can all be resident at once: at most 4 CTAs a cluster and 128 CTAs a launch, or
+# 8 clusters of 8 (measured split sizes, m = 16, k = 4096)
+@pytest.mark.parametrize("n,split,grid", [(512, 8, 32), (1024, 8, 64), (2048, 4, 64), (3072, 4, 96),
+                                          (4096, 4, 128), (5120, 3, 120), (6144, 2, 96), (8192, 2, 128),
+                                          (12288, 1, 96), (14336, 1, 112)])
+def test_splitk_cluster_residency(g, n, split, grid):
+    p = pv(g, 16, n, 4096, "f16", "gelu_bias", "col", "nk")
+    assert p["kernel"] == g.KERNEL_SPLITK
+    assert (p["split_k"], p["cluster"], p["grid"]) == (split, split, grid)
+
+
+def test_splitk_m64_split_limit(g):
+    # NM = 64: splits up to 4
+    p = pv(g, 64, 1024, 4096, "f16", "gelu_bias", "col", "nk")
+    assert (p["kernel"], p["block_m"], p["split_k"], p["grid"]) == (g.KERNEL_SPLITK, 64, 4, 32)
