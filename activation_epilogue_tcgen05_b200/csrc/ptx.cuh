@@ -2,9 +2,10 @@
 // waits, TMA tiled copies, tcgen05 (tensor memory, MMA, commit, loads) and
 // the shared-memory / instruction descriptors the MMA reads.
 //
-// Only forms from the public PTX ISA are used.  No TMA load here carries
-// .multicast::cluster: every load reads this GPU's own global memory into the
-// issuing CTA's shared memory.
+// Only forms from the public PTX ISA are used.  No TMA load here is a cluster
+// multicast: every load reads this GPU's own global memory into the issuing
+// CTA's shared memory (or, in the CTA-pair form, its own half of the pair's
+// tile, signalled on the leader's barrier).
 #pragma once
 #include <cstdint>
 #include <cuda.h>
