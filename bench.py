@@ -285,11 +285,15 @@ def oracle_rows_rate(wl, prob, target_s: float, max_rows=None):
         return time.perf_counter() - t0
 
     threads = oracle.threads()
-    rows = min(wl.m, max(1, threads))
+    cap = wl.m if max_rows is None else min(wl.m, max_rows)
+    rows = min(cap, max(1, threads))
+    run(rows)                      # warm-up (thread start-up, first touch), not timed
     dt = run(rows)
-    if dt < target_s:
-        rows = int(min(wl.m if max_rows is None else max_rows,
-                       max(rows, rows * target_s / max(dt, 1e-6))))
+    # grow the sample towards target_s (a few rounds: the first timings are the noisiest)
+    for _ in range(4):
+        if dt >= 0.8 * target_s or rows >= cap:
+            break
+        rows = int(min(cap, max(rows + 1, rows * target_s / max(dt, 1e-6))))
         dt = run(rows)
     flops = 2.0 * rows * wl.n * wl.k
     return flops / dt / 1e12, rows, dt, threads
