@@ -145,7 +145,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         *abort_flag = 0;
         ptx::fence_mbarrier_init();
         // the one arrival of red_bar's phase, with the bytes every CTA of the cluster will send
-        if (groups > 0) ptx::mbar_arrive_expect_tx(red_bar, (uint32_t)(groups * (int)csize * C::SLOT_BYTES));
+        if (groups > 0 && csize > 1u)
+            ptx::mbar_arrive_expect_tx(red_bar, (uint32_t)(groups * (int)csize * C::SLOT_BYTES));
     }
     if (warp == 1) {
         ptx::tmem_alloc<1>(ptx::smem_addr(tmem_slot), C::TMEM_COLS);
@@ -264,6 +265,51 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // -------------------------------------------------------------- epilogue
     // warps 2..5: thread (q, lane) owns accumulator lane 32q + lane = output column n0 + 32q + lane.
     const int q = warp & 3;
+    using O = OutT<C::DT>;
+    using T = typename O::type;
+    T *D = reinterpret_cast<T *>(p.D);
+    const bool has_bias = p.bias != nullptr;
+    float amax_l = 0.0f;
+    // The fused epilogue of rows 4u .. 4u+3 of column group `grp` (this thread's column
+    // n0 + 32 grp + lane), from their fp32 sums `part`: the four rows' values first, without
+    // branches, then their stores.
+    auto emit4 = [&](int grp, int u, const float (&part)[4], float cb) {
+        const int col = n0 + 32 * grp + lane;
+        const bool col_ok = col < p.n;
+        // every word of the mask pitch belongs to exactly one group of one tile;
+        // columns at or past n contribute 0 bits, so padding words come out 0
+        const int64_t word = (col - lane) / 32;
+        float y[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int i = 4 * u + c;
+            float x = part[c] * alpha;
+            if constexpr (C::EPI != EPI_NONE) {
+                if constexpr (C::AXIS == AXIS_COL) x += cb;
+                else if (has_bias && i < p.m) x += O::load(p.bias, i);
+            }
+            if constexpr (C::EPI == EPI_RELU_AUX) {
+                const uint32_t bits = __ballot_sync(0xFFFFFFFFu, col_ok && x > 0.0f);
+                if (lane == 0 && i < p.m) p.aux[(int64_t)i * p.aux_pitch_words + word] = bits;
+            }
+            y[c] = activate<C::EPI>(x);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int i = 4 * u + c;
+            if (col_ok && i < p.m) {
+                if constexpr (C::QOUT) {
+                    // e4m3 code, round to nearest even, saturating at +-448
+                    amax_l = fmaxf(amax_l, fabsf(y[c]));
+                    p.dq[(int64_t)i * p.n + col] = __nv_cvt_float_to_fp8(y[c] * inv_out, __NV_SATFINITE, __NV_E4M3);
+                } else if constexpr (C::DT == DT_F16) {
+                    D[(int64_t)i * p.n + col] = __float2half_rn(y[c]);
+                } else {
+                    D[(int64_t)i * p.n + col] = __float2bfloat16_rn(y[c]);
+                }
+            }
+        }
+    };
     __syncwarp();
     ptx::cluster_wait();     // every CTA's red_bar is initialised
     if (epi) {
@@ -287,32 +333,41 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < C::NM; ++j) acc[j] = 0.0f;
         }
-        // this CTA's partial of group q goes to slot (q / S) * S + rank of the group's owner;
-        // a CTA without work (or after an abort) sends zeros, so every owner's count completes
-        const uint32_t owner = (uint32_t)q % csize;
-        const uint32_t slot = ((uint32_t)q / csize) * csize + rank;
-        const uint32_t dst = ptx::mapa(sb + C::OFF_RED + slot * C::SLOT_BYTES + (uint32_t)lane * 16u, owner);
-        const uint32_t dbar = ptx::mapa(red_bar, owner);
+        if (csize == 1u) {
+            // a cluster of one CTA: the accumulator is the whole sum; each warp finishes its own
+            // column group straight from its registers
+            if (have) {
+                float cb = 0.0f;
 #pragma unroll
-        for (int u = 0; u < C::NM / 4; ++u)
-            ptx::st_async_v4(dst + (uint32_t)u * 512u, acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3], dbar);
+                for (int j = 0; j < 4; ++j)
+                    if (j == q) cb = cbias[j];
+#pragma unroll
+                for (int u = 0; u < C::NM / 4; ++u) {
+                    const float part[4] = {acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3]};
+                    emit4(q, u, part, cb);
+                }
+            }
+        } else {
+            // this CTA's partial of group q goes to slot (q / S) * S + rank of the group's owner;
+            // a CTA without work (or after an abort) sends zeros, so every owner's count completes
+            const uint32_t owner = (uint32_t)q % csize;
+            const uint32_t slot = ((uint32_t)q / csize) * csize + rank;
+            const uint32_t dst = ptx::mapa(sb + C::OFF_RED + slot * C::SLOT_BYTES + (uint32_t)lane * 16u, owner);
+            const uint32_t dbar = ptx::mapa(red_bar, owner);
+#pragma unroll
+            for (int u = 0; u < C::NM / 4; ++u)
+                ptx::st_async_v4(dst + (uint32_t)u * 512u, acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3], dbar);
+        }
     }
 
-    if (epi && groups > 0) {
-        using O = OutT<C::DT>;
-        using T = typename O::type;
+    if (epi && groups > 0 && csize > 1u) {
         const int ew = warp - 2;
-        float amax_l = 0.0f;
         if (wait_bounded<true>(red_bar, 0, abort_flag, p.status, ST_TIMEOUT_SPLITK)) {
             if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 28, tile_n, (int)rank);
-            const bool has_bias = p.bias != nullptr;
-            T *D = reinterpret_cast<T *>(p.D);
             constexpr int QUADS = C::NM / 4;
             // work units (owned group, block of 4 rows), dealt round-robin to the 4 epilogue warps
             for (int unit = ew; unit < groups * QUADS; unit += 4) {
                 const int gl = unit / QUADS, u = unit - gl * QUADS;
-                const int col = n0 + 32 * ((int)rank + gl * (int)csize) + lane;
-                const bool col_ok = col < p.n;
                 // the S partials, all loaded first, then added in rank order
                 const float *src = reinterpret_cast<const float *>(smem + C::OFF_RED) +
                                    ((gl * (int)csize) * C::SLOT_BYTES + u * 512 + lane * 16) / 4;
@@ -332,49 +387,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
                 const float part[4] = {sum.x, sum.y, sum.z, sum.w};
                 if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 33, tile_n, unit);
-                // every word of the mask pitch belongs to exactly one group of one tile;
-                // columns at or past n contribute 0 bits, so padding words come out 0
-                const int64_t word = (col - lane) / 32;
                 float cb = 0.0f;
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     if (j == gl) cb = cbias[j];
-                // the four rows' values first, without branches, then their stores
-                float y[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int i = 4 * u + c;
-                    float x = part[c] * alpha;
-                    if constexpr (C::EPI != EPI_NONE) {
-                        if constexpr (C::AXIS == AXIS_COL) x += cb;
-                        else if (has_bias && i < p.m) x += O::load(p.bias, i);
-                    }
-                    if constexpr (C::EPI == EPI_RELU_AUX) {
-                        const uint32_t bits = __ballot_sync(0xFFFFFFFFu, col_ok && x > 0.0f);
-                        if (lane == 0 && i < p.m) p.aux[(int64_t)i * p.aux_pitch_words + word] = bits;
-                    }
-                    y[c] = activate<C::EPI>(x);
-                }
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int i = 4 * u + c;
-                    if (col_ok && i < p.m) {
-                        if constexpr (C::QOUT) {
-                            // e4m3 code, round to nearest even, saturating at +-448
-                            amax_l = fmaxf(amax_l, fabsf(y[c]));
-                            p.dq[(int64_t)i * p.n + col] =
-                                __nv_cvt_float_to_fp8(y[c] * inv_out, __NV_SATFINITE, __NV_E4M3);
-                        } else if constexpr (C::DT == DT_F16) {
-                            D[(int64_t)i * p.n + col] = __float2half_rn(y[c]);
-                        } else {
-                            D[(int64_t)i * p.n + col] = __float2bfloat16_rn(y[c]);
-                        }
-                    }
-                }
+                emit4((int)rank + gl * (int)csize, u, part, cb);
                 if (warp == 2 && lane == 0) trace_stage(p.trace, 2, tr_i, 34, tile_n, unit);
             }
         }
-        if constexpr (C::QOUT) {
+    }
+    if constexpr (C::QOUT) {
+        if (epi && groups > 0) {
             // one atomic per warp: the launch's max |y| (non-negative floats order as their bits)
             const unsigned int wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax_l));
             if (lane == 0 && p.amax != nullptr && wmax != 0u) atomicMax(p.amax, wmax);
