@@ -100,6 +100,17 @@ def check_qout(wl, scale_factor=1.0, **opts):
     return frac_unique, info
 
 
+@pytest.mark.parametrize("split", [1, 3])
+@pytest.mark.parametrize("epilogue", ["gelu_bias", "relu_bias"])
+def test_fp8_out_splitk_cluster_forms(split, epilogue):
+    """e4m3 output from the small-m kernel: one-CTA clusters (finished from registers) and
+    clusters of 3 (partials exchanged), codes and amax against the oracle."""
+    wl = Workload("q_sk", 24, 1008, 1024, "e4m3", epilogue, "col", "kn", seed=72)
+    frac, info = check_qout(wl, kernel="splitk", split_k=split)
+    assert info["kernel"] == g.KERNEL_SPLITK and info["cluster"] == split
+    assert frac > 0.5          # most codes decided uniquely (as in the single-GEMM variants)
+
+
 # ------------------------------------------------------------------ FP8 output, single GEMM
 @pytest.mark.parametrize("layout", ["kn", "nk"])
 @pytest.mark.parametrize("axis", ["row", "col"])

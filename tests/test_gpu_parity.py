@@ -312,6 +312,21 @@ def test_splitk_cluster_sizes(split):
     assert worst <= 1.0
 
 
+@pytest.mark.parametrize("m", [1, 16, 29, 64])
+@pytest.mark.parametrize("dtype,epilogue,axis,layout", [
+    ("f16", "gelu_bias", "col", "nk"), ("bf16", "relu_aux_bias", "row", "kn"),
+    ("bf16", "bias", "col", "nk"), ("e4m3", "relu_bias", "row", "kn"), ("f16", "tanh_bias", "row", "kn")])
+def test_splitk_one_cta_clusters(m, dtype, epilogue, axis, layout):
+    """split_k = 1: each CTA holds its tile's whole sum and every epilogue warp finishes its own
+    32 columns straight from its accumulator registers (no exchange), over ragged n, batch tiles
+    of 16 / 32 / 64 rows and rows past m."""
+    wl = Workload("sk_one", m, 1008, 1000 if dtype != "e4m3" else 1024, dtype, epilogue, axis, layout, seed=71)
+    prob = make_problem(wl)
+    worst, info = check_against_oracle(wl, prob, kernel="splitk", split_k=1)
+    assert info["split_k"] == 1 and info["cluster"] == 1 and info["grid"] == 8
+    assert worst <= 1.0
+
+
 @pytest.mark.parametrize("kernel,block_n", [("tc1", 128), ("tc1", 256), ("tc2", 256), ("tc2", 512)])
 @pytest.mark.parametrize("dtype,b_layout,a_layout", [("bf16", "kn", "mk"), ("f16", "nk", "mk"), ("bf16", "kn", "km"),
                                                      ("e4m3", "kn", "mk"), ("e4m3", "nk", "km")])
