@@ -103,7 +103,9 @@ enum gemm_epi_bias_axis { GEMM_EPI_BIAS_ROW = 0, GEMM_EPI_BIAS_COL = 1 };
  * forward epilogues, not with the backward epilogues or an e4m3 output. */
 enum gemm_epi_b_layout { GEMM_EPI_B_KN = 0, GEMM_EPI_B_NK = 1, GEMM_EPI_A_KM = 2 };
 
-/* Kernel families a plan can use (GEMM_EPI_KERNEL_AUTO lets the plan choose). */
+/* Kernel families a plan can use.  GEMM_EPI_KERNEL_AUTO lets the plan choose: SPLITK for
+ * m <= 64 (forward epilogues, A stored (m, k)), TC2 when there is a 256 x 256 tile for every SM
+ * pair, TC1 otherwise. */
 enum gemm_epi_kernel {
     GEMM_EPI_KERNEL_AUTO = 0,
     GEMM_EPI_KERNEL_TC1 = 1,    /* persistent, one CTA per 128 x block_n tile           */
@@ -141,7 +143,10 @@ typedef struct gemm_epi_options {
                           auto, which takes 512 for TC2 with 16-bit operands, an epilogue
                           without GELU / tanh and at least four waves of 256 x 512 tiles).  TC2 with e4m3 and B stored (k, n) supports
                           256 and 512 only (128 is ERR_UNSUPPORTED)                       */
-    int32_t split_k;   /* SPLITK: CTAs per cluster along k (1..8; 0 = auto).  TC1/TC2:
+    int32_t split_k;   /* SPLITK: CTAs per cluster along k (1..8; 0 = auto: 8 when there are
+                          at most 8 tiles of 128 columns, else the largest of 4, 3, 2, 1 that
+                          keeps the launch at or under 128 CTAs, so that every cluster is
+                          resident at once; capped at the split the batch tile allows).  TC1/TC2:
                           cap on the parts a tail tile is split into (0 = auto: 2 behind
                           whole waves; with fewer tiles than SMs up to 4, at least 8
                           128-byte k-atoms a part).  The parts are whole ring stages
